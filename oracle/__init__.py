@@ -1,0 +1,156 @@
+"""fp64 CPU oracle for the DM0.5 action-expert (suffix) attention.
+
+TEST INFRASTRUCTURE.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this package.  The CUDA library in
+``gqa_prefix_suffix_b200`` never imports it and shares no code with it.
+
+The arithmetic lives in ``oracle.c`` (plain C, double precision); this module
+only compiles it with gcc and marshals numpy arrays through ctypes.  What it
+computes and the readings it takes are stated in the header of ``oracle.c``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_default = None
+
+
+def build(force: bool = False, src: str = _SRC, out: str = _LIB, extra_flags=()) -> str:
+    """Compile oracle.c into a shared library (gcc -O2, OpenMP, no fast-math)."""
+    if (not force and os.path.exists(out)
+            and os.path.getmtime(out) >= os.path.getmtime(src)):
+        return out
+    tmp = out + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-O2", "-fno-fast-math", "-ffp-contract=off", "-fopenmp",
+           "-fPIC", "-shared", "-std=c11", *extra_flags, src, "-o", tmp, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, out)
+    return out
+
+
+def _bits(a) -> np.ndarray:
+    """bf16 data as a contiguous uint16 bit-pattern array.
+
+    Accepts a numpy uint16 array (already bit patterns) or a torch bfloat16
+    tensor on the CPU."""
+    if isinstance(a, np.ndarray):
+        if a.dtype != np.uint16:
+            raise TypeError("numpy inputs must be uint16 bf16 bit patterns")
+        return np.ascontiguousarray(a)
+    import torch  # local: the oracle itself needs only numpy
+    if a.dtype != torch.bfloat16:
+        raise TypeError("torch inputs must be bfloat16")
+    return np.ascontiguousarray(a.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16))
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+class Oracle:
+    """ctypes front end of one compiled copy of oracle.c."""
+
+    def __init__(self, lib_path: str):
+        lib = ctypes.CDLL(lib_path)
+        p = ctypes.c_void_p
+        i = ctypes.c_int
+        lib.oracle_suffix_attn_range.argtypes = [p] * 9 + [i] * 6 + [i, i, i]
+        lib.oracle_suffix_attn_range.restype = i
+        lib.oracle_suffix_attn.argtypes = [p] * 9 + [i] * 6 + [i]
+        lib.oracle_suffix_attn.restype = i
+        lib.oracle_merge_parts.argtypes = [p, p, i, ctypes.c_long, i, p, p]
+        lib.oracle_merge_parts.restype = i
+        lib.oracle_max_threads.argtypes = []
+        lib.oracle_max_threads.restype = i
+        self.lib = lib
+        self.path = lib_path
+
+    def max_threads(self) -> int:
+        return int(self.lib.oracle_max_threads())
+
+    def suffix_attn(self, q, k_prefix, v_prefix, prefix_valid_len, prefix_mask, k_suffix,
+                    v_suffix, B, Hq, Hkv, P, S, D, key_range=None, nthreads: int = 1):
+        """Return (out float64 [B,Hq,S,D], lse float64 [B,Hq,S]).
+
+        key_range=(lo, hi) restricts the keys to the index-space slice [lo, hi)
+        where [0, P) are prefix positions and [P, P+S) suffix positions."""
+        qb, kpb, vpb = _bits(q), _bits(k_prefix), _bits(v_prefix)
+        ksb, vsb = _bits(k_suffix), _bits(v_suffix)
+        if qb.size != B * Hq * S * D or ksb.size != B * Hkv * S * D or vsb.size != B * Hkv * S * D:
+            raise ValueError("q/k_suffix/v_suffix size does not match the dims")
+        if kpb.size != B * Hkv * P * D or vpb.size != B * Hkv * P * D:
+            raise ValueError("k_prefix/v_prefix size does not match the dims")
+        vl = None
+        if prefix_valid_len is not None:
+            vl = np.ascontiguousarray(np.asarray(prefix_valid_len, dtype=np.int32).reshape(B))
+        mk = None
+        if prefix_mask is not None:
+            mk = np.ascontiguousarray(np.asarray(prefix_mask, dtype=np.uint8).reshape(B, P))
+        out = np.zeros((B, Hq, S, D), dtype=np.float64)
+        lse = np.zeros((B, Hq, S), dtype=np.float64)
+        lo, hi = (0, P + S) if key_range is None else key_range
+        rc = self.lib.oracle_suffix_attn_range(
+            _ptr(qb), _ptr(kpb), _ptr(vpb), _ptr(vl), _ptr(mk), _ptr(ksb), _ptr(vsb),
+            _ptr(out), _ptr(lse), B, Hq, Hkv, P, S, D, int(lo), int(hi), int(nthreads))
+        if rc != 0:
+            raise ValueError(f"oracle_suffix_attn_range failed with status {rc}")
+        return out, lse
+
+    def merge_parts(self, o_parts, lse_parts):
+        """Combine partial results over disjoint key sets (log-sum-exp identity).
+
+        o_parts [n, rows, D] float64, lse_parts [n, rows] -> (out [rows, D], lse [rows])."""
+        o_parts = np.ascontiguousarray(o_parts, dtype=np.float64)
+        lse_parts = np.ascontiguousarray(lse_parts, dtype=np.float64)
+        n, rows, D = o_parts.shape
+        out = np.zeros((rows, D), dtype=np.float64)
+        lse = np.zeros((rows,), dtype=np.float64)
+        rc = self.lib.oracle_merge_parts(_ptr(o_parts), _ptr(lse_parts), n, rows, D,
+                                         _ptr(out), _ptr(lse))
+        if rc != 0:
+            raise ValueError(f"oracle_merge_parts failed with status {rc}")
+        return out, lse
+
+    def inputs_call(self, inp, nthreads: int = 1, key_range=None):
+        """Run on an object with the attributes of a SuffixAttnInputs."""
+        return self.suffix_attn(inp.q, inp.k_prefix, inp.v_prefix, inp.prefix_valid_len,
+                                inp.prefix_mask, inp.k_suffix, inp.v_suffix,
+                                inp.B, inp.Hq, inp.Hkv, inp.P, inp.S, inp.D,
+                                key_range=key_range, nthreads=nthreads)
+
+
+def default() -> Oracle:
+    """The oracle built from oracle.c next to this file (compiled on demand)."""
+    global _default
+    with _lock:
+        if _default is None:
+            _default = Oracle(build())
+    return _default
+
+
+def max_threads() -> int:
+    return default().max_threads()
+
+
+def suffix_attn(*args, **kwargs):
+    """Oracle.suffix_attn on the default build."""
+    return default().suffix_attn(*args, **kwargs)
+
+
+def merge_parts(o_parts, lse_parts):
+    """Oracle.merge_parts on the default build."""
+    return default().merge_parts(o_parts, lse_parts)
+
+
+def inputs_call(inp, nthreads: int = 1, key_range=None):
+    """Oracle.inputs_call on the default build."""
+    return default().inputs_call(inp, nthreads=nthreads, key_range=key_range)

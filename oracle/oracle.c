@@ -1,0 +1,247 @@
+/*
+ * oracle.c -- plain fp64 CPU reference for the DM0.5 action-expert (suffix)
+ * attention.  TEST INFRASTRUCTURE: only the tests, the smoke check and the
+ * benchmark's CPU-baseline leg may load this file.  The product path (the
+ * CUDA library) never calls it and shares no code, header, table or helper
+ * with it.
+ *
+ * What it computes (page "TensorRT+Triton+FlexAttention: OpenDM VLA
+ * 快速推理加速栈深度剖析", section 2.2 "Triton 大 Kernel"): the action-expert
+ * (suffix) attention reads the prefix KV cache and the suffix's own K/V at
+ * once, applies the prefix-visibility mask, takes a softmax over the scaled
+ * logits and forms the value-weighted sum.  The suffix path's shape table in
+ * the same section fixes head_dim 256 and 8 query heads over 4 KV heads
+ * (GQA).  The prefix cache is padded to a length bucket (same page, section 3;
+ * page "DM05 推理指南", section "Fast Backend 约束"), hence a valid length.
+ *
+ * Readings taken where the pages are silent (each one is listed with its
+ * reason in the design notes):
+ *   - every suffix key is visible to every suffix query (bidirectional);
+ *   - prefix key j of sample b is visible iff j < clamp(valid_len[b], 0, P)
+ *     and (no mask given or mask[b, j] != 0); the same for every head/query;
+ *   - query head h reads KV head h / (Hq / Hkv) (contiguous groups);
+ *   - logits are scaled by 1 / sqrt(D); no soft-cap, no extra scalar;
+ *   - LSE is the natural-log log-sum-exp of the scaled logits.
+ *
+ * Arithmetic: every bf16 input is widened exactly to double; all sums,
+ * exponentials and logarithms are in double with the host libm (exp, log).
+ * The softmax is the plain two-pass form: max, then sum of exponentials.
+ * There is no blocking, no online rescaling and no reordering beyond that.
+ *
+ * Parity status: pinned (see tests/test_oracle.py): float64 library
+ * scaled-dot-product attention on tiny shapes, closed forms (all-equal
+ * logits, constant V, one visible key), invariants (masked rows ignored,
+ * prefix permutation), and an arbitrary-precision brute force.
+ */
+#include <math.h>
+#include <stddef.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* Exact widening of a bf16 bit pattern: bf16 is the upper half of an IEEE
+ * binary32, so shifting the 16 bits up gives the same value as a float. */
+static double bf16_bits_to_double(uint16_t h)
+{
+    uint32_t bits = ((uint32_t)h) << 16;
+    float f;
+    memcpy(&f, &bits, sizeof f);
+    return (double)f;
+}
+
+static int clamp_valid_len(const int32_t *valid_len, int b, int P)
+{
+    if (valid_len == NULL) return P;
+    int v = valid_len[b];
+    if (v < 0) return 0;
+    if (v > P) return P;
+    return v;
+}
+
+/* Key index space of one sample: [0, P) are the prefix positions, [P, P+S)
+ * the suffix positions.  Returns 1 if key x is visible to every query of
+ * sample b. */
+static int key_visible(int x, int P, int vl, const uint8_t *mask_row)
+{
+    if (x >= P) return 1; /* suffix keys: always visible */
+    if (x >= vl) return 0; /* bucket padding */
+    if (mask_row != NULL && mask_row[x] == 0) return 0;
+    return 1;
+}
+
+/* One (b, h, i) row restricted to keys x in [key_lo, key_hi) of the index
+ * space above.  Writes D outputs and the LSE.  If no key in the range is
+ * visible, writes O = 0 and LSE = -inf. */
+static void attend_row(const uint16_t *q_row, const uint16_t *kp, const uint16_t *vp,
+                       const uint16_t *ks, const uint16_t *vs, const uint8_t *mask_row,
+                       int vl, int P, int S, int D, int key_lo, int key_hi,
+                       double *logit_buf, double *o_row, double *lse_out)
+{
+    const double scale = 1.0 / sqrt((double)D);
+    int n = 0;
+    double m = -INFINITY;
+    /* pass 1: logits of the visible keys and their maximum */
+    for (int x = key_lo; x < key_hi; ++x) {
+        if (!key_visible(x, P, vl, mask_row)) continue;
+        const uint16_t *k_row = (x < P) ? kp + (size_t)x * D : ks + (size_t)(x - P) * D;
+        double dot = 0.0;
+        for (int d = 0; d < D; ++d)
+            dot += bf16_bits_to_double(q_row[d]) * bf16_bits_to_double(k_row[d]);
+        double l = scale * dot;
+        logit_buf[x - key_lo] = l;
+        if (l > m) m = l;
+        ++n;
+    }
+    for (int d = 0; d < D; ++d) o_row[d] = 0.0;
+    if (n == 0) {
+        *lse_out = -INFINITY;
+        return;
+    }
+    /* pass 2: normaliser Z = sum exp(l - m), LSE = m + ln Z */
+    double z = 0.0;
+    for (int x = key_lo; x < key_hi; ++x) {
+        if (!key_visible(x, P, vl, mask_row)) continue;
+        z += exp(logit_buf[x - key_lo] - m);
+    }
+    double lse = m + log(z);
+    /* pass 3: O = sum over visible keys of softmax weight times the V row */
+    for (int x = key_lo; x < key_hi; ++x) {
+        if (!key_visible(x, P, vl, mask_row)) continue;
+        double w = exp(logit_buf[x - key_lo] - lse);
+        const uint16_t *v_row = (x < P) ? vp + (size_t)x * D : vs + (size_t)(x - P) * D;
+        for (int d = 0; d < D; ++d) o_row[d] += w * bf16_bits_to_double(v_row[d]);
+    }
+    *lse_out = lse;
+}
+
+static int check_shape(int B, int Hq, int Hkv, int P, int S, int D)
+{
+    if (B < 1 || Hq < 1 || Hkv < 1 || P < 0 || S < 1 || D < 1) return -2;
+    if (Hq % Hkv != 0) return -2;
+    return 0;
+}
+
+/*
+ * Attention of every (b, h, i) over the keys x in [key_lo, key_hi) of the
+ * index space [0, P+S) (prefix positions, then suffix positions).  With
+ * key_lo = 0 and key_hi = P + S this is the full result.  Layouts (row-major,
+ * bf16 passed as uint16 bit patterns):
+ *   q [B,Hq,S,D], k_prefix/v_prefix [B,Hkv,P,D], k_suffix/v_suffix [B,Hkv,S,D],
+ *   prefix_valid_len int32 [B] or NULL, prefix_mask uint8 [B,P] or NULL,
+ *   out double [B,Hq,S,D], lse double [B,Hq,S].
+ * nthreads > 1 spreads the (b, h) pairs over OpenMP threads.
+ * Returns 0, -1 for a NULL pointer, -2 for a bad shape, -7 for no memory.
+ */
+int oracle_suffix_attn_range(const uint16_t *q, const uint16_t *k_prefix, const uint16_t *v_prefix,
+                             const int32_t *prefix_valid_len, const uint8_t *prefix_mask,
+                             const uint16_t *k_suffix, const uint16_t *v_suffix,
+                             double *out, double *lse,
+                             int B, int Hq, int Hkv, int P, int S, int D,
+                             int key_lo, int key_hi, int nthreads)
+{
+    if (!q || !k_suffix || !v_suffix || !out || !lse) return -1;
+    if (P > 0 && (!k_prefix || !v_prefix)) return -1;
+    int rc = check_shape(B, Hq, Hkv, P, S, D);
+    if (rc) return rc;
+    if (key_lo < 0) key_lo = 0;
+    if (key_hi > P + S) key_hi = P + S;
+    if (key_hi < key_lo) key_hi = key_lo;
+    const int G = Hq / Hkv;
+    const int n_keys = key_hi - key_lo;
+    int failed = 0;
+    if (nthreads < 1) nthreads = 1;
+
+#pragma omp parallel num_threads(nthreads) reduction(| : failed)
+    {
+        double *logit_buf = (double *)malloc(sizeof(double) * (size_t)(n_keys > 0 ? n_keys : 1));
+        if (!logit_buf) {
+            failed = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int bh = 0; bh < B * Hq; ++bh) {
+                const int b = bh / Hq, h = bh % Hq;
+                const int kv = h / G;
+                const int vl = clamp_valid_len(prefix_valid_len, b, P);
+                const uint8_t *mask_row = prefix_mask ? prefix_mask + (size_t)b * P : NULL;
+                const size_t kv_off_p = ((size_t)b * Hkv + kv) * (size_t)P * D;
+                const size_t kv_off_s = ((size_t)b * Hkv + kv) * (size_t)S * D;
+                for (int i = 0; i < S; ++i) {
+                    const size_t row = ((size_t)b * Hq + h) * S + i;
+                    attend_row(q + row * D,
+                               P > 0 ? k_prefix + kv_off_p : NULL,
+                               P > 0 ? v_prefix + kv_off_p : NULL,
+                               k_suffix + kv_off_s, v_suffix + kv_off_s, mask_row,
+                               vl, P, S, D, key_lo, key_hi, logit_buf,
+                               out + row * D, lse + row);
+                }
+            }
+            free(logit_buf);
+        }
+    }
+    return failed ? -7 : 0;
+}
+
+/* The full attention: every visible prefix key and every suffix key. */
+int oracle_suffix_attn(const uint16_t *q, const uint16_t *k_prefix, const uint16_t *v_prefix,
+                       const int32_t *prefix_valid_len, const uint8_t *prefix_mask,
+                       const uint16_t *k_suffix, const uint16_t *v_suffix,
+                       double *out, double *lse,
+                       int B, int Hq, int Hkv, int P, int S, int D, int nthreads)
+{
+    return oracle_suffix_attn_range(q, k_prefix, v_prefix, prefix_valid_len, prefix_mask,
+                                    k_suffix, v_suffix, out, lse, B, Hq, Hkv, P, S, D,
+                                    0, P + S, nthreads);
+}
+
+/*
+ * Combination of n_parts partial results over disjoint key sets into the
+ * result over their union (the log-sum-exp identity):
+ *   LSE = ln sum_s exp(lse_s),   O = sum_s exp(lse_s - LSE) * O_s,
+ * where O_s is the softmax-weighted sum over part s alone (weights summing to
+ * one within the part) and lse_s its log-sum-exp.  A part with lse_s = -inf
+ * (no visible key) contributes nothing.  Inputs are [n_parts][rows][D] and
+ * [n_parts][rows]; outputs [rows][D] and [rows].
+ */
+int oracle_merge_parts(const double *o_parts, const double *lse_parts, int n_parts,
+                       long rows, int D, double *out, double *lse)
+{
+    if (!o_parts || !lse_parts || !out || !lse) return -1;
+    if (n_parts < 1 || rows < 0 || D < 1) return -2;
+    for (long r = 0; r < rows; ++r) {
+        double m = -INFINITY;
+        for (int s = 0; s < n_parts; ++s) {
+            double l = lse_parts[(size_t)s * rows + r];
+            if (l > m) m = l;
+        }
+        for (int d = 0; d < D; ++d) out[r * D + d] = 0.0;
+        if (m == -INFINITY) {
+            lse[r] = -INFINITY;
+            continue;
+        }
+        double z = 0.0;
+        for (int s = 0; s < n_parts; ++s) z += exp(lse_parts[(size_t)s * rows + r] - m);
+        double total = m + log(z);
+        for (int s = 0; s < n_parts; ++s) {
+            double l = lse_parts[(size_t)s * rows + r];
+            if (l == -INFINITY) continue;
+            double w = exp(l - total);
+            const double *o = o_parts + ((size_t)s * rows + r) * D;
+            for (int d = 0; d < D; ++d) out[r * D + d] += w * o[d];
+        }
+        lse[r] = total;
+    }
+    return 0;
+}
+
+/* Number of OpenMP threads this build can use (1 without OpenMP). */
+int oracle_max_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

@@ -1,0 +1,290 @@
+"""Checks that tie the fp64 oracle to facts outside itself.
+
+Each ``pin_*`` function takes an ``oracle.Oracle`` and raises AssertionError
+when the oracle disagrees with a fact that the pages or the mathematics fix:
+a library routine that computes a special case (float64 scaled-dot-product
+attention), a closed form, an invariant, or a brute force in independent
+arithmetic.  ``test_oracle.py`` runs them on the real oracle;
+``test_oracle_mutations.py`` shows that each planted mistake in a copy of the
+oracle fails at least one of them.
+
+The attention these pins describe is the action-expert suffix attention of
+the page "TensorRT+Triton+FlexAttention: OpenDM VLA 快速推理加速栈深度剖析",
+section 2.2: logits over the prefix KV cache and the suffix K/V under the
+prefix-visibility mask, softmax, value-weighted sum; GQA with head_dim 256
+and 8/4 heads (same section's shape table).
+"""
+from __future__ import annotations
+
+import decimal
+import math
+
+import numpy as np
+import torch
+
+BF = torch.bfloat16
+
+
+def bf16_rand(gen, shape, mult=1.0):
+    return (torch.randn(shape, generator=gen, dtype=torch.float32) * mult).to(BF)
+
+
+def rand_case(seed, B, Hq, Hkv, P, S, D, vl=None, mask_p=0.0, mult=1.0):
+    gen = torch.Generator().manual_seed(seed)
+    q = bf16_rand(gen, (B, Hq, S, D), mult)
+    kp = bf16_rand(gen, (B, Hkv, P, D), mult)
+    vp = bf16_rand(gen, (B, Hkv, P, D))
+    ks = bf16_rand(gen, (B, Hkv, S, D), mult)
+    vs = bf16_rand(gen, (B, Hkv, S, D))
+    if vl is None:
+        vlt = torch.randint(0, P + 1, (B,), generator=gen, dtype=torch.int64).to(torch.int32)
+    else:
+        vlt = torch.tensor(vl, dtype=torch.int32)
+    mask = None
+    if mask_p > 0.0:
+        mask = (torch.rand((B, P), generator=gen) >= mask_p).to(torch.uint8)
+    return dict(q=q, k_prefix=kp, v_prefix=vp, prefix_valid_len=vlt, prefix_mask=mask,
+                k_suffix=ks, v_suffix=vs, B=B, Hq=Hq, Hkv=Hkv, P=P, S=S, D=D)
+
+
+def run(orc, c, **kw):
+    return orc.suffix_attn(c["q"], c["k_prefix"], c["v_prefix"], c["prefix_valid_len"],
+                           c["prefix_mask"], c["k_suffix"], c["v_suffix"],
+                           c["B"], c["Hq"], c["Hkv"], c["P"], c["S"], c["D"], **kw)
+
+
+def visible_keys(c, b):
+    """Boolean visibility of the P+S keys of sample b (prefix, then suffix)."""
+    P, S = c["P"], c["S"]
+    vl = P if c["prefix_valid_len"] is None else int(c["prefix_valid_len"][b])
+    vl = max(0, min(P, vl))
+    vis = np.zeros(P + S, dtype=bool)
+    vis[:vl] = True
+    if c["prefix_mask"] is not None:
+        vis[:P] &= c["prefix_mask"][b].numpy() != 0
+    vis[P:] = True
+    return vis
+
+
+def sdpa_reference(c):
+    """float64 torch scaled_dot_product_attention on the concatenated keys.
+
+    The KV heads are expanded to the query heads with repeat_interleave (head
+    h reads KV head h // G).  The LSE comes from the same library call: one
+    extra key with an all-zero K row (logit exactly 0) and a value that is 1
+    in an extra output column receives weight 1 / (1 + Z), where Z is the sum
+    of exp(logit) over the real visible keys; so LSE = ln(1/w - 1)."""
+    B, Hq, Hkv, P, S, D = (c[k] for k in ("B", "Hq", "Hkv", "P", "S", "D"))
+    G = Hq // Hkv
+    f = lambda t: t.to(torch.float64)
+    k = torch.cat([f(c["k_prefix"]), f(c["k_suffix"])], dim=2)      # [B,Hkv,P+S,D]
+    v = torch.cat([f(c["v_prefix"]), f(c["v_suffix"])], dim=2)
+    k = k.repeat_interleave(G, dim=1)
+    v = v.repeat_interleave(G, dim=1)
+    vis = torch.stack([torch.from_numpy(visible_keys(c, b)) for b in range(B)])  # [B,P+S]
+    attn_mask = vis[:, None, None, :].expand(B, Hq, S, P + S)
+    q = f(c["q"])
+    out = torch.nn.functional.scaled_dot_product_attention(q, k, v, attn_mask=attn_mask)
+    # LSE through the extra-key construction
+    k_x = torch.cat([k, torch.zeros(B, Hq, 1, D, dtype=torch.float64)], dim=2)
+    v_x = torch.cat([torch.cat([v, torch.zeros(B, Hq, P + S, 1, dtype=torch.float64)], dim=3),
+                     torch.cat([torch.zeros(B, Hq, 1, D, dtype=torch.float64),
+                                torch.ones(B, Hq, 1, 1, dtype=torch.float64)], dim=3)], dim=2)
+    mask_x = torch.cat([attn_mask, torch.ones(B, Hq, S, 1, dtype=torch.bool)], dim=3)
+    out_x = torch.nn.functional.scaled_dot_product_attention(q, k_x, v_x, attn_mask=mask_x)
+    w = out_x[..., D]
+    lse = torch.log(1.0 / w - 1.0)
+    return out.numpy(), lse.numpy()
+
+
+# --------------------------------------------------------------------------
+
+SDPA_SHAPES = [
+    # seed, B, Hq, Hkv, P, S, D, mask_p
+    (11, 1, 2, 1, 5, 1, 4, 0.0),
+    (12, 2, 4, 2, 7, 3, 8, 0.3),
+    (13, 2, 8, 4, 8, 4, 16, 0.2),
+    (14, 1, 4, 1, 6, 2, 256, 0.4),
+    (15, 2, 2, 2, 3, 4, 8, 0.0),
+    (16, 1, 8, 4, 0, 3, 8, 0.0),
+]
+
+
+def pin_sdpa_float64(orc):
+    """O and LSE equal float64 library attention on tiny random shapes."""
+    for seed, B, Hq, Hkv, P, S, D, mp in SDPA_SHAPES:
+        c = rand_case(seed, B, Hq, Hkv, P, S, D, mask_p=mp)
+        o, lse = run(orc, c)
+        o_ref, lse_ref = sdpa_reference(c)
+        np.testing.assert_allclose(o, o_ref, rtol=0, atol=1e-12,
+                                   err_msg=f"O vs float64 SDPA, case seed {seed}")
+        np.testing.assert_allclose(lse, lse_ref, rtol=0, atol=1e-9,
+                                   err_msg=f"LSE vs float64 SDPA, case seed {seed}")
+
+
+def pin_uniform_logits(orc):
+    """Q = 0 makes every logit 0: O is the mean of the visible V rows and LSE is
+    ln(number of visible keys)."""
+    c = rand_case(21, 2, 4, 2, 9, 3, 8, mask_p=0.3)
+    c["q"] = torch.zeros_like(c["q"])
+    o, lse = run(orc, c)
+    G = c["Hq"] // c["Hkv"]
+    for b in range(c["B"]):
+        vis = visible_keys(c, b)
+        for h in range(c["Hq"]):
+            kv = h // G
+            rows = torch.cat([c["v_prefix"][b, kv], c["v_suffix"][b, kv]], 0).to(torch.float64).numpy()
+            mean = rows[vis].mean(axis=0)
+            for i in range(c["S"]):
+                np.testing.assert_allclose(o[b, h, i], mean, rtol=0, atol=1e-13)
+                assert abs(lse[b, h, i] - math.log(int(vis.sum()))) < 1e-13
+
+
+def pin_constant_v_gqa(orc):
+    """Every V row of KV head g holds the constant c_g: head h must output
+    c_{h // G} (pins the GQA head mapping and the normalisation)."""
+    consts = [0.5, -1.25, 2.0, 3.5]
+    c = rand_case(22, 2, 8, 4, 6, 3, 8, mask_p=0.2)
+    for g, val in enumerate(consts):
+        c["v_prefix"][:, g] = val
+        c["v_suffix"][:, g] = val
+    o, _ = run(orc, c)
+    for h in range(8):
+        np.testing.assert_allclose(o[:, h], consts[h // 2], rtol=0, atol=1e-13,
+                                   err_msg=f"head {h}")
+
+
+def pin_masked_rows_ignored(orc):
+    """Large finite values in masked prefix rows, and NaN in rows at or past
+    the valid length, change nothing."""
+    c = rand_case(23, 2, 4, 2, 10, 2, 8, vl=[7, 4], mask_p=0.3)
+    o0, l0 = run(orc, c)
+    for b in range(c["B"]):
+        vl = int(c["prefix_valid_len"][b])
+        hidden = np.where(c["prefix_mask"][b].numpy()[:vl] == 0)[0]
+        for t in ("k_prefix", "v_prefix"):
+            c[t][b, :, hidden.tolist(), :] = 1.0e4
+            c[t][b, :, vl:, :] = float("nan")
+    o1, l1 = run(orc, c)
+    assert np.array_equal(o0, o1) and np.array_equal(l0, l1)
+
+
+def pin_single_suffix_key(orc):
+    """S = 1 with no visible prefix key: O is the one suffix V row and LSE is
+    its logit <q, k_s> / sqrt(D)."""
+    for P in (0, 4):
+        c = rand_case(24 + P, 1, 2, 1, P, 1, 16, vl=[0])
+        o, lse = run(orc, c)
+        ks = c["k_suffix"][0, 0, 0].to(torch.float64).numpy()
+        vs = c["v_suffix"][0, 0, 0].to(torch.float64).numpy()
+        for h in range(2):
+            q = c["q"][0, h, 0].to(torch.float64).numpy()
+            np.testing.assert_array_equal(o[0, h, 0], vs)
+            assert abs(lse[0, h, 0] - float(np.dot(q, ks)) / 4.0) < 1e-12
+
+
+def pin_dominant_key(orc):
+    """One prefix key aligned with every query and scaled far above the
+    others takes essentially all the weight."""
+    B, Hq, Hkv, P, S, D = 1, 2, 1, 6, 2, 4
+    c = rand_case(25, B, Hq, Hkv, P, S, D, vl=[6])
+    for t in ("q", "k_prefix", "k_suffix"):
+        c[t] = (c[t].to(torch.float32) * 0.01).to(BF)
+    c["q"][..., 0] = 8.0
+    c["k_prefix"][0, 0, 3, :] = 0.0
+    c["k_prefix"][0, 0, 3, 0] = 8.0      # logit exactly 8*8/sqrt(4) = 32 (others ~ 0.04)
+    o, lse = run(orc, c)
+    v3 = c["v_prefix"][0, 0, 3].to(torch.float64).numpy()
+    for h in range(Hq):
+        for i in range(S):
+            np.testing.assert_allclose(o[0, h, i], v3, rtol=0, atol=1e-11)
+            assert abs(lse[0, h, i] - 32.0) < 1e-11
+
+
+def pin_prefix_permutation(orc):
+    """Permuting the prefix rows inside the valid range (with their mask
+    bytes) permutes nothing in the result."""
+    c = rand_case(26, 1, 4, 2, 12, 3, 8, vl=[10], mask_p=0.25)
+    o0, l0 = run(orc, c)
+    perm = torch.randperm(10, generator=torch.Generator().manual_seed(5))
+    full = torch.cat([perm, torch.arange(10, 12)])
+    c["k_prefix"] = c["k_prefix"][:, :, full].contiguous()
+    c["v_prefix"] = c["v_prefix"][:, :, full].contiguous()
+    c["prefix_mask"] = c["prefix_mask"][:, full].contiguous()
+    o1, l1 = run(orc, c)
+    np.testing.assert_allclose(o1, o0, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(l1, l0, rtol=0, atol=1e-13)
+
+
+def pin_split_merge(orc):
+    """Attention over disjoint key ranges merged by the log-sum-exp identity
+    equals attention over the union (the split-KV combine)."""
+    c = rand_case(27, 2, 4, 2, 11, 3, 8, vl=[9, 11], mask_p=0.2)
+    o_full, l_full = run(orc, c)
+    P, S = c["P"], c["S"]
+    cuts = [0, 4, 9, P + 1, P + S]
+    parts_o, parts_l = [], []
+    for lo, hi in zip(cuts[:-1], cuts[1:]):
+        o, l = run(orc, c, key_range=(lo, hi))
+        parts_o.append(o.reshape(-1, c["D"]))
+        parts_l.append(l.reshape(-1))
+    o_m, l_m = orc.merge_parts(np.stack(parts_o), np.stack(parts_l))
+    np.testing.assert_allclose(o_m, o_full.reshape(-1, c["D"]), rtol=0, atol=1e-13)
+    np.testing.assert_allclose(l_m, l_full.reshape(-1), rtol=0, atol=1e-13)
+
+
+def _dec_bf16(t):
+    return [decimal.Decimal(float(x)) for x in t.to(torch.float32).reshape(-1).tolist()]
+
+
+def pin_decimal_bruteforce(orc):
+    """A 60-digit decimal brute force of softmax(q K^T / sqrt(D)) V on a tiny
+    case (every bf16 value is exact in decimal)."""
+    decimal.getcontext().prec = 60
+    c = rand_case(28, 1, 2, 1, 4, 2, 4, vl=[3])
+    c["prefix_mask"] = torch.tensor([[1, 0, 1, 1]], dtype=torch.uint8)
+    o, lse = run(orc, c)
+    P, S, D = 4, 2, 4
+    vis = visible_keys(c, 0)
+    K = _dec_bf16(torch.cat([c["k_prefix"][0, 0], c["k_suffix"][0, 0]], 0))
+    V = _dec_bf16(torch.cat([c["v_prefix"][0, 0], c["v_suffix"][0, 0]], 0))
+    half = decimal.Decimal(1) / decimal.Decimal(D).sqrt()
+    for h in range(2):
+        for i in range(S):
+            qrow = _dec_bf16(c["q"][0, h, i])
+            logits = {}
+            for x in range(P + S):
+                if vis[x]:
+                    logits[x] = half * sum(qrow[d] * K[x * D + d] for d in range(D))
+            z = sum(l.exp() for l in logits.values())
+            want_lse = z.ln()
+            for d in range(D):
+                want = sum((l.exp() / z) * V[x * D + d] for x, l in logits.items())
+                assert abs(float(want) - o[0, h, i, d]) < 1e-14
+            assert abs(float(want_lse) - lse[0, h, i]) < 1e-14
+
+
+def pin_valid_len_clamp_and_boundary(orc):
+    """Valid lengths outside [0, P] clamp to the range; the key at index
+    valid_len - 1 is seen and the key at valid_len is not."""
+    c = rand_case(29, 1, 2, 1, 6, 2, 8, vl=[3])
+    base_o, _ = run(orc, c)
+    for vl, same_as in ((-5, 0), (13, 6)):
+        c1 = dict(c, prefix_valid_len=torch.tensor([vl], dtype=torch.int32))
+        c2 = dict(c, prefix_valid_len=torch.tensor([same_as], dtype=torch.int32))
+        assert np.array_equal(run(orc, c1)[0], run(orc, c2)[0])
+    c3 = dict(c, prefix_valid_len=None)
+    c4 = dict(c, prefix_valid_len=torch.tensor([6], dtype=torch.int32))
+    assert np.array_equal(run(orc, c3)[0], run(orc, c4)[0])
+    # boundary: change row vl-1 -> output moves; change row vl -> it does not
+    c5 = dict(c, v_prefix=c["v_prefix"].clone())
+    c5["v_prefix"][0, 0, 3] = 100.0
+    assert np.array_equal(run(orc, c5)[0], base_o)
+    c6 = dict(c, v_prefix=c["v_prefix"].clone())
+    c6["v_prefix"][0, 0, 2] = 100.0
+    assert not np.allclose(run(orc, c6)[0], base_o)
+
+
+ALL_PINS = [pin_sdpa_float64, pin_uniform_logits, pin_constant_v_gqa, pin_masked_rows_ignored,
+            pin_single_suffix_key, pin_dominant_key, pin_prefix_permutation, pin_split_merge,
+            pin_decimal_bruteforce, pin_valid_len_clamp_and_boundary]

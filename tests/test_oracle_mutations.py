@@ -1,0 +1,53 @@
+"""Planted mistakes in a copy of the oracle must each fail at least one pin.
+
+Each mutation below is a plausible slip (a dropped term, a wrong index or
+sign, a swapped operand).  The copy is edited and compiled under a temporary
+directory; the real oracle source is never touched.
+"""
+import os
+
+import pytest
+
+import oracle
+import pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "oracle.c")
+
+MUTATIONS = {
+    "suffix_keys_dropped": ("if (x >= P) return 1; /* suffix keys: always visible */",
+                            "if (x >= P) return 0;"),
+    "gqa_modulo_mapping": ("const int kv = h / G;", "const int kv = h % Hkv;"),
+    "scale_missing": ("const double scale = 1.0 / sqrt((double)D);", "const double scale = 1.0;"),
+    "valid_len_off_by_one": ("if (x >= vl) return 0; /* bucket padding */",
+                             "if (x > vl) return 0;"),
+    "mask_inverted": ("if (mask_row != NULL && mask_row[x] == 0) return 0;",
+                      "if (mask_row != NULL && mask_row[x] != 0) return 0;"),
+    "lse_without_max": ("double lse = m + log(z);", "double lse = log(z);"),
+    "weights_unnormalised": ("double w = exp(logit_buf[x - key_lo] - lse);",
+                             "double w = exp(logit_buf[x - key_lo] - m);"),
+    "k_used_as_v": ("const uint16_t *v_row = (x < P) ? vp + (size_t)x * D",
+                    "const uint16_t *v_row = (x < P) ? kp + (size_t)x * D"),
+    "merge_weight_sign": ("double w = exp(l - total);", "double w = exp(total - l);"),
+    "dot_drops_last_term": ("for (int d = 0; d < D; ++d)\n            dot +=",
+                            "for (int d = 0; d < D - 1; ++d)\n            dot +="),
+    "merge_skips_first_part": ("for (int s = 0; s < n_parts; ++s) {\n            double l = lse_parts[(size_t)s * rows + r];\n            if (l == -INFINITY) continue;",
+                               "for (int s = 1; s < n_parts; ++s) {\n            double l = lse_parts[(size_t)s * rows + r];\n            if (l == -INFINITY) continue;"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_mutation_is_caught(tmp_path, name):
+    before, after = MUTATIONS[name]
+    src = open(SRC).read()
+    assert src.count(before) == 1, f"mutation anchor for {name} not found exactly once"
+    mutant_src = tmp_path / "oracle_mutant.c"
+    mutant_src.write_text(src.replace(before, after))
+    lib = oracle.build(force=True, src=str(mutant_src), out=str(tmp_path / "libmutant.so"))
+    mutant = oracle.Oracle(lib)
+    caught = []
+    for pin in pins.ALL_PINS:
+        try:
+            pin(mutant)
+        except (AssertionError, ValueError, IndexError):
+            caught.append(pin.__name__)
+    assert caught, f"no pin catches the planted mistake {name}"

@@ -1,0 +1,468 @@
+"""Benchmark of the B200 suffix attention (one JSON line on rank 0).
+
+A step is one dm05_suffix_attn call over one batch of synthetic input of the
+named workload (default: the base-model chunk, B=1, P=1024 bucket with 900
+valid rows, S=50, 8/4 heads, D=256).  Timing: W untimed warm-up calls, then
+exactly K calls replayed from CUDA graphs and bracketed by a barrier and a
+device synchronise, timed with CUDA events on the launching stream, max over
+ranks.  Every call reads a different one of R rotating input sets whose total
+size is more than twice the L2, so each call streams its K/V from HBM.
+
+Multi-GPU: the path has no exchange step; each rank runs independent
+replicas on its own GPU (no collective on the data path) and `value` is the
+whole job's time per call, max-over-ranks time / (K * N).
+
+--impl reference times the fp64 CPU oracle on the host cores (each step one
+bounded sample of query rows of the same workload, scaled to a full call).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "suffix-attn µs/call & achieved HBM GB/s (frac of roofline), P=1024 S=50 B=1"
+UNIT = "us/call"
+KV_ROW_BYTES_PER_HEAD = 2 * 256 * 2   # K and V rows of one KV head, bf16, D=256
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default="base_chunk",
+                    choices=("base_chunk", "libero_tiny", "history_loop", "batched_mask", "bucket_sweep"))
+    ap.add_argument("--splits", type=int, default=0, help="force CTAs per (sample, KV head); 0 = auto")
+    ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU-baseline sample budget")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def workload_inputs(name):
+    from gqa_prefix_suffix_b200 import inputs as gen
+    w = gen.WORKLOADS[name]()
+    if isinstance(w, list):
+        # the history loop reuses one prefix; the sweep: take its largest bucket
+        w = w[0] if name == "history_loop" else w[-1]
+    return w
+
+
+def algorithmic_bytes(inp):
+    """K/V bytes the method must move: visible prefix rows plus the S suffix
+    rows, K and V, every KV head, bf16 (rows past valid_len and hidden rows
+    are not counted)."""
+    import torch
+    total_rows = 0
+    for b in range(inp.B):
+        vl = inp.P if inp.prefix_valid_len is None else max(0, min(inp.P, int(inp.prefix_valid_len[b])))
+        vis = vl if inp.prefix_mask is None else int((inp.prefix_mask[b, :vl] != 0).sum())
+        total_rows += vis + inp.S
+    kv = total_rows * inp.Hkv * KV_ROW_BYTES_PER_HEAD
+    G = inp.Hq // inp.Hkv
+    flops = 4 * total_rows * inp.Hkv * G * inp.S * inp.D
+    del torch
+    return kv, flops
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for rel in ("gqa_prefix_suffix_b200/csrc/suffix_attn_kernel.cuh", "gqa_prefix_suffix_b200/csrc/sm100_ptx.cuh",
+                "gqa_prefix_suffix_b200/csrc/dm05_suffix_attn.cu"):
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            j = json.load(f)
+        e = j.get(workload)
+        if e and e.get("kernel_source_hash") == kernel_source_hash():
+            return float(e["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """Polls SM clock and clock-event reasons through NVML while running."""
+
+    def __init__(self, torch_device):
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._ok = False
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            try:  # the same physical GPU as the torch device, whatever CUDA_VISIBLE_DEVICES says
+                uuid = str(torch.cuda.get_device_properties(torch_device).uuid)
+                self._h = pynvml.nvmlDeviceGetHandleByUUID(("GPU-" + uuid).encode())
+            except Exception:
+                self._h = pynvml.nvmlDeviceGetHandleByIndex(torch_device.index or 0)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._ok = True
+        except Exception:
+            self._ok = False
+
+    def _run(self):
+        nv = self._nv
+        names = {
+            "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+            "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+            "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80, "display_clock_setting": 0x100,
+        }
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for k, bit in names.items():
+                    if r & bit:
+                        self.reasons.add(k)
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self._ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self._ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": len(self.samples)}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+# ----------------------------------------------------------------------------- CPU side
+
+def host_bits(inp):
+    """The workload's tensors as numpy arrays (bf16 as uint16 bit patterns),
+    converted once so that timed oracle calls do no marshalling copies."""
+    import types
+
+    import numpy as np
+    import torch
+
+    def bits(t):
+        return None if t is None else np.ascontiguousarray(t.contiguous().view(torch.int16).numpy().view(np.uint16))
+
+    def plain(t):
+        return None if t is None else np.ascontiguousarray(t.numpy())
+
+    return types.SimpleNamespace(
+        name=inp.name, B=inp.B, Hq=inp.Hq, Hkv=inp.Hkv, P=inp.P, S=inp.S, D=inp.D,
+        q=bits(inp.q), k_prefix=bits(inp.k_prefix), v_prefix=bits(inp.v_prefix), k_suffix=bits(inp.k_suffix),
+        v_suffix=bits(inp.v_suffix), prefix_valid_len=plain(inp.prefix_valid_len), prefix_mask=plain(inp.prefix_mask))
+
+
+def cpu_oracle_rate(inp, seconds, threads):
+    """Times the fp64 oracle on bounded samples of query rows of this workload
+    and scales to a full call.  Returns (us per full call, rows timed, calls)."""
+    import oracle
+    orc = oracle.default()
+    inp = host_bits(inp)
+    n_rows = inp.B * inp.Hq * inp.S
+    chunk = max(1, threads)
+    t_total, rows_done, calls, start = 0.0, 0, 0, 0
+    while t_total < seconds:
+        lo = start % n_rows
+        hi = min(n_rows, lo + chunk)
+        t0 = time.perf_counter()
+        orc.inputs_call(inp, nthreads=threads, row_range=(lo, hi))
+        t_total += time.perf_counter() - t0
+        rows_done += hi - lo
+        calls += 1
+        start = hi
+    return t_total / rows_done * n_rows * 1e6, rows_done, calls
+
+
+def run_reference(args, world, rank):
+    """The reference arm: the fp64 CPU oracle, as it stands, on the host cores."""
+    if rank != 0:
+        return 0
+    import oracle
+    full = workload_inputs(args.workload)
+    inp = host_bits(full)
+    threads = oracle.max_threads()
+    orc = oracle.default()
+    n_rows = inp.B * inp.Hq * inp.S
+    rows_per_step = max(1, threads)
+    for i in range(args.warmup):
+        lo = (i * rows_per_step) % n_rows
+        orc.inputs_call(inp, nthreads=threads, row_range=(lo, min(n_rows, lo + rows_per_step)))
+    t0 = time.perf_counter()
+    rows = 0
+    for i in range(args.steps):
+        lo = (i * rows_per_step) % n_rows
+        hi = min(n_rows, lo + rows_per_step)
+        orc.inputs_call(inp, nthreads=threads, row_range=(lo, hi))
+        rows += hi - lo
+    dt = time.perf_counter() - t0
+    us_per_call = dt / rows * n_rows * 1e6
+    kv, _ = algorithmic_bytes(full)
+    sample = (f"each step: {rows_per_step} query rows (of {n_rows} per call) of {inp.name}, "
+              f"fp64 oracle; value scaled to a full call")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": us_per_call, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(full, None),
+        "cpu_baseline": {"value": us_per_call, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": us_per_call, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "achieved_kv_gbs": kv / (us_per_call * 1e-6) / 1e9,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(inp, extra):
+    vl = None if inp.prefix_valid_len is None else [int(x) for x in inp.prefix_valid_len.tolist()]
+    cfg = {"workload": inp.name, "B": inp.B, "Hq": inp.Hq, "Hkv": inp.Hkv, "P": inp.P, "S": inp.S, "D": inp.D,
+           "valid_len": vl if vl is None or len(vl) <= 4 else f"{len(vl)} values, mean {sum(vl) / len(vl):.1f}",
+           "prefix_mask": inp.prefix_mask is not None}
+    if extra:
+        cfg.update(extra)
+    return cfg
+
+
+# ----------------------------------------------------------------------------- GPU side
+
+def main():
+    args = parse()
+    world, rank, local = dist_setup()
+    if args.impl == "reference":
+        return run_reference(args, world, rank)
+
+    import torch
+    from gqa_prefix_suffix_b200 import binding as bd
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+        pg = dist
+
+    bd.lib()  # fails loudly if the CUDA library is missing
+    inp = workload_inputs(args.workload)
+    B, Hq, Hkv, P, S, D = inp.B, inp.Hq, inp.Hkv, inp.P, inp.S, inp.D
+    kv_bytes, flops = algorithmic_bytes(inp)
+
+    # rotating input sets: total footprint > 2 x L2
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    set_bytes = sum(t.numel() * t.element_size() for t in inp.tensors().values() if t is not None)
+    set_bytes += B * Hq * S * (D * 2 + 4)
+    R = max(2, int(2 * l2 // set_bytes) + 2)
+    base = inp.to(dev)
+    sets = []
+    for r in range(R):
+        t = {k: (None if v is None else v.clone()) for k, v in base.tensors().items()}
+        t["out"] = torch.empty((B, Hq, S, D), dtype=torch.bfloat16, device=dev)
+        t["lse"] = torch.empty((B, Hq, S), dtype=torch.float32, device=dev)
+        sets.append(t)
+    torch.cuda.synchronize()
+
+    stream = torch.cuda.Stream(device=dev)
+    sh = stream.cuda_stream
+    if bd.dm05_set_split_override(args.splits) != 0:
+        raise SystemExit("bad --splits")
+    rc = bd.dm05_suffix_attn_reserve(B, Hq, Hkv, P, S, D, sh)
+    if rc != 0:
+        raise bd.Dm05Error(rc, "reserve")
+    rc, splits, tile_rows = bd.dm05_suffix_attn_plan(B, Hq, Hkv, P, S, D)
+
+    def call(t, s=sh):
+        ptr = lambda x: None if x is None else x.data_ptr()
+        rc = bd.dm05_suffix_attn(ptr(t["q"]), ptr(t["k_prefix"]), ptr(t["v_prefix"]), ptr(t["prefix_valid_len"]),
+                                 ptr(t["prefix_mask"]), ptr(t["k_suffix"]), ptr(t["v_suffix"]), ptr(t["out"]),
+                                 ptr(t["lse"]), B, Hq, Hkv, P, S, D, s)
+        if rc != 0:
+            raise bd.Dm05Error(rc, "dm05_suffix_attn")
+
+    # warm-up (untimed)
+    with torch.cuda.stream(stream):
+        for i in range(max(3, args.warmup)):
+            call(sets[i % R])
+    stream.synchronize()
+
+    # the K timed steps, captured as graphs of up to `chunk` calls each
+    K = args.steps
+    chunk = min(K, 1000)
+    n_full, rem = divmod(K, chunk)
+
+    def capture(n, offset):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(n):
+                call(sets[(offset + i) % R])
+        return g
+
+    g_full = capture(chunk, 0) if n_full else None
+    g_rem = capture(rem, n_full * chunk) if rem else None
+    # one untimed replay of each graph
+    if g_full is not None:
+        g_full.replay()
+    if g_rem is not None:
+        g_rem.replay()
+    stream.synchronize()
+
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    if pg is not None:
+        pg.barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(dev)
+    with sampler:
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(n_full):
+                g_full.replay()
+            if g_rem is not None:
+                g_rem.replay()
+            e1.record(stream)
+        stream.synchronize()
+    torch.cuda.synchronize()
+    if pg is not None:
+        pg.barrier()
+    t_ms = e0.elapsed_time(e1)
+    if pg is not None:
+        tt = torch.tensor([t_ms], device=dev)
+        pg.all_reduce(tt, op=pg.ReduceOp.MAX)
+        t_ms = float(tt.item())
+    rc, word = bd.dm05_get_error_word(sh)
+    if word != 0:
+        raise SystemExit(f"kernel error word {word:#x}")
+
+    us_per_call_device = t_ms * 1e3 / K          # one GPU's time per call
+    value = t_ms * 1e3 / (K * world)              # whole-job time per call
+    achieved = kv_bytes / (us_per_call_device * 1e-6) / 1e9
+    peak, peak_kind = measured_peaks()
+
+    # ---- end to end through the public API: pinned host inputs -> device -> call -> host
+    host = {k: (None if v is None else v.pin_memory()) for k, v in inp.tensors().items()}
+    dev_in = {k: (None if v is None else torch.empty_like(v, device=dev)) for k, v in inp.tensors().items()}
+    out_h = torch.empty((B, Hq, S, D), dtype=torch.bfloat16).pin_memory()
+    lse_h = torch.empty((B, Hq, S), dtype=torch.float32).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
+    d2h = out_h.numel() * 2 + lse_h.numel() * 4
+    E = max(1, min(args.e2e_steps, K))
+
+    def e2e_step():
+        with torch.cuda.stream(stream):
+            for k, v in host.items():
+                if v is not None:
+                    dev_in[k].copy_(v, non_blocking=True)
+            o, l = bd.suffix_attn(dev_in["q"], dev_in["k_prefix"], dev_in["v_prefix"], dev_in["k_suffix"],
+                                  dev_in["v_suffix"], prefix_valid_len=dev_in["prefix_valid_len"],
+                                  prefix_mask=dev_in["prefix_mask"], stream=stream)
+            out_h.copy_(o, non_blocking=True)
+            lse_h.copy_(l, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    stream.synchronize()
+    if pg is not None:
+        pg.barrier()
+    f0 = torch.cuda.Event(enable_timing=True)
+    f1 = torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(E):
+        e2e_step()
+    f1.record(stream)
+    stream.synchronize()
+    e2e_ms = f0.elapsed_time(f1)
+    if pg is not None:
+        tt = torch.tensor([e2e_ms], device=dev)
+        pg.all_reduce(tt, op=pg.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+    e2e_value = e2e_ms * 1e3 / (E * world)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        threads = oracle.max_threads()
+        us, rows, n = cpu_oracle_rate(inp, args.cpu_seconds, threads)
+        cpu = {"value": us, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": f"{rows} query rows of {inp.name} in {n} oracle calls (~{args.cpu_seconds:.0f} s), "
+                         f"fp64, scaled to a full call of {B * Hq * S} rows"}
+
+    clocks = sampler.summary()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+            "ms_per_step": value / 1e3, "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": workload_config(inp, {
+                "splits_per_head": splits, "tile_rows": tile_rows, "parallelism": f"replicas x{world}",
+                "l2": f"{R} rotating input sets, {R * set_bytes / 1e6:.0f} MB > 2 x L2 ({l2 / 1e6:.0f} MB)",
+                "graph_calls": chunk}),
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": profiled_traffic(args.workload),
+                         "peak_source": peak_kind, "algorithmic_bytes": kv_bytes,
+                         "tensor_tflops": flops / (us_per_call_device * 1e-6) / 1e12},
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "steps": E},
+            "gpu_launches": K,
+            "clocks": clocks,
+        }
+        if cpu is not None:
+            line["cpu_baseline"] = cpu
+        print(json.dumps(line), flush=True)
+    del g_full, g_rem
+    if pg is not None:
+        pg.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,167 @@
+"""ctypes binding of the C ABI in include/dm05_suffix_attn.h.
+
+Argument marshalling only: every step of the attention runs in the CUDA
+library.  If the library is missing the import of the entry points fails
+loudly; there is no other implementation behind these names.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdm05_suffix_attn.so")
+
+DM05_OK = 0
+DM05_ERR_NULL = -1
+DM05_ERR_SHAPE = -2
+DM05_ERR_UNSUPPORTED = -3
+DM05_ERR_ALIGN = -4
+DM05_ERR_WORKSPACE = -5
+DM05_ERR_CUDA = -6
+DM05_EW_VALID_LEN_CLAMPED = 0x1
+DM05_EW_WAIT_TIMEOUT = 0x2
+
+EXPORTS = ("dm05_suffix_attn", "dm05_suffix_attn_workspace_bytes", "dm05_suffix_attn_reserve",
+           "dm05_suffix_attn_plan", "dm05_set_split_override", "dm05_get_error_word",
+           "dm05_status_string", "dm05_release")
+
+_lock = threading.Lock()
+_lib = None
+
+
+class Dm05Error(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        super().__init__(f"{what}: {dm05_status_string(status)} ({status})" if what else
+                         f"{dm05_status_string(status)} ({status})")
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                                   "`python -m gqa_prefix_suffix_b200.build` (nvcc, sm_100a)")
+            L = ctypes.CDLL(LIB_PATH)
+            p, i, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+            L.dm05_suffix_attn.argtypes = [p] * 9 + [i] * 6 + [p]
+            L.dm05_suffix_attn.restype = i
+            L.dm05_suffix_attn_workspace_bytes.argtypes = [i] * 6
+            L.dm05_suffix_attn_workspace_bytes.restype = sz
+            L.dm05_suffix_attn_reserve.argtypes = [i] * 6 + [p]
+            L.dm05_suffix_attn_reserve.restype = i
+            L.dm05_suffix_attn_plan.argtypes = [i] * 6 + [ctypes.POINTER(i), ctypes.POINTER(i)]
+            L.dm05_suffix_attn_plan.restype = i
+            L.dm05_set_split_override.argtypes = [i]
+            L.dm05_set_split_override.restype = i
+            L.dm05_get_error_word.argtypes = [p, ctypes.POINTER(ctypes.c_uint32)]
+            L.dm05_get_error_word.restype = i
+            L.dm05_status_string.argtypes = [i]
+            L.dm05_status_string.restype = ctypes.c_char_p
+            L.dm05_release.argtypes = []
+            L.dm05_release.restype = None
+            _lib = L
+    return _lib
+
+
+# ---- the C entry points, same names, integer pointers ------------------------
+
+def dm05_suffix_attn(q, k_prefix, v_prefix, prefix_valid_len, prefix_mask, k_suffix, v_suffix,
+                     out, lse, B, Hq, Hkv, P, S, D, stream) -> int:
+    return lib().dm05_suffix_attn(q, k_prefix, v_prefix, prefix_valid_len, prefix_mask, k_suffix,
+                                  v_suffix, out, lse, B, Hq, Hkv, P, S, D, stream)
+
+
+def dm05_suffix_attn_workspace_bytes(B, Hq, Hkv, P, S, D) -> int:
+    return int(lib().dm05_suffix_attn_workspace_bytes(B, Hq, Hkv, P, S, D))
+
+
+def dm05_suffix_attn_reserve(B, Hq, Hkv, P, S, D, stream) -> int:
+    return lib().dm05_suffix_attn_reserve(B, Hq, Hkv, P, S, D, stream)
+
+
+def dm05_suffix_attn_plan(B, Hq, Hkv, P, S, D):
+    """Returns (status, splits_per_head, tile_rows)."""
+    sp, tr = ctypes.c_int(0), ctypes.c_int(0)
+    rc = lib().dm05_suffix_attn_plan(B, Hq, Hkv, P, S, D, ctypes.byref(sp), ctypes.byref(tr))
+    return rc, sp.value, tr.value
+
+
+def dm05_set_split_override(splits_per_head: int) -> int:
+    return lib().dm05_set_split_override(splits_per_head)
+
+
+def dm05_get_error_word(stream):
+    """Returns (status, error bits); synchronises the stream and clears the bits."""
+    w = ctypes.c_uint32(0)
+    rc = lib().dm05_get_error_word(stream, ctypes.byref(w))
+    return rc, int(w.value)
+
+
+def dm05_status_string(status: int) -> str:
+    return lib().dm05_status_string(status).decode()
+
+
+def dm05_release() -> None:
+    lib().dm05_release()
+
+
+# ---- torch front end (marshalling only) -------------------------------------
+
+def _stream_handle(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def suffix_attn(q, k_prefix, v_prefix, k_suffix, v_suffix, prefix_valid_len=None, prefix_mask=None,
+                out=None, lse=None, want_lse: bool = True, stream=None):
+    """Suffix attention on CUDA torch tensors; returns (out, lse or None).
+
+    q [B,Hq,S,D] bf16; k_prefix/v_prefix [B,Hkv,P,D] bf16; k_suffix/v_suffix
+    [B,Hkv,S,D] bf16; prefix_valid_len int32 [B] or None; prefix_mask uint8
+    [B,P] or None.  out (bf16 [B,Hq,S,D]) and lse (fp32 [B,Hq,S]) are
+    allocated when not given."""
+    import torch
+    B, Hq, S, D = q.shape
+    Hkv, P = k_prefix.shape[1], k_prefix.shape[2]
+    for name, t, dt in (("q", q, torch.bfloat16), ("k_prefix", k_prefix, torch.bfloat16),
+                        ("v_prefix", v_prefix, torch.bfloat16), ("k_suffix", k_suffix, torch.bfloat16),
+                        ("v_suffix", v_suffix, torch.bfloat16)):
+        if not t.is_cuda or t.dtype != dt or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA {dt} tensor")
+    if tuple(k_prefix.shape) != (B, Hkv, P, D) or tuple(v_prefix.shape) != (B, Hkv, P, D):
+        raise ValueError("k_prefix/v_prefix must be [B,Hkv,P,D]")
+    if tuple(k_suffix.shape) != (B, Hkv, S, D) or tuple(v_suffix.shape) != (B, Hkv, S, D):
+        raise ValueError("k_suffix/v_suffix must be [B,Hkv,S,D]")
+    if prefix_valid_len is not None:
+        if not prefix_valid_len.is_cuda or prefix_valid_len.dtype != torch.int32 or prefix_valid_len.numel() != B:
+            raise ValueError("prefix_valid_len must be a CUDA int32 tensor of B values")
+    if prefix_mask is not None:
+        if (not prefix_mask.is_cuda or prefix_mask.dtype != torch.uint8 or tuple(prefix_mask.shape) != (B, P)
+                or not prefix_mask.is_contiguous()):
+            raise ValueError("prefix_mask must be a contiguous CUDA uint8 tensor [B,P]")
+    if out is None:
+        out = torch.empty((B, Hq, S, D), dtype=torch.bfloat16, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq, S), dtype=torch.float32, device=q.device)
+    ptr = lambda t: None if t is None else t.data_ptr()
+    rc = dm05_suffix_attn(ptr(q), ptr(k_prefix), ptr(v_prefix), ptr(prefix_valid_len), ptr(prefix_mask),
+                          ptr(k_suffix), ptr(v_suffix), ptr(out), ptr(lse), B, Hq, Hkv, P, S, D,
+                          _stream_handle(stream))
+    if rc != DM05_OK:
+        raise Dm05Error(rc, "dm05_suffix_attn")
+    return out, lse
+
+
+def reserve_for(q, k_prefix, stream=None) -> None:
+    """dm05_suffix_attn_reserve for the sizes of these tensors (call before graph capture)."""
+    B, Hq, S, D = q.shape
+    rc = dm05_suffix_attn_reserve(B, Hq, k_prefix.shape[1], k_prefix.shape[2], S, D, _stream_handle(stream))
+    if rc != DM05_OK:
+        raise Dm05Error(rc, "dm05_suffix_attn_reserve")

@@ -1,0 +1,324 @@
+// dm05_suffix_attn.cu -- C ABI of the sm_100a suffix attention: argument
+// checks, the split plan, TMA descriptors, the per-device workspace (error
+// word) and the launch.  The operation is specified in
+// include/dm05_suffix_attn.h.
+#include "dm05_suffix_attn.h"
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "suffix_attn_kernel.cuh"
+
+namespace {
+
+constexpr int kTileRows = 64;
+constexpr int kStages = 2;
+using Layout = dm05::SmemLayout<kTileRows, kStages>;
+constexpr size_t kWorkspaceBytes = 256;  // error word (padded to one 256-byte segment)
+constexpr int kMaxUnits = 1 << 24;       // B * Hkv
+constexpr int kMaxPrefix = 1 << 24;      // P
+
+struct DeviceState {
+    uint32_t *err = nullptr;   // device error word
+    bool attrs_set = false;
+    int num_sms = 0;
+    int max_cluster = 0;       // largest cluster size (power of two <= 16) that can be resident
+};
+
+std::mutex g_mu;
+std::vector<DeviceState> g_dev;
+int g_split_override = 0;
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+auto *kKernel = &dm05::suffix_attn_kernel<kTileRows, kStages>;
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_sizes(int B, int Hq, int Hkv, int P, int S, int D)
+{
+    if (B < 1 || Hq < 1 || Hkv < 1 || S < 1 || P < 0) return DM05_ERR_SHAPE;
+    if (Hq % Hkv != 0) return DM05_ERR_SHAPE;
+    if (static_cast<long long>(B) * Hkv > kMaxUnits || P > kMaxPrefix) return DM05_ERR_SHAPE;
+    if (D != dm05::kHeadDim) return DM05_ERR_UNSUPPORTED;
+    if (static_cast<long long>(Hq / Hkv) * S > dm05::kMRows) return DM05_ERR_UNSUPPORTED;
+    return DM05_OK;
+}
+
+// CTAs per (sample, KV head): the largest power of two (<= 16, <= the number
+// of 64-row key tiles) that keeps all CTAs of a call resident at once.
+int choose_splits(int B, int Hkv, int P, int S, int num_sms, int max_cluster)
+{
+    if (g_split_override > 0) return g_split_override;
+    const long long units = static_cast<long long>(B) * Hkv;
+    const int tiles = (P + kTileRows - 1) / kTileRows + (S + kTileRows - 1) / kTileRows;
+    int c = 1;
+    while (c * 2 <= max_cluster && units * (c * 2) <= num_sms && c * 2 <= tiles) c *= 2;
+    return c;
+}
+
+int get_encoder()
+{
+    if (g_encode) return DM05_OK;
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || fn == nullptr)
+        return DM05_ERR_CUDA;
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    return DM05_OK;
+}
+
+// Device state of the current device with kernel attributes set; the error
+// word is created only if `allocate`.  Caller holds g_mu.
+int device_state(bool allocate, DeviceState **out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return DM05_ERR_CUDA;
+    if (dev >= static_cast<int>(g_dev.size())) g_dev.resize(dev + 1);
+    DeviceState &ds = g_dev[dev];
+    if (!ds.attrs_set) {
+        if (cudaDeviceGetAttribute(&ds.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return DM05_ERR_CUDA;
+        if (cudaFuncSetAttribute(kKernel, cudaFuncAttributeMaxDynamicSharedMemorySize, Layout::kAllocBytes) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(kKernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
+            return DM05_ERR_CUDA;
+        // largest cluster the device can hold with this kernel's footprint
+        ds.max_cluster = 1;
+        for (int c = 16; c >= 2; c /= 2) {
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(c, 1, 1);
+            cfg.blockDim = dim3(dm05::kThreads, 1, 1);
+            cfg.dynamicSmemBytes = Layout::kAllocBytes;
+            cudaLaunchAttribute at[1];
+            at[0].id = cudaLaunchAttributeClusterDimension;
+            at[0].val.clusterDim.x = c;
+            at[0].val.clusterDim.y = 1;
+            at[0].val.clusterDim.z = 1;
+            cfg.attrs = at;
+            cfg.numAttrs = 1;
+            int n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, kKernel, &cfg) == cudaSuccess && n > 0) {
+                ds.max_cluster = c;
+                break;
+            }
+            cudaGetLastError();  // clear a refused size
+        }
+        ds.attrs_set = true;
+    }
+    if (allocate && ds.err == nullptr) {
+        void *p = nullptr;
+        if (cudaMalloc(&p, kWorkspaceBytes) != cudaSuccess) return DM05_ERR_CUDA;
+        if (cudaMemset(p, 0, kWorkspaceBytes) != cudaSuccess) {
+            cudaFree(p);
+            return DM05_ERR_CUDA;
+        }
+        ds.err = static_cast<uint32_t *>(p);
+    }
+    *out = &ds;
+    return DM05_OK;
+}
+
+// bf16 tensor viewed as [d2][d1][256], loaded in boxes of 64 columns x box1 rows
+// with 128-byte swizzle; rows past d1 read as zero.
+int encode_3d(CUtensorMap *map, const void *base, uint64_t d1, uint64_t d2, uint32_t box1)
+{
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(dm05::kHeadDim), d1, d2};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(dm05::kHeadDim) * 2, d1 * dm05::kHeadDim * 2};
+    cuuint32_t box[3] = {static_cast<cuuint32_t>(dm05::kChunkElems), box1, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? DM05_OK : DM05_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *dm05_status_string(int status)
+{
+    switch (status) {
+    case DM05_OK: return "DM05_OK";
+    case DM05_ERR_NULL: return "DM05_ERR_NULL: a required pointer is NULL";
+    case DM05_ERR_SHAPE: return "DM05_ERR_SHAPE: invalid sizes";
+    case DM05_ERR_UNSUPPORTED: return "DM05_ERR_UNSUPPORTED: D must be 256 and (Hq/Hkv)*S at most 128";
+    case DM05_ERR_ALIGN: return "DM05_ERR_ALIGN: a bf16 tensor base is not 16-byte aligned";
+    case DM05_ERR_WORKSPACE: return "DM05_ERR_WORKSPACE: no workspace on this device while the stream is capturing";
+    case DM05_ERR_CUDA: return "DM05_ERR_CUDA: a CUDA call failed";
+    default: return "unknown dm05 status";
+    }
+}
+
+size_t dm05_suffix_attn_workspace_bytes(int B, int Hq, int Hkv, int P, int S, int D)
+{
+    return check_sizes(B, Hq, Hkv, P, S, D) == DM05_OK ? kWorkspaceBytes : 0;
+}
+
+int dm05_set_split_override(int splits_per_head)
+{
+    if (splits_per_head != 0 && splits_per_head != 1 && splits_per_head != 2 && splits_per_head != 4 &&
+        splits_per_head != 8 && splits_per_head != 16)
+        return DM05_ERR_SHAPE;
+    std::lock_guard<std::mutex> lk(g_mu);
+    g_split_override = splits_per_head;
+    return DM05_OK;
+}
+
+int dm05_suffix_attn_plan(int B, int Hq, int Hkv, int P, int S, int D, int *splits_per_head, int *tile_rows)
+{
+    int rc = check_sizes(B, Hq, Hkv, P, S, D);
+    if (rc != DM05_OK) return rc;
+    std::lock_guard<std::mutex> lk(g_mu);
+    DeviceState *ds = nullptr;
+    rc = device_state(false, &ds);
+    if (rc != DM05_OK) return rc;
+    if (splits_per_head) *splits_per_head = choose_splits(B, Hkv, P, S, ds->num_sms, ds->max_cluster);
+    if (tile_rows) *tile_rows = kTileRows;
+    return DM05_OK;
+}
+
+int dm05_suffix_attn_reserve(int B, int Hq, int Hkv, int P, int S, int D, cudaStream_t stream)
+{
+    int rc = check_sizes(B, Hq, Hkv, P, S, D);
+    if (rc != DM05_OK) return rc;
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) return DM05_ERR_CUDA;
+    if (cs != cudaStreamCaptureStatusNone) return DM05_ERR_WORKSPACE;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (get_encoder() != DM05_OK) return DM05_ERR_CUDA;
+    DeviceState *ds = nullptr;
+    return device_state(true, &ds);
+}
+
+int dm05_suffix_attn(const void *q, const void *k_prefix, const void *v_prefix, const int32_t *prefix_valid_len,
+                     const uint8_t *prefix_mask, const void *k_suffix, const void *v_suffix, void *out, float *lse,
+                     int B, int Hq, int Hkv, int P, int S, int D, cudaStream_t stream)
+{
+    // ---- host-side checks; nothing is launched on failure
+    if (!q || !k_suffix || !v_suffix || !out) return DM05_ERR_NULL;
+    if (P > 0 && (!k_prefix || !v_prefix)) return DM05_ERR_NULL;
+    int rc = check_sizes(B, Hq, Hkv, P, S, D);
+    if (rc != DM05_OK) return rc;
+    if (!aligned16(q) || !aligned16(k_suffix) || !aligned16(v_suffix) || !aligned16(out) ||
+        (P > 0 && (!aligned16(k_prefix) || !aligned16(v_prefix))))
+        return DM05_ERR_ALIGN;
+    if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u) != 0) return DM05_ERR_ALIGN;
+
+    const int G = Hq / Hkv;
+    const int GS = G * S;
+    const int units = B * Hkv;
+
+    DeviceState *ds = nullptr;
+    int splits = 1;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (get_encoder() != DM05_OK) return DM05_ERR_CUDA;
+        rc = device_state(false, &ds);
+        if (rc != DM05_OK) return rc;
+        if (ds->err == nullptr) {
+            cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+            if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) return DM05_ERR_CUDA;
+            if (cs != cudaStreamCaptureStatusNone) return DM05_ERR_WORKSPACE;
+            rc = device_state(true, &ds);
+            if (rc != DM05_OK) return rc;
+        }
+        splits = choose_splits(B, Hkv, P, S, ds->num_sms, ds->max_cluster);
+        if (splits > ds->max_cluster) splits = ds->max_cluster;
+    }
+
+    // ---- TMA descriptors (the tensor maps travel as kernel parameters)
+    CUtensorMap tm_q, tm_kp, tm_vp, tm_ks, tm_vs;
+    if (encode_3d(&tm_q, q, static_cast<uint64_t>(GS), static_cast<uint64_t>(units), dm05::kMRows) != DM05_OK ||
+        encode_3d(&tm_ks, k_suffix, static_cast<uint64_t>(S), static_cast<uint64_t>(units), kTileRows) != DM05_OK ||
+        encode_3d(&tm_vs, v_suffix, static_cast<uint64_t>(S), static_cast<uint64_t>(units), kTileRows) != DM05_OK)
+        return DM05_ERR_CUDA;
+    if (P > 0) {
+        if (encode_3d(&tm_kp, k_prefix, static_cast<uint64_t>(P), static_cast<uint64_t>(units), kTileRows) !=
+                DM05_OK ||
+            encode_3d(&tm_vp, v_prefix, static_cast<uint64_t>(P), static_cast<uint64_t>(units), kTileRows) != DM05_OK)
+            return DM05_ERR_CUDA;
+    } else {
+        tm_kp = tm_ks;  // never read: no prefix tile exists when P == 0
+        tm_vp = tm_vs;
+    }
+
+    dm05::KernelParams kp;
+    kp.valid_len = prefix_valid_len;
+    kp.mask = prefix_mask;
+    kp.out = static_cast<__nv_bfloat16 *>(out);
+    kp.lse = lse;
+    kp.err = ds->err;
+    kp.Hkv = Hkv;
+    kp.P = P;
+    kp.S = S;
+    kp.GS = GS;
+    kp.splits = splits;
+    kp.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(units * splits), 1, 1);
+    cfg.blockDim = dim3(dm05::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = Layout::kAllocBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute at[2];
+    int na = 0;
+    at[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+    if (splits > 1) {
+        at[na].id = cudaLaunchAttributeClusterDimension;
+        at[na].val.clusterDim.x = static_cast<unsigned>(splits);
+        at[na].val.clusterDim.y = 1;
+        at[na].val.clusterDim.z = 1;
+        ++na;
+    }
+    cfg.attrs = at;
+    cfg.numAttrs = na;
+    if (cudaLaunchKernelEx(&cfg, kKernel, tm_q, tm_kp, tm_vp, tm_ks, tm_vs, kp) != cudaSuccess) return DM05_ERR_CUDA;
+    return DM05_OK;
+}
+
+int dm05_get_error_word(cudaStream_t stream, uint32_t *host_word)
+{
+    if (!host_word) return DM05_ERR_NULL;
+    uint32_t *err = nullptr;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        DeviceState *ds = nullptr;
+        int rc = device_state(false, &ds);
+        if (rc != DM05_OK) return rc;
+        err = ds->err;
+    }
+    *host_word = 0;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return DM05_ERR_CUDA;
+    if (err == nullptr) return DM05_OK;
+    if (cudaMemcpyAsync(host_word, err, sizeof(uint32_t), cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
+        cudaMemsetAsync(err, 0, sizeof(uint32_t), stream) != cudaSuccess || cudaStreamSynchronize(stream) != cudaSuccess)
+        return DM05_ERR_CUDA;
+    return DM05_OK;
+}
+
+void dm05_release(void)
+{
+    std::lock_guard<std::mutex> lk(g_mu);
+    int cur = 0;
+    bool have_cur = cudaGetDevice(&cur) == cudaSuccess;
+    for (size_t d = 0; d < g_dev.size(); ++d) {
+        if (g_dev[d].err != nullptr) {
+            if (cudaSetDevice(static_cast<int>(d)) == cudaSuccess) cudaFree(g_dev[d].err);
+            g_dev[d].err = nullptr;
+        }
+    }
+    if (have_cur) cudaSetDevice(cur);
+}
+
+}  // extern "C"

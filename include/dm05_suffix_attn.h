@@ -1,0 +1,135 @@
+/*
+ * dm05_suffix_attn.h -- C ABI of the B200 (sm_100a) suffix attention of the
+ * DM0.5 action expert.
+ *
+ * The operation (page "TensorRT+Triton+FlexAttention: OpenDM VLA
+ * 快速推理加速栈深度剖析", section 2.2 "Triton 大 Kernel"): the action-chunk
+ * queries attend at once over the prefix KV cache and over the suffix's own
+ * K/V, under the prefix-visibility mask, with a softmax and a value-weighted
+ * sum.  The same section's shape table gives head_dim 256 and 8 query heads
+ * over 4 KV heads (GQA).  The prefix cache is padded to a length bucket
+ * (same page, section 3; page "DM05 推理指南", section "Fast Backend 约束"),
+ * so each sample carries a valid prefix length.
+ *
+ * For every sample b, query head h (KV head g = h / (Hq / Hkv)) and suffix
+ * query i:
+ *   visible keys  = prefix rows j with j < clamp(prefix_valid_len[b], 0, P)
+ *                   and (prefix_mask == NULL or prefix_mask[b*P + j] != 0),
+ *                   plus every suffix row k < S (suffix keys are visible to
+ *                   every suffix query);
+ *   logit(x)      = <q[b,h,i,:], K_x> / sqrt(D);
+ *   lse[b,h,i]    = ln sum_x exp(logit(x))           (natural log, fp32);
+ *   out[b,h,i,:]  = sum_x exp(logit(x) - lse) V_x     (rounded once to bf16).
+ *
+ * Layouts: every tensor is dense, row-major, with the last dimension
+ * contiguous.  All device pointers are addresses in the memory of the CUDA
+ * device that is current on the calling thread.
+ *
+ * Ownership: the caller owns every tensor.  The library keeps no pointer
+ * after a call returns.  The library owns one small device workspace per
+ * device (an error word); it is created by dm05_suffix_attn_reserve or by the
+ * first dm05_suffix_attn on the device that runs outside stream capture, and
+ * freed by dm05_release.
+ *
+ * Errors: every entry point returns a dm05_status.  Arguments are checked on
+ * the host before anything is launched; a failed check launches nothing.
+ * Nothing on the success path synchronises the host.
+ */
+#ifndef DM05_SUFFIX_ATTN_H
+#define DM05_SUFFIX_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    DM05_OK = 0,
+    DM05_ERR_NULL = -1,        /* a required pointer is NULL */
+    DM05_ERR_SHAPE = -2,       /* B, Hq, Hkv, S < 1, P < 0, Hq % Hkv != 0, or sizes too large */
+    DM05_ERR_UNSUPPORTED = -3, /* D != 256, or (Hq/Hkv)*S > 128 */
+    DM05_ERR_ALIGN = -4,       /* a bf16 tensor base is not 16-byte aligned */
+    DM05_ERR_WORKSPACE = -5,   /* no workspace on this device and the stream is capturing */
+    DM05_ERR_CUDA = -6         /* a CUDA call failed (launch, attribute, allocation) */
+} dm05_status;
+
+/* Bits of the device error word (dm05_get_error_word). */
+#define DM05_EW_VALID_LEN_CLAMPED 0x1u /* a prefix_valid_len value was outside [0, P] and was clamped */
+#define DM05_EW_WAIT_TIMEOUT      0x2u /* a kernel wait gave up after its time limit; outputs invalid */
+
+/*
+ * dm05_suffix_attn -- one suffix-attention call, asynchronous on `stream`.
+ *
+ *   q                 bf16  [B, Hq, S, D]    suffix queries
+ *   k_prefix          bf16  [B, Hkv, P, D]   bucket-padded prefix key cache (NULL allowed iff P == 0)
+ *   v_prefix          bf16  [B, Hkv, P, D]   prefix value cache              (NULL allowed iff P == 0)
+ *   prefix_valid_len  int32 [B]     device; NULL = every prefix row is in range.  Values
+ *                                   outside [0, P] are clamped and flagged in the error word.
+ *   prefix_mask       uint8 [B, P]  device; 1 = visible, 0 = hidden; NULL = no extra mask.
+ *   k_suffix          bf16  [B, Hkv, S, D]   suffix keys
+ *   v_suffix          bf16  [B, Hkv, S, D]   suffix values
+ *   out               bf16  [B, Hq, S, D]    result (written)
+ *   lse               fp32  [B, Hq, S]       natural-log LSE of the scaled logits; NULL = not written
+ *   B, Hq, Hkv, P, S, D  sizes; query head h reads KV head h / (Hq / Hkv).
+ *   stream            CUDA stream (0 = legacy default stream).
+ *
+ * Supported: D == 256 and (Hq / Hkv) * S <= 128; P >= 0.  Bases of q,
+ * k_prefix, v_prefix, k_suffix, v_suffix and out must be 16-byte aligned.
+ * Prefix rows at or past the valid length are never used: they may hold any
+ * bits, NaN included.  Hidden rows inside the valid range must hold finite
+ * values (they are multiplied by an exact zero weight).
+ *
+ * The call is deterministic for fixed inputs and sizes, does not
+ * synchronise, and may be captured into a CUDA graph once the device has a
+ * workspace (dm05_suffix_attn_reserve).  Consecutive calls on one stream may
+ * overlap their start-up with the previous kernel (programmatic dependent
+ * launch); each call still waits for all earlier work on the stream before
+ * it reads an input or writes an output.
+ */
+int dm05_suffix_attn(const void *q, const void *k_prefix, const void *v_prefix,
+                     const int32_t *prefix_valid_len, const uint8_t *prefix_mask,
+                     const void *k_suffix, const void *v_suffix,
+                     void *out, float *lse,
+                     int B, int Hq, int Hkv, int P, int S, int D,
+                     cudaStream_t stream);
+
+/* Bytes of device workspace dm05_suffix_attn needs for these sizes (the
+ * per-device error word).  0 if the sizes are invalid. */
+size_t dm05_suffix_attn_workspace_bytes(int B, int Hq, int Hkv, int P, int S, int D);
+
+/* Creates the workspace of the current device for these sizes, and sets the
+ * kernel attributes, outside any stream capture.  Call it before capturing
+ * dm05_suffix_attn into a CUDA graph.  `stream` must not be capturing. */
+int dm05_suffix_attn_reserve(int B, int Hq, int Hkv, int P, int S, int D, cudaStream_t stream);
+
+/* Work decomposition the next call with these sizes will use: the number of
+ * CTAs (one thread-block cluster) per (sample, KV head), and the key rows per
+ * tile.  Either output pointer may be NULL. */
+int dm05_suffix_attn_plan(int B, int Hq, int Hkv, int P, int S, int D,
+                          int *splits_per_head, int *tile_rows);
+
+/* Forces the number of CTAs per (sample, KV head) for later calls on this
+ * process: 1, 2, 4, 8 or 16; 0 restores the automatic choice.  For tuning
+ * and tests.  Returns DM05_ERR_SHAPE for any other value. */
+int dm05_set_split_override(int splits_per_head);
+
+/* Synchronises `stream`, then returns in *host_word the error bits
+ * (DM05_EW_*) that kernels on the current device set since the last read,
+ * and clears them. */
+int dm05_get_error_word(cudaStream_t stream, uint32_t *host_word);
+
+/* Human-readable name of a dm05_status value. */
+const char *dm05_status_string(int status);
+
+/* Frees every workspace the library holds (all devices).  No call may be in
+ * flight. */
+void dm05_release(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DM05_SUFFIX_ATTN_H */

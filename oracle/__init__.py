@@ -65,6 +65,8 @@ class Oracle:
         i = ctypes.c_int
         lib.oracle_suffix_attn_range.argtypes = [p] * 9 + [i] * 6 + [i, i, i]
         lib.oracle_suffix_attn_range.restype = i
+        lib.oracle_suffix_attn_rows.argtypes = [p] * 9 + [i] * 6 + [i, i, ctypes.c_long, ctypes.c_long, i]
+        lib.oracle_suffix_attn_rows.restype = i
         lib.oracle_suffix_attn.argtypes = [p] * 9 + [i] * 6 + [i]
         lib.oracle_suffix_attn.restype = i
         lib.oracle_merge_parts.argtypes = [p, p, i, ctypes.c_long, i, p, p]
@@ -78,11 +80,14 @@ class Oracle:
         return int(self.lib.oracle_max_threads())
 
     def suffix_attn(self, q, k_prefix, v_prefix, prefix_valid_len, prefix_mask, k_suffix,
-                    v_suffix, B, Hq, Hkv, P, S, D, key_range=None, nthreads: int = 1):
+                    v_suffix, B, Hq, Hkv, P, S, D, key_range=None, nthreads: int = 1,
+                    row_range=None):
         """Return (out float64 [B,Hq,S,D], lse float64 [B,Hq,S]).
 
         key_range=(lo, hi) restricts the keys to the index-space slice [lo, hi)
-        where [0, P) are prefix positions and [P, P+S) suffix positions."""
+        where [0, P) are prefix positions and [P, P+S) suffix positions.
+        row_range=(lo, hi) computes only the flat query rows (b*Hq + h)*S + i
+        in [lo, hi); the other rows of the result are left at zero."""
         qb, kpb, vpb = _bits(q), _bits(k_prefix), _bits(v_prefix)
         ksb, vsb = _bits(k_suffix), _bits(v_suffix)
         if qb.size != B * Hq * S * D or ksb.size != B * Hkv * S * D or vsb.size != B * Hkv * S * D:
@@ -98,11 +103,13 @@ class Oracle:
         out = np.zeros((B, Hq, S, D), dtype=np.float64)
         lse = np.zeros((B, Hq, S), dtype=np.float64)
         lo, hi = (0, P + S) if key_range is None else key_range
-        rc = self.lib.oracle_suffix_attn_range(
+        rlo, rhi = (0, B * Hq * S) if row_range is None else row_range
+        rc = self.lib.oracle_suffix_attn_rows(
             _ptr(qb), _ptr(kpb), _ptr(vpb), _ptr(vl), _ptr(mk), _ptr(ksb), _ptr(vsb),
-            _ptr(out), _ptr(lse), B, Hq, Hkv, P, S, D, int(lo), int(hi), int(nthreads))
+            _ptr(out), _ptr(lse), B, Hq, Hkv, P, S, D, int(lo), int(hi), int(rlo), int(rhi),
+            int(nthreads))
         if rc != 0:
-            raise ValueError(f"oracle_suffix_attn_range failed with status {rc}")
+            raise ValueError(f"oracle_suffix_attn_rows failed with status {rc}")
         return out, lse
 
     def merge_parts(self, o_parts, lse_parts):
@@ -120,12 +127,12 @@ class Oracle:
             raise ValueError(f"oracle_merge_parts failed with status {rc}")
         return out, lse
 
-    def inputs_call(self, inp, nthreads: int = 1, key_range=None):
+    def inputs_call(self, inp, nthreads: int = 1, key_range=None, row_range=None):
         """Run on an object with the attributes of a SuffixAttnInputs."""
         return self.suffix_attn(inp.q, inp.k_prefix, inp.v_prefix, inp.prefix_valid_len,
                                 inp.prefix_mask, inp.k_suffix, inp.v_suffix,
                                 inp.B, inp.Hq, inp.Hkv, inp.P, inp.S, inp.D,
-                                key_range=key_range, nthreads=nthreads)
+                                key_range=key_range, nthreads=nthreads, row_range=row_range)
 
 
 def default() -> Oracle:
@@ -151,6 +158,6 @@ def merge_parts(o_parts, lse_parts):
     return default().merge_parts(o_parts, lse_parts)
 
 
-def inputs_call(inp, nthreads: int = 1, key_range=None):
+def inputs_call(inp, nthreads: int = 1, key_range=None, row_range=None):
     """Oracle.inputs_call on the default build."""
-    return default().inputs_call(inp, nthreads=nthreads, key_range=key_range)
+    return default().inputs_call(inp, nthreads=nthreads, key_range=key_range, row_range=row_range)

@@ -125,22 +125,23 @@ static int check_shape(int B, int Hq, int Hkv, int P, int S, int D)
 }
 
 /*
- * Attention of every (b, h, i) over the keys x in [key_lo, key_hi) of the
- * index space [0, P+S) (prefix positions, then suffix positions).  With
- * key_lo = 0 and key_hi = P + S this is the full result.  Layouts (row-major,
- * bf16 passed as uint16 bit patterns):
+ * Attention of the query rows r in [row_lo, row_hi) (flat index
+ * r = (b*Hq + h)*S + i) over the keys x in [key_lo, key_hi) of the index
+ * space [0, P+S) (prefix positions, then suffix positions).  With the full
+ * ranges this is the whole result; rows outside [row_lo, row_hi) are not
+ * written.  Layouts (row-major, bf16 passed as uint16 bit patterns):
  *   q [B,Hq,S,D], k_prefix/v_prefix [B,Hkv,P,D], k_suffix/v_suffix [B,Hkv,S,D],
  *   prefix_valid_len int32 [B] or NULL, prefix_mask uint8 [B,P] or NULL,
  *   out double [B,Hq,S,D], lse double [B,Hq,S].
- * nthreads > 1 spreads the (b, h) pairs over OpenMP threads.
+ * nthreads > 1 spreads the rows over OpenMP threads.
  * Returns 0, -1 for a NULL pointer, -2 for a bad shape, -7 for no memory.
  */
-int oracle_suffix_attn_range(const uint16_t *q, const uint16_t *k_prefix, const uint16_t *v_prefix,
-                             const int32_t *prefix_valid_len, const uint8_t *prefix_mask,
-                             const uint16_t *k_suffix, const uint16_t *v_suffix,
-                             double *out, double *lse,
-                             int B, int Hq, int Hkv, int P, int S, int D,
-                             int key_lo, int key_hi, int nthreads)
+int oracle_suffix_attn_rows(const uint16_t *q, const uint16_t *k_prefix, const uint16_t *v_prefix,
+                            const int32_t *prefix_valid_len, const uint8_t *prefix_mask,
+                            const uint16_t *k_suffix, const uint16_t *v_suffix,
+                            double *out, double *lse,
+                            int B, int Hq, int Hkv, int P, int S, int D,
+                            int key_lo, int key_hi, long row_lo, long row_hi, int nthreads)
 {
     if (!q || !k_suffix || !v_suffix || !out || !lse) return -1;
     if (P > 0 && (!k_prefix || !v_prefix)) return -1;
@@ -149,6 +150,9 @@ int oracle_suffix_attn_range(const uint16_t *q, const uint16_t *k_prefix, const 
     if (key_lo < 0) key_lo = 0;
     if (key_hi > P + S) key_hi = P + S;
     if (key_hi < key_lo) key_hi = key_lo;
+    const long n_rows = (long)B * Hq * S;
+    if (row_lo < 0) row_lo = 0;
+    if (row_hi > n_rows) row_hi = n_rows;
     const int G = Hq / Hkv;
     const int n_keys = key_hi - key_lo;
     int failed = 0;
@@ -160,28 +164,39 @@ int oracle_suffix_attn_range(const uint16_t *q, const uint16_t *k_prefix, const 
         if (!logit_buf) {
             failed = 1;
         } else {
-#pragma omp for schedule(dynamic, 1)
-            for (int bh = 0; bh < B * Hq; ++bh) {
-                const int b = bh / Hq, h = bh % Hq;
+#pragma omp for schedule(static)
+            for (long row = row_lo; row < row_hi; ++row) {
+                const int b = (int)(row / ((long)Hq * S));
+                const int h = (int)((row / S) % Hq);
                 const int kv = h / G;
                 const int vl = clamp_valid_len(prefix_valid_len, b, P);
                 const uint8_t *mask_row = prefix_mask ? prefix_mask + (size_t)b * P : NULL;
                 const size_t kv_off_p = ((size_t)b * Hkv + kv) * (size_t)P * D;
                 const size_t kv_off_s = ((size_t)b * Hkv + kv) * (size_t)S * D;
-                for (int i = 0; i < S; ++i) {
-                    const size_t row = ((size_t)b * Hq + h) * S + i;
-                    attend_row(q + row * D,
-                               P > 0 ? k_prefix + kv_off_p : NULL,
-                               P > 0 ? v_prefix + kv_off_p : NULL,
-                               k_suffix + kv_off_s, v_suffix + kv_off_s, mask_row,
-                               vl, P, S, D, key_lo, key_hi, logit_buf,
-                               out + row * D, lse + row);
-                }
+                attend_row(q + (size_t)row * D,
+                           P > 0 ? k_prefix + kv_off_p : NULL,
+                           P > 0 ? v_prefix + kv_off_p : NULL,
+                           k_suffix + kv_off_s, v_suffix + kv_off_s, mask_row,
+                           vl, P, S, D, key_lo, key_hi, logit_buf,
+                           out + (size_t)row * D, lse + row);
             }
             free(logit_buf);
         }
     }
     return failed ? -7 : 0;
+}
+
+/* Every query row over the keys x in [key_lo, key_hi). */
+int oracle_suffix_attn_range(const uint16_t *q, const uint16_t *k_prefix, const uint16_t *v_prefix,
+                             const int32_t *prefix_valid_len, const uint8_t *prefix_mask,
+                             const uint16_t *k_suffix, const uint16_t *v_suffix,
+                             double *out, double *lse,
+                             int B, int Hq, int Hkv, int P, int S, int D,
+                             int key_lo, int key_hi, int nthreads)
+{
+    return oracle_suffix_attn_rows(q, k_prefix, v_prefix, prefix_valid_len, prefix_mask,
+                                   k_suffix, v_suffix, out, lse, B, Hq, Hkv, P, S, D,
+                                   key_lo, key_hi, 0, (long)B * Hq * S, nthreads);
 }
 
 /* The full attention: every visible prefix key and every suffix key. */

@@ -1,0 +1,113 @@
+"""The C-ABI library without a GPU: it loads, exports every declared entry
+point, and rejects bad arguments on the host before touching CUDA."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from gqa_prefix_suffix_b200 import binding as bd
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dm05_suffix_attn.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(dm05_[a-z_0-9]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from gqa_prefix_suffix_b200 import build
+    build.build()
+    return bd.lib()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert set(names) == set(bd.EXPORTS)
+    out = subprocess.run(["nm", "-D", "--defined-only", bd.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(re.findall(r"\bT (dm05_[a-z_0-9]+)$", out, flags=re.M))
+    for n in names:
+        assert n in exported, n
+        assert hasattr(lib, n)
+
+
+def test_status_strings(lib):
+    for st in (0, -1, -2, -3, -4, -5, -6):
+        assert bd.dm05_status_string(st).startswith("DM05_")
+    assert "unknown" in bd.dm05_status_string(99)
+
+
+FAKE = 0x7f0000001000  # 16-byte aligned, never dereferenced: checks fail first
+
+
+def call(**kw):
+    a = dict(q=FAKE, k_prefix=FAKE, v_prefix=FAKE, prefix_valid_len=None, prefix_mask=None,
+             k_suffix=FAKE, v_suffix=FAKE, out=FAKE, lse=None, B=1, Hq=8, Hkv=4, P=1024, S=50, D=256,
+             stream=None)
+    a.update(kw)
+    return bd.dm05_suffix_attn(a["q"], a["k_prefix"], a["v_prefix"], a["prefix_valid_len"],
+                               a["prefix_mask"], a["k_suffix"], a["v_suffix"], a["out"], a["lse"],
+                               a["B"], a["Hq"], a["Hkv"], a["P"], a["S"], a["D"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), bd.DM05_ERR_NULL),
+    (dict(k_suffix=None), bd.DM05_ERR_NULL),
+    (dict(v_suffix=None), bd.DM05_ERR_NULL),
+    (dict(out=None), bd.DM05_ERR_NULL),
+    (dict(k_prefix=None), bd.DM05_ERR_NULL),
+    (dict(v_prefix=None), bd.DM05_ERR_NULL),
+    (dict(B=0), bd.DM05_ERR_SHAPE),
+    (dict(S=0), bd.DM05_ERR_SHAPE),
+    (dict(P=-1), bd.DM05_ERR_SHAPE),
+    (dict(Hq=6), bd.DM05_ERR_SHAPE),
+    (dict(Hkv=0), bd.DM05_ERR_SHAPE),
+    (dict(P=(1 << 24) + 1), bd.DM05_ERR_SHAPE),
+    (dict(D=128), bd.DM05_ERR_UNSUPPORTED),
+    (dict(S=65), bd.DM05_ERR_UNSUPPORTED),        # G*S = 130 > 128
+    (dict(Hkv=8, S=129), bd.DM05_ERR_UNSUPPORTED),
+    (dict(q=FAKE + 8), bd.DM05_ERR_ALIGN),
+    (dict(k_prefix=FAKE + 2), bd.DM05_ERR_ALIGN),
+    (dict(v_suffix=FAKE + 4), bd.DM05_ERR_ALIGN),
+    (dict(out=FAKE + 8), bd.DM05_ERR_ALIGN),
+    (dict(lse=FAKE + 2), bd.DM05_ERR_ALIGN),
+])
+def test_host_checks_reject(lib, kw, status):
+    assert call(**kw) == status
+
+
+def test_prefix_pointers_optional_when_p_is_zero(lib):
+    # P == 0 accepts NULL prefix pointers: the checks pass, so the call gets
+    # as far as CUDA, which is absent here (or it launches on a GPU machine: not
+    # in this CPU test).
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("would launch on a GPU")
+    assert call(P=0, k_prefix=None, v_prefix=None) == bd.DM05_ERR_CUDA
+
+
+def test_workspace_bytes(lib):
+    assert bd.dm05_suffix_attn_workspace_bytes(1, 8, 4, 1024, 50, 256) > 0
+    assert bd.dm05_suffix_attn_workspace_bytes(1, 8, 4, 1024, 50, 128) == 0
+    assert bd.dm05_suffix_attn_workspace_bytes(0, 8, 4, 1024, 50, 256) == 0
+
+
+def test_split_override_values(lib):
+    for v in (0, 1, 2, 4, 8, 16):
+        assert bd.dm05_set_split_override(v) == bd.DM05_OK
+    for v in (3, 32, -1):
+        assert bd.dm05_set_split_override(v) == bd.DM05_ERR_SHAPE
+    assert bd.dm05_set_split_override(0) == bd.DM05_OK
+
+
+def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
+    monkeypatch.setattr(bd, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(bd, "_lib", None)
+    with pytest.raises(RuntimeError, match="missing"):
+        bd.lib()

@@ -23,3 +23,13 @@ def test_bad_shapes_rejected(orc):
         cc = dict(c, **bad)
         with pytest.raises(ValueError):
             pins.run(orc, cc)
+
+
+def test_row_range_selects_rows(orc):
+    c = pins.rand_case(33, 2, 4, 2, 9, 3, 8, mask_p=0.2)
+    o_full, l_full = pins.run(orc, c)
+    o_part, l_part = pins.run(orc, c, row_range=(5, 17))
+    flat_o, flat_l = o_part.reshape(-1, 8), l_part.reshape(-1)
+    assert np.array_equal(flat_o[5:17], o_full.reshape(-1, 8)[5:17])
+    assert np.array_equal(flat_l[5:17], l_full.reshape(-1)[5:17])
+    assert not flat_o[:5].any() and not flat_o[17:].any()

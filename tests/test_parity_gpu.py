@@ -1,0 +1,311 @@
+"""CUDA path against the fp64 oracle, element by element, on seeded inputs.
+
+Tolerance (bf16 output, fp32 accumulation): |out - O_oracle| <= 1e-2 for
+every element, except elements whose exact value has magnitude >= 4, where a
+correctly rounded bf16 value can already be 2^-6 = 0.0156 away; those are
+held to one bf16 ulp of the exact value.  mean |out - O_oracle| <= 1e-3 and
+|lse - LSE_oracle| <= 1e-3.
+"""
+import math
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gqa_prefix_suffix_b200 import binding as bd
+from gqa_prefix_suffix_b200 import inputs as gen
+
+pytestmark = pytest.mark.gpu
+
+MAX_ABS = 1e-2
+MEAN_ABS = 1e-3
+LSE_ABS = 1e-3
+
+
+def bf16_ulp(x):
+    ax = np.maximum(np.abs(x), 1e-30)
+    return np.exp2(np.floor(np.log2(ax)) - 7)
+
+
+def element_bound(o_ref):
+    return np.where(np.abs(o_ref) >= 4.0, bf16_ulp(o_ref), MAX_ABS)
+
+
+def check_close(out, lse, o_ref, l_ref, what=""):
+    o = out.float().cpu().double().numpy()
+    err = np.abs(o - o_ref)
+    bound = element_bound(o_ref)
+    floor = np.abs(torch.from_numpy(o_ref).to(torch.bfloat16).double().numpy() - o_ref).max()
+    bad = err > bound
+    if bad.any():
+        rows = sorted({tuple(int(v) for v in idx[:3]) for idx in np.argwhere(bad)})
+        raise AssertionError(f"{what}: {int(bad.sum())} elements over the bound in {len(rows)} rows "
+                             f"(b,h,i) {rows[:12]}; max err {err.max():.5f} at "
+                             f"|o|={np.abs(o_ref).flat[err.argmax()]:.3f}; rounding floor {floor:.5f}")
+    assert err.mean() <= MEAN_ABS, f"{what}: mean err {err.mean():.2e}"
+    if lse is not None:
+        le = np.abs(lse.double().cpu().numpy() - l_ref)
+        assert le.max() <= LSE_ABS, f"{what}: lse err {le.max():.2e}"
+    return err.max(), err.mean()
+
+
+@pytest.fixture(scope="module", autouse=True)
+def cuda_ready():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from gqa_prefix_suffix_b200 import build
+    build.build()
+    bd.lib()
+    yield
+    bd.dm05_set_split_override(0)
+
+
+def run_gpu(inp, splits=0, with_lse=True, stream=None):
+    d = inp.to("cuda")
+    assert bd.dm05_set_split_override(splits) == 0
+    try:
+        out, lse = bd.suffix_attn(d.q, d.k_prefix, d.v_prefix, d.k_suffix, d.v_suffix,
+                                  prefix_valid_len=d.prefix_valid_len, prefix_mask=d.prefix_mask,
+                                  want_lse=with_lse, stream=stream)
+        torch.cuda.synchronize()
+    finally:
+        bd.dm05_set_split_override(0)
+    rc, word = bd.dm05_get_error_word(None)
+    assert rc == 0
+    return out.cpu(), (lse.cpu() if lse is not None else None), word
+
+
+def ref(inp):
+    return oracle.inputs_call(inp, nthreads=min(8, oracle.max_threads()))
+
+
+# ---------------------------------------------------------------- small / ragged shapes
+
+SMALL = [
+    # name, B, Hq, Hkv, P, S, valid (None|int|list|'rand'), mask_frac, peak(frac, mult)
+    ("no_prefix", 1, 8, 4, 0, 1, None, 0.0, None),
+    ("one_prefix_row", 1, 8, 4, 1, 1, 1, 0.0, None),
+    ("p63_s10", 2, 8, 4, 63, 10, "rand", 0.0, None),
+    ("p64_s50", 1, 8, 4, 64, 50, 64, 0.0, None),
+    ("p65_s50", 2, 8, 4, 65, 50, [65, 1], 0.0, None),
+    ("p127_s7", 1, 8, 4, 127, 7, 127, 0.2, None),
+    ("p128_s64", 1, 8, 4, 128, 64, [100], 0.0, None),
+    ("p129_s33", 3, 8, 4, 129, 33, "rand", 0.1, (0.05, 3.0)),
+    ("g1_s128", 1, 4, 4, 200, 128, 150, 0.0, None),
+    ("g4_s32", 2, 8, 2, 300, 32, "rand", 0.1, None),
+    ("g8_s16", 1, 8, 1, 333, 16, 321, 0.0, None),
+    ("valid_zero", 2, 8, 4, 256, 20, [0, 0], 0.0, None),
+    ("p576_s10_mask", 2, 8, 4, 576, 10, [512, 300], 0.3, (0.02, 4.0)),
+    ("p1000_s50_peaks", 1, 8, 4, 1000, 50, 999, 0.0, (0.05, 5.0)),
+]
+
+
+def make_small(name, B, Hq, Hkv, P, S, valid, mask_frac, peak, seed=7):
+    kw = {}
+    if valid == "rand":
+        kw["valid_range"] = (0, P)
+    elif valid is not None:
+        kw["valid_len"] = valid
+    if peak is not None:
+        kw["peak_frac"], kw["peak_mult"] = peak
+    return gen.make_inputs(B, Hq, Hkv, P, S, 256, seed + zlib.crc32(name.encode()) % 1000, mask_frac=mask_frac,
+                           name=name, **kw)
+
+
+@pytest.mark.parametrize("case", SMALL, ids=[c[0] for c in SMALL])
+def test_small_shapes(case):
+    inp = make_small(*case)
+    out, lse, word = run_gpu(inp)
+    o_ref, l_ref = ref(inp)
+    check_close(out, lse, o_ref, l_ref, case[0])
+    assert word == 0
+
+
+@pytest.mark.parametrize("splits", [1, 2, 4, 8, 16])
+def test_every_split_count(splits):
+    inp = gen.make_inputs(1, 8, 4, 1024, 50, 256, 99, valid_len=900, peak_frac=0.05, peak_mult=3.0,
+                          mask_frac=0.05)
+    out, lse, _ = run_gpu(inp, splits=splits)
+    o_ref, l_ref = ref(inp)
+    check_close(out, lse, o_ref, l_ref, f"splits={splits}")
+
+
+def test_splits_beyond_tiles():
+    # 16 CTAs for a unit with only 2 tiles: most CTAs get no work
+    inp = gen.make_inputs(2, 8, 4, 64, 10, 256, 5, valid_len=[40, 0])
+    out, lse, _ = run_gpu(inp, splits=16)
+    o_ref, l_ref = ref(inp)
+    check_close(out, lse, o_ref, l_ref, "splits beyond tiles")
+
+
+def ramp_case(top):
+    # K rows scaled by a factor that grows along the prefix, so the running
+    # max of every row moves by more than 2^8 (log2 units) between tiles.
+    inp = gen.make_inputs(1, 8, 4, 512, 20, 256, 11, valid_len=512)
+    ramp = torch.linspace(0.2, top, 512).view(1, 1, 512, 1)
+    inp.k_prefix = (inp.k_prefix.float() * ramp).to(torch.bfloat16)
+    return inp
+
+
+def test_lazy_rescale_path():
+    # x4 (the largest K multiplier of the workloads): every row rescales O
+    # at least once, some twice.
+    inp = ramp_case(4.0)
+    o_ref, l_ref = ref(inp)
+    for splits in (1, 2):
+        out, lse, _ = run_gpu(inp, splits=splits)
+        check_close(out, lse, o_ref, l_ref, f"ramp x4 splits={splits}")
+
+
+def test_peaked_precision_model():
+    """On a sharper input (K up to x6) the error is still the one the bf16
+    probabilities allow.  With p_j rounded to bf16 (relative error
+    u = 2^-8) and O normalised by the sum of the rounded p_j, to first order
+    |O_gpu - O| <= 2u max_j |v_j - O|; the output adds half a bf16 ulp."""
+    inp = ramp_case(6.0)
+    o_ref, l_ref = ref(inp)
+    G = inp.Hq // inp.Hkv
+    v_all = torch.cat([inp.v_prefix, inp.v_suffix], dim=2).double().numpy()   # [B,Hkv,P+S,D]
+    vmax = np.abs(v_all).max(axis=2)                                           # [B,Hkv,D]
+    vmax_q = np.repeat(vmax, G, axis=1)[:, :, None, :]                         # [B,Hq,1,D]
+    bound = 0.5 * bf16_ulp(o_ref) + 2.0 ** -7 * (vmax_q + np.abs(o_ref)) + 1e-5
+    for splits in (1, 2):
+        out, lse, _ = run_gpu(inp, splits=splits)
+        err = np.abs(out.float().double().numpy() - o_ref)
+        assert (err <= bound).all(), f"splits={splits}: max err {err.max():.5f}"
+        assert err.mean() <= MEAN_ABS
+        assert np.abs(lse.double().numpy() - l_ref).max() <= LSE_ABS
+
+
+def test_rows_past_valid_len_are_never_used():
+    inp = gen.make_inputs(2, 8, 4, 200, 30, 256, 12, valid_len=[130, 65], mask_frac=0.1)
+    o_ref, l_ref = ref(inp)
+    for b, vl in enumerate((130, 65)):
+        inp.k_prefix[b, :, vl:] = float("nan")
+        inp.v_prefix[b, :, vl:] = float("nan")
+        hidden = (inp.prefix_mask[b, :vl] == 0).nonzero().flatten()
+        inp.k_prefix[b, :, hidden] = 1.0e4
+        inp.v_prefix[b, :, hidden] = 1.0e4
+    for splits in (0, 1, 4):
+        out, lse, _ = run_gpu(inp, splits=splits)
+        assert torch.isfinite(out.float()).all()
+        check_close(out, lse, o_ref, l_ref, f"nan padding splits={splits}")
+
+
+def test_valid_len_out_of_range_is_clamped_and_flagged():
+    inp = gen.make_inputs(2, 8, 4, 128, 10, 256, 13, valid_len=[-5, 500])
+    out, lse, word = run_gpu(inp)
+    assert word & bd.DM05_EW_VALID_LEN_CLAMPED
+    o_ref, l_ref = ref(inp)  # the oracle clamps to [0, P] too
+    check_close(out, lse, o_ref, l_ref, "clamped")
+
+
+def test_no_valid_len_and_no_lse():
+    inp = gen.make_inputs(1, 8, 4, 96, 12, 256, 14, valid_len=None)
+    out, lse, _ = run_gpu(inp, with_lse=False)
+    assert lse is None
+    o_ref, l_ref = ref(inp)
+    check_close(out, None, o_ref, l_ref, "no valid_len")
+
+
+def test_deterministic():
+    inp = gen.base_chunk()
+    a, la, _ = run_gpu(inp)
+    b, lb, _ = run_gpu(inp)
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    assert torch.equal(la, lb)
+
+
+def test_no_writes_outside_outputs():
+    inp = gen.make_inputs(2, 8, 4, 300, 50, 256, 15, valid_range=(0, 300))
+    d = inp.to("cuda")
+    n_out = 2 * 8 * 50 * 256
+    pad = 4096
+    canary = torch.full((n_out + 2 * pad,), 7.0, dtype=torch.bfloat16, device="cuda")
+    lcan = torch.full((2 * 8 * 50 + 2 * pad,), 7.0, dtype=torch.float32, device="cuda")
+    out = canary[pad:pad + n_out].view(2, 8, 50, 256)
+    lse = lcan[pad:pad + 2 * 8 * 50].view(2, 8, 50)
+    for splits in (1, 16):
+        bd.dm05_set_split_override(splits)
+        bd.suffix_attn(d.q, d.k_prefix, d.v_prefix, d.k_suffix, d.v_suffix,
+                       prefix_valid_len=d.prefix_valid_len, out=out, lse=lse)
+        torch.cuda.synchronize()
+        bd.dm05_set_split_override(0)
+        assert bool((canary[:pad] == 7.0).all()) and bool((canary[pad + n_out:] == 7.0).all())
+        assert bool((lcan[:pad] == 7.0).all()) and bool((lcan[pad + 2 * 8 * 50:] == 7.0).all())
+    o_ref, l_ref = ref(inp)
+    check_close(out.cpu(), lse.cpu(), o_ref, l_ref, "canary")
+
+
+def test_waits_for_the_producer_of_its_inputs():
+    # q is written by a torch kernel right before the call on the same stream;
+    # the call (launched with programmatic dependent launch) must see it.
+    inp = gen.base_chunk()
+    d = inp.to("cuda")
+    q2 = torch.empty_like(d.q)
+    out = torch.empty_like(d.q)
+    for _ in range(3):
+        torch.mul(d.q, -1.0, out=q2)
+        bd.suffix_attn(q2, d.k_prefix, d.v_prefix, d.k_suffix, d.v_suffix,
+                       prefix_valid_len=d.prefix_valid_len, out=out, want_lse=False)
+    torch.cuda.synchronize()
+    inp2 = gen.base_chunk()
+    inp2.q = -inp2.q
+    o_ref, l_ref = ref(inp2)
+    check_close(out.cpu(), None, o_ref, l_ref, "pdl producer")
+
+
+def test_cuda_graph_capture_and_replay():
+    calls = gen.history_loop(3)
+    ds = [c.to("cuda") for c in calls]
+    s = torch.cuda.Stream()
+    bd.reserve_for(ds[0].q, ds[0].k_prefix, stream=s)
+    outs = [torch.empty_like(d.q) for d in ds]
+    lses = [torch.empty(d.q.shape[:3], dtype=torch.float32, device="cuda") for d in ds]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        for d, o, l in zip(ds, outs, lses):
+            bd.suffix_attn(d.q, d.k_prefix, d.v_prefix, d.k_suffix, d.v_suffix,
+                           prefix_valid_len=d.prefix_valid_len, out=o, lse=l, stream=s)
+    for o in outs:
+        o.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    for c, o, l in zip(calls, outs, lses):
+        o_ref, l_ref = ref(c)
+        check_close(o.cpu(), l.cpu(), o_ref, l_ref, c.name)
+
+
+# ---------------------------------------------------------------- the five workloads, full size
+
+def test_libero_tiny():
+    inp = gen.libero_tiny()
+    out, lse, _ = run_gpu(inp)
+    check_close(out, lse, *ref(inp), what=inp.name)
+
+
+def test_base_chunk():
+    inp = gen.base_chunk()
+    out, lse, _ = run_gpu(inp)
+    check_close(out, lse, *ref(inp), what=inp.name)
+
+
+def test_bucket_sweep():
+    for inp in gen.bucket_sweep():
+        out, lse, _ = run_gpu(inp)
+        check_close(out, lse, *ref(inp), what=inp.name)
+
+
+def test_history_loop():
+    for inp in gen.history_loop():
+        out, lse, _ = run_gpu(inp)
+        check_close(out, lse, *ref(inp), what=inp.name)
+
+
+def test_batched_mask():
+    inp = gen.batched_mask()
+    out, lse, _ = run_gpu(inp)
+    mx, mean = check_close(out, lse, *ref(inp), what=inp.name)
+    assert math.isfinite(mx)

@@ -25,7 +25,7 @@ DM05_EW_WAIT_TIMEOUT = 0x2
 
 EXPORTS = ("dm05_suffix_attn", "dm05_suffix_attn_workspace_bytes", "dm05_suffix_attn_reserve",
            "dm05_suffix_attn_plan", "dm05_set_split_override", "dm05_get_error_word",
-           "dm05_status_string", "dm05_release")
+           "dm05_status_string", "dm05_release", "dm05_suffix_attn_noalloc")
 
 _lock = threading.Lock()
 _lib = None
@@ -64,6 +64,8 @@ def lib() -> ctypes.CDLL:
             L.dm05_status_string.restype = ctypes.c_char_p
             L.dm05_release.argtypes = []
             L.dm05_release.restype = None
+            L.dm05_suffix_attn_noalloc.argtypes = [p] * 9 + [i] * 6 + [p]
+            L.dm05_suffix_attn_noalloc.restype = i
             _lib = L
     return _lib
 
@@ -74,6 +76,14 @@ def dm05_suffix_attn(q, k_prefix, v_prefix, prefix_valid_len, prefix_mask, k_suf
                      out, lse, B, Hq, Hkv, P, S, D, stream) -> int:
     return lib().dm05_suffix_attn(q, k_prefix, v_prefix, prefix_valid_len, prefix_mask, k_suffix,
                                   v_suffix, out, lse, B, Hq, Hkv, P, S, D, stream)
+
+
+def dm05_suffix_attn_noalloc(q, k_prefix, v_prefix, prefix_valid_len, prefix_mask, k_suffix, v_suffix,
+                             out, lse, B, Hq, Hkv, P, S, D, stream) -> int:
+    """The allocation-free entry point (for callers that must not allocate
+    device memory); same arguments as dm05_suffix_attn."""
+    return lib().dm05_suffix_attn_noalloc(q, k_prefix, v_prefix, prefix_valid_len, prefix_mask, k_suffix,
+                                          v_suffix, out, lse, B, Hq, Hkv, P, S, D, stream)
 
 
 def dm05_suffix_attn_workspace_bytes(B, Hq, Hkv, P, S, D) -> int:

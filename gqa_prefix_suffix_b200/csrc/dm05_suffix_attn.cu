@@ -287,6 +287,125 @@ int dm05_suffix_attn(const void *q, const void *k_prefix, const void *v_prefix, 
     return DM05_OK;
 }
 
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant.  Its scratch (the kernel's error word) lives in a
+// file-scope device array instead of a cudaMalloc'd workspace.  In host code
+// the array's name is only a host-side stand-in, never a device address: the
+// address the kernel gets comes from cudaGetSymbolAddress, looked up once per
+// device with that device current.
+namespace {
+static __device__ __align__(256) uint32_t g_noalloc_scratch[DM05_NOALLOC_SCRATCH_BYTES / sizeof(uint32_t)];
+std::vector<uint32_t *> g_noalloc_addr;  // per device ordinal: device address of g_noalloc_scratch
+
+// Caller holds g_mu.  Looks up (and on first use clears) this device's copy
+// of the scratch array.  Allocates nothing.
+int noalloc_scratch(cudaStream_t stream, uint32_t **out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return DM05_ERR_CUDA;
+    if (dev >= static_cast<int>(g_noalloc_addr.size())) g_noalloc_addr.resize(dev + 1, nullptr);
+    if (g_noalloc_addr[dev] == nullptr) {
+        cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+        if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) return DM05_ERR_CUDA;
+        if (cs != cudaStreamCaptureStatusNone) return DM05_ERR_WORKSPACE;
+        void *ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) return DM05_ERR_CUDA;
+        if (cudaMemset(ptr, 0, DM05_NOALLOC_SCRATCH_BYTES) != cudaSuccess) return DM05_ERR_CUDA;
+        g_noalloc_addr[dev] = static_cast<uint32_t *>(ptr);
+    }
+    *out = g_noalloc_addr[dev];
+    return DM05_OK;
+}
+}  // namespace
+
+extern "C" {
+
+int dm05_suffix_attn_noalloc(const void *q, const void *k_prefix, const void *v_prefix,
+                             const int32_t *prefix_valid_len, const uint8_t *prefix_mask, const void *k_suffix,
+                             const void *v_suffix, void *out, float *lse, int B, int Hq, int Hkv, int P, int S,
+                             int D, cudaStream_t stream)
+{
+    if (!q || !k_suffix || !v_suffix || !out) return DM05_ERR_NULL;
+    if (P > 0 && (!k_prefix || !v_prefix)) return DM05_ERR_NULL;
+    int rc = check_sizes(B, Hq, Hkv, P, S, D);
+    if (rc != DM05_OK) return rc;
+    if (!aligned16(q) || !aligned16(k_suffix) || !aligned16(v_suffix) || !aligned16(out) ||
+        (P > 0 && (!aligned16(k_prefix) || !aligned16(v_prefix))))
+        return DM05_ERR_ALIGN;
+    if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u) != 0) return DM05_ERR_ALIGN;
+    // scratch this call needs, against the fixed array
+    if (dm05_suffix_attn_workspace_bytes(B, Hq, Hkv, P, S, D) > DM05_NOALLOC_SCRATCH_BYTES) return DM05_ERR_WORKSPACE;
+
+    const int G = Hq / Hkv;
+    const int GS = G * S;
+    const int units = B * Hkv;
+    DeviceState *ds = nullptr;
+    uint32_t *scratch = nullptr;
+    int splits = 1;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (get_encoder() != DM05_OK) return DM05_ERR_CUDA;
+        rc = device_state(false, &ds);  // kernel attributes only; allocates nothing
+        if (rc != DM05_OK) return rc;
+        rc = noalloc_scratch(stream, &scratch);
+        if (rc != DM05_OK) return rc;
+        splits = choose_splits(B, Hkv, P, S, ds->num_sms, ds->max_cluster);
+        if (splits > ds->max_cluster) splits = ds->max_cluster;
+    }
+
+    CUtensorMap tm_q, tm_kp, tm_vp, tm_ks, tm_vs;
+    if (encode_3d(&tm_q, q, static_cast<uint64_t>(GS), static_cast<uint64_t>(units), dm05::kMRows) != DM05_OK ||
+        encode_3d(&tm_ks, k_suffix, static_cast<uint64_t>(S), static_cast<uint64_t>(units), kTileRows) != DM05_OK ||
+        encode_3d(&tm_vs, v_suffix, static_cast<uint64_t>(S), static_cast<uint64_t>(units), kTileRows) != DM05_OK)
+        return DM05_ERR_CUDA;
+    if (P > 0) {
+        if (encode_3d(&tm_kp, k_prefix, static_cast<uint64_t>(P), static_cast<uint64_t>(units), kTileRows) !=
+                DM05_OK ||
+            encode_3d(&tm_vp, v_prefix, static_cast<uint64_t>(P), static_cast<uint64_t>(units), kTileRows) != DM05_OK)
+            return DM05_ERR_CUDA;
+    } else {
+        tm_kp = tm_ks;
+        tm_vp = tm_vs;
+    }
+
+    dm05::KernelParams kp;
+    kp.valid_len = prefix_valid_len;
+    kp.mask = prefix_mask;
+    kp.out = static_cast<__nv_bfloat16 *>(out);
+    kp.lse = lse;
+    kp.err = scratch;
+    kp.Hkv = Hkv;
+    kp.P = P;
+    kp.S = S;
+    kp.GS = GS;
+    kp.splits = splits;
+    kp.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(units * splits), 1, 1);
+    cfg.blockDim = dim3(dm05::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = Layout::kAllocBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute at[2];
+    int na = 0;
+    at[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+    if (splits > 1) {
+        at[na].id = cudaLaunchAttributeClusterDimension;
+        at[na].val.clusterDim.x = static_cast<unsigned>(splits);
+        at[na].val.clusterDim.y = 1;
+        at[na].val.clusterDim.z = 1;
+        ++na;
+    }
+    cfg.attrs = at;
+    cfg.numAttrs = na;
+    if (cudaLaunchKernelEx(&cfg, kKernel, tm_q, tm_kp, tm_vp, tm_ks, tm_vs, kp) != cudaSuccess) return DM05_ERR_CUDA;
+    return DM05_OK;
+}
+
 int dm05_get_error_word(cudaStream_t stream, uint32_t *host_word)
 {
     if (!host_word) return DM05_ERR_NULL;

@@ -116,6 +116,45 @@ int dm05_suffix_attn_plan(int B, int Hq, int Hkv, int P, int S, int D,
  * and tests.  Returns DM05_ERR_SHAPE for any other value. */
 int dm05_set_split_override(int splits_per_head);
 
+/*
+ * dm05_suffix_attn_noalloc -- the same attention as dm05_suffix_attn, for
+ * callers that must not allocate device memory.  The source pages have no
+ * counterpart of this entry point; it exists for embedding.
+ *
+ * Who needs it: a process whose device memory is carved up in advance (a
+ * serving stack that reserves almost all of HBM for its KV cache, or an
+ * arena-only deployment where every byte is budgeted), and a real-time
+ * control loop that cannot afford cudaMalloc's implicit device
+ * synchronisation and unbounded latency.  Such a caller still passes every
+ * input and output; the one piece of scratch the kernel needs (its error
+ * word) lives in a fixed array of DM05_NOALLOC_SCRATCH_BYTES compiled into
+ * the library, which every GPU that loads the library holds until exit.
+ *
+ * Arguments, layouts, supported sizes and results are those of
+ * dm05_suffix_attn.  This entry point never calls cudaMalloc, cudaFree or any
+ * allocating routine.  It returns DM05_ERR_WORKSPACE for sizes whose scratch
+ * would not fit the fixed array (the current kernel needs one error word for
+ * any valid size, so valid sizes always fit).
+ *
+ * Set-up: the first call on each device looks up the array's device address
+ * and clears it (a synchronous cudaMemset), so make that first call before
+ * any stream capture on that device; a first call on a capturing stream
+ * returns DM05_ERR_WORKSPACE and does nothing.
+ *
+ * Sharing: every call on a device uses the same array and it keeps what the
+ * last call left there.  The kernel only ever sets time-out bits in it (they
+ * stay set; they are not visible through dm05_get_error_word), so results
+ * never depend on it; still, calls whose kernels overlap on the GPU race on
+ * that word.
+ */
+#define DM05_NOALLOC_SCRATCH_BYTES 256
+int dm05_suffix_attn_noalloc(const void *q, const void *k_prefix, const void *v_prefix,
+                             const int32_t *prefix_valid_len, const uint8_t *prefix_mask,
+                             const void *k_suffix, const void *v_suffix,
+                             void *out, float *lse,
+                             int B, int Hq, int Hkv, int P, int S, int D,
+                             cudaStream_t stream);
+
 /* Synchronises `stream`, then returns in *host_word the error bits
  * (DM05_EW_*) that kernels on the current device set since the last read,
  * and clears them. */

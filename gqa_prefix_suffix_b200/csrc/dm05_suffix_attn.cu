@@ -21,7 +21,8 @@ namespace {
 constexpr int kTileRows = 64;
 constexpr int kStages = 2;
 using Layout = dm05::SmemLayout<kTileRows, kStages>;
-constexpr size_t kWorkspaceBytes = 256;  // error word (padded to one 256-byte segment)
+constexpr size_t kErrBytes = 256;        // error word (padded to one 256-byte segment)
+constexpr size_t kPartRowBytes = dm05::kHeadDim * 4 + 16;  // one partial row: D fp32 of O + float4 stats
 constexpr int kMaxUnits = 1 << 24;       // B * Hkv
 constexpr int kMaxPrefix = 1 << 24;      // P
 
@@ -32,14 +33,31 @@ struct DeviceState {
     int max_cluster = 0;       // largest cluster size (power of two <= 16) that can be resident
 };
 
+// Partial-result workspace of one (device, stream): concurrent streams never
+// share one.
+struct StreamWorkspace {
+    int dev = -1;
+    cudaStream_t stream = nullptr;
+    void *base = nullptr;
+    size_t bytes = 0;
+};
+
 std::mutex g_mu;
 std::vector<DeviceState> g_dev;
+std::vector<StreamWorkspace> g_ws;
 int g_split_override = 0;
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
 auto *kKernel = &dm05::suffix_attn_kernel<kTileRows, kStages>;
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Bytes of partial results a call with `splits` CTAs per unit exchanges:
+// [units][splits][GS] rows of D fp32 followed by a float4 of statistics.
+size_t partial_bytes(long long units, int splits, int GS)
+{
+    return splits > 1 ? static_cast<size_t>(units) * splits * GS * kPartRowBytes : 0;
+}
 
 int check_sizes(int B, int Hq, int Hkv, int P, int S, int D)
 {
@@ -115,14 +133,50 @@ int device_state(bool allocate, DeviceState **out)
     }
     if (allocate && ds.err == nullptr) {
         void *p = nullptr;
-        if (cudaMalloc(&p, kWorkspaceBytes) != cudaSuccess) return DM05_ERR_CUDA;
-        if (cudaMemset(p, 0, kWorkspaceBytes) != cudaSuccess) {
+        if (cudaMalloc(&p, kErrBytes) != cudaSuccess) return DM05_ERR_CUDA;
+        if (cudaMemset(p, 0, kErrBytes) != cudaSuccess) {
             cudaFree(p);
             return DM05_ERR_CUDA;
         }
         ds.err = static_cast<uint32_t *>(p);
     }
     *out = &ds;
+    return DM05_OK;
+}
+
+// Workspace of (current device, stream) with at least `need` bytes.  Grows
+// only outside stream capture.  Caller holds g_mu.
+int stream_workspace(cudaStream_t stream, size_t need, void **out)
+{
+    *out = nullptr;
+    if (need == 0) return DM05_OK;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return DM05_ERR_CUDA;
+    StreamWorkspace *w = nullptr;
+    for (auto &e : g_ws)
+        if (e.dev == dev && e.stream == stream) w = &e;
+    if (w == nullptr) {
+        g_ws.push_back(StreamWorkspace{});
+        w = &g_ws.back();
+        w->dev = dev;
+        w->stream = stream;
+    }
+    if (w->bytes < need) {
+        cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+        if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) return DM05_ERR_CUDA;
+        if (cs != cudaStreamCaptureStatusNone) return DM05_ERR_WORKSPACE;
+        if (w->base != nullptr) {
+            // cudaFree waits for the device, so no kernel still uses the old buffer
+            cudaFree(w->base);
+            w->base = nullptr;
+            w->bytes = 0;
+        }
+        void *p = nullptr;
+        if (cudaMalloc(&p, need) != cudaSuccess) return DM05_ERR_CUDA;
+        w->base = p;
+        w->bytes = need;
+    }
+    *out = w->base;
     return DM05_OK;
 }
 
@@ -160,7 +214,9 @@ const char *dm05_status_string(int status)
 
 size_t dm05_suffix_attn_workspace_bytes(int B, int Hq, int Hkv, int P, int S, int D)
 {
-    return check_sizes(B, Hq, Hkv, P, S, D) == DM05_OK ? kWorkspaceBytes : 0;
+    if (check_sizes(B, Hq, Hkv, P, S, D) != DM05_OK) return 0;
+    // the largest split count the library ever uses is 16
+    return kErrBytes + partial_bytes(static_cast<long long>(B) * Hkv, 16, (Hq / Hkv) * S);
 }
 
 int dm05_set_split_override(int splits_per_head)
@@ -196,7 +252,11 @@ int dm05_suffix_attn_reserve(int B, int Hq, int Hkv, int P, int S, int D, cudaSt
     std::lock_guard<std::mutex> lk(g_mu);
     if (get_encoder() != DM05_OK) return DM05_ERR_CUDA;
     DeviceState *ds = nullptr;
-    return device_state(true, &ds);
+    rc = device_state(true, &ds);
+    if (rc != DM05_OK) return rc;
+    const int splits = choose_splits(B, Hkv, P, S, ds->num_sms, ds->max_cluster);
+    void *ws = nullptr;
+    return stream_workspace(stream, partial_bytes(static_cast<long long>(B) * Hkv, splits, (Hq / Hkv) * S), &ws);
 }
 
 int dm05_suffix_attn(const void *q, const void *k_prefix, const void *v_prefix, const int32_t *prefix_valid_len,
@@ -219,6 +279,7 @@ int dm05_suffix_attn(const void *q, const void *k_prefix, const void *v_prefix, 
 
     DeviceState *ds = nullptr;
     int splits = 1;
+    void *part_ws = nullptr;
     {
         std::lock_guard<std::mutex> lk(g_mu);
         if (get_encoder() != DM05_OK) return DM05_ERR_CUDA;
@@ -233,6 +294,8 @@ int dm05_suffix_attn(const void *q, const void *k_prefix, const void *v_prefix, 
         }
         splits = choose_splits(B, Hkv, P, S, ds->num_sms, ds->max_cluster);
         if (splits > ds->max_cluster) splits = ds->max_cluster;
+        rc = stream_workspace(stream, partial_bytes(units, splits, GS), &part_ws);
+        if (rc != DM05_OK) return rc;
     }
 
     // ---- TMA descriptors (the tensor maps travel as kernel parameters)
@@ -257,6 +320,7 @@ int dm05_suffix_attn(const void *q, const void *k_prefix, const void *v_prefix, 
     kp.out = static_cast<__nv_bfloat16 *>(out);
     kp.lse = lse;
     kp.err = ds->err;
+    kp.part = static_cast<float *>(part_ws);
     kp.Hkv = Hkv;
     kp.P = P;
     kp.S = S;
@@ -296,6 +360,7 @@ int dm05_suffix_attn(const void *q, const void *k_prefix, const void *v_prefix, 
 // address the kernel gets comes from cudaGetSymbolAddress, looked up once per
 // device with that device current.
 namespace {
+// [error word: kErrBytes][partial results: the rest]
 static __device__ __align__(256) uint32_t g_noalloc_scratch[DM05_NOALLOC_SCRATCH_BYTES / sizeof(uint32_t)];
 std::vector<uint32_t *> g_noalloc_addr;  // per device ordinal: device address of g_noalloc_scratch
 
@@ -312,7 +377,7 @@ int noalloc_scratch(cudaStream_t stream, uint32_t **out)
         if (cs != cudaStreamCaptureStatusNone) return DM05_ERR_WORKSPACE;
         void *ptr = nullptr;
         if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) return DM05_ERR_CUDA;
-        if (cudaMemset(ptr, 0, DM05_NOALLOC_SCRATCH_BYTES) != cudaSuccess) return DM05_ERR_CUDA;
+        if (cudaMemset(ptr, 0, kErrBytes) != cudaSuccess) return DM05_ERR_CUDA;  // the error word starts at zero
         g_noalloc_addr[dev] = static_cast<uint32_t *>(ptr);
     }
     *out = g_noalloc_addr[dev];
@@ -335,8 +400,8 @@ int dm05_suffix_attn_noalloc(const void *q, const void *k_prefix, const void *v_
         (P > 0 && (!aligned16(k_prefix) || !aligned16(v_prefix))))
         return DM05_ERR_ALIGN;
     if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u) != 0) return DM05_ERR_ALIGN;
-    // scratch this call needs, against the fixed array
-    if (dm05_suffix_attn_workspace_bytes(B, Hq, Hkv, P, S, D) > DM05_NOALLOC_SCRATCH_BYTES) return DM05_ERR_WORKSPACE;
+    // the error word must fit the fixed array (the partials are sized below)
+    if (kErrBytes > DM05_NOALLOC_SCRATCH_BYTES) return DM05_ERR_WORKSPACE;
 
     const int G = Hq / Hkv;
     const int GS = G * S;
@@ -353,6 +418,8 @@ int dm05_suffix_attn_noalloc(const void *q, const void *k_prefix, const void *v_
         if (rc != DM05_OK) return rc;
         splits = choose_splits(B, Hkv, P, S, ds->num_sms, ds->max_cluster);
         if (splits > ds->max_cluster) splits = ds->max_cluster;
+        // fewer CTAs per unit until the partial results fit the fixed array
+        while (splits > 1 && partial_bytes(units, splits, GS) > DM05_NOALLOC_SCRATCH_BYTES - kErrBytes) splits /= 2;
     }
 
     CUtensorMap tm_q, tm_kp, tm_vp, tm_ks, tm_vs;
@@ -376,6 +443,7 @@ int dm05_suffix_attn_noalloc(const void *q, const void *k_prefix, const void *v_
     kp.out = static_cast<__nv_bfloat16 *>(out);
     kp.lse = lse;
     kp.err = scratch;
+    kp.part = splits > 1 ? reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(scratch) + kErrBytes) : nullptr;
     kp.Hkv = Hkv;
     kp.P = P;
     kp.S = S;
@@ -437,6 +505,10 @@ void dm05_release(void)
             g_dev[d].err = nullptr;
         }
     }
+    for (auto &w : g_ws) {
+        if (w.base != nullptr && cudaSetDevice(w.dev) == cudaSuccess) cudaFree(w.base);
+    }
+    g_ws.clear();
     if (have_cur) cudaSetDevice(cur);
 }
 

@@ -27,12 +27,14 @@
 //   * The running max is updated lazily: O and l are rescaled only when the
 //     tile max exceeds the current max by more than 2^8 (exact: O and l use
 //     the same stale max, and p <= 2^8 stays well inside fp32/bf16 range).
-//   * Splits of one unit form a thread-block cluster.  At the end every CTA
-//     scales its O by exp2(m_self - M) / L (M, L from the cluster's stats via
-//     distributed shared memory), stages it in its own shared memory, and
-//     each CTA sums one column slice over the cluster and writes bf16 output:
-//     the split-KV merge happens on chip, with no workspace and no second
-//     kernel.
+//   * Splits of one unit form a thread-block cluster (the hardware barrier
+//     that orders the merge, and a guarantee that all splits are resident).
+//     Each CTA publishes its unnormalised partial O with its per-row
+//     (m, l, l_hat) to a workspace in L2 (one 1040-byte bulk TMA store per
+//     row); after one cluster barrier CTA r loads rows [r*GS/C, (r+1)*GS/C)
+//     of every partial with one bulk copy per partial and combines them by
+//     the log-sum-exp rule.  (Distributed shared memory was measured at ~10 GB/s per SM for
+//     this traffic, L2 through the TMA engine several times faster.)
 //   * Every wait is bounded (2 s): on time-out the kernel records
 //     DM05_EW_WAIT_TIMEOUT in the error word, drains its own copies and MMAs
 //     (again bounded), frees TMEM and returns.
@@ -69,6 +71,7 @@ struct KernelParams {
     __nv_bfloat16 *out;        // [B*Hkv, GS, D]
     float *lse;                // [B*Hkv, GS] or nullptr
     uint32_t *err;             // device error word
+    float *part;               // splits > 1: partial rows [units][splits][GS], each D fp32 + {m, l, l_hat, 0}
     int Hkv, P, S, GS;         // GS = (Hq / Hkv) * S query rows of a unit
     int splits;                // CTAs per unit (cluster size)
     float scale_log2;          // log2(e) / sqrt(D)
@@ -96,14 +99,21 @@ struct SmemLayout {
     static constexpr int kBarPFree = kBarPReady + kSBufs;    // per S/P buffer
     static constexpr int kBarODone = kBarPFree + kSBufs;
     static constexpr int kBarMmaFinal = kBarODone + 1;
-    static constexpr int kNumBars = kBarMmaFinal + 1;
+    static constexpr int kBarMerge = kBarMmaFinal + 1;
+    static constexpr int kNumBars = kBarMerge + 1;
     static constexpr int kBarOff = kDataEnd;
     static constexpr int kTmemSlotOff = kBarOff + kNumBars * 8;
-    static constexpr int kStatOff = (kTmemSlotOff + 16 + 15) / 16 * 16;  // m, l, l_hat [128] each
-    static constexpr int kEnd = kStatOff + 3 * kMRows * 4;
+    // merge: weights of the rows this CTA reduces (at most
+    // splits * ceil(GS / splits) <= kMRows + 16 entries)
+    static constexpr int kMergeEntries = kMRows + 16;
+    static constexpr int kMergeWOff = (kTmemSlotOff + 16 + 15) / 16 * 16;
+    static constexpr int kEnd = kMergeWOff + kMergeEntries * 4;
     static constexpr int kAllocBytes = kEnd + 1024;                  // slack for 1 KB alignment
-    // The cluster merge stages G*S rows x 1 KB of fp32 in the data region.
-    static_assert(kDataEnd >= kMRows * kHeadDim * 4, "staging area must fit in the data region");
+    // The merge stages up to 128 rows at kStageStride bytes, then receives
+    // at most (128 + 16) rows of 1 KB, both inside the data region.
+    static constexpr int kStageStride = kHeadDim * 4 + 16;           // padded: conflict-free row writes
+    static_assert(kDataEnd >= kMRows * kStageStride, "staging area must fit in the data region");
+    static_assert(kDataEnd >= kMergeEntries * kStageStride, "receive area must fit in the data region");
 };
 
 struct TileInfo {
@@ -147,6 +157,38 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi, float &sum_r
     return *reinterpret_cast<uint32_t *>(&h);
 }
 
+// out[rr][:] = bf16( sum_c w[c][rr] * recv[c][rr][:] ) for the nr rows a CTA
+// merges; the C partial rows are kStageStride bytes apart in shared memory.
+template <int C, class L>
+__device__ __forceinline__ void merge_rows(const uint8_t *recv, const float *mw, int nr, __nv_bfloat16 *out)
+{
+    const int items = nr * (kHeadDim / 4);
+    for (int i = threadIdx.x; i < items; i += kThreads) {
+        const int rr = i / (kHeadDim / 4), ch = i - rr * (kHeadDim / 4);
+        float w[C];
+        float4 v[C];
+#pragma unroll
+        for (int c = 0; c < C; ++c) {
+            w[c] = mw[c * nr + rr];
+            v[c] = *reinterpret_cast<const float4 *>(recv + (c * nr + rr) * L::kStageStride + ch * 16);
+        }
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int c = 0; c < C; ++c) {
+            if (w[c] != 0.0f) {  // a partial without visible keys holds no valid O
+                acc.x += w[c] * v[c].x;
+                acc.y += w[c] * v[c].y;
+                acc.z += w[c] * v[c].z;
+                acc.w += w[c] * v[c].w;
+            }
+        }
+        __nv_bfloat162 h0 = __floats2bfloat162_rn(acc.x, acc.y);
+        __nv_bfloat162 h1 = __floats2bfloat162_rn(acc.z, acc.w);
+        *reinterpret_cast<uint2 *>(out + static_cast<size_t>(rr) * kHeadDim + ch * 4) =
+            make_uint2(*reinterpret_cast<uint32_t *>(&h0), *reinterpret_cast<uint32_t *>(&h1));
+    }
+}
+
 template <int NT, int STAGES>
 __global__ void __launch_bounds__(kThreads, 1)
     suffix_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kp,
@@ -158,9 +200,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kBarOff);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kTmemSlotOff);
-    float *stat_m = reinterpret_cast<float *>(smem + L::kStatOff);
-    float *stat_l = stat_m + kMRows;
-    float *stat_lh = stat_l + kMRows;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -185,6 +224,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         ptx::mbar_init(&bars[L::kBarODone], 1);
         ptx::mbar_init(&bars[L::kBarMmaFinal], 1);
+        ptx::mbar_init(&bars[L::kBarMerge], 1);
         ptx::fence_mbar_init();
     }
     if (warp == kProducerWarp && lane == 0) {
@@ -207,6 +247,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---- from here on inputs are read: wait for the preceding grid
     ptx::griddep_wait();
 
+    uint8_t *sQ = smem + L::kQOff;
+    uint8_t *sK = smem + L::kKOff;
+    uint8_t *sV = smem + L::kVOff;
+    if (warp == kProducerWarp && lane == 0) {
+        // Q does not depend on valid_len: start it before that read.
+        ptx::mbar_arrive_expect_tx(&bars[L::kBarQFull], L::kQBytes);
+        for (int c = 0; c < kChunks; ++c)
+            ptx::tma_load_3d(sQ + c * L::kQChunkBytes, &tm_q, &bars[L::kBarQFull], c * kChunkElems, 0, unit);
+    }
+
     int vl = p.P;
     if (p.valid_len != nullptr) {
         const int raw = __ldg(p.valid_len + b);
@@ -220,18 +270,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int t_end = static_cast<int>((static_cast<long long>(t_all) * (rank + 1)) / C);
     const int T = t_end - t_begin;
 
-    uint8_t *sQ = smem + L::kQOff;
-    uint8_t *sK = smem + L::kKOff;
-    uint8_t *sV = smem + L::kVOff;
     bool failed = false;
 
     if (warp == kProducerWarp) {
         // ================================================== TMA producer
-        if (lane == 0 && T > 0) {
+        if (lane == 0) {
             const uint64_t pol = ptx::policy_evict_first();
-            ptx::mbar_arrive_expect_tx(&bars[L::kBarQFull], L::kQBytes);
-            for (int c = 0; c < kChunks; ++c)
-                ptx::tma_load_3d(sQ + c * L::kQChunkBytes, &tm_q, &bars[L::kBarQFull], c * kChunkElems, 0, unit);
             int k_issued = 0, v_issued = 0;
             for (int t = 0; t < T && !failed; ++t) {
                 const int s = t % STAGES, n = t / STAGES;
@@ -268,7 +312,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == kMmaWarp) {
         // ================================================== MMA issuer
         if (lane == 0 && T > 0) {
-            constexpr uint32_t idesc_qk = ptx::idesc_bf16_f32(kMRows, NT, false);
             constexpr uint32_t idesc_pv = ptx::idesc_bf16_f32(kMRows, kHeadDim, true);
             const uint32_t q_base = ptx::smem_addr(sQ);
             const uint32_t k_base = ptx::smem_addr(sK);
@@ -281,8 +324,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ptx::tc_fence_after_sync();
                 const uint32_t vb = v_base + s * L::kTileBytes;
                 const uint32_t p_tmem = tmem + kTmemS + pb * NT;
+                // only the 16-row k-steps that hold valid keys (a partial tile
+                // stops early; the rows after its last valid key up to the
+                // k-step end are zero)
+                const int nk = (tile_of<NT>(t_begin + u, TP, vl, p.S).n_valid + 15) / 16;
 #pragma unroll
                 for (int kk = 0; kk < NT / 16; ++kk) {
+                    if (kk >= nk) break;
                     // B = V rows [16kk, 16kk+16) of the tile, all 256 columns:
                     // 128-byte rows (16 B units), column chunks LBO apart,
                     // 8-row groups SBO apart.
@@ -313,6 +361,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ptx::tc_fence_after_sync();
                 const uint32_t kb = k_base + s * L::kTileBytes;
                 const uint32_t d = tmem + kTmemS + sb * NT;
+                // N = the valid keys of the tile rounded up to 16; the
+                // softmax masks every column past the valid ones anyway.
+                const int nv16 = (tile_of<NT>(t_begin + t, TP, vl, p.S).n_valid + 15) / 16 * 16;
+                const uint32_t idesc_qk = ptx::idesc_bf16_f32(kMRows, nv16, false);
 #pragma unroll
                 for (int kk = 0; kk < kHeadDim / 16; ++kk) {
                     // K-major, 128-byte swizzle: 16 elements = 32 bytes along
@@ -423,16 +475,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             ptx::tmem_st_wait();
-            if (ti.prefix && ti.n_valid < NT) {
+            if (ti.prefix && (ti.n_valid & 15) != 0) {
                 // Rows at or past valid_len may hold anything (NaN too) and
-                // would poison O through 0 * NaN: clear them in the V tile.
+                // would poison O through 0 * NaN: clear the ones the last PV
+                // k-step reads.
                 const int st = t % STAGES;
                 if (!warp_wait(&bars[L::kBarVFull + st], (t / STAGES) & 1)) {
                     failed = true;
                     break;
                 }
                 uint8_t *vt = sV + st * L::kTileBytes;
-                const int rows = NT - ti.n_valid;
+                const int rows = (ti.n_valid + 15) / 16 * 16 - ti.n_valid;  // read by the last PV k-step
                 const int units = kChunks * rows * 8;  // 16-byte units
                 for (int i = row; i < units; i += kSoftmaxWarps * 32) {
                     const int c = i / (rows * 8);
@@ -476,98 +529,96 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (row < p.GS && p.lse != nullptr) p.lse[out_row] = (m_used + ptx::lg2(l)) * 0.69314718055994531f;
         } else {
-            stat_m[row] = m_used;
-            stat_l[row] = l;
-            stat_lh[row] = lh;
+            // ---------------------------------------- split: publish this CTA's partial
+            // Row `row` of the partial: D fp32 of unnormalised O, then
+            // {m, l, l_hat, 0}; one bulk TMA store per thread.
+            const size_t prow = (static_cast<size_t>(unit) * C + rank) * p.GS + row;
+            uint8_t *srow = smem + row * L::kStageStride;
+            const bool write_o = T > 0 && !failed;
+            if (write_o) {
+#pragma unroll 1
+                for (int j = 0; j < kHeadDim / 64; ++j) {
+                    uint32_t o[4][16];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) ptx::tmem_ld16(tmem + lane_base + kTmemO + j * 64 + q * 16, o[q]);
+                    ptx::tmem_ld_wait();
+                    if (row < p.GS) {
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            uint4 *d = reinterpret_cast<uint4 *>(srow + (j * 64 + q * 16) * 4);
+                            d[0] = make_uint4(o[q][0], o[q][1], o[q][2], o[q][3]);
+                            d[1] = make_uint4(o[q][4], o[q][5], o[q][6], o[q][7]);
+                            d[2] = make_uint4(o[q][8], o[q][9], o[q][10], o[q][11]);
+                            d[3] = make_uint4(o[q][12], o[q][13], o[q][14], o[q][15]);
+                        }
+                    }
+                }
+            }
+            if (row < p.GS) {
+                *reinterpret_cast<float4 *>(srow + kHeadDim * 4) = make_float4(m_used, l, write_o ? lh : 0.0f, 0.0f);
+                ptx::fence_proxy_async_smem();
+                ptx::bulk_store_s2g(reinterpret_cast<uint8_t *>(p.part) + prow * L::kStageStride, ptx::smem_addr(srow),
+                                    L::kStageStride);
+                ptx::bulk_commit();
+                ptx::bulk_wait_all();
+                ptx::fence_proxy_async_global();
+            }
         }
     }
 
     __syncwarp();
     if (C > 1) {
-        // ================================================== on-chip split merge
-        ptx::cluster_sync();  // stats of every CTA published
-        float4 *stage = reinterpret_cast<float4 *>(smem);  // [128 rows][64 chunks], chunk index swizzled
-        float lse_row = 0.0f;
-        if (warp < kSoftmaxWarps) {
-            const int row = warp * 32 + lane;
-            const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-            const float m_self = stat_m[row], lh_self = stat_lh[row];
-            float mr[16], lr[16], lhr[16];
-            float M = -INFINITY;
-#pragma unroll
-            for (int r = 0; r < 16; ++r) {
-                if (r < C) {
-                    mr[r] = ptx::ld_dsmem_f32(ptx::mapa(ptx::smem_addr(&stat_m[row]), r));
-                    lr[r] = ptx::ld_dsmem_f32(ptx::mapa(ptx::smem_addr(&stat_l[row]), r));
-                    lhr[r] = ptx::ld_dsmem_f32(ptx::mapa(ptx::smem_addr(&stat_lh[row]), r));
-                    M = fmaxf(M, mr[r]);
-                }
-            }
-            float Lsum = 0.0f, LHsum = 0.0f;
-#pragma unroll
-            for (int r = 0; r < 16; ++r) {
-                if (r < C && lhr[r] > 0.0f) {
-                    const float f = ptx::ex2(mr[r] - M);
-                    Lsum += lr[r] * f;
-                    LHsum += lhr[r] * f;
-                }
-            }
-            const float wgt = (lh_self > 0.0f) ? ptx::ex2(m_self - M) / LHsum : 0.0f;
-            lse_row = (M + ptx::lg2(Lsum)) * 0.69314718055994531f;
-            ptx::fence_proxy_async_smem();
-            const bool read_o = T > 0 && !failed && wgt != 0.0f;
-#pragma unroll 1
-            for (int j = 0; j < kHeadDim / 16; ++j) {
-                uint32_t o[16];
-                if (__any_sync(0xffffffffu, read_o)) {
-                    ptx::tmem_ld16(tmem + lane_base + kTmemO + j * 16, o);
-                    ptx::tmem_ld_wait();
-                }
-                if (row < p.GS) {
-#pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
-                        const int c = j * 4 + q4;
-                        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-                        if (read_o) {
-                            v.x = __uint_as_float(o[4 * q4 + 0]) * wgt;
-                            v.y = __uint_as_float(o[4 * q4 + 1]) * wgt;
-                            v.z = __uint_as_float(o[4 * q4 + 2]) * wgt;
-                            v.w = __uint_as_float(o[4 * q4 + 3]) * wgt;
-                        }
-                        stage[row * 64 + (c ^ (row & 7))] = v;
-                    }
-                }
+        // ================================================== split merge (rows)
+        // Every CTA of the unit has published its partial; CTA `rank` now
+        // combines rows [r_lo, r_hi) of all C partials:
+        //   M = max_c m_c,  LH = sum_c lh_c 2^(m_c - M),  L = sum_c l_c 2^(m_c - M)
+        //   out = sum_c 2^(m_c - M) O_c / LH,   lse = (M + log2 L) ln 2.
+        ptx::cluster_sync();
+        const int r_lo = (p.GS * rank) / C;
+        const int r_hi = (p.GS * (rank + 1)) / C;
+        const int nr = r_hi - r_lo;
+        const uint8_t *recv = smem;  // [C][nr] rows of kStageStride bytes
+        float *mw = reinterpret_cast<float *>(smem + L::kMergeWOff);  // [C][nr] weights
+        if (nr > 0 && warp == 0) {
+            if (lane == 0) ptx::mbar_arrive_expect_tx(&bars[L::kBarMerge], static_cast<uint32_t>(C * nr * L::kStageStride));
+            __syncwarp();
+            if (lane < C) {
+                ptx::fence_proxy_async_global();
+                ptx::bulk_load_g2s(ptx::smem_addr(smem) + static_cast<uint32_t>(lane * nr * L::kStageStride),
+                                   reinterpret_cast<const uint8_t *>(p.part) +
+                                       ((static_cast<size_t>(unit) * C + lane) * p.GS + r_lo) * L::kStageStride,
+                                   static_cast<uint32_t>(nr * L::kStageStride), &bars[L::kBarMerge]);
             }
         }
-        ptx::cluster_sync();  // every CTA's scaled O staged
-        {
-            const int per = 64 / C;  // 16-byte column chunks owned by this CTA
-            const int c_lo = rank * per;
-            const int items = p.GS * per;
-            const uint32_t stage_base = ptx::smem_addr(stage);
-            for (int i = threadIdx.x; i < items; i += kThreads) {
-                const int r = i / per;
-                const int c = c_lo + (i - r * per);
-                const uint32_t off = stage_base + static_cast<uint32_t>((r * 64 + (c ^ (r & 7))) * 16);
-                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-                for (int src = 0; src < C; ++src) {
-                    const float4 v = ptx::ld_dsmem_f32x4(ptx::mapa(off, src));
-                    acc.x += v.x;
-                    acc.y += v.y;
-                    acc.z += v.z;
-                    acc.w += v.w;
+        if (nr > 0) {
+            if (!warp_wait(&bars[L::kBarMerge], 0)) failed = true;
+            // weights: one warp per row, lane c holds partial c
+            for (int rr = warp; rr < nr; rr += kThreads / 32) {
+                float4 st = make_float4(-INFINITY, 0.f, 0.f, 0.f);
+                if (lane < C) st = *reinterpret_cast<const float4 *>(recv + (lane * nr + rr) * L::kStageStride + kHeadDim * 4);
+                const bool has = lane < C && st.z > 0.0f;
+                float M = has ? st.x : -INFINITY;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+                const float f = has ? ptx::ex2(st.x - M) : 0.0f;
+                float Ls = st.y * f, LHs = st.z * f;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    Ls += __shfl_xor_sync(0xffffffffu, Ls, o);
+                    LHs += __shfl_xor_sync(0xffffffffu, LHs, o);
                 }
-                __nv_bfloat162 h0 = __floats2bfloat162_rn(acc.x, acc.y);
-                __nv_bfloat162 h1 = __floats2bfloat162_rn(acc.z, acc.w);
-                uint2 w2 = make_uint2(*reinterpret_cast<uint32_t *>(&h0), *reinterpret_cast<uint32_t *>(&h1));
-                *reinterpret_cast<uint2 *>(p.out + (static_cast<size_t>(unit) * p.GS + r) * kHeadDim + c * 4) = w2;
+                if (lane < C) mw[lane * nr + rr] = f / LHs;
+                if (lane == 0 && p.lse != nullptr)
+                    p.lse[static_cast<size_t>(unit) * p.GS + r_lo + rr] = (M + ptx::lg2(Ls)) * 0.69314718055994531f;
+            }
+            __syncthreads();
+            switch (C) {
+            case 2: merge_rows<2, L>(recv, mw, nr, p.out + (static_cast<size_t>(unit) * p.GS + r_lo) * kHeadDim); break;
+            case 4: merge_rows<4, L>(recv, mw, nr, p.out + (static_cast<size_t>(unit) * p.GS + r_lo) * kHeadDim); break;
+            case 8: merge_rows<8, L>(recv, mw, nr, p.out + (static_cast<size_t>(unit) * p.GS + r_lo) * kHeadDim); break;
+            default: merge_rows<16, L>(recv, mw, nr, p.out + (static_cast<size_t>(unit) * p.GS + r_lo) * kHeadDim); break;
             }
         }
-        if (warp < kSoftmaxWarps && rank == 0 && p.lse != nullptr) {
-            const int row = warp * 32 + lane;
-            if (row < p.GS) p.lse[static_cast<size_t>(unit) * p.GS + row] = lse_row;
-        }
-        ptx::cluster_sync();  // no CTA leaves while a peer may still read its shared memory
     }
 
     if (failed) atomicOr(p.err, kEwTimeout);

@@ -26,10 +26,11 @@
  * device that is current on the calling thread.
  *
  * Ownership: the caller owns every tensor.  The library keeps no pointer
- * after a call returns.  The library owns one small device workspace per
- * device (an error word); it is created by dm05_suffix_attn_reserve or by the
- * first dm05_suffix_attn on the device that runs outside stream capture, and
- * freed by dm05_release.
+ * after a call returns.  The library owns an error word per device and, per
+ * (device, stream), a workspace for the partial results of split calls (at
+ * most dm05_suffix_attn_workspace_bytes).  They are created by
+ * dm05_suffix_attn_reserve or by a dm05_suffix_attn that runs outside stream
+ * capture, grow only outside capture, and are freed by dm05_release.
  *
  * Errors: every entry point returns a dm05_status.  Arguments are checked on
  * the host before anything is launched; a failed check launches nothing.
@@ -96,13 +97,15 @@ int dm05_suffix_attn(const void *q, const void *k_prefix, const void *v_prefix,
                      int B, int Hq, int Hkv, int P, int S, int D,
                      cudaStream_t stream);
 
-/* Bytes of device workspace dm05_suffix_attn needs for these sizes (the
- * per-device error word).  0 if the sizes are invalid. */
+/* Upper bound of the device workspace dm05_suffix_attn uses for these sizes:
+ * the error word plus the partial results of the largest split (16 CTAs per
+ * (sample, KV head)).  0 if the sizes are invalid. */
 size_t dm05_suffix_attn_workspace_bytes(int B, int Hq, int Hkv, int P, int S, int D);
 
-/* Creates the workspace of the current device for these sizes, and sets the
- * kernel attributes, outside any stream capture.  Call it before capturing
- * dm05_suffix_attn into a CUDA graph.  `stream` must not be capturing. */
+/* Creates the workspace of (current device, `stream`) for these sizes and
+ * sets the kernel attributes, outside any stream capture.  Call it before
+ * capturing dm05_suffix_attn on `stream` into a CUDA graph.  `stream` must not
+ * be capturing. */
 int dm05_suffix_attn_reserve(int B, int Hq, int Hkv, int P, int S, int D, cudaStream_t stream);
 
 /* Work decomposition the next call with these sizes will use: the number of
@@ -126,15 +129,17 @@ int dm05_set_split_override(int splits_per_head);
  * arena-only deployment where every byte is budgeted), and a real-time
  * control loop that cannot afford cudaMalloc's implicit device
  * synchronisation and unbounded latency.  Such a caller still passes every
- * input and output; the one piece of scratch the kernel needs (its error
- * word) lives in a fixed array of DM05_NOALLOC_SCRATCH_BYTES compiled into
- * the library, which every GPU that loads the library holds until exit.
+ * input and output; the kernel's scratch (its error word and the partial
+ * results of split calls) lives in a fixed array of
+ * DM05_NOALLOC_SCRATCH_BYTES compiled into the library, which every GPU that
+ * loads the library holds until exit.
  *
  * Arguments, layouts, supported sizes and results are those of
  * dm05_suffix_attn.  This entry point never calls cudaMalloc, cudaFree or any
- * allocating routine.  It returns DM05_ERR_WORKSPACE for sizes whose scratch
- * would not fit the fixed array (the current kernel needs one error word for
- * any valid size, so valid sizes always fit).
+ * allocating routine.  When the automatic split would need more partial
+ * scratch than the array holds, the call splits each (sample, KV head) over
+ * fewer CTAs (down to one, which needs none), so valid sizes always fit;
+ * DM05_ERR_WORKSPACE is returned only if the error word itself did not fit.
  *
  * Set-up: the first call on each device looks up the array's device address
  * and clears it (a synchronous cudaMemset), so make that first call before
@@ -142,12 +147,13 @@ int dm05_set_split_override(int splits_per_head);
  * returns DM05_ERR_WORKSPACE and does nothing.
  *
  * Sharing: every call on a device uses the same array and it keeps what the
- * last call left there.  The kernel only ever sets time-out bits in it (they
- * stay set; they are not visible through dm05_get_error_word), so results
- * never depend on it; still, calls whose kernels overlap on the GPU race on
- * that word.
+ * last call left there.  A call writes all the partial results it later reads,
+ * and the error word only collects time-out bits (they stay set and are not
+ * visible through dm05_get_error_word).  Calls whose kernels overlap on the
+ * GPU (for example on two streams) race on the array and may corrupt each
+ * other's results: serialise them.
  */
-#define DM05_NOALLOC_SCRATCH_BYTES 256
+#define DM05_NOALLOC_SCRATCH_BYTES (8u << 20)
 int dm05_suffix_attn_noalloc(const void *q, const void *k_prefix, const void *v_prefix,
                              const int32_t *prefix_valid_len, const uint8_t *prefix_mask,
                              const void *k_suffix, const void *v_suffix,

@@ -15,13 +15,15 @@
 //     then the S suffix rows.  The CTAs of one unit split that list evenly
 //     (the split depends on valid_len, read on the device, so a captured
 //     graph stays valid for any valid_len).
-//   * Warp roles: warp 4 issues TMA loads (Q once, then a ring of K and V
-//     tiles); warp 5 allocates TMEM and issues tcgen05 MMAs from one thread;
-//     warps 0-3 (one thread per query row = TMEM lane) run the softmax.
-//   * S = Q K^T goes to TMEM (three rotating buffers).  The softmax thread of
-//     row i reads its row with tcgen05.ld, applies the mask and the scale,
-//     keeps a running max m and sum l, and writes P (bf16) back into the same
-//     TMEM columns.  O += P V is a tcgen05 MMA with A = P read from TMEM and B
+//   * Warp roles: warp 8 issues TMA loads (Q once, then a ring of K and V
+//     tiles); warp 9 allocates TMEM and issues tcgen05 MMAs from one thread;
+//     warps 0-7 run the softmax: warps w and w+4 share TMEM lane quarter w
+//     (32 query rows) and each takes half of every tile's columns.
+//   * S = Q K^T goes to TMEM (three rotating buffers).  Each softmax thread
+//     reads half of its row with tcgen05.ld, applies the mask and the scale,
+//     combines its half's maximum with the partner warp's (shared memory and
+//     a bounded pair barrier), keeps the running max m and its half of the
+//     sums, and writes P (bf16) back into the same TMEM columns.  O += P V is a tcgen05 MMA with A = P read from TMEM and B
 //     = the V tile in shared memory (MN-major).  O (128 x 256 fp32) lives in
 //     TMEM for the whole pass.
 //   * The running max is updated lazily: O and l are rescaled only when the
@@ -52,10 +54,10 @@ constexpr int kHeadDim = 256;
 constexpr int kMRows = 128;                       // MMA M: query rows (padded)
 constexpr int kChunkElems = 64;                   // bf16 per 128-byte swizzle row
 constexpr int kChunks = kHeadDim / kChunkElems;   // 4 column chunks of a row
-constexpr int kSoftmaxWarps = 4;
-constexpr int kProducerWarp = 4;
-constexpr int kMmaWarp = 5;
-constexpr int kThreads = 192;
+constexpr int kSoftmaxWarps = 8;   // 2 per TMEM lane quarter: rows x column halves
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kThreads = 320;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemO = 0;                    // O: columns [0, 256)
 constexpr uint32_t kTmemS = 256;                  // S/P buffers: [256, 256 + kSBufs*NT)
@@ -100,14 +102,17 @@ struct SmemLayout {
     static constexpr int kBarODone = kBarPFree + kSBufs;
     static constexpr int kBarMmaFinal = kBarODone + 1;
     static constexpr int kBarMerge = kBarMmaFinal + 1;
-    static constexpr int kNumBars = kBarMerge + 1;
+    static constexpr int kBarPair = kBarMerge + 1;          // per TMEM lane quarter: its 2 softmax warps
+    static constexpr int kNumBars = kBarPair + 4;
     static constexpr int kBarOff = kDataEnd;
     static constexpr int kTmemSlotOff = kBarOff + kNumBars * 8;
     // merge: weights of the rows this CTA reduces (at most
     // splits * ceil(GS / splits) <= kMRows + 16 entries)
     static constexpr int kMergeEntries = kMRows + 16;
     static constexpr int kMergeWOff = (kTmemSlotOff + 16 + 15) / 16 * 16;
-    static constexpr int kEnd = kMergeWOff + kMergeEntries * 4;
+    // softmax half exchange: row maxima [2][2][128], sums [2][128] x 2
+    static constexpr int kXchgOff = kMergeWOff + kMergeEntries * 4;
+    static constexpr int kEnd = kXchgOff + (4 + 2 + 2) * kMRows * 4;
     static constexpr int kAllocBytes = kEnd + 1024;                  // slack for 1 KB alignment
     // The merge stages up to 128 rows at kStageStride bytes, then receives
     // at most (128 + 16) rows of 1 KB, both inside the data region.
@@ -225,6 +230,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::mbar_init(&bars[L::kBarODone], 1);
         ptx::mbar_init(&bars[L::kBarMmaFinal], 1);
         ptx::mbar_init(&bars[L::kBarMerge], 1);
+        for (int i = 0; i < 4; ++i) ptx::mbar_init(&bars[L::kBarPair + i], 64);
         ptx::fence_mbar_init();
     }
     if (warp == kProducerWarp && lane == 0) {
@@ -389,12 +395,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ================================================== softmax warps
-        const int row = warp * 32 + lane;
-        const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+        // Warp w owns TMEM lanes 32*(w%4).. (its 32 query rows) and half
+        // hf = w/4 of every S tile's columns and of O's columns; the two
+        // warps of a lane quarter exchange their row maxima and sums.
+        const int q4 = warp & 3;
+        const int hf = warp >> 2;
+        const int row = q4 * 32 + lane;
+        const int tid = hf * 128 + row;  // 0..255 over the softmax threads
+        const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
         const uint8_t *mask_row = p.mask ? p.mask + static_cast<size_t>(b) * p.P : nullptr;
+        float *xmax = reinterpret_cast<float *>(smem + L::kXchgOff);  // [2 tile parity][2 half][128 rows]
+        float *xl = xmax + 2 * 2 * kMRows;                             // [2 half][128]
+        float *xlh = xl + 2 * kMRows;                                  // [2 half][128]
+        uint64_t *pair_bar = &bars[L::kBarPair + q4];
+        int pair_phase = 0;
+        auto pair_sync = [&]() -> bool {  // both warps of this lane quarter
+            ptx::mbar_arrive(pair_bar);
+            const bool ok = warp_wait(pair_bar, pair_phase & 1);
+            ++pair_phase;
+            return ok;
+        };
+        constexpr int NH = NT / 2;  // columns of a tile per half
         float m_used = -INFINITY;
-        float l = 0.0f;   // sum of fp32 probabilities (for the LSE)
-        float lh = 0.0f;  // sum of the bf16-rounded probabilities (for O)
+        float l = 0.0f;   // this half's sum of fp32 probabilities (for the LSE)
+        float lh = 0.0f;  // this half's sum of bf16-rounded probabilities (for O)
         for (int t = 0; t < T; ++t) {
             const int sb = t % kSBufs;
             if (!warp_wait(&bars[L::kBarSFull + sb], (t / kSBufs) & 1)) {
@@ -403,54 +427,62 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             ptx::tc_fence_after_sync();
             const uint32_t scol = tmem + lane_base + kTmemS + sb * NT;
-            uint32_t raw[NT / 16][16];
+            uint32_t raw[NH / 16][16];
 #pragma unroll
-            for (int j = 0; j < NT / 16; ++j) ptx::tmem_ld16(scol + j * 16, raw[j]);
+            for (int j = 0; j < NH / 16; ++j) ptx::tmem_ld16(scol + hf * NH + j * 16, raw[j]);
             ptx::tmem_ld_wait();
 
             const TileInfo ti = tile_of<NT>(t_begin + t, TP, vl, p.S);
-            // visibility of the NT keys of this tile, same for every row
-            uint32_t vis[NT / 32];
+            // visibility of this half's keys (same for every row)
+            uint32_t vis[NH / 32];
 #pragma unroll
-            for (int w = 0; w < NT / 32; ++w) {
-                const int c = w * 32 + lane;
+            for (int w = 0; w < NH / 32; ++w) {
+                const int c = hf * NH + w * 32 + lane;
                 bool v = c < ti.n_valid;
                 if (v && ti.prefix && mask_row != nullptr) v = __ldg(mask_row + ti.row0 + c) != 0;
                 vis[w] = __ballot_sync(0xffffffffu, v);
             }
-            float s[NT];
-            float tmax = -INFINITY;
+            float s[NH];
+            float hmax = -INFINITY;
 #pragma unroll
-            for (int c = 0; c < NT; ++c) {
+            for (int c = 0; c < NH; ++c) {
                 const float x = __uint_as_float(raw[c / 16][c % 16]) * p.scale_log2;
                 s[c] = ((vis[c / 32] >> (c % 32)) & 1u) ? x : -INFINITY;
-                tmax = fmaxf(tmax, s[c]);
+                hmax = fmaxf(hmax, s[c]);
             }
+            // the row max over both halves
+            xmax[((t & 1) * 2 + hf) * kMRows + row] = hmax;
+            if (!pair_sync()) {
+                failed = true;
+                break;
+            }
+            const float tmax = fmaxf(hmax, xmax[((t & 1) * 2 + (hf ^ 1)) * kMRows + row]);
+            // identical decision in both halves (same inputs)
             float factor = 1.0f;
             bool rescale_o = false;
             if (t == 0) {
                 m_used = tmax;
             } else if (tmax > m_used + kRescaleThreshold) {
                 factor = ptx::ex2(m_used - tmax);  // 0 when m_used is -inf
-                rescale_o = lh > 0.0f;             // otherwise O holds exact zeros
+                rescale_o = true;
                 l *= factor;
                 lh *= factor;
                 m_used = tmax;
             }
             const float msub = (m_used == -INFINITY) ? 0.0f : m_used;
             float lsum = 0.0f, lhsum = 0.0f;
-            uint32_t pk[NT / 2];
+            uint32_t pk[NH / 2];
 #pragma unroll
-            for (int c = 0; c < NT; c += 2)
+            for (int c = 0; c < NH; c += 2)
                 pk[c / 2] = pack_bf16x2(ptx::ex2(s[c] - msub), ptx::ex2(s[c + 1] - msub), lhsum, lsum);
             l += lsum;
             lh += lhsum;
 #pragma unroll
-            for (int j = 0; j < NT / 32; ++j) {
+            for (int j = 0; j < NH / 32; ++j) {
                 uint32_t chunk[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) chunk[e] = pk[j * 16 + e];
-                ptx::tmem_st16(scol + j * 16, chunk);
+                ptx::tmem_st16(scol + hf * (NH / 2) + j * 16, chunk);
             }
             if (t > 0) {
                 // Every warp observes every PV completion in order (PV(t-1)
@@ -462,15 +494,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                     break;
                 }
                 if (__any_sync(0xffffffffu, rescale_o)) {
+                    // this half's 128 columns of O (an all-zero O stays zero)
                     ptx::tc_fence_after_sync();
 #pragma unroll 1
-                    for (int j = 0; j < kHeadDim / 16; ++j) {
+                    for (int j = 0; j < kHeadDim / 32; ++j) {
                         uint32_t o[16];
-                        ptx::tmem_ld16(tmem + lane_base + kTmemO + j * 16, o);
+                        const uint32_t oc = tmem + lane_base + kTmemO + hf * (kHeadDim / 2) + j * 16;
+                        ptx::tmem_ld16(oc, o);
                         ptx::tmem_ld_wait();
 #pragma unroll
                         for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * factor);
-                        ptx::tmem_st16(tmem + lane_base + kTmemO + j * 16, o);
+                        ptx::tmem_st16(oc, o);
                     }
                 }
             }
@@ -486,8 +520,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 uint8_t *vt = sV + st * L::kTileBytes;
                 const int rows = (ti.n_valid + 15) / 16 * 16 - ti.n_valid;  // read by the last PV k-step
-                const int units = kChunks * rows * 8;  // 16-byte units
-                for (int i = row; i < units; i += kSoftmaxWarps * 32) {
+                const int units = kChunks * rows * 8;                       // 16-byte units
+                for (int i = tid; i < units; i += kSoftmaxWarps * 32) {
                     const int c = i / (rows * 8);
                     const int rem = i - c * rows * 8;
                     const int r = ti.n_valid + rem / 8;
@@ -505,14 +539,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!warp_wait(&bars[L::kBarODone], (T - 1) & 1)) failed = true;
             ptx::tc_fence_after_sync();
         }
+        // row sums over both halves
+        xl[hf * kMRows + row] = l;
+        xlh[hf * kMRows + row] = lh;
+        if (!failed && !pair_sync()) failed = true;
+        const float l_row = l + xl[(hf ^ 1) * kMRows + row];
+        const float lh_row = lh + xlh[(hf ^ 1) * kMRows + row];
         const size_t out_row = static_cast<size_t>(unit) * p.GS + row;
         if (C == 1) {
-            // ---------------------------------------- single CTA: normalise and store
-            const float inv_l = 1.0f / lh;
+            // ---------------------------------------- single CTA: normalise and store this half
+            const float inv_l = 1.0f / lh_row;
 #pragma unroll 1
-            for (int j = 0; j < kHeadDim / 16; ++j) {
+            for (int j = 0; j < kHeadDim / 32; ++j) {
                 uint32_t o[16];
-                ptx::tmem_ld16(tmem + lane_base + kTmemO + j * 16, o);
+                ptx::tmem_ld16(tmem + lane_base + kTmemO + hf * (kHeadDim / 2) + j * 16, o);
                 ptx::tmem_ld_wait();
                 if (row < p.GS) {
                     uint32_t w[8];
@@ -522,41 +562,50 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                                  __uint_as_float(o[2 * e + 1]) * inv_l);
                         w[e] = *reinterpret_cast<uint32_t *>(&h);
                     }
-                    uint4 *dst = reinterpret_cast<uint4 *>(p.out + out_row * kHeadDim + j * 16);
+                    uint4 *dst = reinterpret_cast<uint4 *>(p.out + out_row * kHeadDim + hf * (kHeadDim / 2) + j * 16);
                     dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
                     dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
                 }
             }
-            if (row < p.GS && p.lse != nullptr) p.lse[out_row] = (m_used + ptx::lg2(l)) * 0.69314718055994531f;
+            if (hf == 0 && row < p.GS && p.lse != nullptr)
+                p.lse[out_row] = (m_used + ptx::lg2(l_row)) * 0.69314718055994531f;
         } else {
             // ---------------------------------------- split: publish this CTA's partial
             // Row `row` of the partial: D fp32 of unnormalised O, then
-            // {m, l, l_hat, 0}; one bulk TMA store per thread.
+            // {m, l, l_hat, 0}; each half stages its 128 columns, then one
+            // bulk TMA store per row.
             const size_t prow = (static_cast<size_t>(unit) * C + rank) * p.GS + row;
             uint8_t *srow = smem + row * L::kStageStride;
             const bool write_o = T > 0 && !failed;
             if (write_o) {
 #pragma unroll 1
                 for (int j = 0; j < kHeadDim / 64; ++j) {
-                    uint32_t o[4][16];
+                    uint32_t o[2][16];
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) ptx::tmem_ld16(tmem + lane_base + kTmemO + j * 64 + q * 16, o[q]);
+                    for (int qq = 0; qq < 2; ++qq)
+                        ptx::tmem_ld16(tmem + lane_base + kTmemO + hf * (kHeadDim / 2) + j * 32 + qq * 16, o[qq]);
                     ptx::tmem_ld_wait();
                     if (row < p.GS) {
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            uint4 *d = reinterpret_cast<uint4 *>(srow + (j * 64 + q * 16) * 4);
-                            d[0] = make_uint4(o[q][0], o[q][1], o[q][2], o[q][3]);
-                            d[1] = make_uint4(o[q][4], o[q][5], o[q][6], o[q][7]);
-                            d[2] = make_uint4(o[q][8], o[q][9], o[q][10], o[q][11]);
-                            d[3] = make_uint4(o[q][12], o[q][13], o[q][14], o[q][15]);
+                        for (int qq = 0; qq < 2; ++qq) {
+                            uint4 *d = reinterpret_cast<uint4 *>(srow + (hf * (kHeadDim / 2) + j * 32 + qq * 16) * 4);
+                            d[0] = make_uint4(o[qq][0], o[qq][1], o[qq][2], o[qq][3]);
+                            d[1] = make_uint4(o[qq][4], o[qq][5], o[qq][6], o[qq][7]);
+                            d[2] = make_uint4(o[qq][8], o[qq][9], o[qq][10], o[qq][11]);
+                            d[3] = make_uint4(o[qq][12], o[qq][13], o[qq][14], o[qq][15]);
                         }
                     }
                 }
             }
             if (row < p.GS) {
-                *reinterpret_cast<float4 *>(srow + kHeadDim * 4) = make_float4(m_used, l, write_o ? lh : 0.0f, 0.0f);
+                if (hf == 0)
+                    *reinterpret_cast<float4 *>(srow + kHeadDim * 4) =
+                        make_float4(m_used, l_row, write_o ? lh_row : 0.0f, 0.0f);
                 ptx::fence_proxy_async_smem();
+            }
+            // both halves of the row staged
+            if (!failed && !pair_sync()) failed = true;
+            if (row < p.GS && hf == 0) {
                 ptx::bulk_store_s2g(reinterpret_cast<uint8_t *>(p.part) + prow * L::kStageStride, ptx::smem_addr(srow),
                                     L::kStageStride);
                 ptx::bulk_commit();

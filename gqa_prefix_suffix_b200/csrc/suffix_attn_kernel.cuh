@@ -11,10 +11,12 @@
 //   * The two query heads of a GQA group form one MMA A operand:
 //     M = G*S <= 128 rows (padded to 128 by TMA zero fill), K = D = 256.
 //     Every K/V tile is therefore loaded once and used by both heads.
-//   * Key rows are a list of 64-row tiles: the prefix rows [0, valid_len),
-//     then the S suffix rows.  The CTAs of one unit split that list evenly
-//     (the split depends on valid_len, read on the device, so a captured
-//     graph stays valid for any valid_len).
+//   * Key rows are a list of 64-row tiles: the S suffix rows, then the
+//     prefix rows [0, valid_len).  The CTAs of one unit split that list
+//     evenly (the split depends on valid_len, read on the device, so a
+//     captured graph stays valid for any valid_len).  Each CTA requests its
+//     first tile's K/V before the valid_len read returns (the tile it would
+//     get if valid_len were P, which is nearly always the same one).
 //   * Warp roles: warp 8 issues TMA loads (Q once, then a ring of K and V
 //     tiles); warp 9 allocates TMEM and issues tcgen05 MMAs from one thread;
 //     warps 0-7 run the softmax: warps w and w+4 share TMEM lane quarter w
@@ -127,18 +129,21 @@ struct TileInfo {
     int n_valid;  // rows of the tile that are in range
 };
 
+// Tile g of a unit's key list: the TS suffix tiles first, then the prefix
+// tiles of [0, vl).  A tile's rows (row0) do not depend on vl, only how many
+// of them are valid.
 template <int NT>
-__device__ __forceinline__ TileInfo tile_of(int g, int TP, int vl, int S)
+__device__ __forceinline__ TileInfo tile_of(int g, int TS, int vl, int S)
 {
     TileInfo ti;
-    if (g < TP) {
-        ti.prefix = true;
-        ti.row0 = g * NT;
-        ti.n_valid = min(NT, vl - ti.row0);
-    } else {
+    if (g < TS) {
         ti.prefix = false;
-        ti.row0 = (g - TP) * NT;
+        ti.row0 = g * NT;
         ti.n_valid = min(NT, S - ti.row0);
+    } else {
+        ti.prefix = true;
+        ti.row0 = (g - TS) * NT;
+        ti.n_valid = min(NT, vl - ti.row0);
     }
     return ti;
 }
@@ -256,11 +261,33 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t *sQ = smem + L::kQOff;
     uint8_t *sK = smem + L::kKOff;
     uint8_t *sV = smem + L::kVOff;
+    // This CTA's first tile if valid_len were P (the bucket): it does not
+    // depend on valid_len, so its K/V are requested before that read returns.
+    // With the suffix tiles first it is the true first tile unless the split
+    // boundaries move; then the slot is drained and released (shift below).
+    const int TS = (p.S + NT - 1) / NT;
+    const int t_bucket = TS + (p.P + NT - 1) / NT;
+    const int g_spec = static_cast<int>((static_cast<long long>(t_bucket) * rank) / C);
+    const bool spec = g_spec < static_cast<int>((static_cast<long long>(t_bucket) * (rank + 1)) / C);
+    uint64_t pol = 0;
     if (warp == kProducerWarp && lane == 0) {
-        // Q does not depend on valid_len: start it before that read.
+        pol = ptx::policy_evict_first();
         ptx::mbar_arrive_expect_tx(&bars[L::kBarQFull], L::kQBytes);
         for (int c = 0; c < kChunks; ++c)
             ptx::tma_load_3d(sQ + c * L::kQChunkBytes, &tm_q, &bars[L::kBarQFull], c * kChunkElems, 0, unit);
+        if (spec) {
+            const TileInfo ti = tile_of<NT>(g_spec, TS, p.P, p.S);
+            const CUtensorMap *mk = ti.prefix ? &tm_kp : &tm_ks;
+            const CUtensorMap *mv = ti.prefix ? &tm_vp : &tm_vs;
+            ptx::mbar_arrive_expect_tx(&bars[L::kBarKFull], L::kTileBytes);
+            for (int c = 0; c < kChunks; ++c)
+                ptx::tma_load_3d_hint(sK + c * L::kTileChunkBytes, mk, &bars[L::kBarKFull], c * kChunkElems, ti.row0,
+                                      unit, pol);
+            ptx::mbar_arrive_expect_tx(&bars[L::kBarVFull], L::kTileBytes);
+            for (int c = 0; c < kChunks; ++c)
+                ptx::tma_load_3d_hint(sV + c * L::kTileChunkBytes, mv, &bars[L::kBarVFull], c * kChunkElems, ti.row0,
+                                      unit, pol);
+        }
     }
 
     int vl = p.P;
@@ -269,23 +296,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         vl = min(max(raw, 0), p.P);
         if (raw != vl && rank == 0 && threadIdx.x == 0) atomicOr(p.err, kEwClamped);
     }
-    const int TP = (vl + NT - 1) / NT;
-    const int TS = (p.S + NT - 1) / NT;
-    const int t_all = TP + TS;
+    const int t_all = TS + (vl + NT - 1) / NT;
     const int t_begin = static_cast<int>((static_cast<long long>(t_all) * rank) / C);
     const int t_end = static_cast<int>((static_cast<long long>(t_all) * (rank + 1)) / C);
     const int T = t_end - t_begin;
+    // K/V ring slot of tile t is t + shift: 0 when the early request was the
+    // first tile, 1 when it was not (its slot is then skipped).
+    const int shift = (spec && !(T > 0 && t_begin == g_spec)) ? 1 : 0;
 
     bool failed = false;
 
     if (warp == kProducerWarp) {
         // ================================================== TMA producer
         if (lane == 0) {
-            const uint64_t pol = ptx::policy_evict_first();
-            int k_issued = 0, v_issued = 0;
-            for (int t = 0; t < T && !failed; ++t) {
-                const int s = t % STAGES, n = t / STAGES;
-                const TileInfo ti = tile_of<NT>(t_begin + t, TP, vl, p.S);
+            int slots = spec ? 1 : 0;  // ring slots requested so far
+            if (shift == 1) {
+                // the early request is not one of this CTA's tiles: let it
+                // land, then release its slot as its consumer would
+                if (!ptx::mbar_wait(&bars[L::kBarKFull], 0, kWaitLimitNs) ||
+                    !ptx::mbar_wait(&bars[L::kBarVFull], 0, kWaitLimitNs))
+                    failed = true;
+                ptx::mbar_arrive(&bars[L::kBarKEmpty]);
+                ptx::mbar_arrive(&bars[L::kBarVEmpty]);
+            }
+            int k_issued = slots, v_issued = slots;
+            for (int t = slots - shift; t < T && !failed; ++t) {
+                const int slot = t + shift;
+                const int s = slot % STAGES, n = slot / STAGES;
+                const TileInfo ti = tile_of<NT>(t_begin + t, TS, vl, p.S);
                 const CUtensorMap *mk = ti.prefix ? &tm_kp : &tm_ks;
                 const CUtensorMap *mv = ti.prefix ? &tm_vp : &tm_vs;
                 if (n > 0 && !ptx::mbar_wait(&bars[L::kBarKEmpty + s], (n - 1) & 1, kWaitLimitNs)) {
@@ -296,7 +334,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int c = 0; c < kChunks; ++c)
                     ptx::tma_load_3d_hint(sK + s * L::kTileBytes + c * L::kTileChunkBytes, mk, &bars[L::kBarKFull + s],
                                           c * kChunkElems, ti.row0, unit, pol);
-                k_issued = t + 1;
+                k_issued = slot + 1;
                 if (n > 0 && !ptx::mbar_wait(&bars[L::kBarVEmpty + s], (n - 1) & 1, kWaitLimitNs)) {
                     failed = true;
                     break;
@@ -305,7 +343,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int c = 0; c < kChunks; ++c)
                     ptx::tma_load_3d_hint(sV + s * L::kTileBytes + c * L::kTileChunkBytes, mv, &bars[L::kBarVFull + s],
                                           c * kChunkElems, ti.row0, unit, pol);
-                v_issued = t + 1;
+                v_issued = slot + 1;
             }
             // Drain: every copy this thread issued must have landed before the
             // CTA may exit (normally all phases are long complete here).
@@ -323,17 +361,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t k_base = ptx::smem_addr(sK);
             const uint32_t v_base = ptx::smem_addr(sV);
             auto issue_pv = [&](int u) -> bool {
-                const int s = u % STAGES;
+                const int s = (u + shift) % STAGES;
                 const int pb = u % kSBufs;
                 if (!ptx::mbar_wait(&bars[L::kBarPReady + pb], (u / kSBufs) & 1, kWaitLimitNs)) return false;
-                if (!ptx::mbar_wait(&bars[L::kBarVFull + s], (u / STAGES) & 1, kWaitLimitNs)) return false;
+                if (!ptx::mbar_wait(&bars[L::kBarVFull + s], ((u + shift) / STAGES) & 1, kWaitLimitNs)) return false;
                 ptx::tc_fence_after_sync();
                 const uint32_t vb = v_base + s * L::kTileBytes;
                 const uint32_t p_tmem = tmem + kTmemS + pb * NT;
                 // only the 16-row k-steps that hold valid keys (a partial tile
                 // stops early; the rows after its last valid key up to the
                 // k-step end are zero)
-                const int nk = (tile_of<NT>(t_begin + u, TP, vl, p.S).n_valid + 15) / 16;
+                const int nk = (tile_of<NT>(t_begin + u, TS, vl, p.S).n_valid + 15) / 16;
 #pragma unroll
                 for (int kk = 0; kk < NT / 16; ++kk) {
                     if (kk >= nk) break;
@@ -350,9 +388,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             };
             bool ok = ptx::mbar_wait(&bars[L::kBarQFull], 0, kWaitLimitNs);
             for (int t = 0; t < T && ok; ++t) {
-                const int s = t % STAGES;
+                const int s = (t + shift) % STAGES;
                 const int sb = t % kSBufs;
-                if (!ptx::mbar_wait(&bars[L::kBarKFull + s], (t / STAGES) & 1, kWaitLimitNs)) {
+                if (!ptx::mbar_wait(&bars[L::kBarKFull + s], ((t + shift) / STAGES) & 1, kWaitLimitNs)) {
                     ok = false;
                     break;
                 }
@@ -369,7 +407,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t d = tmem + kTmemS + sb * NT;
                 // N = the valid keys of the tile rounded up to 16; the
                 // softmax masks every column past the valid ones anyway.
-                const int nv16 = (tile_of<NT>(t_begin + t, TP, vl, p.S).n_valid + 15) / 16 * 16;
+                const int nv16 = (tile_of<NT>(t_begin + t, TS, vl, p.S).n_valid + 15) / 16 * 16;
                 const uint32_t idesc_qk = ptx::idesc_bf16_f32(kMRows, nv16, false);
 #pragma unroll
                 for (int kk = 0; kk < kHeadDim / 16; ++kk) {
@@ -432,7 +470,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int j = 0; j < NH / 16; ++j) ptx::tmem_ld16(scol + hf * NH + j * 16, raw[j]);
             ptx::tmem_ld_wait();
 
-            const TileInfo ti = tile_of<NT>(t_begin + t, TP, vl, p.S);
+            const TileInfo ti = tile_of<NT>(t_begin + t, TS, vl, p.S);
             // visibility of this half's keys (same for every row)
             uint32_t vis[NH / 32];
 #pragma unroll
@@ -513,8 +551,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // Rows at or past valid_len may hold anything (NaN too) and
                 // would poison O through 0 * NaN: clear the ones the last PV
                 // k-step reads.
-                const int st = t % STAGES;
-                if (!warp_wait(&bars[L::kBarVFull + st], (t / STAGES) & 1)) {
+                const int st = (t + shift) % STAGES;
+                if (!warp_wait(&bars[L::kBarVFull + st], ((t + shift) / STAGES) & 1)) {
                     failed = true;
                     break;
                 }
@@ -534,6 +572,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::mbar_arrive(&bars[L::kBarPReady + sb]);
         }
 
+        if (T == 0) {
+            // Nothing to compute, but the early requests (Q, and the K/V of
+            // the tile guessed before valid_len was known) still land in the
+            // shared memory the split epilogue reuses: wait for them first.
+            // (A CTA with tiles consumed them all before getting here.)
+            if (!warp_wait(&bars[L::kBarQFull], 0)) failed = true;
+            if (spec && (!warp_wait(&bars[L::kBarKFull], 0) || !warp_wait(&bars[L::kBarVFull], 0))) failed = true;
+        }
         const bool have_o = T > 0 && !failed;
         if (have_o) {
             if (!warp_wait(&bars[L::kBarODone], (T - 1) & 1)) failed = true;

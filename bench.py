@@ -319,7 +319,7 @@ def main():
     rc = bd.dm05_suffix_attn_reserve(B, Hq, Hkv, P, S, D, sh)
     if rc != 0:
         raise bd.Dm05Error(rc, "reserve")
-    rc, splits, tile_rows = bd.dm05_suffix_attn_plan(B, Hq, Hkv, P, S, D)
+    rc, splits, tile_rows, row_blocks = bd.dm05_suffix_attn_plan(B, Hq, Hkv, P, S, D)
 
     def call(t, s=sh):
         ptr = lambda x: None if x is None else x.data_ptr()
@@ -443,7 +443,8 @@ def main():
             "ms_per_step": value / 1e3, "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
             "config": workload_config(inp, {
-                "splits_per_head": splits, "tile_rows": tile_rows, "parallelism": f"replicas x{world}",
+                "splits_per_head": splits, "row_blocks": row_blocks, "tile_rows": tile_rows,
+                "parallelism": f"replicas x{world}",
                 "l2": f"{R} rotating input sets, {R * set_bytes / 1e6:.0f} MB > 2 x L2 ({l2 / 1e6:.0f} MB)",
                 "graph_calls": chunk}),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",

@@ -54,7 +54,7 @@ def lib() -> ctypes.CDLL:
             L.dm05_suffix_attn_workspace_bytes.restype = sz
             L.dm05_suffix_attn_reserve.argtypes = [i] * 6 + [p]
             L.dm05_suffix_attn_reserve.restype = i
-            L.dm05_suffix_attn_plan.argtypes = [i] * 6 + [ctypes.POINTER(i), ctypes.POINTER(i)]
+            L.dm05_suffix_attn_plan.argtypes = [i] * 6 + [ctypes.POINTER(i)] * 3
             L.dm05_suffix_attn_plan.restype = i
             L.dm05_set_split_override.argtypes = [i]
             L.dm05_set_split_override.restype = i
@@ -95,10 +95,10 @@ def dm05_suffix_attn_reserve(B, Hq, Hkv, P, S, D, stream) -> int:
 
 
 def dm05_suffix_attn_plan(B, Hq, Hkv, P, S, D):
-    """Returns (status, splits_per_head, tile_rows)."""
-    sp, tr = ctypes.c_int(0), ctypes.c_int(0)
-    rc = lib().dm05_suffix_attn_plan(B, Hq, Hkv, P, S, D, ctypes.byref(sp), ctypes.byref(tr))
-    return rc, sp.value, tr.value
+    """Returns (status, splits_per_head, tile_rows, row_blocks)."""
+    sp, tr, rb = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int(0)
+    rc = lib().dm05_suffix_attn_plan(B, Hq, Hkv, P, S, D, ctypes.byref(sp), ctypes.byref(tr), ctypes.byref(rb))
+    return rc, sp.value, tr.value, rb.value
 
 
 def dm05_set_split_override(splits_per_head: int) -> int:

@@ -10,6 +10,7 @@
 
 #include <cmath>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <vector>
@@ -31,6 +32,7 @@ struct DeviceState {
     bool attrs_set = false;
     int num_sms = 0;
     int max_cluster = 0;       // largest cluster size (power of two <= 16) that can be resident
+    int active[5] = {0, 0, 0, 0, 0};  // co-resident clusters of size 1, 2, 4, 8, 16
 };
 
 // Partial-result workspace of one (device, stream): concurrent streams never
@@ -52,11 +54,17 @@ auto *kKernel = &dm05::suffix_attn_kernel<kTileRows, kStages>;
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Bytes of partial results a call with `splits` CTAs per unit exchanges:
-// [units][splits][GS] rows of D fp32 followed by a float4 of statistics.
-size_t partial_bytes(long long units, int splits, int GS)
+struct Plan {
+    int splits = 1;      // CTAs per (unit, query block): a cluster
+    int row_blocks = 1;  // query blocks per unit
+    int SQ = 1;          // queries per head per block
+};
+
+// Bytes of partial results a call exchanges: [units * row_blocks][splits]
+// [G * SQ] rows of D fp32, each followed by a float4 of statistics.
+size_t partial_bytes(long long units, const Plan &pl, int G)
 {
-    return splits > 1 ? static_cast<size_t>(units) * splits * GS * kPartRowBytes : 0;
+    return pl.splits > 1 ? static_cast<size_t>(units) * pl.row_blocks * pl.splits * G * pl.SQ * kPartRowBytes : 0;
 }
 
 int check_sizes(int B, int Hq, int Hkv, int P, int S, int D)
@@ -69,16 +77,72 @@ int check_sizes(int B, int Hq, int Hkv, int P, int S, int D)
     return DM05_OK;
 }
 
-// CTAs per (sample, KV head): the largest power of two (<= 16, <= the number
-// of 64-row key tiles) that keeps all CTAs of a call resident at once.
-int choose_splits(int B, int Hkv, int P, int S, int num_sms, int max_cluster)
+// Work decomposition: CTAs per (sample, KV head) (a cluster that splits its
+// key tiles and merges the partial results) and query row blocks per unit
+// (each CTA then carries fewer query rows, so fewer partial rows to merge).
+// Among the plans whose clusters are all resident at once, the one with the
+// lowest estimated cost.
+int log2_pow2(int c) { return c >= 16 ? 4 : c >= 8 ? 3 : c >= 4 ? 2 : c >= 2 ? 1 : 0; }
+
+int env_row_blocks()
 {
-    if (g_split_override > 0) return g_split_override;
+    static const int v = [] {
+        const char *e = std::getenv("DM05_ROW_BLOCKS");
+        return e ? std::atoi(e) : 0;
+    }();
+    return v;
+}
+
+Plan make_plan(int B, int Hq, int Hkv, int P, int S, const DeviceState &ds)
+{
     const long long units = static_cast<long long>(B) * Hkv;
+    const int G = Hq / Hkv;
     const int tiles = (P + kTileRows - 1) / kTileRows + (S + kTileRows - 1) / kTileRows;
-    int c = 1;
-    while (c * 2 <= max_cluster && units * (c * 2) <= num_sms && c * 2 <= tiles) c *= 2;
-    return c;
+    // every cluster of the call resident at once (no second wave)
+    auto fits = [&](int c, long long blocks) {
+        if (c == 1) return true;
+        return units * blocks * c <= ds.num_sms && units * blocks <= ds.active[log2_pow2(c)];
+    };
+    // Estimated cost in microseconds, fitted on B200 measurements of this
+    // kernel: ~1.2 per key tile a CTA streams, and for a split unit a fixed
+    // ~2 for the merge plus ~0.04 per partial row a CTA publishes.
+    auto cost = [&](int c, int sq) {
+        double t = 1.2 * ((tiles + c - 1) / c);
+        if (c > 1) t += 2.0 + 0.04 * G * sq;
+        return t;
+    };
+    const int want_rb = env_row_blocks();
+    Plan best;
+    best.SQ = S;
+    double best_cost = 1e30;
+    for (int c = 1; c <= 16; c *= 2) {
+        if (g_split_override > 0 && c != g_split_override) continue;
+        if (g_split_override == 0 && (c > ds.max_cluster || !fits(c, 1))) continue;
+        for (int r = 1; r <= 16; r *= 2) {
+            if (c == 1 && r > 1) break;
+            const int sq = (S + r - 1) / r;
+            if (r > 1 && (sq < 8 || G * ((sq + 7) / 8 * 8) > dm05::kMRows)) break;
+            if (want_rb > 0 ? r != want_rb && !(r == 1 && c == 1) : !fits(c, r)) continue;
+            const double t = cost(c, sq);
+            if (t < best_cost) {
+                best_cost = t;
+                best.splits = c;
+                best.SQ = sq;
+                best.row_blocks = (S + sq - 1) / sq;  // no empty trailing block
+            }
+        }
+    }
+    if (best_cost > 1e29) {  // forced split count that nothing above accepted
+        best.splits = g_split_override > 0 ? g_split_override : 1;
+        best.row_blocks = 1;
+        best.SQ = S;
+    }
+    if (best.splits > ds.max_cluster) {
+        best.splits = ds.max_cluster;
+        best.row_blocks = 1;
+        best.SQ = S;
+    }
+    return best;
 }
 
 int get_encoder()
@@ -108,9 +172,11 @@ int device_state(bool allocate, DeviceState **out)
                 cudaSuccess ||
             cudaFuncSetAttribute(kKernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
             return DM05_ERR_CUDA;
-        // largest cluster the device can hold with this kernel's footprint
+        // how many clusters of each size the device holds at once with this
+        // kernel's footprint (a plan never exceeds it: no second wave)
         ds.max_cluster = 1;
-        for (int c = 16; c >= 2; c /= 2) {
+        ds.active[0] = ds.num_sms;
+        for (int c = 16, li = 4; c >= 2; c /= 2, --li) {
             cudaLaunchConfig_t cfg = {};
             cfg.gridDim = dim3(c, 1, 1);
             cfg.blockDim = dim3(dm05::kThreads, 1, 1);
@@ -124,10 +190,11 @@ int device_state(bool allocate, DeviceState **out)
             cfg.numAttrs = 1;
             int n = 0;
             if (cudaOccupancyMaxActiveClusters(&n, kKernel, &cfg) == cudaSuccess && n > 0) {
-                ds.max_cluster = c;
-                break;
+                ds.active[li] = n;
+                if (ds.max_cluster == 1) ds.max_cluster = c;
+            } else {
+                cudaGetLastError();  // clear a refused size
             }
-            cudaGetLastError();  // clear a refused size
         }
         ds.attrs_set = true;
     }
@@ -215,8 +282,13 @@ const char *dm05_status_string(int status)
 size_t dm05_suffix_attn_workspace_bytes(int B, int Hq, int Hkv, int P, int S, int D)
 {
     if (check_sizes(B, Hq, Hkv, P, S, D) != DM05_OK) return 0;
-    // the largest split count the library ever uses is 16
-    return kErrBytes + partial_bytes(static_cast<long long>(B) * Hkv, 16, (Hq / Hkv) * S);
+    // the largest split count the library ever uses is 16; row blocks only
+    // round each block's queries up (SQ * row_blocks < S + 16)
+    Plan worst;
+    worst.splits = 16;
+    worst.row_blocks = 1;
+    worst.SQ = S + 16;  // at most 16 blocks of >= 8 queries
+    return kErrBytes + partial_bytes(static_cast<long long>(B) * Hkv, worst, Hq / Hkv);
 }
 
 int dm05_set_split_override(int splits_per_head)
@@ -229,7 +301,8 @@ int dm05_set_split_override(int splits_per_head)
     return DM05_OK;
 }
 
-int dm05_suffix_attn_plan(int B, int Hq, int Hkv, int P, int S, int D, int *splits_per_head, int *tile_rows)
+int dm05_suffix_attn_plan(int B, int Hq, int Hkv, int P, int S, int D, int *splits_per_head, int *tile_rows,
+                          int *row_blocks)
 {
     int rc = check_sizes(B, Hq, Hkv, P, S, D);
     if (rc != DM05_OK) return rc;
@@ -237,8 +310,10 @@ int dm05_suffix_attn_plan(int B, int Hq, int Hkv, int P, int S, int D, int *spli
     DeviceState *ds = nullptr;
     rc = device_state(false, &ds);
     if (rc != DM05_OK) return rc;
-    if (splits_per_head) *splits_per_head = choose_splits(B, Hkv, P, S, ds->num_sms, ds->max_cluster);
+    const Plan pl = make_plan(B, Hq, Hkv, P, S, *ds);
+    if (splits_per_head) *splits_per_head = pl.splits;
     if (tile_rows) *tile_rows = kTileRows;
+    if (row_blocks) *row_blocks = pl.row_blocks;
     return DM05_OK;
 }
 
@@ -254,9 +329,9 @@ int dm05_suffix_attn_reserve(int B, int Hq, int Hkv, int P, int S, int D, cudaSt
     DeviceState *ds = nullptr;
     rc = device_state(true, &ds);
     if (rc != DM05_OK) return rc;
-    const int splits = choose_splits(B, Hkv, P, S, ds->num_sms, ds->max_cluster);
+    const Plan pl = make_plan(B, Hq, Hkv, P, S, *ds);
     void *ws = nullptr;
-    return stream_workspace(stream, partial_bytes(static_cast<long long>(B) * Hkv, splits, (Hq / Hkv) * S), &ws);
+    return stream_workspace(stream, partial_bytes(static_cast<long long>(B) * Hkv, pl, Hq / Hkv), &ws);
 }
 
 int dm05_suffix_attn(const void *q, const void *k_prefix, const void *v_prefix, const int32_t *prefix_valid_len,
@@ -278,7 +353,7 @@ int dm05_suffix_attn(const void *q, const void *k_prefix, const void *v_prefix, 
     const int units = B * Hkv;
 
     DeviceState *ds = nullptr;
-    int splits = 1;
+    Plan pl;
     void *part_ws = nullptr;
     {
         std::lock_guard<std::mutex> lk(g_mu);
@@ -292,15 +367,15 @@ int dm05_suffix_attn(const void *q, const void *k_prefix, const void *v_prefix, 
             rc = device_state(true, &ds);
             if (rc != DM05_OK) return rc;
         }
-        splits = choose_splits(B, Hkv, P, S, ds->num_sms, ds->max_cluster);
-        if (splits > ds->max_cluster) splits = ds->max_cluster;
-        rc = stream_workspace(stream, partial_bytes(units, splits, GS), &part_ws);
+        pl = make_plan(B, Hq, Hkv, P, S, *ds);
+        rc = stream_workspace(stream, partial_bytes(units, pl, G), &part_ws);
         if (rc != DM05_OK) return rc;
     }
 
     // ---- TMA descriptors (the tensor maps travel as kernel parameters)
     CUtensorMap tm_q, tm_kp, tm_vp, tm_ks, tm_vs;
-    if (encode_3d(&tm_q, q, static_cast<uint64_t>(GS), static_cast<uint64_t>(units), dm05::kMRows) != DM05_OK ||
+    if (encode_3d(&tm_q, q, static_cast<uint64_t>(GS), static_cast<uint64_t>(units),
+                  pl.row_blocks == 1 ? dm05::kMRows : static_cast<uint32_t>(pl.SQ)) != DM05_OK ||
         encode_3d(&tm_ks, k_suffix, static_cast<uint64_t>(S), static_cast<uint64_t>(units), kTileRows) != DM05_OK ||
         encode_3d(&tm_vs, v_suffix, static_cast<uint64_t>(S), static_cast<uint64_t>(units), kTileRows) != DM05_OK)
         return DM05_ERR_CUDA;
@@ -325,11 +400,14 @@ int dm05_suffix_attn(const void *q, const void *k_prefix, const void *v_prefix, 
     kp.P = P;
     kp.S = S;
     kp.GS = GS;
-    kp.splits = splits;
+    kp.G = G;
+    kp.row_blocks = pl.row_blocks;
+    kp.SQ = pl.SQ;
+    kp.splits = pl.splits;
     kp.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
 
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(units * splits), 1, 1);
+    cfg.gridDim = dim3(static_cast<unsigned>(units * pl.row_blocks * pl.splits), 1, 1);
     cfg.blockDim = dim3(dm05::kThreads, 1, 1);
     cfg.dynamicSmemBytes = Layout::kAllocBytes;
     cfg.stream = stream;
@@ -338,9 +416,9 @@ int dm05_suffix_attn(const void *q, const void *k_prefix, const void *v_prefix, 
     at[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     at[na].val.programmaticStreamSerializationAllowed = 1;
     ++na;
-    if (splits > 1) {
+    if (pl.splits > 1) {
         at[na].id = cudaLaunchAttributeClusterDimension;
-        at[na].val.clusterDim.x = static_cast<unsigned>(splits);
+        at[na].val.clusterDim.x = static_cast<unsigned>(pl.splits);
         at[na].val.clusterDim.y = 1;
         at[na].val.clusterDim.z = 1;
         ++na;
@@ -408,7 +486,7 @@ int dm05_suffix_attn_noalloc(const void *q, const void *k_prefix, const void *v_
     const int units = B * Hkv;
     DeviceState *ds = nullptr;
     uint32_t *scratch = nullptr;
-    int splits = 1;
+    Plan pl;
     {
         std::lock_guard<std::mutex> lk(g_mu);
         if (get_encoder() != DM05_OK) return DM05_ERR_CUDA;
@@ -416,14 +494,18 @@ int dm05_suffix_attn_noalloc(const void *q, const void *k_prefix, const void *v_
         if (rc != DM05_OK) return rc;
         rc = noalloc_scratch(stream, &scratch);
         if (rc != DM05_OK) return rc;
-        splits = choose_splits(B, Hkv, P, S, ds->num_sms, ds->max_cluster);
-        if (splits > ds->max_cluster) splits = ds->max_cluster;
+        pl = make_plan(B, Hq, Hkv, P, S, *ds);
         // fewer CTAs per unit until the partial results fit the fixed array
-        while (splits > 1 && partial_bytes(units, splits, GS) > DM05_NOALLOC_SCRATCH_BYTES - kErrBytes) splits /= 2;
+        while (pl.splits > 1 && partial_bytes(units, pl, G) > DM05_NOALLOC_SCRATCH_BYTES - kErrBytes) pl.splits /= 2;
+        if (pl.splits == 1) {
+            pl.row_blocks = 1;
+            pl.SQ = S;
+        }
     }
 
     CUtensorMap tm_q, tm_kp, tm_vp, tm_ks, tm_vs;
-    if (encode_3d(&tm_q, q, static_cast<uint64_t>(GS), static_cast<uint64_t>(units), dm05::kMRows) != DM05_OK ||
+    if (encode_3d(&tm_q, q, static_cast<uint64_t>(GS), static_cast<uint64_t>(units),
+                  pl.row_blocks == 1 ? dm05::kMRows : static_cast<uint32_t>(pl.SQ)) != DM05_OK ||
         encode_3d(&tm_ks, k_suffix, static_cast<uint64_t>(S), static_cast<uint64_t>(units), kTileRows) != DM05_OK ||
         encode_3d(&tm_vs, v_suffix, static_cast<uint64_t>(S), static_cast<uint64_t>(units), kTileRows) != DM05_OK)
         return DM05_ERR_CUDA;
@@ -443,16 +525,19 @@ int dm05_suffix_attn_noalloc(const void *q, const void *k_prefix, const void *v_
     kp.out = static_cast<__nv_bfloat16 *>(out);
     kp.lse = lse;
     kp.err = scratch;
-    kp.part = splits > 1 ? reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(scratch) + kErrBytes) : nullptr;
+    kp.part = pl.splits > 1 ? reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(scratch) + kErrBytes) : nullptr;
     kp.Hkv = Hkv;
     kp.P = P;
     kp.S = S;
     kp.GS = GS;
-    kp.splits = splits;
+    kp.G = G;
+    kp.row_blocks = pl.row_blocks;
+    kp.SQ = pl.SQ;
+    kp.splits = pl.splits;
     kp.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
 
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(units * splits), 1, 1);
+    cfg.gridDim = dim3(static_cast<unsigned>(units * pl.row_blocks * pl.splits), 1, 1);
     cfg.blockDim = dim3(dm05::kThreads, 1, 1);
     cfg.dynamicSmemBytes = Layout::kAllocBytes;
     cfg.stream = stream;
@@ -461,9 +546,9 @@ int dm05_suffix_attn_noalloc(const void *q, const void *k_prefix, const void *v_
     at[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     at[na].val.programmaticStreamSerializationAllowed = 1;
     ++na;
-    if (splits > 1) {
+    if (pl.splits > 1) {
         at[na].id = cudaLaunchAttributeClusterDimension;
-        at[na].val.clusterDim.x = static_cast<unsigned>(splits);
+        at[na].val.clusterDim.x = static_cast<unsigned>(pl.splits);
         at[na].val.clusterDim.y = 1;
         at[na].val.clusterDim.z = 1;
         ++na;

@@ -8,9 +8,12 @@
 // KV heads (GQA), head_dim 256 (same section's shape table).
 //
 // Design (one CTA = one slice of the key rows of one (sample, KV head) unit):
-//   * The two query heads of a GQA group form one MMA A operand:
-//     M = G*S <= 128 rows (padded to 128 by TMA zero fill), K = D = 256.
-//     Every K/V tile is therefore loaded once and used by both heads.
+//   * The query heads of a GQA group form one MMA A operand: M = G*S <= 128
+//     rows (padded to 128 by TMA zero fill), K = D = 256, so every K/V tile
+//     is loaded once and used by both heads.  When a unit is split over a
+//     cluster and SMs are left over, its S queries are also split into
+//     row blocks (each CTA then holds both heads' SQ queries of one block),
+//     which halves the partial results each CTA must merge.
 //   * Key rows are a list of 64-row tiles: the S suffix rows, then the
 //     prefix rows [0, valid_len).  The CTAs of one unit split that list
 //     evenly (the split depends on valid_len, read on the device, so a
@@ -75,9 +78,12 @@ struct KernelParams {
     __nv_bfloat16 *out;        // [B*Hkv, GS, D]
     float *lse;                // [B*Hkv, GS] or nullptr
     uint32_t *err;             // device error word
-    float *part;               // splits > 1: partial rows [units][splits][GS], each D fp32 + {m, l, l_hat, 0}
+    float *part;               // splits > 1: partial rows [units*row_blocks][splits][G*SQ], each D fp32 + {m, l, l_hat, 0}
     int Hkv, P, S, GS;         // GS = (Hq / Hkv) * S query rows of a unit
-    int splits;                // CTAs per unit (cluster size)
+    int G;                     // query heads per KV head
+    int row_blocks;            // query blocks per unit (1: all S queries in one CTA)
+    int SQ;                    // queries per head per block (S when row_blocks == 1)
+    int splits;                // CTAs per (unit, query block): the cluster size
     float scale_log2;          // log2(e) / sqrt(D)
 };
 
@@ -167,10 +173,19 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi, float &sum_r
     return *reinterpret_cast<uint32_t *>(&h);
 }
 
-// out[rr][:] = bf16( sum_c w[c][rr] * recv[c][rr][:] ) for the nr rows a CTA
-// merges; the C partial rows are kStageStride bytes apart in shared memory.
+// out row of compact row k = h * nq + j of a query block: head h, query q0 + j
+__device__ __forceinline__ size_t block_out_row(size_t unit_row0, int k, int nq, int S, int q0)
+{
+    const int h = k / nq;
+    return unit_row0 + static_cast<size_t>(h) * S + q0 + (k - h * nq);
+}
+
+// out[row(k_lo + rr)][:] = bf16( sum_c w[c][rr] * recv[c][rr][:] ) for the
+// nr rows a CTA merges; the C partial rows are kStageStride bytes apart in
+// shared memory.
 template <int C, class L>
-__device__ __forceinline__ void merge_rows(const uint8_t *recv, const float *mw, int nr, __nv_bfloat16 *out)
+__device__ __forceinline__ void merge_rows(const uint8_t *recv, const float *mw, int nr, __nv_bfloat16 *out,
+                                           size_t unit_row0, int k_lo, int nq, int S, int q0)
 {
     const int items = nr * (kHeadDim / 4);
     for (int i = threadIdx.x; i < items; i += kThreads) {
@@ -194,7 +209,7 @@ __device__ __forceinline__ void merge_rows(const uint8_t *recv, const float *mw,
         }
         __nv_bfloat162 h0 = __floats2bfloat162_rn(acc.x, acc.y);
         __nv_bfloat162 h1 = __floats2bfloat162_rn(acc.z, acc.w);
-        *reinterpret_cast<uint2 *>(out + static_cast<size_t>(rr) * kHeadDim + ch * 4) =
+        *reinterpret_cast<uint2 *>(out + block_out_row(unit_row0, k_lo + rr, nq, S, q0) * kHeadDim + ch * 4) =
             make_uint2(*reinterpret_cast<uint32_t *>(&h0), *reinterpret_cast<uint32_t *>(&h1));
     }
 }
@@ -214,9 +229,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int C = p.splits;
-    const int unit = blockIdx.x / C;
-    const int rank = blockIdx.x - unit * C;
+    const int cl = blockIdx.x / C;  // cluster: one query block of one unit
+    const int rank = blockIdx.x - cl * C;
+    const int unit = cl / p.row_blocks;
+    const int rb = cl - unit * p.row_blocks;
     const int b = unit / p.Hkv;
+    // TMEM row m <-> head m / rph, query q0 + m % rph (valid if that is < nq);
+    // compact row k = head * nq + (m % rph) indexes the valid rows.
+    const int q0 = rb * p.SQ;
+    const int nq = min(p.SQ, p.S - q0);
+    const int rph = p.row_blocks == 1 ? p.S : (p.SQ + 7) / 8 * 8;
+    const int NR = p.G * nq;
+    const size_t unit_row0 = static_cast<size_t>(unit) * p.GS;
 
     // ---- set-up that reads no input (overlaps the previous kernel under PDL)
     if (threadIdx.x == 0) {
@@ -272,9 +296,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t pol = 0;
     if (warp == kProducerWarp && lane == 0) {
         pol = ptx::policy_evict_first();
-        ptx::mbar_arrive_expect_tx(&bars[L::kBarQFull], L::kQBytes);
-        for (int c = 0; c < kChunks; ++c)
-            ptx::tma_load_3d(sQ + c * L::kQChunkBytes, &tm_q, &bars[L::kBarQFull], c * kChunkElems, 0, unit);
+        if (p.row_blocks == 1) {
+            // both heads' S queries are contiguous: one 128-row box per chunk
+            ptx::mbar_arrive_expect_tx(&bars[L::kBarQFull], L::kQBytes);
+            for (int c = 0; c < kChunks; ++c)
+                ptx::tma_load_3d(sQ + c * L::kQChunkBytes, &tm_q, &bars[L::kBarQFull], c * kChunkElems, 0, unit);
+        } else {
+            // one SQ-row box per head and chunk, at 8-row-aligned rows h * rph
+            ptx::mbar_arrive_expect_tx(&bars[L::kBarQFull], static_cast<uint32_t>(p.G * kChunks * p.SQ * 128));
+            for (int h = 0; h < p.G; ++h)
+                for (int c = 0; c < kChunks; ++c)
+                    ptx::tma_load_3d(sQ + c * L::kQChunkBytes + h * rph * 128, &tm_q, &bars[L::kBarQFull],
+                                     c * kChunkElems, h * p.S + q0, unit);
+        }
         if (spec) {
             const TileInfo ti = tile_of<NT>(g_spec, TS, p.P, p.S);
             const CUtensorMap *mk = ti.prefix ? &tm_kp : &tm_ks;
@@ -591,7 +625,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!failed && !pair_sync()) failed = true;
         const float l_row = l + xl[(hf ^ 1) * kMRows + row];
         const float lh_row = lh + xlh[(hf ^ 1) * kMRows + row];
-        const size_t out_row = static_cast<size_t>(unit) * p.GS + row;
+        const int row_h = row / rph;
+        const int row_j = row - row_h * rph;
+        const bool row_valid = row_h < p.G && row_j < nq;
+        const int row_k = row_h * nq + row_j;  // compact row (when valid)
+        const size_t out_row = unit_row0 + static_cast<size_t>(row_h) * p.S + q0 + row_j;
         if (C == 1) {
             // ---------------------------------------- single CTA: normalise and store this half
             const float inv_l = 1.0f / lh_row;
@@ -600,7 +638,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 uint32_t o[16];
                 ptx::tmem_ld16(tmem + lane_base + kTmemO + hf * (kHeadDim / 2) + j * 16, o);
                 ptx::tmem_ld_wait();
-                if (row < p.GS) {
+                if (row_valid) {
                     uint32_t w[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
@@ -613,14 +651,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
                 }
             }
-            if (hf == 0 && row < p.GS && p.lse != nullptr)
+            if (hf == 0 && row_valid && p.lse != nullptr)
                 p.lse[out_row] = (m_used + ptx::lg2(l_row)) * 0.69314718055994531f;
         } else {
             // ---------------------------------------- split: publish this CTA's partial
             // Row `row` of the partial: D fp32 of unnormalised O, then
             // {m, l, l_hat, 0}; each half stages its 128 columns, then one
             // bulk TMA store per row.
-            const size_t prow = (static_cast<size_t>(unit) * C + rank) * p.GS + row;
+            const size_t prow = (static_cast<size_t>(cl) * C + rank) * (p.G * p.SQ) + row_k;
             uint8_t *srow = smem + row * L::kStageStride;
             const bool write_o = T > 0 && !failed;
             if (write_o) {
@@ -631,7 +669,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int qq = 0; qq < 2; ++qq)
                         ptx::tmem_ld16(tmem + lane_base + kTmemO + hf * (kHeadDim / 2) + j * 32 + qq * 16, o[qq]);
                     ptx::tmem_ld_wait();
-                    if (row < p.GS) {
+                    if (row_valid) {
 #pragma unroll
                         for (int qq = 0; qq < 2; ++qq) {
                             uint4 *d = reinterpret_cast<uint4 *>(srow + (hf * (kHeadDim / 2) + j * 32 + qq * 16) * 4);
@@ -643,7 +681,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             }
-            if (row < p.GS) {
+            if (row_valid) {
                 if (hf == 0)
                     *reinterpret_cast<float4 *>(srow + kHeadDim * 4) =
                         make_float4(m_used, l_row, write_o ? lh_row : 0.0f, 0.0f);
@@ -651,7 +689,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             // both halves of the row staged
             if (!failed && !pair_sync()) failed = true;
-            if (row < p.GS && hf == 0) {
+            if (row_valid && hf == 0) {
                 ptx::bulk_store_s2g(reinterpret_cast<uint8_t *>(p.part) + prow * L::kStageStride, ptx::smem_addr(srow),
                                     L::kStageStride);
                 ptx::bulk_commit();
@@ -669,8 +707,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         //   M = max_c m_c,  LH = sum_c lh_c 2^(m_c - M),  L = sum_c l_c 2^(m_c - M)
         //   out = sum_c 2^(m_c - M) O_c / LH,   lse = (M + log2 L) ln 2.
         ptx::cluster_sync();
-        const int r_lo = (p.GS * rank) / C;
-        const int r_hi = (p.GS * (rank + 1)) / C;
+        const int r_lo = (NR * rank) / C;  // compact rows of this query block
+        const int r_hi = (NR * (rank + 1)) / C;
         const int nr = r_hi - r_lo;
         const uint8_t *recv = smem;  // [C][nr] rows of kStageStride bytes
         float *mw = reinterpret_cast<float *>(smem + L::kMergeWOff);  // [C][nr] weights
@@ -681,7 +719,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ptx::fence_proxy_async_global();
                 ptx::bulk_load_g2s(ptx::smem_addr(smem) + static_cast<uint32_t>(lane * nr * L::kStageStride),
                                    reinterpret_cast<const uint8_t *>(p.part) +
-                                       ((static_cast<size_t>(unit) * C + lane) * p.GS + r_lo) * L::kStageStride,
+                                       ((static_cast<size_t>(cl) * C + lane) * (p.G * p.SQ) + r_lo) * L::kStageStride,
                                    static_cast<uint32_t>(nr * L::kStageStride), &bars[L::kBarMerge]);
             }
         }
@@ -704,14 +742,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 if (lane < C) mw[lane * nr + rr] = f / LHs;
                 if (lane == 0 && p.lse != nullptr)
-                    p.lse[static_cast<size_t>(unit) * p.GS + r_lo + rr] = (M + ptx::lg2(Ls)) * 0.69314718055994531f;
+                    p.lse[block_out_row(unit_row0, r_lo + rr, nq, p.S, q0)] = (M + ptx::lg2(Ls)) * 0.69314718055994531f;
             }
             __syncthreads();
             switch (C) {
-            case 2: merge_rows<2, L>(recv, mw, nr, p.out + (static_cast<size_t>(unit) * p.GS + r_lo) * kHeadDim); break;
-            case 4: merge_rows<4, L>(recv, mw, nr, p.out + (static_cast<size_t>(unit) * p.GS + r_lo) * kHeadDim); break;
-            case 8: merge_rows<8, L>(recv, mw, nr, p.out + (static_cast<size_t>(unit) * p.GS + r_lo) * kHeadDim); break;
-            default: merge_rows<16, L>(recv, mw, nr, p.out + (static_cast<size_t>(unit) * p.GS + r_lo) * kHeadDim); break;
+            case 2: merge_rows<2, L>(recv, mw, nr, p.out, unit_row0, r_lo, nq, p.S, q0); break;
+            case 4: merge_rows<4, L>(recv, mw, nr, p.out, unit_row0, r_lo, nq, p.S, q0); break;
+            case 8: merge_rows<8, L>(recv, mw, nr, p.out, unit_row0, r_lo, nq, p.S, q0); break;
+            default: merge_rows<16, L>(recv, mw, nr, p.out, unit_row0, r_lo, nq, p.S, q0); break;
             }
         }
     }

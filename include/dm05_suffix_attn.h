@@ -109,10 +109,11 @@ size_t dm05_suffix_attn_workspace_bytes(int B, int Hq, int Hkv, int P, int S, in
 int dm05_suffix_attn_reserve(int B, int Hq, int Hkv, int P, int S, int D, cudaStream_t stream);
 
 /* Work decomposition the next call with these sizes will use: the number of
- * CTAs (one thread-block cluster) per (sample, KV head), and the key rows per
- * tile.  Either output pointer may be NULL. */
+ * CTAs (one thread-block cluster) per (sample, KV head, query block), the key
+ * rows per tile, and the number of query blocks each (sample, KV head)'s S
+ * queries are cut into.  Any output pointer may be NULL. */
 int dm05_suffix_attn_plan(int B, int Hq, int Hkv, int P, int S, int D,
-                          int *splits_per_head, int *tile_rows);
+                          int *splits_per_head, int *tile_rows, int *row_blocks);
 
 /* Forces the number of CTAs per (sample, KV head) for later calls on this
  * process: 1, 2, 4, 8 or 16; 0 restores the automatic choice.  For tuning

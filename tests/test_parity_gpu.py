@@ -3,8 +3,9 @@
 Tolerance (bf16 output, fp32 accumulation): |out - O_oracle| <= 1e-2 for
 every element, except elements whose exact value has magnitude >= 4, where a
 correctly rounded bf16 value can already be 2^-6 = 0.0156 away; those are
-held to one bf16 ulp of the exact value.  mean |out - O_oracle| <= 1e-3 and
-|lse - LSE_oracle| <= 1e-3.
+held to one bf16 ulp of the exact value.  mean |out - O_oracle| <= 1e-3, or
+1.5x the mean error of the correctly rounded result when that floor is
+itself near 1e-3 (a handful of keys), and |lse - LSE_oracle| <= 1e-3.
 """
 import math
 import zlib
@@ -44,7 +45,11 @@ def check_close(out, lse, o_ref, l_ref, what=""):
         raise AssertionError(f"{what}: {int(bad.sum())} elements over the bound in {len(rows)} rows "
                              f"(b,h,i) {rows[:12]}; max err {err.max():.5f} at "
                              f"|o|={np.abs(o_ref).flat[err.argmax()]:.3f}; rounding floor {floor:.5f}")
-    assert err.mean() <= MEAN_ABS, f"{what}: mean err {err.mean():.2e}"
+    # With only a few keys |O| is O(1) and the mean error of the correctly
+    # rounded bf16 result itself approaches 1e-3; the mean bound then follows
+    # that floor (realistic inputs have a floor near 1e-4, well under 1e-3).
+    floor_mean = np.abs(torch.from_numpy(o_ref).to(torch.bfloat16).double().numpy() - o_ref).mean()
+    assert err.mean() <= max(MEAN_ABS, 1.5 * floor_mean), f"{what}: mean err {err.mean():.2e}, floor {floor_mean:.2e}"
     if lse is not None:
         le = np.abs(lse.double().cpu().numpy() - l_ref)
         assert le.max() <= LSE_ABS, f"{what}: lse err {le.max():.2e}"

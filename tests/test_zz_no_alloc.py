@@ -63,5 +63,10 @@ def test_noalloc_rejects_bad_arguments_before_launch():
     bad = list(args)
     bad[0] = None
     assert bd.dm05_suffix_attn_noalloc(*bad, 1, 8, 4, 1024, 50, 256, None) == bd.DM05_ERR_NULL
-    # the base-model chunk's split plan fits the fixed scratch array (8 MiB)
-    np.testing.assert_equal(bd.dm05_suffix_attn_workspace_bytes(1, 8, 4, 1024, 50, 256) <= 8 << 20, True)
+    # the base-model chunk's split plan fits the fixed scratch array (8 MiB), so the
+    # allocation-free call runs the same decomposition as the allocating one
+    rc, splits, _, row_blocks = bd.dm05_suffix_attn_plan(1, 8, 4, 1024, 50, 256)
+    assert rc == bd.DM05_OK
+    sq = -(-50 // row_blocks)
+    need = 256 + (4 * row_blocks * splits * 2 * sq * 1040 if splits > 1 else 0)
+    np.testing.assert_equal(need <= 8 << 20, True)

@@ -247,6 +247,23 @@ int stream_workspace(cudaStream_t stream, size_t need, void **out)
     return DM05_OK;
 }
 
+// bf16 tensor [d2][d1][256] viewed as 4-D [d2][d1][4][64]: the 4 column
+// chunks (128 bytes apart) as a dimension inside the row (512 bytes).  A box
+// of {64, box1, 4, 1} lands as 4 chunk-major [box1 x 128 B] blocks with
+// 128-byte swizzle, the layout the tensor-core descriptors read.
+int encode_4d(CUtensorMap *map, const void *base, uint64_t d1, uint64_t d2, uint32_t box1)
+{
+    cuuint64_t dims[4] = {static_cast<cuuint64_t>(dm05::kChunkElems), d1, static_cast<cuuint64_t>(dm05::kChunks), d2};
+    cuuint64_t strides[3] = {static_cast<cuuint64_t>(dm05::kHeadDim) * 2, static_cast<cuuint64_t>(dm05::kChunkElems) * 2,
+                             d1 * dm05::kHeadDim * 2};
+    cuuint32_t box[4] = {static_cast<cuuint32_t>(dm05::kChunkElems), box1, static_cast<cuuint32_t>(dm05::kChunks), 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? DM05_OK : DM05_ERR_CUDA;
+}
+
 // bf16 tensor viewed as [d2][d1][256], loaded in boxes of 64 columns x box1 rows
 // with 128-byte swizzle; rows past d1 read as zero.
 int encode_3d(CUtensorMap *map, const void *base, uint64_t d1, uint64_t d2, uint32_t box1)
@@ -374,15 +391,20 @@ int dm05_suffix_attn(const void *q, const void *k_prefix, const void *v_prefix, 
 
     // ---- TMA descriptors (the tensor maps travel as kernel parameters)
     CUtensorMap tm_q, tm_kp, tm_vp, tm_ks, tm_vs;
-    if (encode_3d(&tm_q, q, static_cast<uint64_t>(GS), static_cast<uint64_t>(units),
-                  pl.row_blocks == 1 ? dm05::kMRows : static_cast<uint32_t>(pl.SQ)) != DM05_OK ||
-        encode_3d(&tm_ks, k_suffix, static_cast<uint64_t>(S), static_cast<uint64_t>(units), kTileRows) != DM05_OK ||
-        encode_3d(&tm_vs, v_suffix, static_cast<uint64_t>(S), static_cast<uint64_t>(units), kTileRows) != DM05_OK)
+    // Q: one 128-row box of all four chunks when the block is the whole unit,
+    // else one SQ-row box per head and chunk (3-D)
+    const int rq = pl.row_blocks == 1
+                       ? encode_4d(&tm_q, q, static_cast<uint64_t>(GS), static_cast<uint64_t>(units), dm05::kMRows)
+                       : encode_3d(&tm_q, q, static_cast<uint64_t>(GS), static_cast<uint64_t>(units),
+                                   static_cast<uint32_t>(pl.SQ));
+    if (rq != DM05_OK ||
+        encode_4d(&tm_ks, k_suffix, static_cast<uint64_t>(S), static_cast<uint64_t>(units), kTileRows) != DM05_OK ||
+        encode_4d(&tm_vs, v_suffix, static_cast<uint64_t>(S), static_cast<uint64_t>(units), kTileRows) != DM05_OK)
         return DM05_ERR_CUDA;
     if (P > 0) {
-        if (encode_3d(&tm_kp, k_prefix, static_cast<uint64_t>(P), static_cast<uint64_t>(units), kTileRows) !=
+        if (encode_4d(&tm_kp, k_prefix, static_cast<uint64_t>(P), static_cast<uint64_t>(units), kTileRows) !=
                 DM05_OK ||
-            encode_3d(&tm_vp, v_prefix, static_cast<uint64_t>(P), static_cast<uint64_t>(units), kTileRows) != DM05_OK)
+            encode_4d(&tm_vp, v_prefix, static_cast<uint64_t>(P), static_cast<uint64_t>(units), kTileRows) != DM05_OK)
             return DM05_ERR_CUDA;
     } else {
         tm_kp = tm_ks;  // never read: no prefix tile exists when P == 0
@@ -504,15 +526,20 @@ int dm05_suffix_attn_noalloc(const void *q, const void *k_prefix, const void *v_
     }
 
     CUtensorMap tm_q, tm_kp, tm_vp, tm_ks, tm_vs;
-    if (encode_3d(&tm_q, q, static_cast<uint64_t>(GS), static_cast<uint64_t>(units),
-                  pl.row_blocks == 1 ? dm05::kMRows : static_cast<uint32_t>(pl.SQ)) != DM05_OK ||
-        encode_3d(&tm_ks, k_suffix, static_cast<uint64_t>(S), static_cast<uint64_t>(units), kTileRows) != DM05_OK ||
-        encode_3d(&tm_vs, v_suffix, static_cast<uint64_t>(S), static_cast<uint64_t>(units), kTileRows) != DM05_OK)
+    // Q: one 128-row box of all four chunks when the block is the whole unit,
+    // else one SQ-row box per head and chunk (3-D)
+    const int rq = pl.row_blocks == 1
+                       ? encode_4d(&tm_q, q, static_cast<uint64_t>(GS), static_cast<uint64_t>(units), dm05::kMRows)
+                       : encode_3d(&tm_q, q, static_cast<uint64_t>(GS), static_cast<uint64_t>(units),
+                                   static_cast<uint32_t>(pl.SQ));
+    if (rq != DM05_OK ||
+        encode_4d(&tm_ks, k_suffix, static_cast<uint64_t>(S), static_cast<uint64_t>(units), kTileRows) != DM05_OK ||
+        encode_4d(&tm_vs, v_suffix, static_cast<uint64_t>(S), static_cast<uint64_t>(units), kTileRows) != DM05_OK)
         return DM05_ERR_CUDA;
     if (P > 0) {
-        if (encode_3d(&tm_kp, k_prefix, static_cast<uint64_t>(P), static_cast<uint64_t>(units), kTileRows) !=
+        if (encode_4d(&tm_kp, k_prefix, static_cast<uint64_t>(P), static_cast<uint64_t>(units), kTileRows) !=
                 DM05_OK ||
-            encode_3d(&tm_vp, v_prefix, static_cast<uint64_t>(P), static_cast<uint64_t>(units), kTileRows) != DM05_OK)
+            encode_4d(&tm_vp, v_prefix, static_cast<uint64_t>(P), static_cast<uint64_t>(units), kTileRows) != DM05_OK)
             return DM05_ERR_CUDA;
     } else {
         tm_kp = tm_ks;

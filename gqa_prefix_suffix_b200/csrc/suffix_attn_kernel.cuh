@@ -298,9 +298,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         pol = ptx::policy_evict_first();
         if (p.row_blocks == 1) {
             // both heads' S queries are contiguous: one 128-row box per chunk
+            // (4-D view [units][rows][4 chunks][64]: one request lands all
+            // four 64-column chunks, chunk-major, in the MMA layout)
             ptx::mbar_arrive_expect_tx(&bars[L::kBarQFull], L::kQBytes);
-            for (int c = 0; c < kChunks; ++c)
-                ptx::tma_load_3d(sQ + c * L::kQChunkBytes, &tm_q, &bars[L::kBarQFull], c * kChunkElems, 0, unit);
+            ptx::tma_load_4d(sQ, &tm_q, &bars[L::kBarQFull], 0, 0, 0, unit);
         } else {
             // one SQ-row box per head and chunk, at 8-row-aligned rows h * rph
             ptx::mbar_arrive_expect_tx(&bars[L::kBarQFull], static_cast<uint32_t>(p.G * kChunks * p.SQ * 128));
@@ -314,13 +315,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const CUtensorMap *mk = ti.prefix ? &tm_kp : &tm_ks;
             const CUtensorMap *mv = ti.prefix ? &tm_vp : &tm_vs;
             ptx::mbar_arrive_expect_tx(&bars[L::kBarKFull], L::kTileBytes);
-            for (int c = 0; c < kChunks; ++c)
-                ptx::tma_load_3d_hint(sK + c * L::kTileChunkBytes, mk, &bars[L::kBarKFull], c * kChunkElems, ti.row0,
-                                      unit, pol);
+            ptx::tma_load_4d_hint(sK, mk, &bars[L::kBarKFull], 0, ti.row0, 0, unit, pol);
             ptx::mbar_arrive_expect_tx(&bars[L::kBarVFull], L::kTileBytes);
-            for (int c = 0; c < kChunks; ++c)
-                ptx::tma_load_3d_hint(sV + c * L::kTileChunkBytes, mv, &bars[L::kBarVFull], c * kChunkElems, ti.row0,
-                                      unit, pol);
+            ptx::tma_load_4d_hint(sV, mv, &bars[L::kBarVFull], 0, ti.row0, 0, unit, pol);
         }
     }
 
@@ -365,18 +362,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     break;
                 }
                 ptx::mbar_arrive_expect_tx(&bars[L::kBarKFull + s], L::kTileBytes);
-                for (int c = 0; c < kChunks; ++c)
-                    ptx::tma_load_3d_hint(sK + s * L::kTileBytes + c * L::kTileChunkBytes, mk, &bars[L::kBarKFull + s],
-                                          c * kChunkElems, ti.row0, unit, pol);
+                ptx::tma_load_4d_hint(sK + s * L::kTileBytes, mk, &bars[L::kBarKFull + s], 0, ti.row0, 0, unit, pol);
                 k_issued = slot + 1;
                 if (n > 0 && !ptx::mbar_wait(&bars[L::kBarVEmpty + s], (n - 1) & 1, kWaitLimitNs)) {
                     failed = true;
                     break;
                 }
                 ptx::mbar_arrive_expect_tx(&bars[L::kBarVFull + s], L::kTileBytes);
-                for (int c = 0; c < kChunks; ++c)
-                    ptx::tma_load_3d_hint(sV + s * L::kTileBytes + c * L::kTileChunkBytes, mv, &bars[L::kBarVFull + s],
-                                          c * kChunkElems, ti.row0, unit, pol);
+                ptx::tma_load_4d_hint(sV + s * L::kTileBytes, mv, &bars[L::kBarVFull + s], 0, ti.row0, 0, unit, pol);
                 v_issued = slot + 1;
             }
             // Drain: every copy this thread issued must have landed before the

@@ -154,14 +154,24 @@ def ramp_case(top):
     return inp
 
 
-def test_lazy_rescale_path():
-    # x4 (the largest K multiplier of the workloads): every row rescales O
-    # at least once, some twice.
+def test_growing_logits():
+    # x4, the largest K multiplier of the workloads: every row rescales O at
+    # least once
     inp = ramp_case(4.0)
     o_ref, l_ref = ref(inp)
     for splits in (1, 2):
         out, lse, _ = run_gpu(inp, splits=splits)
         check_close(out, lse, o_ref, l_ref, f"ramp x4 splits={splits}")
+
+
+def test_lazy_rescale_path():
+    # K up to x40: the row maxima grow by far more than 2^8 over the prefix,
+    # so O and the sums are rescaled, most rows several times
+    inp = ramp_case(40.0)
+    o_ref, l_ref = ref(inp)
+    for splits in (1, 2):
+        out, lse, _ = run_gpu(inp, splits=splits)
+        check_close(out, lse, o_ref, l_ref, f"ramp x40 splits={splits}")
 
 
 def test_peaked_precision_model():

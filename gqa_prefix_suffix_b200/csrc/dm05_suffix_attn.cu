@@ -20,7 +20,7 @@
 namespace {
 
 constexpr int kTileRows = 64;
-constexpr int kStages = 2;
+constexpr int kStages = 3;
 using Layout = dm05::SmemLayout<kTileRows, kStages>;
 constexpr size_t kErrBytes = 256;        // error word (padded to one 256-byte segment)
 constexpr size_t kPartRowBytes = dm05::kHeadDim * 4 + 16;  // one partial row: D fp32 of O + float4 stats

@@ -21,16 +21,20 @@
 //     first tile's K/V before the valid_len read returns (the tile it would
 //     get if valid_len were P, which is nearly always the same one).
 //   * Warp roles: warp 8 issues TMA loads (Q once, then a ring of K and V
-//     tiles); warp 9 allocates TMEM and issues tcgen05 MMAs from one thread;
-//     warps 0-7 run the softmax: warps w and w+4 share TMEM lane quarter w
-//     (32 query rows) and each takes half of every tile's columns.
-//   * S = Q K^T goes to TMEM (three rotating buffers).  Each softmax thread
-//     reads half of its row with tcgen05.ld, applies the mask and the scale,
-//     combines its half's maximum with the partner warp's (shared memory and
-//     a bounded pair barrier), keeps the running max m and its half of the
-//     sums, and writes P (bf16) back into the same TMEM columns.  O += P V is a tcgen05 MMA with A = P read from TMEM and B
-//     = the V tile in shared memory (MN-major).  O (128 x 256 fp32) lives in
-//     TMEM for the whole pass.
+//     tiles); warp 9 allocates TMEM, copies Q from shared memory into TMEM
+//     (where it stays, so its shared memory becomes the ring's third
+//     stage) and issues tcgen05 MMAs from one thread; warps 0-7 run the
+//     softmax: warps w and w+4 share TMEM lane quarter w (32 query rows) and
+//     each takes half of every tile's columns.
+//   * S = Q K^T (A = Q from TMEM, B = the K tile in shared memory) goes to
+//     TMEM (two rotating buffers).  Each softmax thread reads half of its
+//     row with tcgen05.ld, applies the mask, combines its half's maximum
+//     with the partner warp's (shared memory and a bounded pair barrier),
+//     computes p = 2^(s * scale - m) with paired fp32 arithmetic, keeps the
+//     running max m and its half of the sums, and writes P (bf16) back into
+//     the same TMEM columns.  O += P V is a tcgen05 MMA with A = P read from
+//     TMEM and B = the V tile in shared memory (MN-major).  O (128 x 256
+//     fp32) lives in TMEM for the whole pass.
 //   * The running max is updated lazily: O and l are rescaled only when the
 //     tile max exceeds the current max by more than 2^8 (exact: O and l use
 //     the same stale max, and p <= 2^8 stays well inside fp32/bf16 range).
@@ -40,8 +44,9 @@
 //     (m, l, l_hat) to a workspace in L2 (one 1040-byte bulk TMA store per
 //     row); after one cluster barrier CTA r loads rows [r*GS/C, (r+1)*GS/C)
 //     of every partial with one bulk copy per partial and combines them by
-//     the log-sum-exp rule.  (Distributed shared memory was measured at ~10 GB/s per SM for
-//     this traffic, L2 through the TMA engine several times faster.)
+//     the log-sum-exp rule.  (Distributed shared memory, as loads and as
+//     bulk pushes, and plain stores and loads through L2 were measured
+//     slower for this traffic.)
 //   * Every wait is bounded (2 s): on time-out the kernel records
 //     DM05_EW_WAIT_TIMEOUT in the error word, drains its own copies and MMAs
 //     (again bounded), frees TMEM and returns.
@@ -65,8 +70,9 @@ constexpr int kMmaWarp = 9;
 constexpr int kThreads = 320;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemO = 0;                    // O: columns [0, 256)
-constexpr uint32_t kTmemS = 256;                  // S/P buffers: [256, 256 + kSBufs*NT)
-constexpr int kSBufs = 3;                         // S/P TMEM buffers in flight
+constexpr uint32_t kTmemQ = 256;                  // Q as bf16 pairs: columns [256, 384)
+constexpr uint32_t kTmemS = 384;                  // S/P buffers: [384, 384 + kSBufs*NT)
+constexpr int kSBufs = 2;                         // S/P TMEM buffers in flight
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait
 constexpr float kRescaleThreshold = 8.0f;         // log2 units: p <= 2^8 between rescales
 constexpr uint32_t kEwClamped = 0x1u;
@@ -94,13 +100,16 @@ struct SmemLayout {
     static constexpr int kQBytes = kChunks * kQChunkBytes;            // 64 KB
     static constexpr int kTileChunkBytes = NT * 128;
     static constexpr int kTileBytes = kChunks * kTileChunkBytes;      // NT * 512
-    static constexpr int kQOff = 0;
-    static constexpr int kKOff = kQBytes;
-    static constexpr int kVOff = kKOff + STAGES * kTileBytes;
-    static constexpr int kDataEnd = kVOff + STAGES * kTileBytes;
+    // ring stage s: the K tile at s * kStageBytes, the V tile right after it
+    static constexpr int kStageBytes = 2 * kTileBytes;
+    static constexpr int kDataEnd = STAGES * kStageBytes;
+    // Q lands in the last stage and stays there until it is copied to TMEM
+    static constexpr int kQOff = (STAGES - 1) * kStageBytes;
+    static_assert(kStageBytes >= kQBytes, "Q must fit in one ring stage");
     // barriers
     static constexpr int kBarQFull = 0;
-    static constexpr int kBarKFull = 1;
+    static constexpr int kBarQFree = kBarQFull + 1;         // Q copied to TMEM: its stage may be reused
+    static constexpr int kBarKFull = kBarQFree + 1;
     static constexpr int kBarKEmpty = kBarKFull + STAGES;
     static constexpr int kBarVFull = kBarKEmpty + STAGES;
     static constexpr int kBarVEmpty = kBarVFull + STAGES;
@@ -161,15 +170,13 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity)
     return __all_sync(0xffffffffu, ok);
 }
 
-// Packs two probabilities as bf16 (the MMA operand) and adds them to two
-// running sums: the rounded values (which normalise O, so that O is an exact
-// convex combination of V rows with the weights the MMA used) and the fp32
-// values (which give the LSE).
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi, float &sum_rounded, float &sum_exact)
+// Two probabilities rounded to bf16 (the MMA operand), low half = lo.  The
+// rounded values are summed too: they normalise O, so that O is an exact
+// convex combination of V rows with the weights the MMA used; the fp32
+// values give the LSE.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 {
     __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-    sum_rounded += __low2float(h) + __high2float(h);
-    sum_exact += lo + hi;
     return *reinterpret_cast<uint32_t *>(&h);
 }
 
@@ -245,6 +252,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---- set-up that reads no input (overlaps the previous kernel under PDL)
     if (threadIdx.x == 0) {
         ptx::mbar_init(&bars[L::kBarQFull], 1);
+        ptx::mbar_init(&bars[L::kBarQFree], 1);
         for (int s = 0; s < STAGES; ++s) {
             ptx::mbar_init(&bars[L::kBarKFull + s], 1);
             ptx::mbar_init(&bars[L::kBarKEmpty + s], 1);
@@ -283,8 +291,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::griddep_wait();
 
     uint8_t *sQ = smem + L::kQOff;
-    uint8_t *sK = smem + L::kKOff;
-    uint8_t *sV = smem + L::kVOff;
+    auto sK = [&](int s) { return smem + s * L::kStageBytes; };
+    auto sV = [&](int s) { return smem + s * L::kStageBytes + L::kTileBytes; };
     // This CTA's first tile if valid_len were P (the bucket): it does not
     // depend on valid_len, so its K/V are requested before that read returns.
     // With the suffix tiles first it is the true first tile unless the split
@@ -315,9 +323,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const CUtensorMap *mk = ti.prefix ? &tm_kp : &tm_ks;
             const CUtensorMap *mv = ti.prefix ? &tm_vp : &tm_vs;
             ptx::mbar_arrive_expect_tx(&bars[L::kBarKFull], L::kTileBytes);
-            ptx::tma_load_4d_hint(sK, mk, &bars[L::kBarKFull], 0, ti.row0, 0, unit, pol);
+            ptx::tma_load_4d_hint(sK(0), mk, &bars[L::kBarKFull], 0, ti.row0, 0, unit, pol);
             ptx::mbar_arrive_expect_tx(&bars[L::kBarVFull], L::kTileBytes);
-            ptx::tma_load_4d_hint(sV, mv, &bars[L::kBarVFull], 0, ti.row0, 0, unit, pol);
+            ptx::tma_load_4d_hint(sV(0), mv, &bars[L::kBarVFull], 0, ti.row0, 0, unit, pol);
         }
     }
 
@@ -361,15 +369,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                     failed = true;
                     break;
                 }
+                // the last stage first holds Q: wait until it is in TMEM
+                if (slot == STAGES - 1 && !ptx::mbar_wait(&bars[L::kBarQFree], 0, kWaitLimitNs)) {
+                    failed = true;
+                    break;
+                }
                 ptx::mbar_arrive_expect_tx(&bars[L::kBarKFull + s], L::kTileBytes);
-                ptx::tma_load_4d_hint(sK + s * L::kTileBytes, mk, &bars[L::kBarKFull + s], 0, ti.row0, 0, unit, pol);
+                ptx::tma_load_4d_hint(sK(s), mk, &bars[L::kBarKFull + s], 0, ti.row0, 0, unit, pol);
                 k_issued = slot + 1;
                 if (n > 0 && !ptx::mbar_wait(&bars[L::kBarVEmpty + s], (n - 1) & 1, kWaitLimitNs)) {
                     failed = true;
                     break;
                 }
                 ptx::mbar_arrive_expect_tx(&bars[L::kBarVFull + s], L::kTileBytes);
-                ptx::tma_load_4d_hint(sV + s * L::kTileBytes, mv, &bars[L::kBarVFull + s], 0, ti.row0, 0, unit, pol);
+                ptx::tma_load_4d_hint(sV(s), mv, &bars[L::kBarVFull + s], 0, ti.row0, 0, unit, pol);
                 v_issued = slot + 1;
             }
             // Drain: every copy this thread issued must have landed before the
@@ -385,15 +398,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0 && T > 0) {
             constexpr uint32_t idesc_pv = ptx::idesc_bf16_f32(kMRows, kHeadDim, true);
             const uint32_t q_base = ptx::smem_addr(sQ);
-            const uint32_t k_base = ptx::smem_addr(sK);
-            const uint32_t v_base = ptx::smem_addr(sV);
+            const uint32_t k_base = ptx::smem_addr(sK(0));
+            const uint32_t v_base = ptx::smem_addr(sV(0));
             auto issue_pv = [&](int u) -> bool {
                 const int s = (u + shift) % STAGES;
                 const int pb = u % kSBufs;
                 if (!ptx::mbar_wait(&bars[L::kBarPReady + pb], (u / kSBufs) & 1, kWaitLimitNs)) return false;
                 if (!ptx::mbar_wait(&bars[L::kBarVFull + s], ((u + shift) / STAGES) & 1, kWaitLimitNs)) return false;
                 ptx::tc_fence_after_sync();
-                const uint32_t vb = v_base + s * L::kTileBytes;
+                const uint32_t vb = v_base + s * L::kStageBytes;
                 const uint32_t p_tmem = tmem + kTmemS + pb * NT;
                 // only the 16-row k-steps that hold valid keys (a partial tile
                 // stops early; the rows after its last valid key up to the
@@ -414,6 +427,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 return true;
             };
             bool ok = ptx::mbar_wait(&bars[L::kBarQFull], 0, kWaitLimitNs);
+            if (ok) {
+                // Q -> TMEM once (row m to lane m, 16-column k-steps as 8
+                // columns of bf16 pairs: the A layout of the QK MMAs below),
+                // then the last ring stage is released to the producer.
+                ptx::tc_fence_after_sync();
+#pragma unroll
+                for (int kk = 0; kk < kHeadDim / 16; ++kk)
+                    ptx::tmem_cp_128x256b(tmem + kTmemQ + kk * 8,
+                                          ptx::sw128_desc(q_base + (kk >> 2) * L::kQChunkBytes + (kk & 3) * 32, 16, 1024));
+                ptx::mma_commit(&bars[L::kBarQFree]);
+            }
             for (int t = 0; t < T && ok; ++t) {
                 const int s = (t + shift) % STAGES;
                 const int sb = t % kSBufs;
@@ -430,7 +454,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     break;
                 }
                 ptx::tc_fence_after_sync();
-                const uint32_t kb = k_base + s * L::kTileBytes;
+                const uint32_t kb = k_base + s * L::kStageBytes;
                 const uint32_t d = tmem + kTmemS + sb * NT;
                 // N = the valid keys of the tile rounded up to 16; the
                 // softmax masks every column past the valid ones anyway.
@@ -441,9 +465,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // K-major, 128-byte swizzle: 16 elements = 32 bytes along
                     // the row; chunk kk/4 holds columns [64(kk/4), 64(kk/4)+64).
                     const uint32_t koff = (kk & 3) * 32;
-                    const uint64_t adesc = ptx::sw128_desc(q_base + (kk >> 2) * L::kQChunkBytes + koff, 16, 1024);
                     const uint64_t bdesc = ptx::sw128_desc(kb + (kk >> 2) * L::kTileChunkBytes + koff, 16, 1024);
-                    ptx::mma_bf16_ss(d, adesc, bdesc, idesc_qk, kk > 0 ? 1u : 0u);
+                    ptx::mma_bf16_ts(d, tmem + kTmemQ + kk * 8, bdesc, idesc_qk, kk > 0 ? 1u : 0u);
                 }
                 ptx::mma_commit(&bars[L::kBarKEmpty + s]);
                 ptx::mma_commit(&bars[L::kBarSFull + sb]);
@@ -498,23 +521,31 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::tmem_ld_wait();
 
             const TileInfo ti = tile_of<NT>(t_begin + t, TS, vl, p.S);
-            // visibility of this half's keys (same for every row)
-            uint32_t vis[NH / 32];
+            float s[NH];  // raw logits <q, k>; the scale is applied inside the exponent
 #pragma unroll
-            for (int w = 0; w < NH / 32; ++w) {
-                const int c = hf * NH + w * 32 + lane;
-                bool v = c < ti.n_valid;
-                if (v && ti.prefix && mask_row != nullptr) v = __ldg(mask_row + ti.row0 + c) != 0;
-                vis[w] = __ballot_sync(0xffffffffu, v);
-            }
-            float s[NH];
-            float hmax = -INFINITY;
+            for (int c = 0; c < NH; ++c) s[c] = __uint_as_float(raw[c / 16][c % 16]);
+            if (ti.n_valid < NT || (ti.prefix && mask_row != nullptr)) {
+                // keys of this half that are out of range or hidden (the same
+                // for every row) become -inf; a full tile without a mask has none
+                uint32_t vis[NH / 32];
 #pragma unroll
-            for (int c = 0; c < NH; ++c) {
-                const float x = __uint_as_float(raw[c / 16][c % 16]) * p.scale_log2;
-                s[c] = ((vis[c / 32] >> (c % 32)) & 1u) ? x : -INFINITY;
-                hmax = fmaxf(hmax, s[c]);
+                for (int w = 0; w < NH / 32; ++w) {
+                    const int c = hf * NH + w * 32 + lane;
+                    bool v = c < ti.n_valid;
+                    if (v && ti.prefix && mask_row != nullptr) v = __ldg(mask_row + ti.row0 + c) != 0;
+                    vis[w] = __ballot_sync(0xffffffffu, v);
+                }
+#pragma unroll
+                for (int c = 0; c < NH; ++c)
+                    if (!((vis[c / 32] >> (c % 32)) & 1u)) s[c] = -INFINITY;
             }
+            // four independent chains, then combined (max is exact in any order)
+            float m4[4] = {s[0], s[1], s[2], s[3]};
+#pragma unroll
+            for (int c = 4; c < NH; ++c) m4[c % 4] = fmaxf(m4[c % 4], s[c]);
+            float hmax = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+            // log2 units; rounding is monotone, so this is the max of the scaled logits
+            hmax *= p.scale_log2;
             // the row max over both halves
             xmax[((t & 1) * 2 + hf) * kMRows + row] = hmax;
             if (!pair_sync()) {
@@ -535,13 +566,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                 m_used = tmax;
             }
             const float msub = (m_used == -INFINITY) ? 0.0f : m_used;
-            float lsum = 0.0f, lhsum = 0.0f;
+            // p = 2^(s * scale - m) for a pair of columns at a time: the
+            // exponent argument and both running sums use paired fp32 ops
+            const uint64_t scale2 = ptx::f32x2(p.scale_log2, p.scale_log2);
+            const uint64_t nm2 = ptx::f32x2(-msub, -msub);
+            uint64_t l2 = ptx::f32x2(0.0f, 0.0f), lh2 = l2;
             uint32_t pk[NH / 2];
 #pragma unroll
-            for (int c = 0; c < NH; c += 2)
-                pk[c / 2] = pack_bf16x2(ptx::ex2(s[c] - msub), ptx::ex2(s[c + 1] - msub), lhsum, lsum);
-            l += lsum;
-            lh += lhsum;
+            for (int c = 0; c < NH; c += 2) {
+                const float2 a = ptx::unpack_f32x2(ptx::fma_f32x2(ptx::f32x2(s[c], s[c + 1]), scale2, nm2));
+                const float p0 = ptx::ex2(a.x), p1 = ptx::ex2(a.y);
+                const uint32_t hb = pack_bf16x2(p0, p1);
+                pk[c / 2] = hb;
+                l2 = ptx::add_f32x2(l2, ptx::f32x2(p0, p1));
+                lh2 = ptx::add_f32x2(lh2, ptx::f32x2(__uint_as_float(hb << 16), __uint_as_float(hb & 0xffff0000u)));
+            }
+            const float2 lp = ptx::unpack_f32x2(l2), lhp = ptx::unpack_f32x2(lh2);
+            l += lp.x + lp.y;
+            lh += lhp.x + lhp.y;
 #pragma unroll
             for (int j = 0; j < NH / 32; ++j) {
                 uint32_t chunk[16];
@@ -583,7 +625,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     failed = true;
                     break;
                 }
-                uint8_t *vt = sV + st * L::kTileBytes;
+                uint8_t *vt = sV(st);
                 const int rows = (ti.n_valid + 15) / 16 * 16 - ti.n_valid;  // read by the last PV k-step
                 const int units = kChunks * rows * 8;                       // 16-byte units
                 for (int i = tid; i < units; i += kSoftmaxWarps * 32) {

@@ -116,26 +116,21 @@ struct SmemLayout {
     static constexpr int kBarSFull = kBarVEmpty + STAGES;    // per S/P buffer
     static constexpr int kBarPReady = kBarSFull + kSBufs;    // per S/P buffer
     static constexpr int kBarPFree = kBarPReady + kSBufs;    // per S/P buffer
-    static constexpr int kBarODone = kBarPFree + kSBufs;
-    static constexpr int kBarMmaFinal = kBarODone + 1;
+    static constexpr int kBarMmaFinal = kBarPFree + kSBufs;
     static constexpr int kBarMerge = kBarMmaFinal + 1;
     static constexpr int kBarPair = kBarMerge + 1;          // per TMEM lane quarter: its 2 softmax warps
     static constexpr int kNumBars = kBarPair + 4;
     static constexpr int kBarOff = kDataEnd;
     static constexpr int kTmemSlotOff = kBarOff + kNumBars * 8;
-    // merge: weights of the rows this CTA reduces (at most
-    // splits * ceil(GS / splits) <= kMRows + 16 entries)
-    static constexpr int kMergeEntries = kMRows + 16;
-    static constexpr int kMergeWOff = (kTmemSlotOff + 16 + 15) / 16 * 16;
     // softmax half exchange: row maxima [2][2][128], sums [2][128] x 2
-    static constexpr int kXchgOff = kMergeWOff + kMergeEntries * 4;
+    static constexpr int kXchgOff = (kTmemSlotOff + 16 + 15) / 16 * 16;
     static constexpr int kEnd = kXchgOff + (4 + 2 + 2) * kMRows * 4;
     static constexpr int kAllocBytes = kEnd + 1024;                  // slack for 1 KB alignment
     // The merge stages up to 128 rows at kStageStride bytes, then receives
     // at most (128 + 16) rows of 1 KB, both inside the data region.
     static constexpr int kStageStride = kHeadDim * 4 + 16;           // padded: conflict-free row writes
     static_assert(kDataEnd >= kMRows * kStageStride, "staging area must fit in the data region");
-    static_assert(kDataEnd >= kMergeEntries * kStageStride, "receive area must fit in the data region");
+    static_assert(kDataEnd >= (kMRows + 16) * kStageStride, "receive area must fit in the data region");
 };
 
 struct TileInfo {
@@ -187,37 +182,53 @@ __device__ __forceinline__ size_t block_out_row(size_t unit_row0, int k, int nq,
     return unit_row0 + static_cast<size_t>(h) * S + q0 + (k - h * nq);
 }
 
-// out[row(k_lo + rr)][:] = bf16( sum_c w[c][rr] * recv[c][rr][:] ) for the
-// nr rows a CTA merges; the C partial rows are kStageStride bytes apart in
-// shared memory.
+// Combines the nr partial rows this CTA owns: partial c's row rr sits at
+// recv + (c * nr + rr) * kStageStride (D fp32 of unnormalised O, then
+// {m, l, l_hat, 0}).  One item per (row, 4-column quad); every item derives
+// its row's weights from the C statistics (a shared-memory broadcast within
+// the warp):
+//   M = max_c m_c,  w_c = 2^(m_c - M),  LH = sum_c l_hat_c w_c,  L = sum_c l_c w_c,
+//   out = sum_c w_c O_c / LH,  lse = (M + log2 L) ln 2.
+// A partial without visible keys (l_hat == 0) holds no O and gets no weight.
 template <int C, class L>
-__device__ __forceinline__ void merge_rows(const uint8_t *recv, const float *mw, int nr, __nv_bfloat16 *out,
+__device__ __forceinline__ void merge_rows(const uint8_t *recv, int nr, __nv_bfloat16 *out, float *lse,
                                            size_t unit_row0, int k_lo, int nq, int S, int q0)
 {
     const int items = nr * (kHeadDim / 4);
     for (int i = threadIdx.x; i < items; i += kThreads) {
         const int rr = i / (kHeadDim / 4), ch = i - rr * (kHeadDim / 4);
-        float w[C];
-        float4 v[C];
+        float4 st[C], v[C];
 #pragma unroll
         for (int c = 0; c < C; ++c) {
-            w[c] = mw[c * nr + rr];
-            v[c] = *reinterpret_cast<const float4 *>(recv + (c * nr + rr) * L::kStageStride + ch * 16);
+            const uint8_t *row = recv + (c * nr + rr) * L::kStageStride;
+            st[c] = *reinterpret_cast<const float4 *>(row + kHeadDim * 4);
+            v[c] = *reinterpret_cast<const float4 *>(row + ch * 16);
         }
+        float M = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < C; ++c)
+            if (st[c].z > 0.0f) M = fmaxf(M, st[c].x);
+        float Ls = 0.0f, LHs = 0.0f;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
         for (int c = 0; c < C; ++c) {
-            if (w[c] != 0.0f) {  // a partial without visible keys holds no valid O
-                acc.x += w[c] * v[c].x;
-                acc.y += w[c] * v[c].y;
-                acc.z += w[c] * v[c].z;
-                acc.w += w[c] * v[c].w;
+            if (st[c].z > 0.0f) {
+                const float w = ptx::ex2(st[c].x - M);
+                Ls += st[c].y * w;
+                LHs += st[c].z * w;
+                acc.x += w * v[c].x;
+                acc.y += w * v[c].y;
+                acc.z += w * v[c].z;
+                acc.w += w * v[c].w;
             }
         }
-        __nv_bfloat162 h0 = __floats2bfloat162_rn(acc.x, acc.y);
-        __nv_bfloat162 h1 = __floats2bfloat162_rn(acc.z, acc.w);
-        *reinterpret_cast<uint2 *>(out + block_out_row(unit_row0, k_lo + rr, nq, S, q0) * kHeadDim + ch * 4) =
+        const float inv = 1.0f / LHs;
+        __nv_bfloat162 h0 = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+        __nv_bfloat162 h1 = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+        const size_t orow = block_out_row(unit_row0, k_lo + rr, nq, S, q0);
+        *reinterpret_cast<uint2 *>(out + orow * kHeadDim + ch * 4) =
             make_uint2(*reinterpret_cast<uint32_t *>(&h0), *reinterpret_cast<uint32_t *>(&h1));
+        if (ch == 0 && lse != nullptr) lse[orow] = (M + ptx::lg2(Ls)) * 0.69314718055994531f;
     }
 }
 
@@ -264,7 +275,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::mbar_init(&bars[L::kBarPReady + i], kSoftmaxWarps * 32);
             ptx::mbar_init(&bars[L::kBarPFree + i], 1);
         }
-        ptx::mbar_init(&bars[L::kBarODone], 1);
         ptx::mbar_init(&bars[L::kBarMmaFinal], 1);
         ptx::mbar_init(&bars[L::kBarMerge], 1);
         for (int i = 0; i < 4; ++i) ptx::mbar_init(&bars[L::kBarPair + i], 64);
@@ -422,7 +432,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ptx::mma_bf16_ts(tmem + kTmemO, p_tmem + kk * 8, bdesc, idesc_pv, (u > 0 || kk > 0) ? 1u : 0u);
                 }
                 ptx::mma_commit(&bars[L::kBarVEmpty + s]);
-                ptx::mma_commit(&bars[L::kBarODone]);
                 ptx::mma_commit(&bars[L::kBarPFree + pb]);
                 return true;
             };
@@ -507,8 +516,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         float m_used = -INFINITY;
         float l = 0.0f;   // this half's sum of fp32 probabilities (for the LSE)
         float lh = 0.0f;  // this half's sum of bf16-rounded probabilities (for O)
+        // Prefix-mask bytes of this thread's columns of tile t (1 where no
+        // mask applies), requested one tile ahead so that their latency hides
+        // behind the previous tile instead of stalling the softmax.
+        uint32_t mask_next[NH / 32];
+        auto load_mask = [&](int t, uint32_t (&m)[NH / 32]) {
+#pragma unroll
+            for (int w = 0; w < NH / 32; ++w) m[w] = 1u;
+            if (mask_row == nullptr || t >= T) return;
+            const TileInfo tn = tile_of<NT>(t_begin + t, TS, vl, p.S);
+            if (!tn.prefix) return;
+#pragma unroll
+            for (int w = 0; w < NH / 32; ++w) {
+                const int c = hf * NH + w * 32 + lane;
+                if (c < tn.n_valid) m[w] = __ldg(mask_row + tn.row0 + c);
+            }
+        };
+        load_mask(0, mask_next);
         for (int t = 0; t < T; ++t) {
             const int sb = t % kSBufs;
+            uint32_t mask_cur[NH / 32];
+#pragma unroll
+            for (int w = 0; w < NH / 32; ++w) mask_cur[w] = mask_next[w];
+            load_mask(t + 1, mask_next);
             if (!warp_wait(&bars[L::kBarSFull + sb], (t / kSBufs) & 1)) {
                 failed = true;
                 break;
@@ -531,8 +561,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int w = 0; w < NH / 32; ++w) {
                     const int c = hf * NH + w * 32 + lane;
-                    bool v = c < ti.n_valid;
-                    if (v && ti.prefix && mask_row != nullptr) v = __ldg(mask_row + ti.row0 + c) != 0;
+                    const bool v = c < ti.n_valid && mask_cur[w] != 0u;
                     vis[w] = __ballot_sync(0xffffffffu, v);
                 }
 #pragma unroll
@@ -591,16 +620,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int e = 0; e < 16; ++e) chunk[e] = pk[j * 16 + e];
                 ptx::tmem_st16(scol + hf * (NH / 2) + j * 16, chunk);
             }
-            if (t > 0) {
-                // Every warp observes every PV completion in order (PV(t-1)
-                // here), so the single o_done barrier is never two phases
-                // ahead of a waiter and its parity is exact.  PV(t) cannot
-                // start before this warp arrives on p_ready below.
-                if (!warp_wait(&bars[L::kBarODone], (t - 1) & 1)) {
+            if (t > 0 && __any_sync(0xffffffffu, rescale_o)) {
+                // O must hold the sum through PV(t-1), the last PV issued
+                // (PV(t) waits for this warp's p_ready below): wait for its
+                // completion on the free barrier of its S/P buffer.  The
+                // parity is exact: PV(t-3), the previous use of that buffer,
+                // completed before QK(t) could start, and PV(t+1) cannot
+                // start before P(t+1) exists.
+                if (!warp_wait(&bars[L::kBarPFree + (t - 1) % kSBufs], ((t - 1) / kSBufs) & 1)) {
                     failed = true;
                     break;
                 }
-                if (__any_sync(0xffffffffu, rescale_o)) {
+                {
                     // this half's 128 columns of O (an all-zero O stays zero)
                     ptx::tc_fence_after_sync();
 #pragma unroll 1
@@ -651,7 +682,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const bool have_o = T > 0 && !failed;
         if (have_o) {
-            if (!warp_wait(&bars[L::kBarODone], (T - 1) & 1)) failed = true;
+            // the last PV (every earlier MMA completed before it)
+            if (!warp_wait(&bars[L::kBarPFree + (T - 1) % kSBufs], ((T - 1) / kSBufs) & 1)) failed = true;
             ptx::tc_fence_after_sync();
         }
         // row sums over both halves
@@ -746,7 +778,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int r_hi = (NR * (rank + 1)) / C;
         const int nr = r_hi - r_lo;
         const uint8_t *recv = smem;  // [C][nr] rows of kStageStride bytes
-        float *mw = reinterpret_cast<float *>(smem + L::kMergeWOff);  // [C][nr] weights
         if (nr > 0 && warp == 0) {
             if (lane == 0) ptx::mbar_arrive_expect_tx(&bars[L::kBarMerge], static_cast<uint32_t>(C * nr * L::kStageStride));
             __syncwarp();
@@ -760,31 +791,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (nr > 0) {
             if (!warp_wait(&bars[L::kBarMerge], 0)) failed = true;
-            // weights: one warp per row, lane c holds partial c
-            for (int rr = warp; rr < nr; rr += kThreads / 32) {
-                float4 st = make_float4(-INFINITY, 0.f, 0.f, 0.f);
-                if (lane < C) st = *reinterpret_cast<const float4 *>(recv + (lane * nr + rr) * L::kStageStride + kHeadDim * 4);
-                const bool has = lane < C && st.z > 0.0f;
-                float M = has ? st.x : -INFINITY;
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-                const float f = has ? ptx::ex2(st.x - M) : 0.0f;
-                float Ls = st.y * f, LHs = st.z * f;
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) {
-                    Ls += __shfl_xor_sync(0xffffffffu, Ls, o);
-                    LHs += __shfl_xor_sync(0xffffffffu, LHs, o);
-                }
-                if (lane < C) mw[lane * nr + rr] = f / LHs;
-                if (lane == 0 && p.lse != nullptr)
-                    p.lse[block_out_row(unit_row0, r_lo + rr, nq, p.S, q0)] = (M + ptx::lg2(Ls)) * 0.69314718055994531f;
-            }
-            __syncthreads();
             switch (C) {
-            case 2: merge_rows<2, L>(recv, mw, nr, p.out, unit_row0, r_lo, nq, p.S, q0); break;
-            case 4: merge_rows<4, L>(recv, mw, nr, p.out, unit_row0, r_lo, nq, p.S, q0); break;
-            case 8: merge_rows<8, L>(recv, mw, nr, p.out, unit_row0, r_lo, nq, p.S, q0); break;
-            default: merge_rows<16, L>(recv, mw, nr, p.out, unit_row0, r_lo, nq, p.S, q0); break;
+            case 2: merge_rows<2, L>(recv, nr, p.out, p.lse, unit_row0, r_lo, nq, p.S, q0); break;
+            case 4: merge_rows<4, L>(recv, nr, p.out, p.lse, unit_row0, r_lo, nq, p.S, q0); break;
+            case 8: merge_rows<8, L>(recv, nr, p.out, p.lse, unit_row0, r_lo, nq, p.S, q0); break;
+            default: merge_rows<16, L>(recv, nr, p.out, p.lse, unit_row0, r_lo, nq, p.S, q0); break;
             }
         }
     }

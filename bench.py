@@ -200,6 +200,115 @@ def host_bits(inp):
         v_suffix=bits(inp.v_suffix), prefix_valid_len=plain(inp.prefix_valid_len), prefix_mask=plain(inp.prefix_mask))
 
 
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def history_warm(args, dev, stream, bd):
+    """The history/long-prefix loop as the pages run it: one prefix cache on
+    the device, 10 sequential denoising-step calls with fresh suffix inputs,
+    replayed from one graph (the prefix stays warm in L2 across the steps)."""
+    import torch
+    from gqa_prefix_suffix_b200 import inputs as gen
+    steps = gen.WORKLOADS["history_loop"]()
+    d0 = steps[0].to(dev)
+    sets = []
+    for st in steps:
+        d = st.to(dev)
+        sets.append({"q": d.q, "ks": d.k_suffix, "vs": d.v_suffix,
+                     "out": torch.empty((st.B, st.Hq, st.S, st.D), dtype=torch.bfloat16, device=dev),
+                     "lse": torch.empty((st.B, st.Hq, st.S), dtype=torch.float32, device=dev)})
+    B, Hq, Hkv, P, S, D = d0.B, d0.Hq, d0.Hkv, d0.P, d0.S, d0.D
+    vl = d0.prefix_valid_len
+
+    def ten():
+        for t in sets:
+            rc = bd.dm05_suffix_attn(t["q"].data_ptr(), d0.k_prefix.data_ptr(),
+                                     d0.v_prefix.data_ptr(), None if vl is None else vl.data_ptr(), None,
+                                     t["ks"].data_ptr(), t["vs"].data_ptr(), t["out"].data_ptr(),
+                                     t["lse"].data_ptr(), B, Hq, Hkv, P, S, D, stream.cuda_stream)
+            if rc != 0:
+                raise bd.Dm05Error(rc, "dm05_suffix_attn")
+
+    with torch.cuda.stream(stream):
+        ten()
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        ten()
+    reps = 100
+    with torch.cuda.stream(stream):
+        g.replay()
+        ea = torch.cuda.Event(enable_timing=True)
+        eb = torch.cuda.Event(enable_timing=True)
+        ea.record(stream)
+        for _ in range(reps):
+            g.replay()
+        eb.record(stream)
+    stream.synchronize()
+    ms = ea.elapsed_time(eb)
+    del g
+    return {"warm_per_call": ms * 1e3 / (reps * len(sets)), "per_10_steps": ms * 1e3 / reps, "unit": UNIT,
+            "note": "one prefix kept on the device, 10 fresh suffix sets; value is the cold figure "
+                    "(prefix rotated through more than 2 x L2)"}
+
+
+def bucket_times(args, dev, stream, bd, l2):
+    """µs/call per prefix bucket of the sweep (5 calls per bucket with their
+    own valid lengths, copies rotated through more than 2 x L2)."""
+    import torch
+    from gqa_prefix_suffix_b200 import inputs as gen
+    calls = gen.WORKLOADS["bucket_sweep"]()
+    by_p = {}
+    for c in calls:
+        by_p.setdefault(c.P, []).append(c)
+    res = {}
+    for P, group in sorted(by_p.items()):
+        one = sum(t.numel() * t.element_size() for c in group for t in c.tensors().values() if t is not None)
+        copies = max(1, int(2 * l2 // max(1, one)) + 1)
+        sets = []
+        for _ in range(copies):
+            for c in group:
+                d = c.to(dev)
+                sets.append((d, torch.empty((d.B, d.Hq, d.S, d.D), dtype=torch.bfloat16, device=dev),
+                             torch.empty((d.B, d.Hq, d.S), dtype=torch.float32, device=dev)))
+
+        def run_all():
+            for d, o, l in sets:
+                rc = bd.dm05_suffix_attn(d.q.data_ptr(), d.k_prefix.data_ptr(), d.v_prefix.data_ptr(),
+                                         None if d.prefix_valid_len is None else d.prefix_valid_len.data_ptr(),
+                                         None, d.k_suffix.data_ptr(), d.v_suffix.data_ptr(), o.data_ptr(),
+                                         l.data_ptr(), d.B, d.Hq, d.Hkv, d.P, d.S, d.D, stream.cuda_stream)
+                if rc != 0:
+                    raise bd.Dm05Error(rc, "dm05_suffix_attn")
+
+        with torch.cuda.stream(stream):
+            run_all()
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            run_all()
+        with torch.cuda.stream(stream):
+            g.replay()
+            ea = torch.cuda.Event(enable_timing=True)
+            eb = torch.cuda.Event(enable_timing=True)
+            ea.record(stream)
+            for _ in range(10):
+                g.replay()
+            eb.record(stream)
+        stream.synchronize()
+        res[str(P)] = ea.elapsed_time(eb) * 1e3 / (10 * len(sets))
+        del g, sets
+    return {"us_per_call": res, "calls_per_bucket": len(calls) // max(1, len(by_p))}
+
+
 def cpu_oracle_rate(inp, seconds, threads):
     """Times the fp64 oracle on bounded samples of query rows of this workload
     and scales to a full call.  Returns (us per full call, rows timed, calls)."""
@@ -356,25 +465,26 @@ def main():
         g_rem.replay()
     stream.synchronize()
 
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
+    # one event between consecutive replays: the total spans all K calls, and
+    # each replay gives one sample of the per-call time for the spread
+    replays = [(g_full, chunk)] * n_full + ([(g_rem, rem)] if g_rem is not None else [])
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(replays) + 1)]
     if pg is not None:
         pg.barrier()
     torch.cuda.synchronize()
     sampler = ClockSampler(dev)
     with sampler:
         with torch.cuda.stream(stream):
-            e0.record(stream)
-            for _ in range(n_full):
-                g_full.replay()
-            if g_rem is not None:
-                g_rem.replay()
-            e1.record(stream)
+            evs[0].record(stream)
+            for i, (g, _) in enumerate(replays):
+                g.replay()
+                evs[i + 1].record(stream)
         stream.synchronize()
     torch.cuda.synchronize()
     if pg is not None:
         pg.barrier()
-    t_ms = e0.elapsed_time(e1)
+    t_ms = evs[0].elapsed_time(evs[-1])
+    per_replay = sorted(evs[i].elapsed_time(evs[i + 1]) * 1e3 / n for i, (_, n) in enumerate(replays))
     if pg is not None:
         tt = torch.tensor([t_ms], device=dev)
         pg.all_reduce(tt, op=pg.ReduceOp.MAX)
@@ -382,6 +492,51 @@ def main():
     rc, word = bd.dm05_get_error_word(sh)
     if word != 0:
         raise SystemExit(f"kernel error word {word:#x}")
+
+    def pct(xs, q):
+        return xs[min(len(xs) - 1, max(0, int(round(q * (len(xs) - 1)))))]
+
+    latency = {"median": statistics.median(per_replay), "p10": pct(per_replay, 0.1), "p90": pct(per_replay, 0.9),
+               "replays": len(per_replay), "unit": UNIT}
+    # a single call launched on its own (no graph, no neighbour to overlap with)
+    singles = []
+    for i in range(20):
+        ea = torch.cuda.Event(enable_timing=True)
+        eb = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            ea.record(stream)
+            call(sets[i % R])
+            eb.record(stream)
+        stream.synchronize()
+        singles.append(ea.elapsed_time(eb) * 1e3)
+    latency["eager_single"] = statistics.median(singles)
+    # the launch floor of this machine: a graph of 1000 one-element kernels
+    z = torch.zeros(1, device=dev)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            z.add_(1.0)
+    stream.synchronize()
+    g_floor = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_floor, stream=stream):
+        for _ in range(1000):
+            z.add_(1.0)
+    with torch.cuda.stream(stream):
+        g_floor.replay()
+        ea = torch.cuda.Event(enable_timing=True)
+        eb = torch.cuda.Event(enable_timing=True)
+        ea.record(stream)
+        for _ in range(3):
+            g_floor.replay()
+        eb.record(stream)
+    stream.synchronize()
+    latency["launch_floor"] = ea.elapsed_time(eb) * 1e3 / 3000
+    del g_floor
+
+    extra = {}
+    if args.workload == "history_loop":
+        extra["history"] = history_warm(args, dev, stream, bd)
+    if args.workload == "bucket_sweep":
+        extra["buckets"] = bucket_times(args, dev, stream, bd, l2)
 
     us_per_call_device = t_ms * 1e3 / K          # one GPU's time per call
     value = t_ms * 1e3 / (K * world)              # whole-job time per call
@@ -435,6 +590,11 @@ def main():
         cpu = {"value": us, "unit": UNIT, "cores": threads, "kind": "oracle",
                "sample": f"{rows} query rows of {inp.name} in {n} oracle calls (~{args.cpu_seconds:.0f} s), "
                          f"fp64, scaled to a full call of {B * Hq * S} rows"}
+        one_s = min(3.0, args.cpu_seconds)
+        us1, rows1, _ = cpu_oracle_rate(inp, one_s, 1)
+        cpu["value_1_thread"] = us1
+        cpu["sample_1_thread"] = f"{rows1} query rows on 1 thread (~{one_s:.0f} s), scaled the same way"
+        cpu["cpu_model"] = cpu_model()
 
     clocks = sampler.summary()
     if rank == 0:
@@ -455,7 +615,9 @@ def main():
                     "steps": E},
             "gpu_launches": K,
             "clocks": clocks,
+            "latency": latency,
         }
+        line.update(extra)
         if cpu is not None:
             line["cpu_baseline"] = cpu
         print(json.dumps(line), flush=True)

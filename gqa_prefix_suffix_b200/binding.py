@@ -25,7 +25,8 @@ DM05_EW_WAIT_TIMEOUT = 0x2
 
 EXPORTS = ("dm05_suffix_attn", "dm05_suffix_attn_workspace_bytes", "dm05_suffix_attn_reserve",
            "dm05_suffix_attn_plan", "dm05_set_split_override", "dm05_get_error_word",
-           "dm05_status_string", "dm05_release", "dm05_suffix_attn_noalloc")
+           "dm05_status_string", "dm05_release", "dm05_suffix_attn_noalloc", "dm05_suffix_attn_host",
+           "dm05_suffix_attn_host_copy_bytes")
 
 _lock = threading.Lock()
 _lib = None
@@ -66,6 +67,10 @@ def lib() -> ctypes.CDLL:
             L.dm05_release.restype = None
             L.dm05_suffix_attn_noalloc.argtypes = [p] * 9 + [i] * 6 + [p]
             L.dm05_suffix_attn_noalloc.restype = i
+            L.dm05_suffix_attn_host.argtypes = [p] * 9 + [i] * 6 + [p]
+            L.dm05_suffix_attn_host.restype = i
+            L.dm05_suffix_attn_host_copy_bytes.argtypes = [p] + [i] * 8 + [ctypes.POINTER(sz)] * 2
+            L.dm05_suffix_attn_host_copy_bytes.restype = i
             _lib = L
     return _lib
 
@@ -84,6 +89,22 @@ def dm05_suffix_attn_noalloc(q, k_prefix, v_prefix, prefix_valid_len, prefix_mas
     device memory); same arguments as dm05_suffix_attn."""
     return lib().dm05_suffix_attn_noalloc(q, k_prefix, v_prefix, prefix_valid_len, prefix_mask, k_suffix,
                                           v_suffix, out, lse, B, Hq, Hkv, P, S, D, stream)
+
+
+def dm05_suffix_attn_host(q, k_prefix, v_prefix, prefix_valid_len, prefix_mask, k_suffix, v_suffix,
+                          out, lse, B, Hq, Hkv, P, S, D, stream) -> int:
+    """The host-buffer entry point: every pointer is a host address."""
+    return lib().dm05_suffix_attn_host(q, k_prefix, v_prefix, prefix_valid_len, prefix_mask, k_suffix,
+                                       v_suffix, out, lse, B, Hq, Hkv, P, S, D, stream)
+
+
+def dm05_suffix_attn_host_copy_bytes(prefix_valid_len, has_prefix_mask, want_lse, B, Hq, Hkv, P, S, D):
+    """Returns (status, host-to-device bytes, device-to-host bytes) of one
+    dm05_suffix_attn_host call; prefix_valid_len is a host address or None."""
+    h, d = ctypes.c_size_t(0), ctypes.c_size_t(0)
+    rc = lib().dm05_suffix_attn_host_copy_bytes(prefix_valid_len, int(bool(has_prefix_mask)), int(bool(want_lse)),
+                                                B, Hq, Hkv, P, S, D, ctypes.byref(h), ctypes.byref(d))
+    return rc, int(h.value), int(d.value)
 
 
 def dm05_suffix_attn_workspace_bytes(B, Hq, Hkv, P, S, D) -> int:
@@ -166,6 +187,49 @@ def suffix_attn(q, k_prefix, v_prefix, k_suffix, v_suffix, prefix_valid_len=None
                           _stream_handle(stream))
     if rc != DM05_OK:
         raise Dm05Error(rc, "dm05_suffix_attn")
+    return out, lse
+
+
+def suffix_attn_host(q, k_prefix, v_prefix, k_suffix, v_suffix, prefix_valid_len=None, prefix_mask=None,
+                     out=None, lse=None, want_lse: bool = True, stream=None):
+    """Suffix attention on CPU torch tensors (page-locked for asynchronous
+    copies) through dm05_suffix_attn_host; returns (out, lse or None), host
+    tensors that hold the result once `stream` has passed the call.
+
+    Shapes and dtypes are those of suffix_attn; every tensor, out and lse
+    included, must be a contiguous CPU tensor."""
+    import torch
+    B, Hq, S, D = q.shape
+    Hkv, P = k_prefix.shape[1], k_prefix.shape[2]
+    for name, t, dt in (("q", q, torch.bfloat16), ("k_prefix", k_prefix, torch.bfloat16),
+                        ("v_prefix", v_prefix, torch.bfloat16), ("k_suffix", k_suffix, torch.bfloat16),
+                        ("v_suffix", v_suffix, torch.bfloat16)):
+        if t.is_cuda or t.dtype != dt or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CPU {dt} tensor")
+    if tuple(k_prefix.shape) != (B, Hkv, P, D) or tuple(v_prefix.shape) != (B, Hkv, P, D):
+        raise ValueError("k_prefix/v_prefix must be [B,Hkv,P,D]")
+    if tuple(k_suffix.shape) != (B, Hkv, S, D) or tuple(v_suffix.shape) != (B, Hkv, S, D):
+        raise ValueError("k_suffix/v_suffix must be [B,Hkv,S,D]")
+    if prefix_valid_len is not None and (prefix_valid_len.is_cuda or prefix_valid_len.dtype != torch.int32
+                                         or prefix_valid_len.numel() != B or not prefix_valid_len.is_contiguous()):
+        raise ValueError("prefix_valid_len must be a contiguous CPU int32 tensor of B values")
+    if prefix_mask is not None and (prefix_mask.is_cuda or prefix_mask.dtype != torch.uint8
+                                    or tuple(prefix_mask.shape) != (B, P) or not prefix_mask.is_contiguous()):
+        raise ValueError("prefix_mask must be a contiguous CPU uint8 tensor [B,P]")
+    pin = q.is_pinned()
+    if out is None:
+        out = torch.empty((B, Hq, S, D), dtype=torch.bfloat16, pin_memory=pin)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq, S), dtype=torch.float32, pin_memory=pin)
+    for name, t, shape, dt in (("out", out, (B, Hq, S, D), torch.bfloat16), ("lse", lse, (B, Hq, S), torch.float32)):
+        if t is not None and (t.is_cuda or t.dtype != dt or tuple(t.shape) != shape or not t.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous CPU {dt} tensor {list(shape)}")
+    ptr = lambda t: None if t is None else t.data_ptr()
+    rc = dm05_suffix_attn_host(ptr(q), ptr(k_prefix), ptr(v_prefix), ptr(prefix_valid_len), ptr(prefix_mask),
+                               ptr(k_suffix), ptr(v_suffix), ptr(out), ptr(lse), B, Hq, Hkv, P, S, D,
+                               _stream_handle(stream))
+    if rc != DM05_OK:
+        raise Dm05Error(rc, "dm05_suffix_attn_host")
     return out, lse
 
 

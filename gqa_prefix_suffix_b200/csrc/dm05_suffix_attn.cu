@@ -47,6 +47,7 @@ struct StreamWorkspace {
 std::mutex g_mu;
 std::vector<DeviceState> g_dev;
 std::vector<StreamWorkspace> g_ws;
+std::vector<StreamWorkspace> g_stage;  // device copies of host-buffer calls, per (device, stream)
 int g_split_override = 0;
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
@@ -245,6 +246,71 @@ int stream_workspace(cudaStream_t stream, size_t need, void **out)
     }
     *out = w->base;
     return DM05_OK;
+}
+
+// Device staging buffer of (current device, stream) for the host-buffer
+// entry point, at least `need` bytes.  Caller holds g_mu and has checked that
+// the stream is not capturing.
+int stream_staging(cudaStream_t stream, size_t need, uint8_t **out)
+{
+    *out = nullptr;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return DM05_ERR_CUDA;
+    StreamWorkspace *w = nullptr;
+    for (auto &e : g_stage)
+        if (e.dev == dev && e.stream == stream) w = &e;
+    if (w == nullptr) {
+        g_stage.push_back(StreamWorkspace{});
+        w = &g_stage.back();
+        w->dev = dev;
+        w->stream = stream;
+    }
+    if (w->bytes < need) {
+        if (w->base != nullptr) {
+            cudaFree(w->base);  // waits for the device: no earlier call still reads it
+            w->base = nullptr;
+            w->bytes = 0;
+        }
+        void *p = nullptr;
+        if (cudaMalloc(&p, need) != cudaSuccess) return DM05_ERR_CUDA;
+        w->base = p;
+        w->bytes = need;
+    }
+    *out = static_cast<uint8_t *>(w->base);
+    return DM05_OK;
+}
+
+// Places of the tensors in the staging buffer (256-byte aligned offsets).
+struct StageLayout {
+    size_t q, kp, vp, ks, vs, out, lse, vl, mask, total;
+};
+
+StageLayout stage_layout(int B, int Hq, int Hkv, int P, int S, int D)
+{
+    auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+    const size_t row = static_cast<size_t>(D) * 2;
+    StageLayout L{};
+    size_t o = 0;
+    L.q = o;    o += up(static_cast<size_t>(B) * Hq * S * row);
+    L.kp = o;   o += up(static_cast<size_t>(B) * Hkv * P * row);
+    L.vp = o;   o += up(static_cast<size_t>(B) * Hkv * P * row);
+    L.ks = o;   o += up(static_cast<size_t>(B) * Hkv * S * row);
+    L.vs = o;   o += up(static_cast<size_t>(B) * Hkv * S * row);
+    L.out = o;  o += up(static_cast<size_t>(B) * Hq * S * row);
+    L.lse = o;  o += up(static_cast<size_t>(B) * Hq * S * 4);
+    L.vl = o;   o += up(static_cast<size_t>(B) * 4);
+    L.mask = o; o += up(static_cast<size_t>(B) * P);
+    L.total = o;
+    return L;
+}
+
+// Prefix rows [0, n) of sample b that a host-buffer call copies: the clamped
+// valid length, or every row when there is no valid-length array.
+int host_rows(const int32_t *valid_len, int b, int P)
+{
+    if (valid_len == nullptr) return P;
+    const int32_t v = valid_len[b];
+    return v < 0 ? 0 : v > P ? P : static_cast<int>(v);
 }
 
 // bf16 tensor [d2][d1][256] viewed as 4-D [d2][d1][4][64]: the 4 column
@@ -451,6 +517,96 @@ int dm05_suffix_attn(const void *q, const void *k_prefix, const void *v_prefix, 
     return DM05_OK;
 }
 
+int dm05_suffix_attn_host_copy_bytes(const int32_t *prefix_valid_len, int has_prefix_mask, int want_lse, int B,
+                                     int Hq, int Hkv, int P, int S, int D, size_t *h2d_bytes, size_t *d2h_bytes)
+{
+    int rc = check_sizes(B, Hq, Hkv, P, S, D);
+    if (rc != DM05_OK) return rc;
+    const size_t row = static_cast<size_t>(D) * 2;
+    size_t in = static_cast<size_t>(B) * Hq * S * row + 2 * static_cast<size_t>(B) * Hkv * S * row;
+    for (int b = 0; b < B; ++b) in += 2 * static_cast<size_t>(Hkv) * host_rows(prefix_valid_len, b, P) * row;
+    if (prefix_valid_len != nullptr) in += static_cast<size_t>(B) * 4;
+    if (has_prefix_mask) in += static_cast<size_t>(B) * P;
+    size_t outb = static_cast<size_t>(B) * Hq * S * row;
+    if (want_lse) outb += static_cast<size_t>(B) * Hq * S * 4;
+    if (h2d_bytes) *h2d_bytes = in;
+    if (d2h_bytes) *d2h_bytes = outb;
+    return DM05_OK;
+}
+
+int dm05_suffix_attn_host(const void *q, const void *k_prefix, const void *v_prefix, const int32_t *prefix_valid_len,
+                          const uint8_t *prefix_mask, const void *k_suffix, const void *v_suffix, void *out,
+                          float *lse, int B, int Hq, int Hkv, int P, int S, int D, cudaStream_t stream)
+{
+    if (!q || !k_suffix || !v_suffix || !out) return DM05_ERR_NULL;
+    if (P > 0 && (!k_prefix || !v_prefix)) return DM05_ERR_NULL;
+    int rc = check_sizes(B, Hq, Hkv, P, S, D);
+    if (rc != DM05_OK) return rc;
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) return DM05_ERR_CUDA;
+    if (cs != cudaStreamCaptureStatusNone) return DM05_ERR_UNSUPPORTED;  // valid lengths are read now
+
+    const StageLayout L = stage_layout(B, Hq, Hkv, P, S, D);
+    uint8_t *dv = nullptr;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        rc = stream_staging(stream, L.total, &dv);
+        if (rc != DM05_OK) return rc;
+    }
+    const size_t row = static_cast<size_t>(D) * 2;
+    const size_t q_bytes = static_cast<size_t>(B) * Hq * S * row;
+    const size_t suf_bytes = static_cast<size_t>(B) * Hkv * S * row;
+    auto h2d = [&](size_t off, const void *src, size_t n) {
+        return n == 0 || cudaMemcpyAsync(dv + off, src, n, cudaMemcpyHostToDevice, stream) == cudaSuccess;
+    };
+    bool ok = h2d(L.q, q, q_bytes) && h2d(L.ks, k_suffix, suf_bytes) && h2d(L.vs, v_suffix, suf_bytes);
+    if (ok && prefix_valid_len != nullptr) ok = h2d(L.vl, prefix_valid_len, static_cast<size_t>(B) * 4);
+    if (ok && prefix_mask != nullptr) ok = h2d(L.mask, prefix_mask, static_cast<size_t>(B) * P);
+    // Prefix K/V: rows [0, clamped valid length) of every (sample, KV head);
+    // the kernel reads no row past it.  Runs of samples whose whole bucket is
+    // in range are copied as one contiguous block; any other sample as one
+    // 2-D copy per tensor (Hkv slabs of n rows at a pitch of P rows).
+    const size_t pitch = static_cast<size_t>(P) * row;
+    const size_t sample = static_cast<size_t>(Hkv) * pitch;
+    const bool pitch_ok = pitch <= static_cast<size_t>(INT32_MAX);
+    int run0 = 0;  // first sample of the pending run of whole-bucket samples
+    for (int b = 0; ok && P > 0 && b <= B; ++b) {
+        const int n = b < B ? host_rows(prefix_valid_len, b, P) : -1;
+        if (n == P) continue;
+        if (b > run0) {
+            const size_t off = static_cast<size_t>(run0) * sample, len = static_cast<size_t>(b - run0) * sample;
+            ok = h2d(L.kp + off, static_cast<const uint8_t *>(k_prefix) + off, len) &&
+                 h2d(L.vp + off, static_cast<const uint8_t *>(v_prefix) + off, len);
+        }
+        run0 = b + 1;
+        if (!ok || n <= 0) continue;
+        const size_t off = static_cast<size_t>(b) * sample, width = static_cast<size_t>(n) * row;
+        for (int t = 0; ok && t < 2; ++t) {
+            const uint8_t *src = static_cast<const uint8_t *>(t == 0 ? k_prefix : v_prefix) + off;
+            uint8_t *dst = dv + (t == 0 ? L.kp : L.vp) + off;
+            if (pitch_ok) {
+                ok = cudaMemcpy2DAsync(dst, pitch, src, pitch, width, static_cast<size_t>(Hkv),
+                                       cudaMemcpyHostToDevice, stream) == cudaSuccess;
+            } else {
+                for (int h = 0; ok && h < Hkv; ++h)
+                    ok = cudaMemcpyAsync(dst + h * pitch, src + h * pitch, width, cudaMemcpyHostToDevice, stream) ==
+                         cudaSuccess;
+            }
+        }
+    }
+    if (!ok) return DM05_ERR_CUDA;
+    rc = dm05_suffix_attn(dv + L.q, P > 0 ? dv + L.kp : nullptr, P > 0 ? dv + L.vp : nullptr,
+                          prefix_valid_len ? reinterpret_cast<const int32_t *>(dv + L.vl) : nullptr,
+                          prefix_mask ? dv + L.mask : nullptr, dv + L.ks, dv + L.vs, dv + L.out,
+                          lse ? reinterpret_cast<float *>(dv + L.lse) : nullptr, B, Hq, Hkv, P, S, D, stream);
+    if (rc != DM05_OK) return rc;
+    if (cudaMemcpyAsync(out, dv + L.out, q_bytes, cudaMemcpyDeviceToHost, stream) != cudaSuccess) return DM05_ERR_CUDA;
+    if (lse != nullptr && cudaMemcpyAsync(lse, dv + L.lse, static_cast<size_t>(B) * Hq * S * 4,
+                                          cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+        return DM05_ERR_CUDA;
+    return DM05_OK;
+}
+
 }  // extern "C"
 
 // ---------------------------------------------------------------------------
@@ -621,6 +777,10 @@ void dm05_release(void)
         if (w.base != nullptr && cudaSetDevice(w.dev) == cudaSuccess) cudaFree(w.base);
     }
     g_ws.clear();
+    for (auto &w : g_stage) {
+        if (w.base != nullptr && cudaSetDevice(w.dev) == cudaSuccess) cudaFree(w.base);
+    }
+    g_stage.clear();
     if (have_cur) cudaSetDevice(cur);
 }
 

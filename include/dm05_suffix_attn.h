@@ -162,6 +162,53 @@ int dm05_suffix_attn_noalloc(const void *q, const void *k_prefix, const void *v_
                              int B, int Hq, int Hkv, int P, int S, int D,
                              cudaStream_t stream);
 
+/*
+ * dm05_suffix_attn_host -- the same attention with every tensor in HOST
+ * memory: the call for a caller whose inputs are on the host and who wants
+ * the result back there (one request at a time, as a control loop issues
+ * them).  The source pages have no counterpart; it exists so that a whole
+ * request (copies in, attention, copies out) is one library call.
+ *
+ * Arguments, sizes and results are those of dm05_suffix_attn, but q,
+ * k_prefix, v_prefix, prefix_valid_len, prefix_mask, k_suffix, v_suffix,
+ * out and lse are host addresses; no alignment is required.  The call
+ * enqueues on `stream`, in order: host-to-device copies of the inputs into a
+ * staging buffer the library owns per (device, stream), the attention
+ * kernel, and device-to-host copies of out (and of lse unless it is NULL).
+ *
+ * prefix_valid_len is read on the host during the call: only the prefix
+ * rows [0, clamp(prefix_valid_len[b], 0, P)) of each sample are copied
+ * (every row when it is NULL), since no other row is used.  The clamp is
+ * flagged in the error word as in dm05_suffix_attn.
+ *
+ * With page-locked host buffers (cudaHostAlloc / cudaHostRegister) every
+ * copy is asynchronous: the inputs must stay unchanged, and out / lse must
+ * not be read, until `stream` has passed the call (cudaStreamSynchronize).
+ * Pageable buffers also work, but the CUDA runtime then blocks the host
+ * inside the copies.
+ *
+ * The staging buffer is allocated (cudaMalloc) by the first call with these
+ * sizes on the stream, grows when sizes grow (cudaFree, which waits for the
+ * device) and is freed by dm05_release.  The call cannot be captured into a
+ * CUDA graph (it reads valid lengths on the host): on a capturing stream it
+ * returns DM05_ERR_UNSUPPORTED and enqueues nothing.
+ */
+int dm05_suffix_attn_host(const void *q, const void *k_prefix, const void *v_prefix,
+                          const int32_t *prefix_valid_len, const uint8_t *prefix_mask,
+                          const void *k_suffix, const void *v_suffix,
+                          void *out, float *lse,
+                          int B, int Hq, int Hkv, int P, int S, int D,
+                          cudaStream_t stream);
+
+/* Bytes one dm05_suffix_attn_host call with these arguments copies to the
+ * device (*h2d_bytes) and back to the host (*d2h_bytes).  prefix_valid_len
+ * is the same host array (or NULL); has_prefix_mask and want_lse say whether
+ * prefix_mask and lse would be non-NULL.  Host-only: touches no device.
+ * Either output pointer may be NULL. */
+int dm05_suffix_attn_host_copy_bytes(const int32_t *prefix_valid_len, int has_prefix_mask, int want_lse,
+                                     int B, int Hq, int Hkv, int P, int S, int D,
+                                     size_t *h2d_bytes, size_t *d2h_bytes);
+
 /* Synchronises `stream`, then returns in *host_word the error bits
  * (DM05_EW_*) that kernels on the current device set since the last read,
  * and clears them. */
@@ -170,8 +217,8 @@ int dm05_get_error_word(cudaStream_t stream, uint32_t *host_word);
 /* Human-readable name of a dm05_status value. */
 const char *dm05_status_string(int status);
 
-/* Frees every workspace the library holds (all devices).  No call may be in
- * flight. */
+/* Frees every workspace and staging buffer the library holds (all
+ * devices).  No call may be in flight. */
 void dm05_release(void);
 
 #ifdef __cplusplus

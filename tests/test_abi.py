@@ -111,3 +111,74 @@ def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(bd, "_lib", None)
     with pytest.raises(RuntimeError, match="missing"):
         bd.lib()
+
+
+def call_host(**kw):
+    a = dict(q=FAKE, k_prefix=FAKE, v_prefix=FAKE, prefix_valid_len=None, prefix_mask=None,
+             k_suffix=FAKE, v_suffix=FAKE, out=FAKE, lse=None, B=1, Hq=8, Hkv=4, P=1024, S=50, D=256,
+             stream=None)
+    a.update(kw)
+    return bd.dm05_suffix_attn_host(a["q"], a["k_prefix"], a["v_prefix"], a["prefix_valid_len"],
+                                    a["prefix_mask"], a["k_suffix"], a["v_suffix"], a["out"], a["lse"],
+                                    a["B"], a["Hq"], a["Hkv"], a["P"], a["S"], a["D"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), bd.DM05_ERR_NULL),
+    (dict(out=None), bd.DM05_ERR_NULL),
+    (dict(v_prefix=None), bd.DM05_ERR_NULL),
+    (dict(B=0), bd.DM05_ERR_SHAPE),
+    (dict(Hq=6), bd.DM05_ERR_SHAPE),
+    (dict(D=128), bd.DM05_ERR_UNSUPPORTED),
+    (dict(S=65), bd.DM05_ERR_UNSUPPORTED),
+])
+def test_host_entry_checks_reject(lib, kw, status):
+    # the host-buffer entry point checks its arguments before any CUDA call
+    assert call_host(**kw) == status
+
+
+def test_host_entry_takes_unaligned_host_buffers(lib):
+    # host addresses need no alignment: an odd address passes the checks and
+    # the call reaches CUDA (absent here)
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("would copy from fake host addresses on a GPU")
+    assert call_host(q=FAKE + 2, out=FAKE + 6, lse=FAKE + 1) == bd.DM05_ERR_CUDA
+
+
+def expected_copy_bytes(valid_len, has_mask, want_lse, B, Hq, Hkv, P, S, D):
+    """Bytes the host entry point moves, counted tensor by tensor: Q and the
+    suffix K/V whole, the prefix K/V rows below the clamped valid length, the
+    valid-length and mask arrays when given; O (and the LSE) back."""
+    row = D * 2
+    rows = [P] * B if valid_len is None else [min(max(int(v), 0), P) for v in valid_len]
+    h2d = B * Hq * S * row                      # q
+    h2d += 2 * B * Hkv * S * row                # k_suffix, v_suffix
+    h2d += sum(2 * Hkv * n * row for n in rows)  # k_prefix, v_prefix rows in range
+    h2d += 0 if valid_len is None else 4 * B
+    h2d += B * P if has_mask else 0
+    d2h = B * Hq * S * row + (B * Hq * S * 4 if want_lse else 0)
+    return h2d, d2h
+
+
+@pytest.mark.parametrize("valid_len,has_mask,want_lse,B,P,S", [
+    (None, False, True, 1, 1024, 50),
+    ([900], False, True, 1, 1024, 50),
+    ([900], True, False, 1, 1024, 50),
+    ([0], False, True, 1, 576, 10),
+    ([-5, 2000, 700, 1024], True, True, 4, 1024, 50),   # clamped both ways
+    (None, False, False, 2, 0, 10),
+])
+def test_host_copy_bytes(lib, valid_len, has_mask, want_lse, B, P, S):
+    arr = None
+    if valid_len is not None:
+        arr = (ctypes.c_int32 * B)(*valid_len)
+    rc, h2d, d2h = bd.dm05_suffix_attn_host_copy_bytes(
+        None if arr is None else ctypes.addressof(arr), has_mask, want_lse, B, 8, 4, P, S, 256)
+    assert rc == bd.DM05_OK
+    assert (h2d, d2h) == expected_copy_bytes(valid_len, has_mask, want_lse, B, 8, 4, P, S, 256)
+
+
+def test_host_copy_bytes_checks_sizes(lib):
+    assert bd.dm05_suffix_attn_host_copy_bytes(None, 0, 1, 1, 8, 4, 1024, 50, 128)[0] == bd.DM05_ERR_UNSUPPORTED
+    assert bd.dm05_suffix_attn_host_copy_bytes(None, 0, 1, 0, 8, 4, 1024, 50, 256)[0] == bd.DM05_ERR_SHAPE

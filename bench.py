@@ -173,6 +173,23 @@ class ClockSampler:
                 "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
 
 
+def max_over_ranks(dist, value, device):
+    """The largest of the ranks' values (each rank passes its own); the value
+    itself when there is no process group."""
+    if dist is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_us_per_call(max_ms, calls_per_rank, world):
+    """Whole-job time per call: the slowest rank's time over every call that
+    all replicas made."""
+    return max_ms * 1e3 / (calls_per_rank * world)
+
+
 def dist_setup():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -487,10 +504,7 @@ def main():
         pg.barrier()
     t_ms = evs[0].elapsed_time(evs[-1])
     per_replay = sorted(evs[i].elapsed_time(evs[i + 1]) * 1e3 / n for i, (_, n) in enumerate(replays))
-    if pg is not None:
-        tt = torch.tensor([t_ms], device=dev)
-        pg.all_reduce(tt, op=pg.ReduceOp.MAX)
-        t_ms = float(tt.item())
+    t_ms = max_over_ranks(pg, t_ms, dev)
     rc, word = bd.dm05_get_error_word(sh)
     if word != 0:
         raise SystemExit(f"kernel error word {word:#x}")
@@ -541,7 +555,7 @@ def main():
         extra["buckets"] = bucket_times(args, dev, stream, bd, l2)
 
     us_per_call_device = t_ms * 1e3 / K          # one GPU's time per call
-    value = t_ms * 1e3 / (K * world)              # whole-job time per call
+    value = whole_job_us_per_call(t_ms, K, world)  # whole-job time per call
     achieved = kv_bytes / (us_per_call_device * 1e-6) / 1e9
     peak, peak_kind = measured_peaks()
 
@@ -581,12 +595,8 @@ def main():
         evs[c + 1].record(stream)
     stream.synchronize()
     chunk_us = sorted(evs[c].elapsed_time(evs[c + 1]) * 1e3 / per for c in range(n_chunks))
-    e2e_us = chunk_us[len(chunk_us) // 2]
-    if pg is not None:
-        tt = torch.tensor([e2e_us], device=dev)
-        pg.all_reduce(tt, op=pg.ReduceOp.MAX)
-        e2e_us = float(tt.item())
-    e2e_value = e2e_us / world
+    e2e_us = max_over_ranks(pg, chunk_us[len(chunk_us) // 2], dev)
+    e2e_value = whole_job_us_per_call(e2e_us / 1e3, 1, world)
     E = per * n_chunks
 
     cpu = None

@@ -304,6 +304,32 @@ StageLayout stage_layout(int B, int Hq, int Hkv, int P, int S, int D)
     return L;
 }
 
+// Device address of the host buffer [p, p + n) when the device can store to
+// all of it directly (page-locked memory mapped into the device's address
+// space, as every cudaHostAlloc / cudaMallocHost buffer is on a 64-bit
+// system) and p has the alignment the kernel's stores need; else nullptr.
+// Both ends must be mapped and map n - 1 bytes apart, so a buffer that runs
+// off its allocation is never written from the device.
+void *device_view(void *p, size_t n, size_t align)
+{
+    if (p == nullptr || n == 0 || reinterpret_cast<uintptr_t>(p) % align != 0) return nullptr;
+    uint8_t *first = static_cast<uint8_t *>(p);
+    uint8_t *last = first + (n - 1);
+    cudaPointerAttributes a{}, z{};
+    if (cudaPointerGetAttributes(&a, first) != cudaSuccess || cudaPointerGetAttributes(&z, last) != cudaSuccess) {
+        cudaGetLastError();  // an unknown pointer is not an error of the call
+        return nullptr;
+    }
+    if (a.type != cudaMemoryTypeHost || z.type != cudaMemoryTypeHost || a.devicePointer == nullptr ||
+        z.devicePointer == nullptr)
+        return nullptr;
+    if (static_cast<uint8_t *>(z.devicePointer) - static_cast<uint8_t *>(a.devicePointer) !=
+        static_cast<ptrdiff_t>(n - 1))
+        return nullptr;
+    if (reinterpret_cast<uintptr_t>(a.devicePointer) % align != 0) return nullptr;
+    return a.devicePointer;
+}
+
 // Prefix rows [0, n) of sample b that a host-buffer call copies: the clamped
 // valid length, or every row when there is no valid-length array.
 int host_rows(const int32_t *valid_len, int b, int P)
@@ -595,14 +621,21 @@ int dm05_suffix_attn_host(const void *q, const void *k_prefix, const void *v_pre
         }
     }
     if (!ok) return DM05_ERR_CUDA;
+    // O and the LSE go from the kernel straight into the caller's buffers
+    // when the device can address both; otherwise through the staging buffer
+    // and a copy back.
+    const size_t lse_bytes = static_cast<size_t>(B) * Hq * S * 4;
+    void *out_dev = device_view(out, q_bytes, 16);
+    void *lse_dev = lse != nullptr ? device_view(lse, lse_bytes, 4) : nullptr;
+    const bool direct = out_dev != nullptr && (lse == nullptr || lse_dev != nullptr);
     rc = dm05_suffix_attn(dv + L.q, P > 0 ? dv + L.kp : nullptr, P > 0 ? dv + L.vp : nullptr,
                           prefix_valid_len ? reinterpret_cast<const int32_t *>(dv + L.vl) : nullptr,
-                          prefix_mask ? dv + L.mask : nullptr, dv + L.ks, dv + L.vs, dv + L.out,
-                          lse ? reinterpret_cast<float *>(dv + L.lse) : nullptr, B, Hq, Hkv, P, S, D, stream);
-    if (rc != DM05_OK) return rc;
+                          prefix_mask ? dv + L.mask : nullptr, dv + L.ks, dv + L.vs, direct ? out_dev : dv + L.out,
+                          lse == nullptr ? nullptr : static_cast<float *>(direct ? lse_dev : dv + L.lse), B, Hq, Hkv,
+                          P, S, D, stream);
+    if (rc != DM05_OK || direct) return rc;
     if (cudaMemcpyAsync(out, dv + L.out, q_bytes, cudaMemcpyDeviceToHost, stream) != cudaSuccess) return DM05_ERR_CUDA;
-    if (lse != nullptr && cudaMemcpyAsync(lse, dv + L.lse, static_cast<size_t>(B) * Hq * S * 4,
-                                          cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+    if (lse != nullptr && cudaMemcpyAsync(lse, dv + L.lse, lse_bytes, cudaMemcpyDeviceToHost, stream) != cudaSuccess)
         return DM05_ERR_CUDA;
     return DM05_OK;
 }

@@ -187,6 +187,13 @@ int dm05_suffix_attn_noalloc(const void *q, const void *k_prefix, const void *v_
  * Pageable buffers also work, but the CUDA runtime then blocks the host
  * inside the copies.
  *
+ * When out (16-byte aligned) and lse (if not NULL) are page-locked memory
+ * that the device can address (cudaHostAlloc / cudaMallocHost on a 64-bit
+ * system, or cudaHostRegister with cudaHostRegisterMapped), the kernel
+ * stores O and the LSE into them directly and no copy back is enqueued;
+ * otherwise both come back from the staging buffer by copies.  out and lse
+ * must each lie inside one allocation.
+ *
  * The staging buffer is allocated (cudaMalloc) by the first call with these
  * sizes on the stream, grows when sizes grow (cudaFree, which waits for the
  * device) and is freed by dm05_release.  The call cannot be captured into a

@@ -161,3 +161,39 @@ def test_host_copy_bytes_match_the_copies():
     kv = int(rows.sum()) * 4 * 2 * 512
     assert h2d == inp.q.numel() * 2 + inp.k_suffix.numel() * 4 + kv + 4 * inp.B + inp.prefix_mask.numel()
     assert d2h == inp.q.numel() * 2 + inp.B * 8 * inp.S * 4
+
+
+def pinned_view(shape, dtype, offset, pad=256, fill=0xA5):
+    """A contiguous view at byte `offset` inside a larger page-locked buffer
+    filled with a guard pattern; returns (view, whole buffer)."""
+    n = int(np.prod(shape)) * torch.empty((), dtype=dtype).element_size()
+    buf = torch.full((offset + n + pad,), fill, dtype=torch.uint8).pin_memory()
+    return buf[offset:offset + n].view(dtype).view(shape), buf
+
+
+@pytest.mark.parametrize("out_off,lse_off,pin_lse", [
+    (16, 4, True),      # device writes O and the LSE straight into the views
+    (48, 12, True),
+    (8, 4, True),       # O not 16-byte aligned: staging and a copy back
+    (16, 4, False),     # LSE pageable: staging and a copy back for both
+])
+def test_host_entry_output_buffers(out_off, lse_off, pin_lse):
+    inp = make_case(*CASES[5])
+    B, Hq, S = inp.B, inp.Hq, inp.S
+    h = {k: (None if v is None else v.pin_memory()) for k, v in inp.tensors().items()}
+    out, out_buf = pinned_view((B, Hq, S, 256), torch.bfloat16, out_off)
+    if pin_lse:
+        lse, lse_buf = pinned_view((B, Hq, S), torch.float32, lse_off)
+    else:
+        lse_buf = torch.full((lse_off + B * Hq * S * 4 + 256,), 0xA5, dtype=torch.uint8)
+        lse = lse_buf[lse_off:lse_off + B * Hq * S * 4].view(torch.float32).view(B, Hq, S)
+    bd.suffix_attn_host(h["q"], h["k_prefix"], h["v_prefix"], h["k_suffix"], h["v_suffix"],
+                        prefix_valid_len=h["prefix_valid_len"], prefix_mask=h["prefix_mask"], out=out, lse=lse)
+    torch.cuda.synchronize()
+    o_d, l_d, _ = run_gpu(inp)
+    assert same_bits(out, o_d)
+    assert torch.equal(lse, l_d)
+    n_out = out.numel() * 2
+    assert (out_buf[:out_off] == 0xA5).all() and (out_buf[out_off + n_out:] == 0xA5).all()
+    n_lse = lse.numel() * 4
+    assert (lse_buf[:lse_off] == 0xA5).all() and (lse_buf[lse_off + n_lse:] == 0xA5).all()

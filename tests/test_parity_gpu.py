@@ -324,3 +324,33 @@ def test_batched_mask():
     out, lse, _ = run_gpu(inp)
     mx, mean = check_close(out, lse, *ref(inp), what=inp.name)
     assert math.isfinite(mx)
+
+
+# ---------------------------------------------------------------- size limits
+
+def test_longest_prefix():
+    # P = 65535, the longest prefix the supported range is read to cover:
+    # 1024 key tiles per (sample, KV head), the last one ragged (63 rows)
+    inp = gen.make_inputs(1, 8, 4, 65535, 4, 256, 61, valid_len=65535, mask_frac=0.02)
+    plan = bd.dm05_suffix_attn_plan(1, 8, 4, 65535, 4, 256)
+    assert plan[0] == 0
+    out, lse, word = run_gpu(inp)
+    assert word == 0
+    check_close(out, lse, *ref(inp), what=f"P=65535 plan {plan[1:]}")
+
+
+def test_many_units_several_waves():
+    # 1024 (sample, KV head) units: one CTA each, about seven waves on 148 SMs
+    inp = gen.make_inputs(256, 8, 4, 256, 10, 256, 62, valid_range=(0, 256), mask_frac=0.1)
+    out, lse, word = run_gpu(inp)
+    assert word == 0
+    check_close(out, lse, *ref(inp), what="B=256")
+
+
+def test_long_prefix_every_split():
+    # a long valid range cut 1..16 ways: up to 469 tiles per CTA
+    inp = gen.make_inputs(1, 8, 4, 30016, 16, 256, 63, valid_len=30001, peak_frac=0.01, peak_mult=4.0)
+    o_ref, l_ref = ref(inp)
+    for splits in (1, 4, 16):
+        out, lse, _ = run_gpu(inp, splits=splits)
+        check_close(out, lse, o_ref, l_ref, f"P=30016 splits={splits}")

@@ -197,3 +197,16 @@ def test_host_entry_output_buffers(out_off, lse_off, pin_lse):
     assert (out_buf[:out_off] == 0xA5).all() and (out_buf[out_off + n_out:] == 0xA5).all()
     n_lse = lse.numel() * 4
     assert (lse_buf[:lse_off] == 0xA5).all() and (lse_buf[lse_off + n_lse:] == 0xA5).all()
+
+
+def test_release_then_call_again():
+    # dm05_release frees the staging buffers and workspaces; the next calls
+    # (host and device entry points) allocate them again
+    inp = make_case(*CASES[0])
+    o1, l1, _ = run_host(inp)
+    torch.cuda.synchronize()
+    bd.dm05_release()
+    o2, l2, _ = run_host(inp)
+    o3, l3, _ = run_gpu(inp)
+    assert same_bits(o1, o2) and torch.equal(l1, l2)
+    assert same_bits(o2, o3) and torch.equal(l2, l3)

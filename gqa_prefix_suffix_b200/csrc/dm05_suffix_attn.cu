@@ -461,7 +461,8 @@ int dm05_suffix_attn(const void *q, const void *k_prefix, const void *v_prefix, 
     const int GS = G * S;
     const int units = B * Hkv;
 
-    DeviceState *ds = nullptr;
+    DeviceState *ds = nullptr;  // points into g_dev: used only while g_mu is held
+    uint32_t *err_word = nullptr;
     Plan pl;
     void *part_ws = nullptr;
     {
@@ -477,6 +478,7 @@ int dm05_suffix_attn(const void *q, const void *k_prefix, const void *v_prefix, 
             if (rc != DM05_OK) return rc;
         }
         pl = make_plan(B, Hq, Hkv, P, S, *ds);
+        err_word = ds->err;
         rc = stream_workspace(stream, partial_bytes(units, pl, G), &part_ws);
         if (rc != DM05_OK) return rc;
     }
@@ -508,7 +510,7 @@ int dm05_suffix_attn(const void *q, const void *k_prefix, const void *v_prefix, 
     kp.mask = prefix_mask;
     kp.out = static_cast<__nv_bfloat16 *>(out);
     kp.lse = lse;
-    kp.err = ds->err;
+    kp.err = err_word;
     kp.part = static_cast<float *>(part_ws);
     kp.Hkv = Hkv;
     kp.P = P;

@@ -13,6 +13,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <thread>
 #include <vector>
 
 #include "suffix_attn_kernel.cuh"
@@ -36,13 +37,20 @@ struct DeviceState {
 };
 
 // Partial-result workspace of one (device, stream): concurrent streams never
-// share one.
+// share one.  cudaStreamPerThread is a different stream on every thread, so
+// for that handle the calling thread is part of the key.
 struct StreamWorkspace {
     int dev = -1;
     cudaStream_t stream = nullptr;
+    std::thread::id thread;  // default (no thread) unless stream == cudaStreamPerThread
     void *base = nullptr;
     size_t bytes = 0;
 };
+
+std::thread::id stream_owner(cudaStream_t stream)
+{
+    return stream == cudaStreamPerThread ? std::this_thread::get_id() : std::thread::id();
+}
 
 std::mutex g_mu;
 std::vector<DeviceState> g_dev;
@@ -220,14 +228,16 @@ int stream_workspace(cudaStream_t stream, size_t need, void **out)
     if (need == 0) return DM05_OK;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return DM05_ERR_CUDA;
+    const std::thread::id owner = stream_owner(stream);
     StreamWorkspace *w = nullptr;
     for (auto &e : g_ws)
-        if (e.dev == dev && e.stream == stream) w = &e;
+        if (e.dev == dev && e.stream == stream && e.thread == owner) w = &e;
     if (w == nullptr) {
         g_ws.push_back(StreamWorkspace{});
         w = &g_ws.back();
         w->dev = dev;
         w->stream = stream;
+        w->thread = owner;
     }
     if (w->bytes < need) {
         cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
@@ -256,14 +266,16 @@ int stream_staging(cudaStream_t stream, size_t need, uint8_t **out)
     *out = nullptr;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return DM05_ERR_CUDA;
+    const std::thread::id owner = stream_owner(stream);
     StreamWorkspace *w = nullptr;
     for (auto &e : g_stage)
-        if (e.dev == dev && e.stream == stream) w = &e;
+        if (e.dev == dev && e.stream == stream && e.thread == owner) w = &e;
     if (w == nullptr) {
         g_stage.push_back(StreamWorkspace{});
         w = &g_stage.back();
         w->dev = dev;
         w->stream = stream;
+        w->thread = owner;
     }
     if (w->bytes < need) {
         if (w->base != nullptr) {

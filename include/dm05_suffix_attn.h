@@ -28,7 +28,9 @@
  * Ownership: the caller owns every tensor.  The library keeps no pointer
  * after a call returns.  The library owns an error word per device and, per
  * (device, stream), a workspace for the partial results of split calls (at
- * most dm05_suffix_attn_workspace_bytes).  They are created by
+ * most dm05_suffix_attn_workspace_bytes); for the handle cudaStreamPerThread
+ * the calling thread is part of the key, since that handle names a different
+ * stream on every thread.  They are created by
  * dm05_suffix_attn_reserve or by a dm05_suffix_attn that runs outside stream
  * capture, grow only outside capture, and are freed by dm05_release.
  *

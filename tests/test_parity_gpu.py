@@ -354,3 +354,47 @@ def test_long_prefix_every_split():
     for splits in (1, 4, 16):
         out, lse, _ = run_gpu(inp, splits=splits)
         check_close(out, lse, o_ref, l_ref, f"P=30016 splits={splits}")
+
+
+def test_per_thread_streams_from_two_threads():
+    # cudaStreamPerThread is a different stream on each thread: two threads
+    # issuing split calls through it at the same time must not share a
+    # workspace.  Every result must equal the single-threaded one bit for bit.
+    import threading
+    cases = [gen.make_inputs(1, 8, 4, 1024, 50, 256, 71, valid_len=900),
+             gen.make_inputs(2, 8, 4, 640, 30, 256, 72, valid_range=(0, 640), mask_frac=0.1)]
+    refs = [run_gpu(c)[:2] for c in cases]
+    per_thread = 2  # cudaStreamPerThread
+    n_calls = 30
+    devs = [c.to("cuda") for c in cases]
+    outs = [[(torch.empty_like(d.q), torch.empty(d.q.shape[:3], dtype=torch.float32, device="cuda"))
+             for _ in range(n_calls)] for d in devs]
+    torch.cuda.synchronize()
+    ptr = lambda x: None if x is None else x.data_ptr()
+    errors = []
+
+    def worker(i):
+        try:
+            d = devs[i]
+            B, Hq, S, D = d.q.shape
+            for o, l in outs[i]:
+                rc = bd.dm05_suffix_attn(ptr(d.q), ptr(d.k_prefix), ptr(d.v_prefix), ptr(d.prefix_valid_len),
+                                         ptr(d.prefix_mask), ptr(d.k_suffix), ptr(d.v_suffix), ptr(o), ptr(l),
+                                         B, Hq, d.k_prefix.shape[1], d.k_prefix.shape[2], S, D, per_thread)
+                assert rc == 0, rc
+            rc, word = bd.dm05_get_error_word(per_thread)  # synchronises this thread's stream
+            assert rc == 0 and word == 0, (rc, word)
+        except Exception as e:  # reported below
+            errors.append(e)
+
+    threads = [threading.Thread(target=worker, args=(i,)) for i in range(2)]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join(timeout=120)
+    torch.cuda.synchronize()
+    assert not errors, errors
+    for i in range(2):
+        for o, l in outs[i]:
+            assert torch.equal(o.cpu().view(torch.int16), refs[i][0].view(torch.int16))
+            assert torch.equal(l.cpu(), refs[i][1])

@@ -26,7 +26,7 @@ DM05_EW_WAIT_TIMEOUT = 0x2
 EXPORTS = ("dm05_suffix_attn", "dm05_suffix_attn_workspace_bytes", "dm05_suffix_attn_reserve",
            "dm05_suffix_attn_plan", "dm05_set_split_override", "dm05_get_error_word",
            "dm05_status_string", "dm05_release", "dm05_suffix_attn_noalloc", "dm05_suffix_attn_host",
-           "dm05_suffix_attn_host_copy_bytes")
+           "dm05_suffix_attn_host_copy_bytes", "dm05_selftest_wait_timeout")
 
 _lock = threading.Lock()
 _lib = None
@@ -71,6 +71,8 @@ def lib() -> ctypes.CDLL:
             L.dm05_suffix_attn_host.restype = i
             L.dm05_suffix_attn_host_copy_bytes.argtypes = [p] + [i] * 8 + [ctypes.POINTER(sz)] * 2
             L.dm05_suffix_attn_host_copy_bytes.restype = i
+            L.dm05_selftest_wait_timeout.argtypes = [i, p]
+            L.dm05_selftest_wait_timeout.restype = i
             _lib = L
     return _lib
 
@@ -124,6 +126,11 @@ def dm05_suffix_attn_plan(B, Hq, Hkv, P, S, D):
 
 def dm05_set_split_override(splits_per_head: int) -> int:
     return lib().dm05_set_split_override(splits_per_head)
+
+
+def dm05_selftest_wait_timeout(limit_ms: int, stream) -> int:
+    """Launches the bounded-wait self-test (a wait that must run out)."""
+    return lib().dm05_selftest_wait_timeout(limit_ms, stream)
 
 
 def dm05_get_error_word(stream):

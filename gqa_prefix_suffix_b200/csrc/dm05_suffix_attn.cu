@@ -258,6 +258,20 @@ int stream_workspace(cudaStream_t stream, size_t need, void **out)
     return DM05_OK;
 }
 
+// Failure-detection self-test: one thread waits, with the attention
+// kernel's bounded wait, on a barrier that nothing arrives on (phase 0 of a
+// fresh barrier never completes), and records the time-out in the error word
+// as the attention kernel does.
+__global__ void wait_timeout_selftest_kernel(uint32_t *err, uint64_t limit_ns)
+{
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        dm05::ptx::mbar_init(&bar, 1);
+        dm05::ptx::fence_mbar_init();
+        if (!dm05::ptx::mbar_wait(&bar, 0, limit_ns)) atomicOr(err, dm05::kEwTimeout);
+    }
+}
+
 // Device staging buffer of (current device, stream) for the host-buffer
 // entry point, at least `need` bytes.  Caller holds g_mu and has checked that
 // the stream is not capturing.
@@ -555,6 +569,24 @@ int dm05_suffix_attn(const void *q, const void *k_prefix, const void *v_prefix, 
     cfg.numAttrs = na;
     if (cudaLaunchKernelEx(&cfg, kKernel, tm_q, tm_kp, tm_vp, tm_ks, tm_vs, kp) != cudaSuccess) return DM05_ERR_CUDA;
     return DM05_OK;
+}
+
+int dm05_selftest_wait_timeout(int limit_ms, cudaStream_t stream)
+{
+    if (limit_ms < 1 || limit_ms > 2000) return DM05_ERR_SHAPE;
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) return DM05_ERR_CUDA;
+    if (cs != cudaStreamCaptureStatusNone) return DM05_ERR_UNSUPPORTED;
+    uint32_t *err = nullptr;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        DeviceState *ds = nullptr;
+        const int rc = device_state(true, &ds);
+        if (rc != DM05_OK) return rc;
+        err = ds->err;
+    }
+    wait_timeout_selftest_kernel<<<1, 32, 0, stream>>>(err, static_cast<uint64_t>(limit_ms) * 1000000ull);
+    return cudaGetLastError() == cudaSuccess ? DM05_OK : DM05_ERR_CUDA;
 }
 
 int dm05_suffix_attn_host_copy_bytes(const int32_t *prefix_valid_len, int has_prefix_mask, int want_lse, int B,

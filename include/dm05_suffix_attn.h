@@ -218,6 +218,19 @@ int dm05_suffix_attn_host_copy_bytes(const int32_t *prefix_valid_len, int has_pr
                                      int B, int Hq, int Hkv, int P, int S, int D,
                                      size_t *h2d_bytes, size_t *d2h_bytes);
 
+/*
+ * dm05_selftest_wait_timeout -- exercises the failure detection without a
+ * GPU fault.  It launches, on `stream`, one thread that waits on a barrier
+ * nothing completes, with the same bounded wait every kernel wait uses but a
+ * limit of limit_ms milliseconds (1..2000); the wait gives up and sets
+ * DM05_EW_WAIT_TIMEOUT in the device error word, as an attention kernel
+ * whose wait ran out does, and the kernel returns normally.  Read the word
+ * with dm05_get_error_word.  Creates the error word if needed, so it must not
+ * be called on a capturing stream (DM05_ERR_UNSUPPORTED).  Returns
+ * DM05_ERR_SHAPE for a limit out of range.
+ */
+int dm05_selftest_wait_timeout(int limit_ms, cudaStream_t stream);
+
 /* Synchronises `stream`, then returns in *host_word the error bits
  * (DM05_EW_*) that kernels on the current device set since the last read,
  * and clears them. */

@@ -182,3 +182,11 @@ def test_host_copy_bytes(lib, valid_len, has_mask, want_lse, B, P, S):
 def test_host_copy_bytes_checks_sizes(lib):
     assert bd.dm05_suffix_attn_host_copy_bytes(None, 0, 1, 1, 8, 4, 1024, 50, 128)[0] == bd.DM05_ERR_UNSUPPORTED
     assert bd.dm05_suffix_attn_host_copy_bytes(None, 0, 1, 0, 8, 4, 1024, 50, 256)[0] == bd.DM05_ERR_SHAPE
+
+
+def test_selftest_wait_timeout_checks_its_limit(lib):
+    for bad in (0, -1, 2001):
+        assert bd.dm05_selftest_wait_timeout(bad, None) == bd.DM05_ERR_SHAPE
+    import torch
+    if not torch.cuda.is_available():
+        assert bd.dm05_selftest_wait_timeout(10, None) == bd.DM05_ERR_CUDA  # no device here

@@ -398,3 +398,24 @@ def test_per_thread_streams_from_two_threads():
         for o, l in outs[i]:
             assert torch.equal(o.cpu().view(torch.int16), refs[i][0].view(torch.int16))
             assert torch.equal(l.cpu(), refs[i][1])
+
+
+def test_wait_timeout_is_reported_and_the_context_stays_usable():
+    # A wait that runs out (a barrier nothing completes, 50 ms limit) sets
+    # DM05_EW_WAIT_TIMEOUT and returns; the next attention call on the same
+    # context then runs normally with a clean error word.
+    s = torch.cuda.Stream()
+    sh = s.cuda_stream
+    assert bd.dm05_get_error_word(sh)[0] == 0  # clears earlier bits
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    assert bd.dm05_selftest_wait_timeout(50, sh) == 0
+    e1.record(s)
+    rc, word = bd.dm05_get_error_word(sh)
+    assert rc == 0 and word & bd.DM05_EW_WAIT_TIMEOUT, word
+    assert e0.elapsed_time(e1) >= 45.0
+    inp = gen.make_inputs(1, 8, 4, 200, 10, 256, 81, valid_len=150)
+    out, lse, word = run_gpu(inp)
+    assert word == 0
+    check_close(out, lse, *ref(inp), what="after a wait time-out")

@@ -30,6 +30,12 @@ MUTATIONS = {
     "merge_weight_sign": ("double w = exp(l - total);", "double w = exp(total - l);"),
     "dot_drops_last_term": ("for (int d = 0; d < D; ++d)\n            dot +=",
                             "for (int d = 0; d < D - 1; ++d)\n            dot +="),
+    "lse_in_log2": ("double lse = m + log(z);", "double lse = m + log2(z);"),
+    "query_head_modulo_kv_heads": ("const int h = (int)((row / S) % Hq);",
+                                   "const int h = (int)((row / S) % Hkv);"),
+    "normaliser_without_max": ("z += exp(logit_buf[x - key_lo] - m);", "z += exp(logit_buf[x - key_lo]);"),
+    "scale_one_over_d": ("const double scale = 1.0 / sqrt((double)D);", "const double scale = 1.0 / (double)D;"),
+    "merge_total_is_max": ("double total = m + log(z);", "double total = m;"),
     "merge_skips_first_part": ("for (int s = 0; s < n_parts; ++s) {\n            double l = lse_parts[(size_t)s * rows + r];\n            if (l == -INFINITY) continue;",
                                "for (int s = 1; s < n_parts; ++s) {\n            double l = lse_parts[(size_t)s * rows + r];\n            if (l == -INFINITY) continue;"),
 }

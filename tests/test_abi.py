@@ -190,3 +190,35 @@ def test_selftest_wait_timeout_checks_its_limit(lib):
     import torch
     if not torch.cuda.is_available():
         assert bd.dm05_selftest_wait_timeout(10, None) == bd.DM05_ERR_CUDA  # no device here
+
+
+def _host_inputs(B=1, Hq=8, Hkv=4, P=64, S=10, D=256):
+    import torch
+    bf = torch.bfloat16
+    return dict(q=torch.zeros(B, Hq, S, D, dtype=bf), k_prefix=torch.zeros(B, Hkv, P, D, dtype=bf),
+                v_prefix=torch.zeros(B, Hkv, P, D, dtype=bf), k_suffix=torch.zeros(B, Hkv, S, D, dtype=bf),
+                v_suffix=torch.zeros(B, Hkv, S, D, dtype=bf))
+
+
+def _bad_host_argument(case):
+    """One argument of a suffix_attn_host call made wrong, by name."""
+    import torch
+    return {
+        "q": dict(q=torch.zeros(1, 8, 10, 256)),                                   # fp32
+        "k_prefix": dict(k_prefix=torch.zeros(1, 4, 32, 256, dtype=torch.bfloat16)),  # P mismatch
+        "v_suffix": dict(v_suffix=torch.zeros(1, 4, 256, 10, dtype=torch.bfloat16).transpose(2, 3)),
+        "prefix_valid_len": dict(prefix_valid_len=torch.zeros(1, dtype=torch.int64)),
+        "prefix_mask": dict(prefix_mask=torch.ones(1, 63, dtype=torch.uint8)),
+        "out": dict(out=torch.zeros(1, 8, 10, 128, dtype=torch.bfloat16)),
+        "lse": dict(lse=torch.zeros(1, 8, 10, dtype=torch.float64)),
+    }[case]
+
+
+@pytest.mark.parametrize("what", ["q", "k_prefix", "v_suffix", "prefix_valid_len", "prefix_mask", "out", "lse"])
+def test_host_binding_rejects_bad_tensors(lib, what):
+    # the binding checks CPU tensors before it calls the library
+    a = _host_inputs()
+    a.update(_bad_host_argument(what))
+    q, kp, vp, ks, vs = a.pop("q"), a.pop("k_prefix"), a.pop("v_prefix"), a.pop("k_suffix"), a.pop("v_suffix")
+    with pytest.raises(ValueError, match=what):
+        bd.suffix_attn_host(q, kp, vp, ks, vs, **a)

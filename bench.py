@@ -48,6 +48,7 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU-baseline sample budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true", help="skip the per-workload table")
     return ap.parse_args()
 
 
@@ -230,102 +231,113 @@ def cpu_model():
     return "unknown"
 
 
-def history_warm(args, dev, stream, bd):
-    """The history/long-prefix loop as the pages run it: one prefix cache on
-    the device, 10 sequential denoising-step calls with fresh suffix inputs,
-    replayed from one graph (the prefix stays warm in L2 across the steps)."""
+def time_calls(calls, K, W, dev, stream, bd, l2, rotate=True):
+    """Device time per call of K dm05_suffix_attn calls that cycle through
+    `calls` (a list of input sets, one call each), captured as CUDA graphs of
+    up to 1000 calls and timed with CUDA events on the launching stream.
+    With `rotate`, the list is copied until the copies hold more than twice
+    the L2, so every call streams its K/V from HBM; a call list that shares
+    one prefix (the history loop, warm) is timed as is."""
     import torch
-    from gqa_prefix_suffix_b200 import inputs as gen
-    steps = gen.WORKLOADS["history_loop"]()
-    d0 = steps[0].to(dev)
+    one = sum(t.numel() * t.element_size() for c in calls for t in c.tensors().values() if t is not None)
+    copies = max(1, int(2 * l2 // max(1, one)) + 1) if rotate else 1
     sets = []
-    for st in steps:
-        d = st.to(dev)
-        sets.append({"q": d.q, "ks": d.k_suffix, "vs": d.v_suffix,
-                     "out": torch.empty((st.B, st.Hq, st.S, st.D), dtype=torch.bfloat16, device=dev),
-                     "lse": torch.empty((st.B, st.Hq, st.S), dtype=torch.float32, device=dev)})
-    B, Hq, Hkv, P, S, D = d0.B, d0.Hq, d0.Hkv, d0.P, d0.S, d0.D
-    vl = d0.prefix_valid_len
+    for _ in range(copies):
+        prefix_cache = {}
+        for c in calls:
+            # calls that share one prefix cache keep sharing it on the device
+            key = (c.k_prefix.data_ptr(), c.v_prefix.data_ptr())
+            if key not in prefix_cache:
+                prefix_cache[key] = (c.k_prefix.to(dev), c.v_prefix.to(dev))
+            kp, vp = prefix_cache[key]
+            mv = lambda t: None if t is None else t.to(dev)
+            sets.append(dict(q=mv(c.q), k_prefix=kp, v_prefix=vp, prefix_valid_len=mv(c.prefix_valid_len),
+                             prefix_mask=mv(c.prefix_mask), k_suffix=mv(c.k_suffix), v_suffix=mv(c.v_suffix),
+                             out=torch.empty((c.B, c.Hq, c.S, c.D), dtype=torch.bfloat16, device=dev),
+                             lse=torch.empty((c.B, c.Hq, c.S), dtype=torch.float32, device=dev),
+                             dims=(c.B, c.Hq, c.Hkv, c.P, c.S, c.D)))
+    ptr = lambda x: None if x is None else x.data_ptr()
 
-    def ten():
-        for t in sets:
-            rc = bd.dm05_suffix_attn(t["q"].data_ptr(), d0.k_prefix.data_ptr(),
-                                     d0.v_prefix.data_ptr(), None if vl is None else vl.data_ptr(), None,
-                                     t["ks"].data_ptr(), t["vs"].data_ptr(), t["out"].data_ptr(),
-                                     t["lse"].data_ptr(), B, Hq, Hkv, P, S, D, stream.cuda_stream)
-            if rc != 0:
-                raise bd.Dm05Error(rc, "dm05_suffix_attn")
+    def call(t):
+        B, Hq, Hkv, P, S, D = t["dims"]
+        rc = bd.dm05_suffix_attn(ptr(t["q"]), ptr(t["k_prefix"]), ptr(t["v_prefix"]), ptr(t["prefix_valid_len"]),
+                                 ptr(t["prefix_mask"]), ptr(t["k_suffix"]), ptr(t["v_suffix"]), ptr(t["out"]),
+                                 ptr(t["lse"]), B, Hq, Hkv, P, S, D, stream.cuda_stream)
+        if rc != 0:
+            raise bd.Dm05Error(rc, "dm05_suffix_attn")
 
+    n = len(sets)
+    for d in {t["dims"] for t in sets}:
+        rc = bd.dm05_suffix_attn_reserve(*d, stream.cuda_stream)
+        if rc != 0:
+            raise bd.Dm05Error(rc, "reserve")
     with torch.cuda.stream(stream):
-        ten()
+        for i in range(max(3, W)):
+            call(sets[i % n])
     stream.synchronize()
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g, stream=stream):
-        ten()
-    reps = 100
-    with torch.cuda.stream(stream):
-        g.replay()
-        ea = torch.cuda.Event(enable_timing=True)
-        eb = torch.cuda.Event(enable_timing=True)
-        ea.record(stream)
-        for _ in range(reps):
-            g.replay()
-        eb.record(stream)
-    stream.synchronize()
-    ms = ea.elapsed_time(eb)
-    del g
-    return {"warm_per_call": ms * 1e3 / (reps * len(sets)), "per_10_steps": ms * 1e3 / reps, "unit": UNIT,
-            "note": "one prefix kept on the device, 10 fresh suffix sets; value is the cold figure "
-                    "(prefix rotated through more than 2 x L2)"}
-
-
-def bucket_times(args, dev, stream, bd, l2):
-    """µs/call per prefix bucket of the sweep (5 calls per bucket with their
-    own valid lengths, copies rotated through more than 2 x L2)."""
-    import torch
-    from gqa_prefix_suffix_b200 import inputs as gen
-    calls = gen.WORKLOADS["bucket_sweep"]()
-    by_p = {}
-    for c in calls:
-        by_p.setdefault(c.P, []).append(c)
-    res = {}
-    for P, group in sorted(by_p.items()):
-        one = sum(t.numel() * t.element_size() for c in group for t in c.tensors().values() if t is not None)
-        copies = max(1, int(2 * l2 // max(1, one)) + 1)
-        sets = []
-        for _ in range(copies):
-            for c in group:
-                d = c.to(dev)
-                sets.append((d, torch.empty((d.B, d.Hq, d.S, d.D), dtype=torch.bfloat16, device=dev),
-                             torch.empty((d.B, d.Hq, d.S), dtype=torch.float32, device=dev)))
-
-        def run_all():
-            for d, o, l in sets:
-                rc = bd.dm05_suffix_attn(d.q.data_ptr(), d.k_prefix.data_ptr(), d.v_prefix.data_ptr(),
-                                         None if d.prefix_valid_len is None else d.prefix_valid_len.data_ptr(),
-                                         None, d.k_suffix.data_ptr(), d.v_suffix.data_ptr(), o.data_ptr(),
-                                         l.data_ptr(), d.B, d.Hq, d.Hkv, d.P, d.S, d.D, stream.cuda_stream)
-                if rc != 0:
-                    raise bd.Dm05Error(rc, "dm05_suffix_attn")
-
-        with torch.cuda.stream(stream):
-            run_all()
-        stream.synchronize()
+    chunk = min(K, 1000)
+    graphs = []
+    done = 0
+    while done < K:
+        m = min(chunk, K - done)
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
-            run_all()
-        with torch.cuda.stream(stream):
+            for i in range(m):
+                call(sets[(done + i) % n])
+        graphs.append((g, m))
+        done += m
+    for g, _ in graphs:
+        g.replay()
+    stream.synchronize()
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(graphs) + 1)]
+    with torch.cuda.stream(stream):
+        evs[0].record(stream)
+        for i, (g, _) in enumerate(graphs):
             g.replay()
-            ea = torch.cuda.Event(enable_timing=True)
-            eb = torch.cuda.Event(enable_timing=True)
-            ea.record(stream)
-            for _ in range(10):
-                g.replay()
-            eb.record(stream)
-        stream.synchronize()
-        res[str(P)] = ea.elapsed_time(eb) * 1e3 / (10 * len(sets))
-        del g, sets
-    return {"us_per_call": res, "calls_per_bucket": len(calls) // max(1, len(by_p))}
+            evs[i + 1].record(stream)
+    stream.synchronize()
+    us = evs[0].elapsed_time(evs[-1]) * 1e3 / K
+    del graphs, sets
+    return us, copies
+
+
+def workload_table(args, dev, stream, bd, l2, peak):
+    """Every workload of the benchmark timed with the same protocol as the
+    headline (rotating input sets over 2 x L2, K calls from CUDA graphs):
+    µs per call, algorithmic K/V GB/s and its fraction of the HBM peak, and
+    the work plan."""
+    from gqa_prefix_suffix_b200 import inputs as gen
+    K, W = args.steps, args.warmup
+
+    def row(calls, rotate=True, note=None):
+        us, copies = time_calls(calls, K, W, dev, stream, bd, l2, rotate=rotate)
+        kv = sum(algorithmic_bytes(c)[0] for c in calls) / len(calls)
+        c0 = calls[0]
+        _, sp, tr, rb = bd.dm05_suffix_attn_plan(c0.B, c0.Hq, c0.Hkv, c0.P, c0.S, c0.D)
+        gbs = kv / (us * 1e-6) / 1e9
+        r = {"us_per_call": us, "algorithmic_bytes": kv, "achieved_gbs": gbs, "frac": gbs / peak,
+             "plan": {"splits_per_head": sp, "row_blocks": rb, "tile_rows": tr}, "calls": K,
+             "l2": (f"{copies} copies of {len(calls)} input sets" if rotate
+                    else "one shared prefix, L2-warm by design")}
+        if note:
+            r["note"] = note
+        return r
+
+    out = {}
+    out["libero_tiny"] = row([gen.libero_tiny()])
+    sweep = gen.bucket_sweep()
+    by_p = {}
+    for c in sweep:
+        by_p.setdefault(c.P, []).append(c)
+    out["bucket_sweep"] = {str(P): row(g) for P, g in sorted(by_p.items())}
+    hist = gen.history_loop()
+    cold = row(hist, rotate=True, note="prefix cache rotated through more than 2 x L2 (cold)")
+    warm = row(hist, rotate=False, note="one prefix cache, 10 fresh suffix sets per 10 steps (warm, as specified)")
+    cold["per_10_steps"] = 10 * cold["us_per_call"]
+    warm["per_10_steps"] = 10 * warm["us_per_call"]
+    out["history_loop"] = {"cold": cold, "warm": warm}
+    out["batched_mask"] = row([gen.batched_mask()])
+    return out
 
 
 def cpu_oracle_rate(inp, seconds, threads):
@@ -548,16 +560,14 @@ def main():
     latency["launch_floor"] = ea.elapsed_time(eb) * 1e3 / 3000
     del g_floor
 
-    extra = {}
-    if args.workload == "history_loop":
-        extra["history"] = history_warm(args, dev, stream, bd)
-    if args.workload == "bucket_sweep":
-        extra["buckets"] = bucket_times(args, dev, stream, bd, l2)
-
     us_per_call_device = t_ms * 1e3 / K          # one GPU's time per call
     value = whole_job_us_per_call(t_ms, K, world)  # whole-job time per call
     achieved = kv_bytes / (us_per_call_device * 1e-6) / 1e9
     peak, peak_kind = measured_peaks()
+
+    extra = {}
+    if not args.no_workloads:
+        extra["workloads"] = workload_table(args, dev, stream, bd, l2, peak)
 
     # ---- end to end through the public API: one dm05_suffix_attn_host call per
     # step copies the pinned host inputs in, runs the kernel and copies O and

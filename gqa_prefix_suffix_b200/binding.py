@@ -22,9 +22,11 @@ DM05_ERR_WORKSPACE = -5
 DM05_ERR_CUDA = -6
 DM05_EW_VALID_LEN_CLAMPED = 0x1
 DM05_EW_WAIT_TIMEOUT = 0x2
+DM05_EW_BAD_SPLIT = 0x4
 
 EXPORTS = ("dm05_suffix_attn", "dm05_suffix_attn_workspace_bytes", "dm05_suffix_attn_reserve",
-           "dm05_suffix_attn_plan", "dm05_set_split_override", "dm05_get_error_word",
+           "dm05_suffix_attn_plan", "dm05_set_split_override", "dm05_set_row_block_override",
+           "dm05_get_error_word",
            "dm05_status_string", "dm05_release", "dm05_suffix_attn_noalloc", "dm05_suffix_attn_host",
            "dm05_suffix_attn_host_copy_bytes", "dm05_selftest_wait_timeout")
 
@@ -59,6 +61,8 @@ def lib() -> ctypes.CDLL:
             L.dm05_suffix_attn_plan.restype = i
             L.dm05_set_split_override.argtypes = [i]
             L.dm05_set_split_override.restype = i
+            L.dm05_set_row_block_override.argtypes = [i]
+            L.dm05_set_row_block_override.restype = i
             L.dm05_get_error_word.argtypes = [p, ctypes.POINTER(ctypes.c_uint32)]
             L.dm05_get_error_word.restype = i
             L.dm05_status_string.argtypes = [i]
@@ -128,6 +132,10 @@ def dm05_set_split_override(splits_per_head: int) -> int:
     return lib().dm05_set_split_override(splits_per_head)
 
 
+def dm05_set_row_block_override(row_blocks: int) -> int:
+    return lib().dm05_set_row_block_override(row_blocks)
+
+
 def dm05_selftest_wait_timeout(limit_ms: int, stream) -> int:
     """Launches the bounded-wait self-test (a wait that must run out)."""
     return lib().dm05_selftest_wait_timeout(limit_ms, stream)
@@ -178,8 +186,9 @@ def suffix_attn(q, k_prefix, v_prefix, k_suffix, v_suffix, prefix_valid_len=None
     if tuple(k_suffix.shape) != (B, Hkv, S, D) or tuple(v_suffix.shape) != (B, Hkv, S, D):
         raise ValueError("k_suffix/v_suffix must be [B,Hkv,S,D]")
     if prefix_valid_len is not None:
-        if not prefix_valid_len.is_cuda or prefix_valid_len.dtype != torch.int32 or prefix_valid_len.numel() != B:
-            raise ValueError("prefix_valid_len must be a CUDA int32 tensor of B values")
+        if (not prefix_valid_len.is_cuda or prefix_valid_len.dtype != torch.int32 or prefix_valid_len.numel() != B
+                or not prefix_valid_len.is_contiguous()):
+            raise ValueError("prefix_valid_len must be a contiguous CUDA int32 tensor of B values")
     if prefix_mask is not None:
         if (not prefix_mask.is_cuda or prefix_mask.dtype != torch.uint8 or tuple(prefix_mask.shape) != (B, P)
                 or not prefix_mask.is_contiguous()):
@@ -188,6 +197,15 @@ def suffix_attn(q, k_prefix, v_prefix, k_suffix, v_suffix, prefix_valid_len=None
         out = torch.empty((B, Hq, S, D), dtype=torch.bfloat16, device=q.device)
     if lse is None and want_lse:
         lse = torch.empty((B, Hq, S), dtype=torch.float32, device=q.device)
+    # the library writes B*Hq*S rows through these pointers: a smaller or
+    # strided buffer would be overrun
+    for name, t, shape, dt in (("out", out, (B, Hq, S, D), torch.bfloat16), ("lse", lse, (B, Hq, S), torch.float32)):
+        if t is not None and (not t.is_cuda or t.dtype != dt or tuple(t.shape) != shape or not t.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous CUDA {dt} tensor {list(shape)}")
+    for name, t in (("k_prefix", k_prefix), ("v_prefix", v_prefix), ("k_suffix", k_suffix), ("v_suffix", v_suffix),
+                    ("prefix_valid_len", prefix_valid_len), ("prefix_mask", prefix_mask), ("out", out), ("lse", lse)):
+        if t is not None and t.device != q.device:
+            raise ValueError(f"{name} must be on {q.device} like q")
     ptr = lambda t: None if t is None else t.data_ptr()
     rc = dm05_suffix_attn(ptr(q), ptr(k_prefix), ptr(v_prefix), ptr(prefix_valid_len), ptr(prefix_mask),
                           ptr(k_suffix), ptr(v_suffix), ptr(out), ptr(lse), B, Hq, Hkv, P, S, D,

@@ -57,6 +57,7 @@ std::vector<DeviceState> g_dev;
 std::vector<StreamWorkspace> g_ws;
 std::vector<StreamWorkspace> g_stage;  // device copies of host-buffer calls, per (device, stream)
 int g_split_override = 0;
+int g_row_block_override = 0;
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
 auto *kKernel = &dm05::suffix_attn_kernel<kTileRows, kStages>;
@@ -93,15 +94,6 @@ int check_sizes(int B, int Hq, int Hkv, int P, int S, int D)
 // lowest estimated cost.
 int log2_pow2(int c) { return c >= 16 ? 4 : c >= 8 ? 3 : c >= 4 ? 2 : c >= 2 ? 1 : 0; }
 
-int env_row_blocks()
-{
-    static const int v = [] {
-        const char *e = std::getenv("DM05_ROW_BLOCKS");
-        return e ? std::atoi(e) : 0;
-    }();
-    return v;
-}
-
 Plan make_plan(int B, int Hq, int Hkv, int P, int S, const DeviceState &ds)
 {
     const long long units = static_cast<long long>(B) * Hkv;
@@ -120,7 +112,7 @@ Plan make_plan(int B, int Hq, int Hkv, int P, int S, const DeviceState &ds)
         if (c > 1) t += 2.0 + 0.04 * G * sq;
         return t;
     };
-    const int want_rb = env_row_blocks();
+    const int want_rb = g_row_block_override;
     Plan best;
     best.SQ = S;
     double best_cost = 1e30;
@@ -167,8 +159,9 @@ int get_encoder()
 }
 
 // Device state of the current device with kernel attributes set; the error
-// word is created only if `allocate`.  Caller holds g_mu.
-int device_state(bool allocate, DeviceState **out)
+// word is created only if `allocate` (then `stream` must not be capturing).
+// Caller holds g_mu.
+int device_state(bool allocate, DeviceState **out, cudaStream_t stream = nullptr)
 {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return DM05_ERR_CUDA;
@@ -208,9 +201,12 @@ int device_state(bool allocate, DeviceState **out)
         ds.attrs_set = true;
     }
     if (allocate && ds.err == nullptr) {
+        // cleared on the caller's stream and waited for, so that no kernel on
+        // any stream can run before the word holds zero (only ever done
+        // outside stream capture)
         void *p = nullptr;
         if (cudaMalloc(&p, kErrBytes) != cudaSuccess) return DM05_ERR_CUDA;
-        if (cudaMemset(p, 0, kErrBytes) != cudaSuccess) {
+        if (cudaMemsetAsync(p, 0, kErrBytes, stream) != cudaSuccess || cudaStreamSynchronize(stream) != cudaSuccess) {
             cudaFree(p);
             return DM05_ERR_CUDA;
         }
@@ -396,6 +392,85 @@ int encode_3d(CUtensorMap *map, const void *base, uint64_t d1, uint64_t d2, uint
     return r == CUDA_SUCCESS ? DM05_OK : DM05_ERR_CUDA;
 }
 
+
+// Encodes the tensor maps and launches the kernel with plan `pl` on
+// `stream`; `err` is the device error word, `part` the partial-result area
+// (unused when pl.splits == 1).  Sizes and pointers are already checked.
+int launch_attention(const void *q, const void *k_prefix, const void *v_prefix, const int32_t *prefix_valid_len,
+                     const uint8_t *prefix_mask, const void *k_suffix, const void *v_suffix, void *out, float *lse,
+                     int B, int Hq, int Hkv, int P, int S, int D, const Plan &pl, uint32_t *err, void *part,
+                     cudaStream_t stream)
+{
+    const int G = Hq / Hkv;
+    const int GS = G * S;
+    const long long units = static_cast<long long>(B) * Hkv;
+    const long long grid = units * pl.row_blocks * pl.splits;
+    if (grid > 0x7fffffffLL) return DM05_ERR_SHAPE;  // more CTAs than one launch can name
+    if (pl.splits != 1 && pl.splits != 2 && pl.splits != 4 && pl.splits != 8 && pl.splits != 16)
+        return DM05_ERR_SHAPE;  // the kernel merges only these cluster sizes
+
+    // ---- TMA descriptors (the tensor maps travel as kernel parameters)
+    CUtensorMap tm_q, tm_kp, tm_vp, tm_ks, tm_vs;
+    // Q: one 128-row box of all four chunks when the block is the whole unit,
+    // else one SQ-row box per head and chunk (3-D)
+    const int rq = pl.row_blocks == 1
+                       ? encode_4d(&tm_q, q, static_cast<uint64_t>(GS), static_cast<uint64_t>(units), dm05::kMRows)
+                       : encode_3d(&tm_q, q, static_cast<uint64_t>(GS), static_cast<uint64_t>(units),
+                                   static_cast<uint32_t>(pl.SQ));
+    if (rq != DM05_OK ||
+        encode_4d(&tm_ks, k_suffix, static_cast<uint64_t>(S), static_cast<uint64_t>(units), kTileRows) != DM05_OK ||
+        encode_4d(&tm_vs, v_suffix, static_cast<uint64_t>(S), static_cast<uint64_t>(units), kTileRows) != DM05_OK)
+        return DM05_ERR_CUDA;
+    if (P > 0) {
+        if (encode_4d(&tm_kp, k_prefix, static_cast<uint64_t>(P), static_cast<uint64_t>(units), kTileRows) !=
+                DM05_OK ||
+            encode_4d(&tm_vp, v_prefix, static_cast<uint64_t>(P), static_cast<uint64_t>(units), kTileRows) != DM05_OK)
+            return DM05_ERR_CUDA;
+    } else {
+        tm_kp = tm_ks;  // never read: no prefix tile exists when P == 0
+        tm_vp = tm_vs;
+    }
+
+    dm05::KernelParams kp;
+    kp.valid_len = prefix_valid_len;
+    kp.mask = prefix_mask;
+    kp.out = static_cast<__nv_bfloat16 *>(out);
+    kp.lse = lse;
+    kp.err = err;
+    kp.part = pl.splits > 1 ? static_cast<float *>(part) : nullptr;
+    kp.Hkv = Hkv;
+    kp.P = P;
+    kp.S = S;
+    kp.GS = GS;
+    kp.G = G;
+    kp.row_blocks = pl.row_blocks;
+    kp.SQ = pl.SQ;
+    kp.splits = pl.splits;
+    kp.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+    cfg.blockDim = dim3(dm05::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = Layout::kAllocBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute at[2];
+    int na = 0;
+    at[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+    if (pl.splits > 1) {
+        at[na].id = cudaLaunchAttributeClusterDimension;
+        at[na].val.clusterDim.x = static_cast<unsigned>(pl.splits);
+        at[na].val.clusterDim.y = 1;
+        at[na].val.clusterDim.z = 1;
+        ++na;
+    }
+    cfg.attrs = at;
+    cfg.numAttrs = na;
+    if (cudaLaunchKernelEx(&cfg, kKernel, tm_q, tm_kp, tm_vp, tm_ks, tm_vs, kp) != cudaSuccess) return DM05_ERR_CUDA;
+    return DM05_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -436,6 +511,16 @@ int dm05_set_split_override(int splits_per_head)
     return DM05_OK;
 }
 
+int dm05_set_row_block_override(int row_blocks)
+{
+    if (row_blocks != 0 && row_blocks != 1 && row_blocks != 2 && row_blocks != 4 && row_blocks != 8 &&
+        row_blocks != 16)
+        return DM05_ERR_SHAPE;
+    std::lock_guard<std::mutex> lk(g_mu);
+    g_row_block_override = row_blocks;
+    return DM05_OK;
+}
+
 int dm05_suffix_attn_plan(int B, int Hq, int Hkv, int P, int S, int D, int *splits_per_head, int *tile_rows,
                           int *row_blocks)
 {
@@ -462,7 +547,7 @@ int dm05_suffix_attn_reserve(int B, int Hq, int Hkv, int P, int S, int D, cudaSt
     std::lock_guard<std::mutex> lk(g_mu);
     if (get_encoder() != DM05_OK) return DM05_ERR_CUDA;
     DeviceState *ds = nullptr;
-    rc = device_state(true, &ds);
+    rc = device_state(true, &ds, stream);
     if (rc != DM05_OK) return rc;
     const Plan pl = make_plan(B, Hq, Hkv, P, S, *ds);
     void *ws = nullptr;
@@ -484,7 +569,6 @@ int dm05_suffix_attn(const void *q, const void *k_prefix, const void *v_prefix, 
     if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u) != 0) return DM05_ERR_ALIGN;
 
     const int G = Hq / Hkv;
-    const int GS = G * S;
     const int units = B * Hkv;
 
     DeviceState *ds = nullptr;  // points into g_dev: used only while g_mu is held
@@ -500,7 +584,7 @@ int dm05_suffix_attn(const void *q, const void *k_prefix, const void *v_prefix, 
             cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
             if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) return DM05_ERR_CUDA;
             if (cs != cudaStreamCaptureStatusNone) return DM05_ERR_WORKSPACE;
-            rc = device_state(true, &ds);
+            rc = device_state(true, &ds, stream);
             if (rc != DM05_OK) return rc;
         }
         pl = make_plan(B, Hq, Hkv, P, S, *ds);
@@ -509,66 +593,8 @@ int dm05_suffix_attn(const void *q, const void *k_prefix, const void *v_prefix, 
         if (rc != DM05_OK) return rc;
     }
 
-    // ---- TMA descriptors (the tensor maps travel as kernel parameters)
-    CUtensorMap tm_q, tm_kp, tm_vp, tm_ks, tm_vs;
-    // Q: one 128-row box of all four chunks when the block is the whole unit,
-    // else one SQ-row box per head and chunk (3-D)
-    const int rq = pl.row_blocks == 1
-                       ? encode_4d(&tm_q, q, static_cast<uint64_t>(GS), static_cast<uint64_t>(units), dm05::kMRows)
-                       : encode_3d(&tm_q, q, static_cast<uint64_t>(GS), static_cast<uint64_t>(units),
-                                   static_cast<uint32_t>(pl.SQ));
-    if (rq != DM05_OK ||
-        encode_4d(&tm_ks, k_suffix, static_cast<uint64_t>(S), static_cast<uint64_t>(units), kTileRows) != DM05_OK ||
-        encode_4d(&tm_vs, v_suffix, static_cast<uint64_t>(S), static_cast<uint64_t>(units), kTileRows) != DM05_OK)
-        return DM05_ERR_CUDA;
-    if (P > 0) {
-        if (encode_4d(&tm_kp, k_prefix, static_cast<uint64_t>(P), static_cast<uint64_t>(units), kTileRows) !=
-                DM05_OK ||
-            encode_4d(&tm_vp, v_prefix, static_cast<uint64_t>(P), static_cast<uint64_t>(units), kTileRows) != DM05_OK)
-            return DM05_ERR_CUDA;
-    } else {
-        tm_kp = tm_ks;  // never read: no prefix tile exists when P == 0
-        tm_vp = tm_vs;
-    }
-
-    dm05::KernelParams kp;
-    kp.valid_len = prefix_valid_len;
-    kp.mask = prefix_mask;
-    kp.out = static_cast<__nv_bfloat16 *>(out);
-    kp.lse = lse;
-    kp.err = err_word;
-    kp.part = static_cast<float *>(part_ws);
-    kp.Hkv = Hkv;
-    kp.P = P;
-    kp.S = S;
-    kp.GS = GS;
-    kp.G = G;
-    kp.row_blocks = pl.row_blocks;
-    kp.SQ = pl.SQ;
-    kp.splits = pl.splits;
-    kp.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
-
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(units * pl.row_blocks * pl.splits), 1, 1);
-    cfg.blockDim = dim3(dm05::kThreads, 1, 1);
-    cfg.dynamicSmemBytes = Layout::kAllocBytes;
-    cfg.stream = stream;
-    cudaLaunchAttribute at[2];
-    int na = 0;
-    at[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    at[na].val.programmaticStreamSerializationAllowed = 1;
-    ++na;
-    if (pl.splits > 1) {
-        at[na].id = cudaLaunchAttributeClusterDimension;
-        at[na].val.clusterDim.x = static_cast<unsigned>(pl.splits);
-        at[na].val.clusterDim.y = 1;
-        at[na].val.clusterDim.z = 1;
-        ++na;
-    }
-    cfg.attrs = at;
-    cfg.numAttrs = na;
-    if (cudaLaunchKernelEx(&cfg, kKernel, tm_q, tm_kp, tm_vp, tm_ks, tm_vs, kp) != cudaSuccess) return DM05_ERR_CUDA;
-    return DM05_OK;
+    return launch_attention(q, k_prefix, v_prefix, prefix_valid_len, prefix_mask, k_suffix, v_suffix, out, lse, B,
+                            Hq, Hkv, P, S, D, pl, err_word, part_ws, stream);
 }
 
 int dm05_selftest_wait_timeout(int limit_ms, cudaStream_t stream)
@@ -581,7 +607,7 @@ int dm05_selftest_wait_timeout(int limit_ms, cudaStream_t stream)
     {
         std::lock_guard<std::mutex> lk(g_mu);
         DeviceState *ds = nullptr;
-        const int rc = device_state(true, &ds);
+        const int rc = device_state(true, &ds, stream);
         if (rc != DM05_OK) return rc;
         err = ds->err;
     }
@@ -700,7 +726,9 @@ static __device__ __align__(256) uint32_t g_noalloc_scratch[DM05_NOALLOC_SCRATCH
 std::vector<uint32_t *> g_noalloc_addr;  // per device ordinal: device address of g_noalloc_scratch
 
 // Caller holds g_mu.  Looks up (and on first use clears) this device's copy
-// of the scratch array.  Allocates nothing.
+// of the scratch array.  Allocates nothing.  The clear is enqueued on the
+// caller's stream and waited for, so every later kernel on any stream sees a
+// zero error word; it runs only outside stream capture.
 int noalloc_scratch(cudaStream_t stream, uint32_t **out)
 {
     int dev = 0;
@@ -712,11 +740,21 @@ int noalloc_scratch(cudaStream_t stream, uint32_t **out)
         if (cs != cudaStreamCaptureStatusNone) return DM05_ERR_WORKSPACE;
         void *ptr = nullptr;
         if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) return DM05_ERR_CUDA;
-        if (cudaMemset(ptr, 0, kErrBytes) != cudaSuccess) return DM05_ERR_CUDA;  // the error word starts at zero
+        if (cudaMemsetAsync(ptr, 0, kErrBytes, stream) != cudaSuccess || cudaStreamSynchronize(stream) != cudaSuccess)
+            return DM05_ERR_CUDA;
         g_noalloc_addr[dev] = static_cast<uint32_t *>(ptr);
     }
     *out = g_noalloc_addr[dev];
     return DM05_OK;
+}
+
+// Device address of this device's scratch array if a call has set it up
+// (else nullptr).  Caller holds g_mu.
+uint32_t *noalloc_word_if_set_up()
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev >= static_cast<int>(g_noalloc_addr.size())) return nullptr;
+    return g_noalloc_addr[dev];
 }
 }  // namespace
 
@@ -739,7 +777,6 @@ int dm05_suffix_attn_noalloc(const void *q, const void *k_prefix, const void *v_
     if (kErrBytes > DM05_NOALLOC_SCRATCH_BYTES) return DM05_ERR_WORKSPACE;
 
     const int G = Hq / Hkv;
-    const int GS = G * S;
     const int units = B * Hkv;
     DeviceState *ds = nullptr;
     uint32_t *scratch = nullptr;
@@ -760,84 +797,35 @@ int dm05_suffix_attn_noalloc(const void *q, const void *k_prefix, const void *v_
         }
     }
 
-    CUtensorMap tm_q, tm_kp, tm_vp, tm_ks, tm_vs;
-    // Q: one 128-row box of all four chunks when the block is the whole unit,
-    // else one SQ-row box per head and chunk (3-D)
-    const int rq = pl.row_blocks == 1
-                       ? encode_4d(&tm_q, q, static_cast<uint64_t>(GS), static_cast<uint64_t>(units), dm05::kMRows)
-                       : encode_3d(&tm_q, q, static_cast<uint64_t>(GS), static_cast<uint64_t>(units),
-                                   static_cast<uint32_t>(pl.SQ));
-    if (rq != DM05_OK ||
-        encode_4d(&tm_ks, k_suffix, static_cast<uint64_t>(S), static_cast<uint64_t>(units), kTileRows) != DM05_OK ||
-        encode_4d(&tm_vs, v_suffix, static_cast<uint64_t>(S), static_cast<uint64_t>(units), kTileRows) != DM05_OK)
-        return DM05_ERR_CUDA;
-    if (P > 0) {
-        if (encode_4d(&tm_kp, k_prefix, static_cast<uint64_t>(P), static_cast<uint64_t>(units), kTileRows) !=
-                DM05_OK ||
-            encode_4d(&tm_vp, v_prefix, static_cast<uint64_t>(P), static_cast<uint64_t>(units), kTileRows) != DM05_OK)
-            return DM05_ERR_CUDA;
-    } else {
-        tm_kp = tm_ks;
-        tm_vp = tm_vs;
-    }
-
-    dm05::KernelParams kp;
-    kp.valid_len = prefix_valid_len;
-    kp.mask = prefix_mask;
-    kp.out = static_cast<__nv_bfloat16 *>(out);
-    kp.lse = lse;
-    kp.err = scratch;
-    kp.part = pl.splits > 1 ? reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(scratch) + kErrBytes) : nullptr;
-    kp.Hkv = Hkv;
-    kp.P = P;
-    kp.S = S;
-    kp.GS = GS;
-    kp.G = G;
-    kp.row_blocks = pl.row_blocks;
-    kp.SQ = pl.SQ;
-    kp.splits = pl.splits;
-    kp.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
-
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(units * pl.row_blocks * pl.splits), 1, 1);
-    cfg.blockDim = dim3(dm05::kThreads, 1, 1);
-    cfg.dynamicSmemBytes = Layout::kAllocBytes;
-    cfg.stream = stream;
-    cudaLaunchAttribute at[2];
-    int na = 0;
-    at[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    at[na].val.programmaticStreamSerializationAllowed = 1;
-    ++na;
-    if (pl.splits > 1) {
-        at[na].id = cudaLaunchAttributeClusterDimension;
-        at[na].val.clusterDim.x = static_cast<unsigned>(pl.splits);
-        at[na].val.clusterDim.y = 1;
-        at[na].val.clusterDim.z = 1;
-        ++na;
-    }
-    cfg.attrs = at;
-    cfg.numAttrs = na;
-    if (cudaLaunchKernelEx(&cfg, kKernel, tm_q, tm_kp, tm_vp, tm_ks, tm_vs, kp) != cudaSuccess) return DM05_ERR_CUDA;
-    return DM05_OK;
+    return launch_attention(q, k_prefix, v_prefix, prefix_valid_len, prefix_mask, k_suffix, v_suffix, out, lse, B,
+                            Hq, Hkv, P, S, D, pl, scratch, reinterpret_cast<uint8_t *>(scratch) + kErrBytes, stream);
 }
 
 int dm05_get_error_word(cudaStream_t stream, uint32_t *host_word)
 {
     if (!host_word) return DM05_ERR_NULL;
-    uint32_t *err = nullptr;
+    // the word of the allocating entry points and the one in the fixed
+    // scratch array of dm05_suffix_attn_noalloc (both, when both exist)
+    uint32_t *words[2] = {nullptr, nullptr};
     {
         std::lock_guard<std::mutex> lk(g_mu);
         DeviceState *ds = nullptr;
         int rc = device_state(false, &ds);
         if (rc != DM05_OK) return rc;
-        err = ds->err;
+        words[0] = ds->err;
+        words[1] = noalloc_word_if_set_up();
     }
     *host_word = 0;
     if (cudaStreamSynchronize(stream) != cudaSuccess) return DM05_ERR_CUDA;
-    if (err == nullptr) return DM05_OK;
-    if (cudaMemcpyAsync(host_word, err, sizeof(uint32_t), cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
-        cudaMemsetAsync(err, 0, sizeof(uint32_t), stream) != cudaSuccess || cudaStreamSynchronize(stream) != cudaSuccess)
-        return DM05_ERR_CUDA;
+    for (uint32_t *w : words) {
+        if (w == nullptr) continue;
+        uint32_t v = 0;
+        if (cudaMemcpyAsync(&v, w, sizeof(uint32_t), cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
+            cudaMemsetAsync(w, 0, sizeof(uint32_t), stream) != cudaSuccess ||
+            cudaStreamSynchronize(stream) != cudaSuccess)
+            return DM05_ERR_CUDA;
+        *host_word |= v;
+    }
     return DM05_OK;
 }
 

@@ -77,6 +77,7 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait
 constexpr float kRescaleThreshold = 8.0f;         // log2 units: p <= 2^8 between rescales
 constexpr uint32_t kEwClamped = 0x1u;
 constexpr uint32_t kEwTimeout = 0x2u;
+constexpr uint32_t kEwBadSplit = 0x4u;
 
 struct KernelParams {
     const int32_t *valid_len;  // [B] or nullptr
@@ -791,11 +792,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (nr > 0) {
             if (!warp_wait(&bars[L::kBarMerge], 0)) failed = true;
+            // the host launches only these cluster sizes; any other is
+            // reported and merges nothing
             switch (C) {
             case 2: merge_rows<2, L>(recv, nr, p.out, p.lse, unit_row0, r_lo, nq, p.S, q0); break;
             case 4: merge_rows<4, L>(recv, nr, p.out, p.lse, unit_row0, r_lo, nq, p.S, q0); break;
             case 8: merge_rows<8, L>(recv, nr, p.out, p.lse, unit_row0, r_lo, nq, p.S, q0); break;
-            default: merge_rows<16, L>(recv, nr, p.out, p.lse, unit_row0, r_lo, nq, p.S, q0); break;
+            case 16: merge_rows<16, L>(recv, nr, p.out, p.lse, unit_row0, r_lo, nq, p.S, q0); break;
+            default:
+                if (threadIdx.x == 0) atomicOr(p.err, kEwBadSplit);
+                break;
             }
         }
     }

@@ -62,6 +62,8 @@ typedef enum {
 /* Bits of the device error word (dm05_get_error_word). */
 #define DM05_EW_VALID_LEN_CLAMPED 0x1u /* a prefix_valid_len value was outside [0, P] and was clamped */
 #define DM05_EW_WAIT_TIMEOUT      0x2u /* a kernel wait gave up after its time limit; outputs invalid */
+#define DM05_EW_BAD_SPLIT         0x4u /* a kernel was launched with a split count it cannot merge (the
+                                          host never does this); outputs invalid */
 
 /*
  * dm05_suffix_attn -- one suffix-attention call, asynchronous on `stream`.
@@ -101,13 +103,23 @@ int dm05_suffix_attn(const void *q, const void *k_prefix, const void *v_prefix,
 
 /* Upper bound of the device workspace dm05_suffix_attn uses for these sizes:
  * the error word plus the partial results of the largest split (16 CTAs per
- * (sample, KV head)).  0 if the sizes are invalid. */
+ * (sample, KV head)).  0 if the sizes are invalid.
+ *
+ * The pages' fast path preallocates its work buffers once
+ * (DM05BigKernelBuffers, page "TensorRT+Triton+FlexAttention: OpenDM VLA
+ * 快速推理加速栈深度剖析", section 2.2) so that no request allocates device
+ * memory; this call tells a caller how much this library's equivalent needs. */
 size_t dm05_suffix_attn_workspace_bytes(int B, int Hq, int Hkv, int P, int S, int D);
 
 /* Creates the workspace of (current device, `stream`) for these sizes and
  * sets the kernel attributes, outside any stream capture.  Call it before
  * capturing dm05_suffix_attn on `stream` into a CUDA graph.  `stream` must not
- * be capturing. */
+ * be capturing.
+ *
+ * This is the step the pages take at start-up: the prefix KV cache has a
+ * static address and every bucket's graph is captured once, then replayed
+ * per request (same page, section 3).  A graph captured after this call
+ * stays valid while the workspace lives (until dm05_release). */
 int dm05_suffix_attn_reserve(int B, int Hq, int Hkv, int P, int S, int D, cudaStream_t stream);
 
 /* Work decomposition the next call with these sizes will use: the number of
@@ -121,6 +133,15 @@ int dm05_suffix_attn_plan(int B, int Hq, int Hkv, int P, int S, int D,
  * process: 1, 2, 4, 8 or 16; 0 restores the automatic choice.  For tuning
  * and tests.  Returns DM05_ERR_SHAPE for any other value. */
 int dm05_set_split_override(int splits_per_head);
+
+/* Forces the number of query blocks each (sample, KV head)'s S queries are
+ * cut into, for later split calls on this process: 1, 2, 4, 8 or 16; 0
+ * restores the automatic choice.  A block holds at least 8 queries per head
+ * and (Hq/Hkv) * (block rounded up to 8) <= 128 rows, so a count that breaks
+ * this (or a call that runs unsplit) uses one block; dm05_suffix_attn_plan
+ * reports what a call will use.  For tuning and tests.  Returns
+ * DM05_ERR_SHAPE for any other value. */
+int dm05_set_row_block_override(int row_blocks);
 
 /*
  * dm05_suffix_attn_noalloc -- the same attention as dm05_suffix_attn, for
@@ -145,16 +166,19 @@ int dm05_set_split_override(int splits_per_head);
  * DM05_ERR_WORKSPACE is returned only if the error word itself did not fit.
  *
  * Set-up: the first call on each device looks up the array's device address
- * and clears it (a synchronous cudaMemset), so make that first call before
- * any stream capture on that device; a first call on a capturing stream
- * returns DM05_ERR_WORKSPACE and does nothing.
+ * and clears its error word (enqueued on `stream`, then the host waits for
+ * it), so make that first call before any stream capture on that device; a
+ * first call on a capturing stream returns DM05_ERR_WORKSPACE and does
+ * nothing.
  *
  * Sharing: every call on a device uses the same array and it keeps what the
- * last call left there.  A call writes all the partial results it later reads,
- * and the error word only collects time-out bits (they stay set and are not
- * visible through dm05_get_error_word).  Calls whose kernels overlap on the
- * GPU (for example on two streams) race on the array and may corrupt each
- * other's results: serialise them.
+ * last call left there.  A call writes all the partial results it later
+ * reads.  The array's error word collects the same bits as the allocating
+ * entry points' word (a clamped prefix_valid_len, a wait time-out) and
+ * keeps them until dm05_get_error_word reads and clears them (it reads this
+ * word too).  After a time-out the call's outputs are invalid.  Calls whose
+ * kernels overlap on the GPU (for example on two streams) race on the array
+ * and may corrupt each other's results: serialise them.
  */
 #define DM05_NOALLOC_SCRATCH_BYTES (8u << 20)
 int dm05_suffix_attn_noalloc(const void *q, const void *k_prefix, const void *v_prefix,
@@ -233,7 +257,9 @@ int dm05_selftest_wait_timeout(int limit_ms, cudaStream_t stream);
 
 /* Synchronises `stream`, then returns in *host_word the error bits
  * (DM05_EW_*) that kernels on the current device set since the last read,
- * and clears them. */
+ * and clears them: the word of dm05_suffix_attn / dm05_suffix_attn_host /
+ * dm05_selftest_wait_timeout and the word in the fixed array of
+ * dm05_suffix_attn_noalloc, ORed together.  Allocates nothing. */
 int dm05_get_error_word(cudaStream_t stream, uint32_t *host_word);
 
 /* Human-readable name of a dm05_status value. */

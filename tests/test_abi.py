@@ -106,6 +106,14 @@ def test_split_override_values(lib):
     assert bd.dm05_set_split_override(0) == bd.DM05_OK
 
 
+def test_row_block_override_values(lib):
+    for v in (0, 1, 2, 4, 8, 16):
+        assert bd.dm05_set_row_block_override(v) == bd.DM05_OK
+    for v in (3, 32, -1):
+        assert bd.dm05_set_row_block_override(v) == bd.DM05_ERR_SHAPE
+    assert bd.dm05_set_row_block_override(0) == bd.DM05_OK
+
+
 def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(bd, "LIB_PATH", str(tmp_path / "missing.so"))
     monkeypatch.setattr(bd, "_lib", None)

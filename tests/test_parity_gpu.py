@@ -1,11 +1,19 @@
 """CUDA path against the fp64 oracle, element by element, on seeded inputs.
 
-Tolerance (bf16 output, fp32 accumulation): |out - O_oracle| <= 1e-2 for
-every element, except elements whose exact value has magnitude >= 4, where a
-correctly rounded bf16 value can already be 2^-6 = 0.0156 away; those are
-held to one bf16 ulp of the exact value.  mean |out - O_oracle| <= 1e-3, or
-1.5x the mean error of the correctly rounded result when that floor is
-itself near 1e-3 (a handful of keys), and |lse - LSE_oracle| <= 1e-3.
+Tolerance (bf16 output, fp32 accumulation; the stated bar is 1e-2 max and
+1e-3 mean absolute error, and 1e-3 on the LSE):
+  * every element whose exact value has magnitude < 4: |out - O| <= 1e-2.
+    In [2, 4) a correctly rounded bf16 value may already be 2^-8 away, so
+    the bar leaves a pre-rounding allowance of DELTA = 1e-2 - 2^-7 for the
+    arithmetic before the final rounding.
+  * elements with |O| >= 4, where half a bf16 ulp alone is 2^-6 = 0.0156 or
+    more, so the 1e-2 bar cannot be met even by the correctly rounded value:
+    half a bf16 ulp of O plus the same allowance DELTA.
+  * mean |out - O| <= 1e-3.  Only for rows with few visible keys (at most
+    FEW_KEYS), where |O| is O(1) and the mean error of the correctly rounded
+    bf16 result itself approaches 1e-3, the mean bound is 1.5x that rounding
+    floor instead.  Each check prints which branch it used.
+  * |lse - LSE| <= 1e-3.
 """
 import math
 import zlib
@@ -23,6 +31,8 @@ pytestmark = pytest.mark.gpu
 MAX_ABS = 1e-2
 MEAN_ABS = 1e-3
 LSE_ABS = 1e-3
+DELTA = MAX_ABS - 2.0 ** -7     # pre-rounding allowance the 1e-2 bar leaves in [2, 4)
+FEW_KEYS = 32
 
 
 def bf16_ulp(x):
@@ -31,25 +41,41 @@ def bf16_ulp(x):
 
 
 def element_bound(o_ref):
-    return np.where(np.abs(o_ref) >= 4.0, bf16_ulp(o_ref), MAX_ABS)
+    return np.where(np.abs(o_ref) >= 4.0, 0.5 * bf16_ulp(o_ref) + DELTA, MAX_ABS)
 
 
-def check_close(out, lse, o_ref, l_ref, what=""):
+def visible_keys(inp):
+    """Fewest visible keys (prefix rows in range and not hidden, plus the S
+    suffix rows) over the samples of an input set."""
+    fewest = None
+    for b in range(inp.B):
+        vl = inp.P if inp.prefix_valid_len is None else max(0, min(inp.P, int(inp.prefix_valid_len[b])))
+        vis = vl if inp.prefix_mask is None else int((inp.prefix_mask[b, :vl] != 0).sum())
+        fewest = vis + inp.S if fewest is None else min(fewest, vis + inp.S)
+    return fewest
+
+
+def check_close(out, lse, o_ref, l_ref, what="", keys=None):
+    """keys: the fewest visible keys of any row (None: many)."""
     o = out.float().cpu().double().numpy()
     err = np.abs(o - o_ref)
     bound = element_bound(o_ref)
-    floor = np.abs(torch.from_numpy(o_ref).to(torch.bfloat16).double().numpy() - o_ref).max()
+    rounded = torch.from_numpy(o_ref).to(torch.bfloat16).double().numpy()
+    floor = np.abs(rounded - o_ref).max()
     bad = err > bound
+    n_big = int((np.abs(o_ref) >= 4.0).sum())
     if bad.any():
         rows = sorted({tuple(int(v) for v in idx[:3]) for idx in np.argwhere(bad)})
         raise AssertionError(f"{what}: {int(bad.sum())} elements over the bound in {len(rows)} rows "
                              f"(b,h,i) {rows[:12]}; max err {err.max():.5f} at "
                              f"|o|={np.abs(o_ref).flat[err.argmax()]:.3f}; rounding floor {floor:.5f}")
-    # With only a few keys |O| is O(1) and the mean error of the correctly
-    # rounded bf16 result itself approaches 1e-3; the mean bound then follows
-    # that floor (realistic inputs have a floor near 1e-4, well under 1e-3).
-    floor_mean = np.abs(torch.from_numpy(o_ref).to(torch.bfloat16).double().numpy() - o_ref).mean()
-    assert err.mean() <= max(MEAN_ABS, 1.5 * floor_mean), f"{what}: mean err {err.mean():.2e}, floor {floor_mean:.2e}"
+    floor_mean = np.abs(rounded - o_ref).mean()
+    few = keys is not None and keys <= FEW_KEYS
+    mean_bound = max(MEAN_ABS, 1.5 * floor_mean) if few else MEAN_ABS
+    print(f"[{what}] max err {err.max():.5f} (elements |O|>=4: {n_big}, bound there half-ulp + {DELTA:.5f}); "
+          f"mean {err.mean():.2e} <= {mean_bound:.2e} "
+          f"({'few-key branch: 1.5 x rounding floor ' + f'{floor_mean:.2e}' if few else 'fixed 1e-3'})")
+    assert err.mean() <= mean_bound, f"{what}: mean err {err.mean():.2e}, floor {floor_mean:.2e}"
     if lse is not None:
         le = np.abs(lse.double().cpu().numpy() - l_ref)
         assert le.max() <= LSE_ABS, f"{what}: lse err {le.max():.2e}"
@@ -65,11 +91,13 @@ def cuda_ready():
     bd.lib()
     yield
     bd.dm05_set_split_override(0)
+    bd.dm05_set_row_block_override(0)
 
 
-def run_gpu(inp, splits=0, with_lse=True, stream=None):
+def run_gpu(inp, splits=0, with_lse=True, stream=None, row_blocks=0):
     d = inp.to("cuda")
     assert bd.dm05_set_split_override(splits) == 0
+    assert bd.dm05_set_row_block_override(row_blocks) == 0
     try:
         out, lse = bd.suffix_attn(d.q, d.k_prefix, d.v_prefix, d.k_suffix, d.v_suffix,
                                   prefix_valid_len=d.prefix_valid_len, prefix_mask=d.prefix_mask,
@@ -77,6 +105,7 @@ def run_gpu(inp, splits=0, with_lse=True, stream=None):
         torch.cuda.synchronize()
     finally:
         bd.dm05_set_split_override(0)
+        bd.dm05_set_row_block_override(0)
     rc, word = bd.dm05_get_error_word(None)
     assert rc == 0
     return out.cpu(), (lse.cpu() if lse is not None else None), word
@@ -124,7 +153,7 @@ def test_small_shapes(case):
     inp = make_small(*case)
     out, lse, word = run_gpu(inp)
     o_ref, l_ref = ref(inp)
-    check_close(out, lse, o_ref, l_ref, case[0])
+    check_close(out, lse, o_ref, l_ref, case[0], keys=visible_keys(inp))
     assert word == 0
 
 
@@ -137,12 +166,61 @@ def test_every_split_count(splits):
     check_close(out, lse, o_ref, l_ref, f"splits={splits}")
 
 
+# Query row blocks forced (the automatic plan picks them from occupancy, so a
+# different SM count would reach other block counts): each (sample, KV head)'s
+# S queries cut into `rb` blocks of ceil(S / rb) queries per head, the last
+# one short, for 1, 2, 4 and 8 query heads per KV head, with a prefix mask.
+ROW_BLOCK_CASES = [
+    # Hq, Hkv, S, row_blocks, splits: queries per head per block, last block
+    (8, 4, 50, 2, 2),    # 25 / 25
+    (8, 4, 50, 4, 8),    # 13 / 13 / 13 / 11
+    (8, 4, 50, 4, 2),
+    (8, 4, 60, 8, 8),    # 8 x 7 / 4
+    (8, 4, 64, 8, 2),    # 8 x 8
+    (4, 4, 50, 4, 8),    # G = 1
+    (4, 4, 100, 8, 2),   # G = 1: 13 x 7 / 9
+    (4, 4, 128, 16, 8),  # G = 1: 16 blocks of 8
+    (8, 2, 30, 2, 8),    # G = 4: 15 / 15
+    (8, 2, 30, 4, 2),    # G = 4: 8 / 8 / 8 / 6
+    (8, 1, 16, 2, 4),    # G = 8: 8 / 8
+]
+
+
+@pytest.mark.parametrize("case", ROW_BLOCK_CASES, ids=[f"G{c[0] // c[1]}_S{c[2]}_rb{c[3]}_c{c[4]}" for c in ROW_BLOCK_CASES])
+def test_forced_row_blocks(case):
+    Hq, Hkv, S, rb, splits = case
+    P = 700
+    inp = gen.make_inputs(2, Hq, Hkv, P, S, 256, 500 + rb * 10 + splits, valid_range=(300, P),
+                          mask_frac=0.1, peak_frac=0.02, peak_mult=4.0)
+    assert bd.dm05_set_split_override(splits) == 0 and bd.dm05_set_row_block_override(rb) == 0
+    try:
+        rc, got_splits, _, got_rb = bd.dm05_suffix_attn_plan(2, Hq, Hkv, P, S, 256)
+    finally:
+        bd.dm05_set_split_override(0)
+        bd.dm05_set_row_block_override(0)
+    assert rc == 0 and (got_splits, got_rb) == (splits, rb), (got_splits, got_rb)
+    out, lse, word = run_gpu(inp, splits=splits, row_blocks=rb)
+    assert word == 0
+    check_close(out, lse, *ref(inp), what=f"G={Hq // Hkv} S={S} row_blocks={rb} splits={splits}")
+
+
+def test_row_block_override_falls_back_when_blocks_would_be_too_small():
+    # 8 blocks of S=50 would hold 7 queries per head (< 8): one block is used
+    assert bd.dm05_set_split_override(4) == 0 and bd.dm05_set_row_block_override(8) == 0
+    try:
+        rc, splits, _, rb = bd.dm05_suffix_attn_plan(1, 8, 4, 1024, 50, 256)
+    finally:
+        bd.dm05_set_split_override(0)
+        bd.dm05_set_row_block_override(0)
+    assert rc == 0 and splits == 4 and rb == 1
+
+
 def test_splits_beyond_tiles():
     # 16 CTAs for a unit with only 2 tiles: most CTAs get no work
     inp = gen.make_inputs(2, 8, 4, 64, 10, 256, 5, valid_len=[40, 0])
     out, lse, _ = run_gpu(inp, splits=16)
     o_ref, l_ref = ref(inp)
-    check_close(out, lse, o_ref, l_ref, "splits beyond tiles")
+    check_close(out, lse, o_ref, l_ref, "splits beyond tiles", keys=visible_keys(inp))
 
 
 def ramp_case(top):

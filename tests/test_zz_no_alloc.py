@@ -3,9 +3,11 @@
 dm05_suffix_attn_noalloc serves callers that must not allocate device memory
 (for example a serving process that has reserved nearly all of HBM for its
 KV cache, or a real-time control loop that cannot take cudaMalloc's implicit
-synchronisation).  It keeps its only scratch, the kernel's error word, in a
-fixed array inside the library.  This file is collected last on purpose: a
-run that stops at the first failure has then already run every other test.
+synchronisation).  Its scratch, the kernel's error word and the partial
+results of split calls, lives in one fixed 8 MiB array inside the library;
+when a split's partials would not fit, the call uses fewer CTAs per
+(sample, KV head).  This file is collected last on purpose: a run that stops
+at the first failure has then already run every other test.
 """
 import numpy as np
 import pytest
@@ -70,3 +72,75 @@ def test_noalloc_rejects_bad_arguments_before_launch():
     sq = -(-50 // row_blocks)
     need = 256 + (4 * row_blocks * splits * 2 * sq * 1040 if splits > 1 else 0)
     np.testing.assert_equal(need <= 8 << 20, True)
+
+
+PART_ROW_BYTES = 256 * 4 + 16   # one partial row: 256 fp32 of O and a float4 of statistics
+SCRATCH_BYTES = 8 << 20
+
+
+def _partial_bytes(units, splits, row_blocks, G, S):
+    sq = -(-S // row_blocks)
+    return units * row_blocks * splits * G * sq * PART_ROW_BYTES if splits > 1 else 0
+
+
+def _call_noalloc(d, out, lse, stream):
+    return bd.dm05_suffix_attn_noalloc(_ptr(d.q), _ptr(d.k_prefix), _ptr(d.v_prefix), _ptr(d.prefix_valid_len),
+                                       _ptr(d.prefix_mask), _ptr(d.k_suffix), _ptr(d.v_suffix), _ptr(out),
+                                       _ptr(lse), d.B, d.Hq, d.Hkv, d.P, d.S, d.D, stream)
+
+
+@pytest.mark.parametrize("B", [2, 32])
+def test_noalloc_uses_fewer_ctas_when_partials_do_not_fit(B):
+    # With 16 CTAs per (sample, KV head) the partial results of B = 2 (about
+    # 13 MB) or B = 32 (about 213 MB) do not fit the 8 MiB array: the call
+    # halves the split count until they do (to 8 for B = 2, to 1 for B = 32)
+    # and must still give the allocating entry point's result.
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    inp = gen.make_inputs(B, 8, 4, 1024, 50, 256, 4100 + B, valid_range=(576, 1024), mask_frac=0.1,
+                          peak_frac=0.01, peak_mult=4.0)
+    d = inp.to("cuda")
+    stream = torch.cuda.current_stream().cuda_stream
+    assert bd.dm05_set_split_override(16) == bd.DM05_OK
+    try:
+        rc, splits, _, row_blocks = bd.dm05_suffix_attn_plan(B, 8, 4, 1024, 50, 256)
+        assert rc == bd.DM05_OK and splits == 16
+        assert _partial_bytes(B * 4, splits, row_blocks, 2, 50) > SCRATCH_BYTES - 256
+        want_out, want_lse = bd.suffix_attn(d.q, d.k_prefix, d.v_prefix, d.k_suffix, d.v_suffix,
+                                            prefix_valid_len=d.prefix_valid_len, prefix_mask=d.prefix_mask)
+        for call in range(2):
+            out = torch.full_like(want_out, float("nan"))
+            lse = torch.full_like(want_lse, float("nan"))
+            assert _call_noalloc(d, out, lse, stream) == bd.DM05_OK
+            torch.cuda.synchronize()
+            rc, word = bd.dm05_get_error_word(stream)
+            assert rc == bd.DM05_OK and word == 0, hex(word)
+            err = (out.float() - want_out.float()).abs()
+            assert bool(torch.isfinite(out.float()).all()), f"call {call}: non-finite output"
+            assert float(err.max()) <= MAX_ABS and float(err.mean()) <= MEAN_ABS, (call, float(err.max()))
+            assert float((lse - want_lse).abs().max()) <= LSE_ABS
+    finally:
+        bd.dm05_set_split_override(0)
+
+
+def test_noalloc_error_bits_are_readable():
+    # A prefix_valid_len outside [0, P] is clamped and flagged in the fixed
+    # array's error word; dm05_get_error_word returns the flag and clears it.
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    inp = gen.make_inputs(2, 8, 4, 128, 10, 256, 4200, valid_len=[-3, 999])
+    d = inp.to("cuda")
+    stream = torch.cuda.current_stream().cuda_stream
+    assert bd.dm05_get_error_word(stream)[0] == bd.DM05_OK  # clears earlier bits
+    out = torch.empty((2, 8, 10, 256), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((2, 8, 10), dtype=torch.float32, device="cuda")
+    assert _call_noalloc(d, out, lse, stream) == bd.DM05_OK
+    rc, word = bd.dm05_get_error_word(stream)
+    assert rc == bd.DM05_OK and word & bd.DM05_EW_VALID_LEN_CLAMPED, hex(word)
+    rc, word = bd.dm05_get_error_word(stream)
+    assert rc == bd.DM05_OK and word == 0, "the bits must be cleared by the read"
+    want_out, want_lse = bd.suffix_attn(d.q, d.k_prefix, d.v_prefix, d.k_suffix, d.v_suffix,
+                                        prefix_valid_len=d.prefix_valid_len)
+    torch.cuda.synchronize()
+    assert float((out.float() - want_out.float()).abs().max()) <= MAX_ABS
+    assert float((lse - want_lse).abs().max()) <= LSE_ABS

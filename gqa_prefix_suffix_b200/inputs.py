@@ -182,6 +182,66 @@ def batched_mask() -> SuffixAttnInputs:
                        name="batched_b32_p1024_s50_mask")
 
 
+# --- prefix prefill (the step that fills the prefix KV cache) ---------------
+
+@dataclass
+class PrefillInputs:
+    """One prefix-prefill attention call: the P prefix positions attend to
+    the prefix K/V of the same call under the prefix-causal mask."""
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    P: int
+    D: int
+    q: torch.Tensor                      # bf16 [B,Hq,P,D]
+    k: torch.Tensor                      # bf16 [B,Hkv,P,D]
+    v: torch.Tensor                      # bf16 [B,Hkv,P,D]
+    valid_len: Optional[torch.Tensor] = None   # int32 [B]
+
+    def to(self, device):
+        mv = lambda t: None if t is None else t.to(device)
+        return PrefillInputs(self.name, self.B, self.Hq, self.Hkv, self.P, self.D, mv(self.q), mv(self.k),
+                             mv(self.v), mv(self.valid_len))
+
+    def tensors(self):
+        return dict(q=self.q, k=self.k, v=self.v, valid_len=self.valid_len)
+
+
+def make_prefill_inputs(B: int, Hq: int, Hkv: int, P: int, D: int, seed: int, *, valid_len=None,
+                        valid_range=None, name: str = "prefill") -> PrefillInputs:
+    """Seeded prefill inputs: valid length (fixed, per-sample list, or drawn
+    from an inclusive range first), then fp32 N(0,1) Q [B,Hq,P,D], K, V
+    [B,Hkv,P,D] in that order, each rounded once to bf16.  Padding rows keep
+    ordinary data."""
+    gen = torch.Generator().manual_seed(int(seed))
+    if valid_range is not None:
+        lo, hi = valid_range
+        vl = torch.randint(int(lo), int(hi) + 1, (B,), generator=gen, dtype=torch.int64).to(torch.int32)
+    elif valid_len is None:
+        vl = None
+    elif isinstance(valid_len, int):
+        vl = torch.full((B,), valid_len, dtype=torch.int32)
+    else:
+        vl = torch.tensor(list(valid_len), dtype=torch.int32)
+    bf = torch.bfloat16
+    q = _randn(gen, (B, Hq, P, D)).to(bf)
+    k = _randn(gen, (B, Hkv, P, D)).to(bf)
+    v = _randn(gen, (B, Hkv, P, D)).to(bf)
+    return PrefillInputs(name, B, Hq, Hkv, P, D, q, k, v, vl)
+
+
+def prefill_base() -> PrefillInputs:
+    """Prefix prefill of the base-model chunk's prefix: B=1, P=1024 bucket
+    with 900 valid positions, 8/4 heads (the prefix decoder's shape), D=256."""
+    return make_prefill_inputs(1, HQ, HKV, 1024, HEAD_DIM, 5001, valid_len=900, name="prefill_b1_p1024_v900")
+
+
+def prefill_history() -> PrefillInputs:
+    """Prefix prefill of the history demo's prefix: B=1, P=2048, 1900 valid."""
+    return make_prefill_inputs(1, HQ, HKV, 2048, HEAD_DIM, 5002, valid_len=1900, name="prefill_b1_p2048_v1900")
+
+
 WORKLOADS = {
     "libero_tiny": libero_tiny,
     "base_chunk": base_chunk,

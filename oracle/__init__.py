@@ -71,6 +71,8 @@ class Oracle:
         lib.oracle_suffix_attn.restype = i
         lib.oracle_merge_parts.argtypes = [p, p, i, ctypes.c_long, i, p, p]
         lib.oracle_merge_parts.restype = i
+        lib.oracle_prefix_causal_attn.argtypes = [p] * 6 + [i] * 6
+        lib.oracle_prefix_causal_attn.restype = i
         lib.oracle_max_threads.argtypes = []
         lib.oracle_max_threads.restype = i
         self.lib = lib
@@ -127,6 +129,27 @@ class Oracle:
             raise ValueError(f"oracle_merge_parts failed with status {rc}")
         return out, lse
 
+    def prefix_causal_attn(self, q, k, v, valid_len, B, Hq, Hkv, P, D, nthreads: int = 1, fill=0.0):
+        """Prefix-prefill attention under the prefix-causal mask.
+
+        q [B,Hq,P,D], k/v [B,Hkv,P,D] (bf16 tensors or uint16 bit patterns),
+        valid_len int32 [B] or None.  Returns (out float64 [B,Hq,P,D], lse
+        float64 [B,Hq,P]); rows at or past a sample's valid length are not
+        computed and keep the value `fill`."""
+        qb, kb, vb = _bits(q), _bits(k), _bits(v)
+        if qb.size != B * Hq * P * D or kb.size != B * Hkv * P * D or vb.size != B * Hkv * P * D:
+            raise ValueError("q/k/v size does not match the dims")
+        vl = None
+        if valid_len is not None:
+            vl = np.ascontiguousarray(np.asarray(valid_len, dtype=np.int32).reshape(B))
+        out = np.full((B, Hq, P, D), fill, dtype=np.float64)
+        lse = np.full((B, Hq, P), fill, dtype=np.float64)
+        rc = self.lib.oracle_prefix_causal_attn(_ptr(qb), _ptr(kb), _ptr(vb), _ptr(vl), _ptr(out), _ptr(lse),
+                                                B, Hq, Hkv, P, D, int(nthreads))
+        if rc != 0:
+            raise ValueError(f"oracle_prefix_causal_attn failed with status {rc}")
+        return out, lse
+
     def inputs_call(self, inp, nthreads: int = 1, key_range=None, row_range=None):
         """Run on an object with the attributes of a SuffixAttnInputs."""
         return self.suffix_attn(inp.q, inp.k_prefix, inp.v_prefix, inp.prefix_valid_len,
@@ -156,6 +179,11 @@ def suffix_attn(*args, **kwargs):
 def merge_parts(o_parts, lse_parts):
     """Oracle.merge_parts on the default build."""
     return default().merge_parts(o_parts, lse_parts)
+
+
+def prefix_causal_attn(*args, **kwargs):
+    """Oracle.prefix_causal_attn on the default build."""
+    return default().prefix_causal_attn(*args, **kwargs)
 
 
 def inputs_call(inp, nthreads: int = 1, key_range=None, row_range=None):

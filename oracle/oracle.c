@@ -251,6 +251,87 @@ int oracle_merge_parts(const double *o_parts, const double *lse_parts, int n_par
     return 0;
 }
 
+/*
+ * Prefix-prefill attention under the prefix-causal mask (page
+ * "TensorRT+Triton+FlexAttention: OpenDM VLA 快速推理加速栈深度剖析", section
+ * 2.3: the prefix stage runs its attention through flex_attention with a
+ * custom causal mask mapping built by _make_prefix_causal_mask_mapping).
+ * The queries are the P prefix positions themselves and the keys/values the
+ * prefix K/V of the same call (the tensors that later form the prefix KV
+ * cache the suffix attention reads).
+ *
+ * Readings where the page is silent (listed in the design notes):
+ *   - "causal" is the standard rule: prefix query i sees prefix key j iff
+ *     j <= i; positions at or past clamp(valid_len[b], 0, P) are bucket
+ *     padding and are never keys;
+ *   - the query rows i >= valid length are padding: they are not computed
+ *     (their out / lse entries are left as they were);
+ *   - a row with no visible key (valid length 0 cannot reach a computed row)
+ *     cannot occur among the computed rows, since key 0 <= i is in range;
+ *   - GQA, scale 1/sqrt(D) and the natural-log LSE as in the suffix call.
+ *
+ * Layouts: q [B,Hq,P,D], k/v [B,Hkv,P,D] bf16 bit patterns, valid_len int32
+ * [B] or NULL (every position in range), out double [B,Hq,P,D], lse double
+ * [B,Hq,P].  Each row takes the same three passes as attend_row: the logits
+ * and their maximum, the normaliser, the weighted sum of the value rows.
+ * Returns 0, -1 for a NULL pointer, -2 for a bad shape, -7 for no memory.
+ */
+int oracle_prefix_causal_attn(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                              const int32_t *valid_len, double *out, double *lse,
+                              int B, int Hq, int Hkv, int P, int D, int nthreads)
+{
+    if (!q || !k || !v || !out || !lse) return -1;
+    if (B < 1 || Hq < 1 || Hkv < 1 || P < 1 || D < 1 || Hq % Hkv != 0) return -2;
+    const int G = Hq / Hkv;
+    const double inv_sqrt_d = 1.0 / sqrt((double)D);
+    const long n_rows = (long)B * Hq * P;
+    int failed = 0;
+    if (nthreads < 1) nthreads = 1;
+
+#pragma omp parallel num_threads(nthreads) reduction(| : failed)
+    {
+        double *logit = (double *)malloc(sizeof(double) * (size_t)P);
+        if (!logit) {
+            failed = 1;
+        } else {
+#pragma omp for schedule(dynamic, 16)
+            for (long row = 0; row < n_rows; ++row) {
+                const int b = (int)(row / ((long)Hq * P));
+                const int h = (int)((row / P) % Hq);
+                const int i = (int)(row % P);
+                const int vl = clamp_valid_len(valid_len, b, P);
+                if (i >= vl) continue; /* padding query: not computed */
+                const size_t kv_off = ((size_t)b * Hkv + h / G) * (size_t)P * D;
+                const uint16_t *q_row = q + (size_t)row * D;
+                /* visible keys: j <= i (and j < vl, implied since i < vl) */
+                const int n = i + 1;
+                double m = -INFINITY;
+                for (int j = 0; j < n; ++j) {
+                    const uint16_t *k_row = k + kv_off + (size_t)j * D;
+                    double dot = 0.0;
+                    for (int d = 0; d < D; ++d)
+                        dot += bf16_bits_to_double(q_row[d]) * bf16_bits_to_double(k_row[d]);
+                    logit[j] = inv_sqrt_d * dot;
+                    if (logit[j] > m) m = logit[j];
+                }
+                double z = 0.0;
+                for (int j = 0; j < n; ++j) z += exp(logit[j] - m);
+                const double l = m + log(z);
+                double *o_row = out + (size_t)row * D;
+                for (int d = 0; d < D; ++d) o_row[d] = 0.0;
+                for (int j = 0; j < n; ++j) {
+                    const double w = exp(logit[j] - l);
+                    const uint16_t *v_row = v + kv_off + (size_t)j * D;
+                    for (int d = 0; d < D; ++d) o_row[d] += w * bf16_bits_to_double(v_row[d]);
+                }
+                lse[row] = l;
+            }
+            free(logit);
+        }
+    }
+    return failed ? -7 : 0;
+}
+
 /* Number of OpenMP threads this build can use (1 without OpenMP). */
 int oracle_max_threads(void)
 {

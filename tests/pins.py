@@ -285,6 +285,134 @@ def pin_valid_len_clamp_and_boundary(orc):
     assert not np.allclose(run(orc, c6)[0], base_o)
 
 
+# --------------------------------------------------------------------------
+# Prefix-prefill attention under the prefix-causal mask (page
+# "TensorRT+Triton+FlexAttention: OpenDM VLA 快速推理加速栈深度剖析", section
+# 2.3): prefix query i sees prefix key j iff j <= i and j < valid length;
+# query rows at or past the valid length are not computed.
+
+def prefill_case(seed, B, Hq, Hkv, P, D, vl=None):
+    gen = torch.Generator().manual_seed(seed)
+    q = bf16_rand(gen, (B, Hq, P, D))
+    k = bf16_rand(gen, (B, Hkv, P, D))
+    v = bf16_rand(gen, (B, Hkv, P, D))
+    vlt = None if vl is None else torch.tensor(vl, dtype=torch.int32)
+    return dict(q=q, k=k, v=v, valid_len=vlt, B=B, Hq=Hq, Hkv=Hkv, P=P, D=D)
+
+
+def run_prefill(orc, c, fill=float("nan"), **kw):
+    return orc.prefix_causal_attn(c["q"], c["k"], c["v"], c["valid_len"], c["B"], c["Hq"], c["Hkv"], c["P"],
+                                  c["D"], fill=fill, **kw)
+
+
+def prefill_sdpa_reference(c):
+    """float64 library attention with a boolean mask built from the rule
+    (key j visible to query i iff j <= i and j < valid length), LSE through
+    the extra all-zero key as in sdpa_reference."""
+    B, Hq, Hkv, P, D = (c[k] for k in ("B", "Hq", "Hkv", "P", "D"))
+    G = Hq // Hkv
+    f = lambda t: t.to(torch.float64)
+    q, k, v = f(c["q"]), f(c["k"]).repeat_interleave(G, 1), f(c["v"]).repeat_interleave(G, 1)
+    vl = [P] * B if c["valid_len"] is None else [max(0, min(P, int(x))) for x in c["valid_len"]]
+    i = torch.arange(P)[:, None]
+    j = torch.arange(P)[None, :]
+    mask = torch.stack([(j <= i) & (j < vl[b]) for b in range(B)])[:, None].expand(B, Hq, P, P)
+    out = torch.nn.functional.scaled_dot_product_attention(q, k, v, attn_mask=mask)
+    k_x = torch.cat([k, torch.zeros(B, Hq, 1, D, dtype=torch.float64)], dim=2)
+    v_x = torch.cat([torch.cat([v, torch.zeros(B, Hq, P, 1, dtype=torch.float64)], dim=3),
+                     torch.cat([torch.zeros(B, Hq, 1, D, dtype=torch.float64),
+                                torch.ones(B, Hq, 1, 1, dtype=torch.float64)], dim=3)], dim=2)
+    mask_x = torch.cat([mask, torch.ones(B, Hq, P, 1, dtype=torch.bool)], dim=3)
+    w = torch.nn.functional.scaled_dot_product_attention(q, k_x, v_x, attn_mask=mask_x)[..., D]
+    return out.numpy(), torch.log(1.0 / w - 1.0).numpy(), vl
+
+
+PREFILL_SHAPES = [
+    # seed, B, Hq, Hkv, P, D, valid lengths
+    (41, 1, 2, 1, 5, 4, None),
+    (42, 2, 4, 2, 7, 8, [7, 3]),
+    (43, 2, 8, 4, 9, 16, [9, 1]),
+    (44, 1, 4, 1, 6, 256, [4]),
+]
+
+
+def pin_prefill_sdpa_float64(orc):
+    """Computed rows equal float64 library attention under the causal and
+    padding mask; rows at or past the valid length are left untouched."""
+    for seed, B, Hq, Hkv, P, D, vl in PREFILL_SHAPES:
+        c = prefill_case(seed, B, Hq, Hkv, P, D, vl)
+        o, lse = run_prefill(orc, c, fill=-7.0)
+        o_ref, l_ref, vls = prefill_sdpa_reference(c)
+        for b in range(B):
+            n = vls[b]
+            np.testing.assert_allclose(o[b, :, :n], o_ref[b, :, :n], rtol=0, atol=1e-12,
+                                       err_msg=f"prefill O vs float64 SDPA, seed {seed}")
+            np.testing.assert_allclose(lse[b, :, :n], l_ref[b, :, :n], rtol=0, atol=1e-9,
+                                       err_msg=f"prefill LSE vs float64 SDPA, seed {seed}")
+            assert (o[b, :, n:] == -7.0).all() and (lse[b, :, n:] == -7.0).all(), "padding rows written"
+
+
+def pin_prefill_first_row_and_uniform(orc):
+    """Row 0 sees only key 0: O = V row 0 and LSE = <q_0, k_0> / sqrt(D).
+    With Q = 0 every visible logit is 0: row i is the mean of V rows 0..i and
+    its LSE is ln(i + 1)."""
+    c = prefill_case(45, 1, 4, 2, 8, 16)
+    o, lse = run_prefill(orc, c)
+    for h in range(4):
+        kv = h // 2
+        q0 = c["q"][0, h, 0].to(torch.float64).numpy()
+        k0 = c["k"][0, kv, 0].to(torch.float64).numpy()
+        np.testing.assert_array_equal(o[0, h, 0], c["v"][0, kv, 0].to(torch.float64).numpy())
+        assert abs(lse[0, h, 0] - float(np.dot(q0, k0)) / 4.0) < 1e-12
+    c["q"] = torch.zeros_like(c["q"])
+    o, lse = run_prefill(orc, c)
+    v = c["v"].to(torch.float64).numpy()
+    for h in range(4):
+        for i in range(8):
+            np.testing.assert_allclose(o[0, h, i], v[0, h // 2, :i + 1].mean(axis=0), rtol=0, atol=1e-13)
+            assert abs(lse[0, h, i] - math.log(i + 1)) < 1e-13
+
+
+def pin_prefill_future_keys_ignored(orc):
+    """NaN in the K/V rows from position t on changes no row before t
+    (causality); NaN at or past the valid length changes no computed row."""
+    c = prefill_case(46, 2, 4, 2, 10, 8, [10, 6])
+    o0, l0 = run_prefill(orc, c, fill=0.0)
+    t = 5
+    c1 = dict(c, k=c["k"].clone(), v=c["v"].clone())
+    c1["k"][:, :, t:] = float("nan")
+    c1["v"][:, :, t:] = float("nan")
+    o1, l1 = run_prefill(orc, c1, fill=0.0)
+    assert np.array_equal(o1[:, :, :t], o0[:, :, :t]) and np.array_equal(l1[:, :, :t], l0[:, :, :t])
+    c2 = dict(c, k=c["k"].clone(), v=c["v"].clone())
+    c2["k"][1, :, 6:] = float("nan")
+    c2["v"][1, :, 6:] = float("nan")
+    o2, l2 = run_prefill(orc, c2, fill=0.0)
+    assert np.array_equal(o2, o0) and np.array_equal(l2, l0)
+
+
+def pin_prefill_decimal_bruteforce(orc):
+    """60-digit decimal brute force of the causal softmax on a tiny case."""
+    decimal.getcontext().prec = 60
+    c = prefill_case(47, 1, 2, 1, 5, 4, [4])
+    o, lse = run_prefill(orc, c)
+    D = 4
+    K = _dec_bf16(c["k"][0, 0])
+    V = _dec_bf16(c["v"][0, 0])
+    half = decimal.Decimal(1) / decimal.Decimal(D).sqrt()
+    for h in range(2):
+        for i in range(4):
+            qrow = _dec_bf16(c["q"][0, h, i])
+            logits = [half * sum(qrow[d] * K[j * D + d] for d in range(D)) for j in range(i + 1)]
+            z = sum(l.exp() for l in logits)
+            for d in range(D):
+                want = sum((l.exp() / z) * V[j * D + d] for j, l in enumerate(logits))
+                assert abs(float(want) - o[0, h, i, d]) < 1e-14
+            assert abs(float(z.ln()) - lse[0, h, i]) < 1e-14
+
+
 ALL_PINS = [pin_sdpa_float64, pin_uniform_logits, pin_constant_v_gqa, pin_masked_rows_ignored,
             pin_single_suffix_key, pin_dominant_key, pin_prefix_permutation, pin_split_merge,
-            pin_decimal_bruteforce, pin_valid_len_clamp_and_boundary]
+            pin_decimal_bruteforce, pin_valid_len_clamp_and_boundary,
+            pin_prefill_sdpa_float64, pin_prefill_first_row_and_uniform, pin_prefill_future_keys_ignored,
+            pin_prefill_decimal_bruteforce]

@@ -28,12 +28,14 @@ def _bad(case):
         "lse": dict(lse=torch.zeros(1, 8, 10, dtype=torch.float64, device=dev)),                    # wrong dtype
         "lse ": dict(lse=torch.zeros(1, 8, 9, dtype=torch.float32, device=dev)),                    # too small
         "out  ": dict(out=torch.zeros(1, 8, 10, 256, dtype=torch.bfloat16)),                        # on the host
-        "prefix_valid_len": dict(prefix_valid_len=torch.zeros(2, dtype=torch.int32, device=dev)[::2]),  # strided
+        "prefix_valid_len": dict(prefix_valid_len=torch.zeros(1, dtype=torch.int64, device=dev)),   # wrong dtype
+        "prefix_valid_len ": dict(prefix_valid_len=torch.zeros(2, dtype=torch.int32, device=dev)),  # B + 1 values
         "prefix_mask": dict(prefix_mask=torch.ones(1, 63, dtype=torch.uint8, device=dev)),
     }[case]
 
 
-@pytest.mark.parametrize("what", ["out", "out ", "out  ", "lse", "lse ", "prefix_valid_len", "prefix_mask"])
+@pytest.mark.parametrize("what", ["out", "out ", "out  ", "lse", "lse ", "prefix_valid_len", "prefix_valid_len ",
+                                  "prefix_mask"])
 def test_device_binding_rejects_bad_tensors(what):
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
@@ -42,3 +44,12 @@ def test_device_binding_rejects_bad_tensors(what):
     q, kp, vp, ks, vs = a.pop("q"), a.pop("k_prefix"), a.pop("v_prefix"), a.pop("k_suffix"), a.pop("v_suffix")
     with pytest.raises(ValueError, match=what.strip()):
         bd.suffix_attn(q, kp, vp, ks, vs, **a)
+
+
+def test_device_binding_rejects_a_strided_valid_len():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    a = _inputs(B=2)
+    vl = torch.zeros(4, dtype=torch.int32, device="cuda")[::2]   # 2 values, stride 2
+    with pytest.raises(ValueError, match="prefix_valid_len"):
+        bd.suffix_attn(a["q"], a["k_prefix"], a["v_prefix"], a["k_suffix"], a["v_suffix"], prefix_valid_len=vl)

@@ -38,6 +38,17 @@ MUTATIONS = {
     "merge_total_is_max": ("double total = m + log(z);", "double total = m;"),
     "merge_skips_first_part": ("for (int s = 0; s < n_parts; ++s) {\n            double l = lse_parts[(size_t)s * rows + r];\n            if (l == -INFINITY) continue;",
                                "for (int s = 1; s < n_parts; ++s) {\n            double l = lse_parts[(size_t)s * rows + r];\n            if (l == -INFINITY) continue;"),
+    # prefix-prefill attention under the prefix-causal mask
+    "prefill_sees_one_key_too_few": ("const int n = i + 1;", "const int n = i;"),
+    "prefill_sees_future_keys": ("const int n = i + 1;", "const int n = vl;"),
+    "prefill_computes_padding_rows": ("if (i >= vl) continue; /* padding query: not computed */",
+                                      "if (i > vl) continue;"),
+    "prefill_gqa_modulo": ("const size_t kv_off = ((size_t)b * Hkv + h / G)",
+                           "const size_t kv_off = ((size_t)b * Hkv + h % Hkv)"),
+    "prefill_scale_missing": ("logit[j] = inv_sqrt_d * dot;", "logit[j] = dot;"),
+    "prefill_lse_without_max": ("const double l = m + log(z);", "const double l = log(z);"),
+    "prefill_k_used_as_v": ("const uint16_t *v_row = v + kv_off + (size_t)j * D;",
+                            "const uint16_t *v_row = k + kv_off + (size_t)j * D;"),
 }
 
 

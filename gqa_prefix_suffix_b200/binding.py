@@ -28,7 +28,8 @@ EXPORTS = ("dm05_suffix_attn", "dm05_suffix_attn_workspace_bytes", "dm05_suffix_
            "dm05_suffix_attn_plan", "dm05_set_split_override", "dm05_set_row_block_override",
            "dm05_get_error_word",
            "dm05_status_string", "dm05_release", "dm05_suffix_attn_noalloc", "dm05_suffix_attn_host",
-           "dm05_suffix_attn_host_copy_bytes", "dm05_selftest_wait_timeout")
+           "dm05_suffix_attn_host_copy_bytes", "dm05_selftest_wait_timeout", "dm05_prefix_prefill_attn",
+           "dm05_prefix_prefill_reserve", "dm05_prefix_prefill_plan")
 
 _lock = threading.Lock()
 _lib = None
@@ -77,6 +78,12 @@ def lib() -> ctypes.CDLL:
             L.dm05_suffix_attn_host_copy_bytes.restype = i
             L.dm05_selftest_wait_timeout.argtypes = [i, p]
             L.dm05_selftest_wait_timeout.restype = i
+            L.dm05_prefix_prefill_attn.argtypes = [p] * 6 + [i] * 5 + [p]
+            L.dm05_prefix_prefill_attn.restype = i
+            L.dm05_prefix_prefill_reserve.argtypes = [i] * 5 + [p]
+            L.dm05_prefix_prefill_reserve.restype = i
+            L.dm05_prefix_prefill_plan.argtypes = [i] * 5 + [ctypes.POINTER(i)] * 3
+            L.dm05_prefix_prefill_plan.restype = i
             _lib = L
     return _lib
 
@@ -111,6 +118,22 @@ def dm05_suffix_attn_host_copy_bytes(prefix_valid_len, has_prefix_mask, want_lse
     rc = lib().dm05_suffix_attn_host_copy_bytes(prefix_valid_len, int(bool(has_prefix_mask)), int(bool(want_lse)),
                                                 B, Hq, Hkv, P, S, D, ctypes.byref(h), ctypes.byref(d))
     return rc, int(h.value), int(d.value)
+
+
+def dm05_prefix_prefill_attn(q, k, v, valid_len, out, lse, B, Hq, Hkv, P, D, stream) -> int:
+    """The prefix-prefill attention under the prefix-causal mask."""
+    return lib().dm05_prefix_prefill_attn(q, k, v, valid_len, out, lse, B, Hq, Hkv, P, D, stream)
+
+
+def dm05_prefix_prefill_reserve(B, Hq, Hkv, P, D, stream) -> int:
+    return lib().dm05_prefix_prefill_reserve(B, Hq, Hkv, P, D, stream)
+
+
+def dm05_prefix_prefill_plan(B, Hq, Hkv, P, D):
+    """Returns (status, splits_per_head, query_block, row_blocks)."""
+    sp, qb, rb = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int(0)
+    rc = lib().dm05_prefix_prefill_plan(B, Hq, Hkv, P, D, ctypes.byref(sp), ctypes.byref(qb), ctypes.byref(rb))
+    return rc, sp.value, qb.value, rb.value
 
 
 def dm05_suffix_attn_workspace_bytes(B, Hq, Hkv, P, S, D) -> int:
@@ -255,6 +278,41 @@ def suffix_attn_host(q, k_prefix, v_prefix, k_suffix, v_suffix, prefix_valid_len
                                _stream_handle(stream))
     if rc != DM05_OK:
         raise Dm05Error(rc, "dm05_suffix_attn_host")
+    return out, lse
+
+
+def prefix_prefill_attn(q, k, v, valid_len=None, out=None, lse=None, want_lse: bool = True, stream=None):
+    """Prefix-prefill attention on CUDA torch tensors; returns (out, lse or None).
+
+    q [B,Hq,P,D] bf16; k/v [B,Hkv,P,D] bf16; valid_len int32 [B] or None.
+    Rows at or past a sample's valid length are not written (a fresh out /
+    lse is allocated uninitialised when not given)."""
+    import torch
+    B, Hq, P, D = q.shape
+    Hkv = k.shape[1]
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA bfloat16 tensor")
+    if tuple(k.shape) != (B, Hkv, P, D) or tuple(v.shape) != (B, Hkv, P, D):
+        raise ValueError("k/v must be [B,Hkv,P,D]")
+    if valid_len is not None and (not valid_len.is_cuda or valid_len.dtype != torch.int32 or valid_len.numel() != B
+                                  or not valid_len.is_contiguous()):
+        raise ValueError("valid_len must be a contiguous CUDA int32 tensor of B values")
+    if out is None:
+        out = torch.empty((B, Hq, P, D), dtype=torch.bfloat16, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq, P), dtype=torch.float32, device=q.device)
+    for name, t, shape, dt in (("out", out, (B, Hq, P, D), torch.bfloat16), ("lse", lse, (B, Hq, P), torch.float32)):
+        if t is not None and (not t.is_cuda or t.dtype != dt or tuple(t.shape) != shape or not t.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous CUDA {dt} tensor {list(shape)}")
+    for name, t in (("k", k), ("v", v), ("valid_len", valid_len), ("out", out), ("lse", lse)):
+        if t is not None and t.device != q.device:
+            raise ValueError(f"{name} must be on {q.device} like q")
+    ptr = lambda t: None if t is None else t.data_ptr()
+    rc = dm05_prefix_prefill_attn(ptr(q), ptr(k), ptr(v), ptr(valid_len), ptr(out), ptr(lse), B, Hq, Hkv, P, D,
+                                  _stream_handle(stream))
+    if rc != DM05_OK:
+        raise Dm05Error(rc, "dm05_prefix_prefill_attn")
     return out, lse
 
 

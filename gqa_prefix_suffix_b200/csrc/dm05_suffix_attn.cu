@@ -146,6 +146,47 @@ Plan make_plan(int B, int Hq, int Hkv, int P, int S, const DeviceState &ds)
     return best;
 }
 
+// Work decomposition of a prefix-prefill call: each (sample, KV head)'s P
+// query positions are cut into blocks of SQ per head (G * SQ <= 128 MMA
+// rows); a block's causal key range is split over `splits` CTAs (a
+// cluster, merged as in the suffix call).  The longest block has all
+// ceil(P / 64) key tiles; the split count is the cheapest by the same cost
+// model among plans whose clusters are all resident at once.
+Plan make_prefill_plan(int B, int Hq, int Hkv, int P, const DeviceState &ds)
+{
+    const long long units = static_cast<long long>(B) * Hkv;
+    const int G = Hq / Hkv;
+    Plan pl;
+    const int sq = (dm05::kMRows / G) / 8 * 8;
+    if (P <= sq) {
+        pl.SQ = P;  // one block: the whole unit
+        pl.row_blocks = 1;
+    } else {
+        pl.SQ = sq;
+        pl.row_blocks = (P + sq - 1) / sq;
+    }
+    const int tiles = (P + kTileRows - 1) / kTileRows;
+    auto cost = [&](int c) {
+        double t = 1.2 * ((tiles + c - 1) / c);
+        if (c > 1) t += 2.0 + 0.04 * G * pl.SQ;
+        return t;
+    };
+    double best = 1e30;
+    for (int c = 1; c <= 16; c *= 2) {
+        if (g_split_override > 0 && c != g_split_override) continue;
+        if (g_split_override == 0 && c > 1 &&
+            (c > ds.max_cluster || units * pl.row_blocks * c > ds.num_sms ||
+             units * pl.row_blocks > ds.active[log2_pow2(c)]))
+            continue;
+        if (cost(c) < best) {
+            best = cost(c);
+            pl.splits = c;
+        }
+    }
+    if (pl.splits > ds.max_cluster) pl.splits = ds.max_cluster;
+    return pl;
+}
+
 int get_encoder()
 {
     if (g_encode) return DM05_OK;
@@ -399,7 +440,7 @@ int encode_3d(CUtensorMap *map, const void *base, uint64_t d1, uint64_t d2, uint
 int launch_attention(const void *q, const void *k_prefix, const void *v_prefix, const int32_t *prefix_valid_len,
                      const uint8_t *prefix_mask, const void *k_suffix, const void *v_suffix, void *out, float *lse,
                      int B, int Hq, int Hkv, int P, int S, int D, const Plan &pl, uint32_t *err, void *part,
-                     cudaStream_t stream)
+                     cudaStream_t stream, bool causal = false)
 {
     const int G = Hq / Hkv;
     const int GS = G * S;
@@ -447,6 +488,7 @@ int launch_attention(const void *q, const void *k_prefix, const void *v_prefix, 
     kp.SQ = pl.SQ;
     kp.splits = pl.splits;
     kp.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
+    kp.causal = causal ? 1 : 0;
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
@@ -595,6 +637,79 @@ int dm05_suffix_attn(const void *q, const void *k_prefix, const void *v_prefix, 
 
     return launch_attention(q, k_prefix, v_prefix, prefix_valid_len, prefix_mask, k_suffix, v_suffix, out, lse, B,
                             Hq, Hkv, P, S, D, pl, err_word, part_ws, stream);
+}
+
+int dm05_prefix_prefill_attn(const void *q, const void *k, const void *v, const int32_t *valid_len, void *out,
+                             float *lse, int B, int Hq, int Hkv, int P, int D, cudaStream_t stream)
+{
+    if (!q || !k || !v || !out) return DM05_ERR_NULL;
+    if (B < 1 || Hq < 1 || Hkv < 1 || P < 1 || Hq % Hkv != 0) return DM05_ERR_SHAPE;
+    if (static_cast<long long>(B) * Hkv > kMaxUnits || P > kMaxPrefix) return DM05_ERR_SHAPE;
+    if (D != dm05::kHeadDim || (Hq / Hkv) * 8 > dm05::kMRows) return DM05_ERR_UNSUPPORTED;
+    if (static_cast<long long>(Hq / Hkv) * P > 0x7fffffffLL) return DM05_ERR_SHAPE;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return DM05_ERR_ALIGN;
+    if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u) != 0) return DM05_ERR_ALIGN;
+    const int G = Hq / Hkv;
+    const int units = B * Hkv;
+    uint32_t *err_word = nullptr;
+    Plan pl;
+    void *part_ws = nullptr;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (get_encoder() != DM05_OK) return DM05_ERR_CUDA;
+        DeviceState *ds = nullptr;
+        int rc = device_state(false, &ds);
+        if (rc != DM05_OK) return rc;
+        if (ds->err == nullptr) {
+            cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+            if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) return DM05_ERR_CUDA;
+            if (cs != cudaStreamCaptureStatusNone) return DM05_ERR_WORKSPACE;
+            rc = device_state(true, &ds, stream);
+            if (rc != DM05_OK) return rc;
+        }
+        pl = make_prefill_plan(B, Hq, Hkv, P, *ds);
+        err_word = ds->err;
+        rc = stream_workspace(stream, partial_bytes(units, pl, G), &part_ws);
+        if (rc != DM05_OK) return rc;
+    }
+    // the queries are the P prefix positions (S = P); no suffix keys exist,
+    // so the suffix maps are never read (the prefix K/V stand in for them)
+    return launch_attention(q, k, v, valid_len, nullptr, k, v, out, lse, B, Hq, Hkv, P, P, D, pl, err_word, part_ws,
+                            stream, true);
+}
+
+int dm05_prefix_prefill_reserve(int B, int Hq, int Hkv, int P, int D, cudaStream_t stream)
+{
+    if (B < 1 || Hq < 1 || Hkv < 1 || P < 1 || Hq % Hkv != 0) return DM05_ERR_SHAPE;
+    if (static_cast<long long>(B) * Hkv > kMaxUnits || P > kMaxPrefix) return DM05_ERR_SHAPE;
+    if (D != dm05::kHeadDim || (Hq / Hkv) * 8 > dm05::kMRows) return DM05_ERR_UNSUPPORTED;
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) return DM05_ERR_CUDA;
+    if (cs != cudaStreamCaptureStatusNone) return DM05_ERR_WORKSPACE;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (get_encoder() != DM05_OK) return DM05_ERR_CUDA;
+    DeviceState *ds = nullptr;
+    int rc = device_state(true, &ds, stream);
+    if (rc != DM05_OK) return rc;
+    const Plan pl = make_prefill_plan(B, Hq, Hkv, P, *ds);
+    void *ws = nullptr;
+    return stream_workspace(stream, partial_bytes(static_cast<long long>(B) * Hkv, pl, Hq / Hkv), &ws);
+}
+
+int dm05_prefix_prefill_plan(int B, int Hq, int Hkv, int P, int D, int *splits_per_head, int *query_block,
+                             int *row_blocks)
+{
+    if (B < 1 || Hq < 1 || Hkv < 1 || P < 1 || Hq % Hkv != 0) return DM05_ERR_SHAPE;
+    if (D != dm05::kHeadDim || (Hq / Hkv) * 8 > dm05::kMRows) return DM05_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lk(g_mu);
+    DeviceState *ds = nullptr;
+    const int rc = device_state(false, &ds);
+    if (rc != DM05_OK) return rc;
+    const Plan pl = make_prefill_plan(B, Hq, Hkv, P, *ds);
+    if (splits_per_head) *splits_per_head = pl.splits;
+    if (query_block) *query_block = pl.SQ;
+    if (row_blocks) *row_blocks = pl.row_blocks;
+    return DM05_OK;
 }
 
 int dm05_selftest_wait_timeout(int limit_ms, cudaStream_t stream)

@@ -60,6 +60,28 @@
 
 namespace dm05 {
 
+// Phase time stamps for timeline studies: compiled in only when DM05_TRACE
+// is defined (never in the library build); each records the SM clock (or,
+// for the first and last slot, the global timer) of one CTA's phase boundary.
+#ifdef DM05_TRACE
+__device__ unsigned long long g_dm05_trace[4096][16];
+#define DM05_TRACE_CLOCK(slot)                                                      \
+    do {                                                                            \
+        if (blockIdx.x < 4096) g_dm05_trace[blockIdx.x][slot] = clock64();          \
+    } while (0)
+#define DM05_TRACE_GTIME(slot)                                                      \
+    do {                                                                            \
+        if (blockIdx.x < 4096) g_dm05_trace[blockIdx.x][slot] = ptx::globaltimer_ns(); \
+    } while (0)
+#else
+#define DM05_TRACE_CLOCK(slot) \
+    do {                       \
+    } while (0)
+#define DM05_TRACE_GTIME(slot) \
+    do {                       \
+    } while (0)
+#endif
+
 constexpr int kHeadDim = 256;
 constexpr int kMRows = 128;                       // MMA M: query rows (padded)
 constexpr int kChunkElems = 64;                   // bf16 per 128-byte swizzle row
@@ -92,6 +114,8 @@ struct KernelParams {
     int SQ;                    // queries per head per block (S when row_blocks == 1)
     int splits;                // CTAs per (unit, query block): the cluster size
     float scale_log2;          // log2(e) / sqrt(D)
+    int causal;                // 0: suffix attention; 1: prefix prefill (queries are the P prefix
+                               // positions, S == P, no suffix keys, key j visible to query i iff j <= i)
 };
 
 template <int NT, int STAGES>
@@ -183,7 +207,8 @@ __device__ __forceinline__ size_t block_out_row(size_t unit_row0, int k, int nq,
     return unit_row0 + static_cast<size_t>(h) * S + q0 + (k - h * nq);
 }
 
-// Combines the nr partial rows this CTA owns: partial c's row rr sits at
+// Combines the nr partial rows this CTA owns (rows whose query index within
+// the block is jlim or more are not written): partial c's row rr sits at
 // recv + (c * nr + rr) * kStageStride (D fp32 of unnormalised O, then
 // {m, l, l_hat, 0}).  One item per (row, 4-column quad); every item derives
 // its row's weights from the C statistics (a shared-memory broadcast within
@@ -193,11 +218,13 @@ __device__ __forceinline__ size_t block_out_row(size_t unit_row0, int k, int nq,
 // A partial without visible keys (l_hat == 0) holds no O and gets no weight.
 template <int C, class L>
 __device__ __forceinline__ void merge_rows(const uint8_t *recv, int nr, __nv_bfloat16 *out, float *lse,
-                                           size_t unit_row0, int k_lo, int nq, int S, int q0)
+                                           size_t unit_row0, int k_lo, int nq, int S, int q0, int jlim)
 {
     const int items = nr * (kHeadDim / 4);
     for (int i = threadIdx.x; i < items; i += kThreads) {
         const int rr = i / (kHeadDim / 4), ch = i - rr * (kHeadDim / 4);
+        // only the queries [0, jlim) of each head of the block are written
+        if ((k_lo + rr) % nq >= jlim) continue;
         float4 st[C], v[C];
 #pragma unroll
         for (int c = 0; c < C; ++c) {
@@ -263,6 +290,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // ---- set-up that reads no input (overlaps the previous kernel under PDL)
     if (threadIdx.x == 0) {
+        DM05_TRACE_GTIME(0);
+        DM05_TRACE_CLOCK(1);
+    }
+    if (threadIdx.x == 0) {
         ptx::mbar_init(&bars[L::kBarQFull], 1);
         ptx::mbar_init(&bars[L::kBarQFree], 1);
         for (int s = 0; s < STAGES; ++s) {
@@ -300,6 +331,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // ---- from here on inputs are read: wait for the preceding grid
     ptx::griddep_wait();
+    if (threadIdx.x == 0) DM05_TRACE_CLOCK(2);
 
     uint8_t *sQ = smem + L::kQOff;
     auto sK = [&](int s) { return smem + s * L::kStageBytes; };
@@ -308,8 +340,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     // depend on valid_len, so its K/V are requested before that read returns.
     // With the suffix tiles first it is the true first tile unless the split
     // boundaries move; then the slot is drained and released (shift below).
-    const int TS = (p.S + NT - 1) / NT;
-    const int t_bucket = TS + (p.P + NT - 1) / NT;
+    // Keys of the unit: the suffix tiles (none in prefill mode), then the
+    // prefix rows [0, key limit).  The key limit is the valid length, or in
+    // prefill mode the causal limit of this query block (no key past its last
+    // query; nothing when the block lies wholly in the padding).
+    const int TS = p.causal ? 0 : (p.S + NT - 1) / NT;
+    auto key_limit = [&](int v) { return p.causal ? (q0 >= v ? 0 : min(v, q0 + nq)) : v; };
+    const int t_bucket = TS + (key_limit(p.P) + NT - 1) / NT;
     const int g_spec = static_cast<int>((static_cast<long long>(t_bucket) * rank) / C);
     const bool spec = g_spec < static_cast<int>((static_cast<long long>(t_bucket) * (rank + 1)) / C);
     uint64_t pol = 0;
@@ -330,7 +367,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                      c * kChunkElems, h * p.S + q0, unit);
         }
         if (spec) {
-            const TileInfo ti = tile_of<NT>(g_spec, TS, p.P, p.S);
+            const TileInfo ti = tile_of<NT>(g_spec, TS, key_limit(p.P), p.S);
             const CUtensorMap *mk = ti.prefix ? &tm_kp : &tm_ks;
             const CUtensorMap *mv = ti.prefix ? &tm_vp : &tm_vs;
             ptx::mbar_arrive_expect_tx(&bars[L::kBarKFull], L::kTileBytes);
@@ -346,7 +383,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         vl = min(max(raw, 0), p.P);
         if (raw != vl && rank == 0 && threadIdx.x == 0) atomicOr(p.err, kEwClamped);
     }
-    const int t_all = TS + (vl + NT - 1) / NT;
+    const int klim = key_limit(vl);
+    // rows of the block that are written: every query, or in prefill mode
+    // the queries before the valid length
+    const int jlim = p.causal ? max(0, min(nq, vl - q0)) : nq;
+    const int t_all = TS + (klim + NT - 1) / NT;
     const int t_begin = static_cast<int>((static_cast<long long>(t_all) * rank) / C);
     const int t_end = static_cast<int>((static_cast<long long>(t_all) * (rank + 1)) / C);
     const int T = t_end - t_begin;
@@ -373,7 +414,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int t = slots - shift; t < T && !failed; ++t) {
                 const int slot = t + shift;
                 const int s = slot % STAGES, n = slot / STAGES;
-                const TileInfo ti = tile_of<NT>(t_begin + t, TS, vl, p.S);
+                const TileInfo ti = tile_of<NT>(t_begin + t, TS, klim, p.S);
                 const CUtensorMap *mk = ti.prefix ? &tm_kp : &tm_ks;
                 const CUtensorMap *mv = ti.prefix ? &tm_vp : &tm_vs;
                 if (n > 0 && !ptx::mbar_wait(&bars[L::kBarKEmpty + s], (n - 1) & 1, kWaitLimitNs)) {
@@ -422,7 +463,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // only the 16-row k-steps that hold valid keys (a partial tile
                 // stops early; the rows after its last valid key up to the
                 // k-step end are zero)
-                const int nk = (tile_of<NT>(t_begin + u, TS, vl, p.S).n_valid + 15) / 16;
+                const int nk = (tile_of<NT>(t_begin + u, TS, klim, p.S).n_valid + 15) / 16;
 #pragma unroll
                 for (int kk = 0; kk < NT / 16; ++kk) {
                     if (kk >= nk) break;
@@ -447,6 +488,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ptx::tmem_cp_128x256b(tmem + kTmemQ + kk * 8,
                                           ptx::sw128_desc(q_base + (kk >> 2) * L::kQChunkBytes + (kk & 3) * 32, 16, 1024));
                 ptx::mma_commit(&bars[L::kBarQFree]);
+                DM05_TRACE_CLOCK(3);
             }
             for (int t = 0; t < T && ok; ++t) {
                 const int s = (t + shift) % STAGES;
@@ -455,6 +497,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ok = false;
                     break;
                 }
+                if (t == 0) DM05_TRACE_CLOCK(14);
                 // S(t) overwrites the TMEM columns that held P(t - kSBufs): the
                 // PV MMA reading them must have completed (issue order alone
                 // does not order one MMA's operand reads before a later MMA's
@@ -468,7 +511,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t d = tmem + kTmemS + sb * NT;
                 // N = the valid keys of the tile rounded up to 16; the
                 // softmax masks every column past the valid ones anyway.
-                const int nv16 = (tile_of<NT>(t_begin + t, TS, vl, p.S).n_valid + 15) / 16 * 16;
+                const int nv16 = (tile_of<NT>(t_begin + t, TS, klim, p.S).n_valid + 15) / 16 * 16;
                 const uint32_t idesc_qk = ptx::idesc_bf16_f32(kMRows, nv16, false);
 #pragma unroll
                 for (int kk = 0; kk < kHeadDim / 16; ++kk) {
@@ -486,9 +529,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             if (ok) ok = issue_pv(T - 1);
+            DM05_TRACE_CLOCK(4);
             // Wait for every MMA issued above before TMEM may be freed.
             ptx::mma_commit(&bars[L::kBarMmaFinal]);
             if (!ptx::mbar_wait(&bars[L::kBarMmaFinal], 0, kWaitLimitNs)) ok = false;
+            DM05_TRACE_CLOCK(5);
             failed = !ok;
         }
     } else {
@@ -499,6 +544,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int q4 = warp & 3;
         const int hf = warp >> 2;
         const int row = q4 * 32 + lane;
+        const int row_h = row / rph;
+        const int row_j = row - row_h * rph;  // query of this row within its head's block
         const int tid = hf * 128 + row;  // 0..255 over the softmax threads
         const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
         const uint8_t *mask_row = p.mask ? p.mask + static_cast<size_t>(b) * p.P : nullptr;
@@ -525,7 +572,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int w = 0; w < NH / 32; ++w) m[w] = 1u;
             if (mask_row == nullptr || t >= T) return;
-            const TileInfo tn = tile_of<NT>(t_begin + t, TS, vl, p.S);
+            const TileInfo tn = tile_of<NT>(t_begin + t, TS, klim, p.S);
             if (!tn.prefix) return;
 #pragma unroll
             for (int w = 0; w < NH / 32; ++w) {
@@ -544,6 +591,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 failed = true;
                 break;
             }
+            if (t == 0 && threadIdx.x == 0) DM05_TRACE_CLOCK(15);
             ptx::tc_fence_after_sync();
             const uint32_t scol = tmem + lane_base + kTmemS + sb * NT;
             uint32_t raw[NH / 16][16];
@@ -551,7 +599,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int j = 0; j < NH / 16; ++j) ptx::tmem_ld16(scol + hf * NH + j * 16, raw[j]);
             ptx::tmem_ld_wait();
 
-            const TileInfo ti = tile_of<NT>(t_begin + t, TS, vl, p.S);
+            const TileInfo ti = tile_of<NT>(t_begin + t, TS, klim, p.S);
             float s[NH];  // raw logits <q, k>; the scale is applied inside the exponent
 #pragma unroll
             for (int c = 0; c < NH; ++c) s[c] = __uint_as_float(raw[c / 16][c % 16]);
@@ -568,6 +616,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int c = 0; c < NH; ++c)
                     if (!((vis[c / 32] >> (c % 32)) & 1u)) s[c] = -INFINITY;
+            }
+            if (p.causal && ti.row0 + NT - 1 > q0) {
+                // prefill: key j is visible to query q0 + row_j only if j <= it
+                const int over = ti.row0 + hf * NH - (q0 + row_j);  // key index - query index at c = 0
+#pragma unroll
+                for (int c = 0; c < NH; ++c)
+                    if (c + over > 0) s[c] = -INFINITY;
             }
             // four independent chains, then combined (max is exact in any order)
             float m4[4] = {s[0], s[1], s[2], s[3]};
@@ -681,21 +736,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!warp_wait(&bars[L::kBarQFull], 0)) failed = true;
             if (spec && (!warp_wait(&bars[L::kBarKFull], 0) || !warp_wait(&bars[L::kBarVFull], 0))) failed = true;
         }
+        if (threadIdx.x == 0) DM05_TRACE_CLOCK(6);
         const bool have_o = T > 0 && !failed;
         if (have_o) {
             // the last PV (every earlier MMA completed before it)
             if (!warp_wait(&bars[L::kBarPFree + (T - 1) % kSBufs], ((T - 1) / kSBufs) & 1)) failed = true;
             ptx::tc_fence_after_sync();
         }
+        if (threadIdx.x == 0) DM05_TRACE_CLOCK(7);
         // row sums over both halves
         xl[hf * kMRows + row] = l;
         xlh[hf * kMRows + row] = lh;
         if (!failed && !pair_sync()) failed = true;
         const float l_row = l + xl[(hf ^ 1) * kMRows + row];
         const float lh_row = lh + xlh[(hf ^ 1) * kMRows + row];
-        const int row_h = row / rph;
-        const int row_j = row - row_h * rph;
-        const bool row_valid = row_h < p.G && row_j < nq;
+        const bool row_valid = row_h < p.G && row_j < jlim;
         const int row_k = row_h * nq + row_j;  // compact row (when valid)
         const size_t out_row = unit_row0 + static_cast<size_t>(row_h) * p.S + q0 + row_j;
         if (C == 1) {
@@ -763,6 +818,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ptx::bulk_commit();
                 ptx::bulk_wait_all();
                 ptx::fence_proxy_async_global();
+                if (threadIdx.x == 0) DM05_TRACE_CLOCK(8);
             }
         }
     }
@@ -774,7 +830,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         // combines rows [r_lo, r_hi) of all C partials:
         //   M = max_c m_c,  LH = sum_c lh_c 2^(m_c - M),  L = sum_c l_c 2^(m_c - M)
         //   out = sum_c 2^(m_c - M) O_c / LH,   lse = (M + log2 L) ln 2.
+        if (threadIdx.x == 0) DM05_TRACE_CLOCK(9);
         ptx::cluster_sync();
+        if (threadIdx.x == 0) DM05_TRACE_CLOCK(10);
         const int r_lo = (NR * rank) / C;  // compact rows of this query block
         const int r_hi = (NR * (rank + 1)) / C;
         const int nr = r_hi - r_lo;
@@ -792,13 +850,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (nr > 0) {
             if (!warp_wait(&bars[L::kBarMerge], 0)) failed = true;
+            if (threadIdx.x == 0) DM05_TRACE_CLOCK(11);
             // the host launches only these cluster sizes; any other is
             // reported and merges nothing
             switch (C) {
-            case 2: merge_rows<2, L>(recv, nr, p.out, p.lse, unit_row0, r_lo, nq, p.S, q0); break;
-            case 4: merge_rows<4, L>(recv, nr, p.out, p.lse, unit_row0, r_lo, nq, p.S, q0); break;
-            case 8: merge_rows<8, L>(recv, nr, p.out, p.lse, unit_row0, r_lo, nq, p.S, q0); break;
-            case 16: merge_rows<16, L>(recv, nr, p.out, p.lse, unit_row0, r_lo, nq, p.S, q0); break;
+            case 2: merge_rows<2, L>(recv, nr, p.out, p.lse, unit_row0, r_lo, nq, p.S, q0, jlim); break;
+            case 4: merge_rows<4, L>(recv, nr, p.out, p.lse, unit_row0, r_lo, nq, p.S, q0, jlim); break;
+            case 8: merge_rows<8, L>(recv, nr, p.out, p.lse, unit_row0, r_lo, nq, p.S, q0, jlim); break;
+            case 16: merge_rows<16, L>(recv, nr, p.out, p.lse, unit_row0, r_lo, nq, p.S, q0, jlim); break;
             default:
                 if (threadIdx.x == 0) atomicOr(p.err, kEwBadSplit);
                 break;
@@ -807,6 +866,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     if (failed) atomicOr(p.err, kEwTimeout);
+    if (threadIdx.x == 0) {
+        DM05_TRACE_CLOCK(12);
+        DM05_TRACE_GTIME(13);
+    }
     __syncwarp();
     ptx::tc_fence_before_sync();
     __syncthreads();

@@ -144,6 +144,53 @@ int dm05_set_split_override(int splits_per_head);
 int dm05_set_row_block_override(int row_blocks);
 
 /*
+ * dm05_prefix_prefill_attn -- the prefix stage's attention under the
+ * prefix-causal mask, asynchronous on `stream`.
+ *
+ * The operation (page "TensorRT+Triton+FlexAttention: OpenDM VLA
+ * 快速推理加速栈深度剖析", section 2.3 "FlexAttention"): the prefix stage runs
+ * its attention with a custom causal mask mapping
+ * (_make_prefix_causal_mask_mapping), with the prefix decoder's 8 / 4 GQA
+ * heads and head_dim 256 (section 2.2 shape table).  The queries are the P
+ * prefix positions, the keys and values the prefix K/V of the same call (the
+ * tensors that then form the prefix KV cache read by dm05_suffix_attn).  For
+ * sample b, query head h (KV head h / (Hq / Hkv)) and prefix position
+ * i < clamp(valid_len[b], 0, P):
+ *   visible keys  = prefix positions j <= i   (causal; j < valid length follows);
+ *   lse[b,h,i]    = ln sum_j exp(<q[b,h,i,:], k[b,g,j,:]> / sqrt(D));
+ *   out[b,h,i,:]  = sum_j exp(logit(j) - lse) v[b,g,j,:]   (rounded once to bf16).
+ * Positions i at or past the valid length are bucket padding: their out and
+ * lse rows are not written.
+ *
+ *   q          bf16  [B, Hq, P, D]
+ *   k, v       bf16  [B, Hkv, P, D]
+ *   valid_len  int32 [B]  device; NULL = every position in range; values
+ *                         outside [0, P] are clamped and flagged in the error word
+ *   out        bf16  [B, Hq, P, D]   (rows < valid length written)
+ *   lse        fp32  [B, Hq, P]      (rows < valid length written); NULL = not written
+ *
+ * Supported: D == 256 and (Hq / Hkv) * 8 <= 128; P >= 1; 16-byte aligned
+ * bases.  Workspace, capture, errors and determinism as in dm05_suffix_attn;
+ * the same per-(device, stream) workspace serves both calls.  Before
+ * capturing this call into a CUDA graph, create it with
+ * dm05_prefix_prefill_reserve.
+ */
+int dm05_prefix_prefill_attn(const void *q, const void *k, const void *v, const int32_t *valid_len,
+                             void *out, float *lse, int B, int Hq, int Hkv, int P, int D,
+                             cudaStream_t stream);
+
+/* Creates the workspace of (current device, `stream`) that a
+ * dm05_prefix_prefill_attn call with these sizes needs, outside any stream
+ * capture (as dm05_suffix_attn_reserve does for the suffix call). */
+int dm05_prefix_prefill_reserve(int B, int Hq, int Hkv, int P, int D, cudaStream_t stream);
+
+/* Work plan of a dm05_prefix_prefill_attn call with these sizes: CTAs per
+ * (sample, KV head, query block), query positions per head in a block, and
+ * the number of blocks.  Any output pointer may be NULL. */
+int dm05_prefix_prefill_plan(int B, int Hq, int Hkv, int P, int D, int *splits_per_head, int *query_block,
+                             int *row_blocks);
+
+/*
  * dm05_suffix_attn_noalloc -- the same attention as dm05_suffix_attn, for
  * callers that must not allocate device memory.  The source pages have no
  * counterpart of this entry point; it exists for embedding.

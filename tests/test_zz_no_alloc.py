@@ -13,8 +13,10 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from gqa_prefix_suffix_b200 import binding as bd
 from gqa_prefix_suffix_b200 import inputs as gen
+from parity import check_close
 
 pytestmark = pytest.mark.gpu
 
@@ -106,19 +108,18 @@ def test_noalloc_uses_fewer_ctas_when_partials_do_not_fit(B):
         rc, splits, _, row_blocks = bd.dm05_suffix_attn_plan(B, 8, 4, 1024, 50, 256)
         assert rc == bd.DM05_OK and splits == 16
         assert _partial_bytes(B * 4, splits, row_blocks, 2, 50) > SCRATCH_BYTES - 256
-        want_out, want_lse = bd.suffix_attn(d.q, d.k_prefix, d.v_prefix, d.k_suffix, d.v_suffix,
-                                            prefix_valid_len=d.prefix_valid_len, prefix_mask=d.prefix_mask)
+        # the allocating call runs 16 splits, this one fewer: the two round
+        # differently, so each is held to the oracle with the shared parity bar
+        o_ref, l_ref = oracle.inputs_call(inp, nthreads=min(8, oracle.max_threads()))
         for call in range(2):
-            out = torch.full_like(want_out, float("nan"))
-            lse = torch.full_like(want_lse, float("nan"))
+            out = torch.full((B, 8, 50, 256), float("nan"), dtype=torch.bfloat16, device="cuda")
+            lse = torch.full((B, 8, 50), float("nan"), dtype=torch.float32, device="cuda")
             assert _call_noalloc(d, out, lse, stream) == bd.DM05_OK
             torch.cuda.synchronize()
             rc, word = bd.dm05_get_error_word(stream)
             assert rc == bd.DM05_OK and word == 0, hex(word)
-            err = (out.float() - want_out.float()).abs()
             assert bool(torch.isfinite(out.float()).all()), f"call {call}: non-finite output"
-            assert float(err.max()) <= MAX_ABS and float(err.mean()) <= MEAN_ABS, (call, float(err.max()))
-            assert float((lse - want_lse).abs().max()) <= LSE_ABS
+            check_close(out.cpu(), lse.cpu(), o_ref, l_ref, f"noalloc B={B} call {call}")
     finally:
         bd.dm05_set_split_override(0)
 

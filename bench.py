@@ -34,6 +34,7 @@ METRIC = "suffix-attn µs/call & achieved HBM GB/s (frac of roofline), P=1024 S=
 UNIT = "us/call"
 KV_ROW_BYTES_PER_HEAD = 2 * 256 * 2   # K and V rows of one KV head, bf16, D=256
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 
 
 def parse():
@@ -240,22 +241,32 @@ def time_calls(calls, K, W, dev, stream, bd, l2, rotate=True):
     one prefix (the history loop, warm) is timed as is."""
     import torch
     one = sum(t.numel() * t.element_size() for c in calls for t in c.tensors().values() if t is not None)
-    copies = max(1, int(2 * l2 // max(1, one)) + 1) if rotate else 1
+    copies = max(2, int(2 * l2 // max(1, one)) + 2) if rotate else 1
+    # one device copy of each call (calls that share a prefix cache keep
+    # sharing it), then on-device clones, as the headline measurement does
+    base, prefix_dev = [], {}
+    for c in calls:
+        key = (c.k_prefix.data_ptr(), c.v_prefix.data_ptr())
+        if key not in prefix_dev:
+            prefix_dev[key] = (c.k_prefix.to(dev), c.v_prefix.to(dev))
+        mv = lambda t: None if t is None else t.to(dev)
+        base.append((key, dict(q=mv(c.q), prefix_valid_len=mv(c.prefix_valid_len), prefix_mask=mv(c.prefix_mask),
+                               k_suffix=mv(c.k_suffix), v_suffix=mv(c.v_suffix)),
+                     (c.B, c.Hq, c.Hkv, c.P, c.S, c.D)))
     sets = []
     for _ in range(copies):
-        prefix_cache = {}
-        for c in calls:
-            # calls that share one prefix cache keep sharing it on the device
-            key = (c.k_prefix.data_ptr(), c.v_prefix.data_ptr())
-            if key not in prefix_cache:
-                prefix_cache[key] = (c.k_prefix.to(dev), c.v_prefix.to(dev))
-            kp, vp = prefix_cache[key]
-            mv = lambda t: None if t is None else t.to(dev)
-            sets.append(dict(q=mv(c.q), k_prefix=kp, v_prefix=vp, prefix_valid_len=mv(c.prefix_valid_len),
-                             prefix_mask=mv(c.prefix_mask), k_suffix=mv(c.k_suffix), v_suffix=mv(c.v_suffix),
-                             out=torch.empty((c.B, c.Hq, c.S, c.D), dtype=torch.bfloat16, device=dev),
-                             lse=torch.empty((c.B, c.Hq, c.S), dtype=torch.float32, device=dev),
-                             dims=(c.B, c.Hq, c.Hkv, c.P, c.S, c.D)))
+        prefix_copy = {k: (kp.clone(), vp.clone()) for k, (kp, vp) in prefix_dev.items()} if rotate else prefix_dev
+        for key, t, dims in base:
+            B, Hq, Hkv, P, S, D = dims
+            kp, vp = prefix_copy[key]
+            sets.append(dict(q=t["q"].clone(), k_prefix=kp, v_prefix=vp,
+                             prefix_valid_len=None if t["prefix_valid_len"] is None else t["prefix_valid_len"].clone(),
+                             prefix_mask=None if t["prefix_mask"] is None else t["prefix_mask"].clone(),
+                             k_suffix=t["k_suffix"].clone(), v_suffix=t["v_suffix"].clone(),
+                             out=torch.empty((B, Hq, S, D), dtype=torch.bfloat16, device=dev),
+                             lse=torch.empty((B, Hq, S), dtype=torch.float32, device=dev), dims=dims))
+    del base, prefix_dev
+    torch.cuda.synchronize()
     ptr = lambda x: None if x is None else x.data_ptr()
 
     def call(t):
@@ -301,6 +312,80 @@ def time_calls(calls, K, W, dev, stream, bd, l2, rotate=True):
     return us, copies
 
 
+def prefill_flops(inp):
+    """Algorithmic FLOPs of a prefix-prefill call: every computed query row
+    i (below its sample's valid length) against its i + 1 visible keys, QK^T
+    and PV at 2 flops per multiply-add."""
+    total = 0
+    for b in range(inp.B):
+        vl = inp.P if inp.valid_len is None else max(0, min(inp.P, int(inp.valid_len[b])))
+        total += 4 * inp.D * inp.Hq * vl * (vl + 1) // 2
+    return total
+
+
+def time_prefill(inp, K, W, dev, stream, bd, l2):
+    """Device time per dm05_prefix_prefill_attn call, the same protocol as
+    time_calls (rotating on-device copies over 2 x L2, graphs of up to 1000
+    calls, CUDA events on the launching stream)."""
+    import torch
+    one = sum(t.numel() * t.element_size() for t in inp.tensors().values() if t is not None)
+    copies = max(2, int(2 * l2 // max(1, one)) + 2)
+    d0 = inp.to(dev)
+    sets = []
+    for _ in range(copies):
+        sets.append(dict(q=d0.q.clone(), k=d0.k.clone(), v=d0.v.clone(),
+                         vl=None if d0.valid_len is None else d0.valid_len.clone(),
+                         out=torch.empty_like(d0.q),
+                         lse=torch.empty((inp.B, inp.Hq, inp.P), dtype=torch.float32, device=dev)))
+    ptr = lambda x: None if x is None else x.data_ptr()
+    rc = bd.dm05_prefix_prefill_reserve(inp.B, inp.Hq, inp.Hkv, inp.P, inp.D, stream.cuda_stream)
+    if rc != 0:
+        raise bd.Dm05Error(rc, "dm05_prefix_prefill_reserve")
+
+    def call(t):
+        rc = bd.dm05_prefix_prefill_attn(ptr(t["q"]), ptr(t["k"]), ptr(t["v"]), ptr(t["vl"]), ptr(t["out"]),
+                                         ptr(t["lse"]), inp.B, inp.Hq, inp.Hkv, inp.P, inp.D, stream.cuda_stream)
+        if rc != 0:
+            raise bd.Dm05Error(rc, "dm05_prefix_prefill_attn")
+
+    with torch.cuda.stream(stream):
+        for i in range(max(3, W)):
+            call(sets[i % copies])
+    stream.synchronize()
+    graphs, done = [], 0
+    while done < K:
+        m = min(1000, K - done)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(m):
+                call(sets[(done + i) % copies])
+        graphs.append(g)
+        done += m
+    for g in graphs:
+        g.replay()
+    stream.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for g in graphs:
+            g.replay()
+        e1.record(stream)
+    stream.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / K
+    del graphs, sets
+    return us, copies
+
+
+def measured_tensor_peak():
+    """Dense bf16 tensor peak in TFLOP/s: the measured burst figure when the
+    driver's MEASURED_PEAKS.json is present, else the recipe's fallback."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, "fallback"
+
+
 def workload_table(args, dev, stream, bd, l2, peak):
     """Every workload of the benchmark timed with the same protocol as the
     headline (rotating input sets over 2 x L2, K calls from CUDA graphs):
@@ -337,6 +422,18 @@ def workload_table(args, dev, stream, bd, l2, peak):
     warm["per_10_steps"] = 10 * warm["us_per_call"]
     out["history_loop"] = {"cold": cold, "warm": warm}
     out["batched_mask"] = row([gen.batched_mask()])
+    # the prefix-prefill attention (prefix-causal mask) on the base chunk's and
+    # the history demo's prefixes: a dense contraction, bound by the tensor cores
+    tpeak, tkind = measured_tensor_peak()
+    for inp in (gen.prefill_base(), gen.prefill_history()):
+        us, copies = time_prefill(inp, K, W, dev, stream, bd, l2)
+        fl = prefill_flops(inp)
+        _, sp, qb, rb = bd.dm05_prefix_prefill_plan(inp.B, inp.Hq, inp.Hkv, inp.P, inp.D)
+        tf = fl / (us * 1e-6) / 1e12
+        out[inp.name] = {"us_per_call": us, "algorithmic_flops": fl, "achieved_tflops": tf,
+                         "roofline": {"bound": "tensor", "peak": tpeak, "peak_source": tkind, "frac": tf / tpeak},
+                         "plan": {"splits_per_head": sp, "query_block": qb, "row_blocks": rb}, "calls": K,
+                         "l2": f"{copies} rotating copies"}
     return out
 
 

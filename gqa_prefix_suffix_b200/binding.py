@@ -24,7 +24,9 @@ DM05_EW_VALID_LEN_CLAMPED = 0x1
 DM05_EW_WAIT_TIMEOUT = 0x2
 DM05_EW_BAD_SPLIT = 0x4
 
-EXPORTS = ("dm05_suffix_attn", "dm05_suffix_attn_workspace_bytes", "dm05_suffix_attn_reserve",
+DM05_FLAG_PREFIX_STATIC = 0x1
+
+EXPORTS = ("dm05_suffix_attn", "dm05_suffix_attn_ex", "dm05_suffix_attn_workspace_bytes", "dm05_suffix_attn_reserve",
            "dm05_suffix_attn_plan", "dm05_set_split_override", "dm05_set_row_block_override",
            "dm05_get_error_word",
            "dm05_status_string", "dm05_release", "dm05_suffix_attn_noalloc", "dm05_suffix_attn_host",
@@ -54,6 +56,8 @@ def lib() -> ctypes.CDLL:
             p, i, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
             L.dm05_suffix_attn.argtypes = [p] * 9 + [i] * 6 + [p]
             L.dm05_suffix_attn.restype = i
+            L.dm05_suffix_attn_ex.argtypes = [p] * 9 + [i] * 6 + [ctypes.c_uint, p]
+            L.dm05_suffix_attn_ex.restype = i
             L.dm05_suffix_attn_workspace_bytes.argtypes = [i] * 6
             L.dm05_suffix_attn_workspace_bytes.restype = sz
             L.dm05_suffix_attn_reserve.argtypes = [i] * 6 + [p]
@@ -94,6 +98,13 @@ def dm05_suffix_attn(q, k_prefix, v_prefix, prefix_valid_len, prefix_mask, k_suf
                      out, lse, B, Hq, Hkv, P, S, D, stream) -> int:
     return lib().dm05_suffix_attn(q, k_prefix, v_prefix, prefix_valid_len, prefix_mask, k_suffix,
                                   v_suffix, out, lse, B, Hq, Hkv, P, S, D, stream)
+
+
+def dm05_suffix_attn_ex(q, k_prefix, v_prefix, prefix_valid_len, prefix_mask, k_suffix, v_suffix,
+                        out, lse, B, Hq, Hkv, P, S, D, flags, stream) -> int:
+    """dm05_suffix_attn with option flags (DM05_FLAG_PREFIX_STATIC)."""
+    return lib().dm05_suffix_attn_ex(q, k_prefix, v_prefix, prefix_valid_len, prefix_mask, k_suffix,
+                                     v_suffix, out, lse, B, Hq, Hkv, P, S, D, flags, stream)
 
 
 def dm05_suffix_attn_noalloc(q, k_prefix, v_prefix, prefix_valid_len, prefix_mask, k_suffix, v_suffix,
@@ -189,7 +200,7 @@ def _stream_handle(stream):
 
 
 def suffix_attn(q, k_prefix, v_prefix, k_suffix, v_suffix, prefix_valid_len=None, prefix_mask=None,
-                out=None, lse=None, want_lse: bool = True, stream=None):
+                out=None, lse=None, want_lse: bool = True, stream=None, prefix_static: bool = False):
     """Suffix attention on CUDA torch tensors; returns (out, lse or None).
 
     q [B,Hq,S,D] bf16; k_prefix/v_prefix [B,Hkv,P,D] bf16; k_suffix/v_suffix
@@ -230,9 +241,9 @@ def suffix_attn(q, k_prefix, v_prefix, k_suffix, v_suffix, prefix_valid_len=None
         if t is not None and t.device != q.device:
             raise ValueError(f"{name} must be on {q.device} like q")
     ptr = lambda t: None if t is None else t.data_ptr()
-    rc = dm05_suffix_attn(ptr(q), ptr(k_prefix), ptr(v_prefix), ptr(prefix_valid_len), ptr(prefix_mask),
-                          ptr(k_suffix), ptr(v_suffix), ptr(out), ptr(lse), B, Hq, Hkv, P, S, D,
-                          _stream_handle(stream))
+    rc = dm05_suffix_attn_ex(ptr(q), ptr(k_prefix), ptr(v_prefix), ptr(prefix_valid_len), ptr(prefix_mask),
+                             ptr(k_suffix), ptr(v_suffix), ptr(out), ptr(lse), B, Hq, Hkv, P, S, D,
+                             DM05_FLAG_PREFIX_STATIC if prefix_static else 0, _stream_handle(stream))
     if rc != DM05_OK:
         raise Dm05Error(rc, "dm05_suffix_attn")
     return out, lse

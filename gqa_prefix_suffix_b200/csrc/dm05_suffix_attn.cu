@@ -32,8 +32,8 @@ struct DeviceState {
     uint32_t *err = nullptr;   // device error word
     bool attrs_set = false;
     int num_sms = 0;
-    int max_cluster = 0;       // largest cluster size (power of two <= 16) that can be resident
-    int active[5] = {0, 0, 0, 0, 0};  // co-resident clusters of size 1, 2, 4, 8, 16
+    int max_cluster = 0;       // largest cluster size (<= 16) that can be resident
+    int active[17] = {};       // active[c]: clusters of c CTAs the device holds at once (0: not allowed)
 };
 
 // Partial-result workspace of one (device, stream): concurrent streams never
@@ -92,7 +92,6 @@ int check_sizes(int B, int Hq, int Hkv, int P, int S, int D)
 // (each CTA then carries fewer query rows, so fewer partial rows to merge).
 // Among the plans whose clusters are all resident at once, the one with the
 // lowest estimated cost.
-int log2_pow2(int c) { return c >= 16 ? 4 : c >= 8 ? 3 : c >= 4 ? 2 : c >= 2 ? 1 : 0; }
 
 Plan make_plan(int B, int Hq, int Hkv, int P, int S, const DeviceState &ds)
 {
@@ -102,7 +101,7 @@ Plan make_plan(int B, int Hq, int Hkv, int P, int S, const DeviceState &ds)
     // every cluster of the call resident at once (no second wave)
     auto fits = [&](int c, long long blocks) {
         if (c == 1) return true;
-        return units * blocks * c <= ds.num_sms && units * blocks <= ds.active[log2_pow2(c)];
+        return units * blocks * c <= ds.num_sms && units * blocks <= ds.active[c];
     };
     // Estimated cost in microseconds, fitted on B200 measurements of this
     // kernel: ~1.2 per key tile a CTA streams, and for a split unit a fixed
@@ -116,20 +115,22 @@ Plan make_plan(int B, int Hq, int Hkv, int P, int S, const DeviceState &ds)
     Plan best;
     best.SQ = S;
     double best_cost = 1e30;
-    for (int c = 1; c <= 16; c *= 2) {
+    for (int c = 1; c <= dm05::kMaxSplits; ++c) {
         if (g_split_override > 0 && c != g_split_override) continue;
         if (g_split_override == 0 && (c > ds.max_cluster || !fits(c, 1))) continue;
-        for (int r = 1; r <= 16; r *= 2) {
+        for (int r = 1; r <= 16; ++r) {
             if (c == 1 && r > 1) break;
             const int sq = (S + r - 1) / r;
-            if (r > 1 && (sq < 8 || G * ((sq + 7) / 8 * 8) > dm05::kMRows)) break;
+            if (r > 1 && sq < 8) break;                        // blocks of at least 8 queries per head
+            if ((S + sq - 1) / sq != r) continue;              // the same blocks as a smaller r
+            if (r > 1 && G * ((sq + 7) / 8 * 8) > dm05::kMRows) continue;
             if (want_rb > 0 ? r != want_rb && !(r == 1 && c == 1) : !fits(c, r)) continue;
             const double t = cost(c, sq);
             if (t < best_cost) {
                 best_cost = t;
                 best.splits = c;
                 best.SQ = sq;
-                best.row_blocks = (S + sq - 1) / sq;  // no empty trailing block
+                best.row_blocks = r;
             }
         }
     }
@@ -172,11 +173,11 @@ Plan make_prefill_plan(int B, int Hq, int Hkv, int P, const DeviceState &ds)
         return t;
     };
     double best = 1e30;
-    for (int c = 1; c <= 16; c *= 2) {
+    for (int c = 1; c <= dm05::kMaxSplits; ++c) {
         if (g_split_override > 0 && c != g_split_override) continue;
         if (g_split_override == 0 && c > 1 &&
             (c > ds.max_cluster || units * pl.row_blocks * c > ds.num_sms ||
-             units * pl.row_blocks > ds.active[log2_pow2(c)]))
+             units * pl.row_blocks > ds.active[c]))
             continue;
         if (cost(c) < best) {
             best = cost(c);
@@ -218,8 +219,8 @@ int device_state(bool allocate, DeviceState **out, cudaStream_t stream = nullptr
         // how many clusters of each size the device holds at once with this
         // kernel's footprint (a plan never exceeds it: no second wave)
         ds.max_cluster = 1;
-        ds.active[0] = ds.num_sms;
-        for (int c = 16, li = 4; c >= 2; c /= 2, --li) {
+        ds.active[1] = ds.num_sms;
+        for (int c = dm05::kMaxSplits; c >= 2; --c) {
             cudaLaunchConfig_t cfg = {};
             cfg.gridDim = dim3(c, 1, 1);
             cfg.blockDim = dim3(dm05::kThreads, 1, 1);
@@ -233,7 +234,7 @@ int device_state(bool allocate, DeviceState **out, cudaStream_t stream = nullptr
             cfg.numAttrs = 1;
             int n = 0;
             if (cudaOccupancyMaxActiveClusters(&n, kKernel, &cfg) == cudaSuccess && n > 0) {
-                ds.active[li] = n;
+                ds.active[c] = n;
                 if (ds.max_cluster == 1) ds.max_cluster = c;
             } else {
                 cudaGetLastError();  // clear a refused size
@@ -440,15 +441,14 @@ int encode_3d(CUtensorMap *map, const void *base, uint64_t d1, uint64_t d2, uint
 int launch_attention(const void *q, const void *k_prefix, const void *v_prefix, const int32_t *prefix_valid_len,
                      const uint8_t *prefix_mask, const void *k_suffix, const void *v_suffix, void *out, float *lse,
                      int B, int Hq, int Hkv, int P, int S, int D, const Plan &pl, uint32_t *err, void *part,
-                     cudaStream_t stream, bool causal = false)
+                     cudaStream_t stream, bool causal = false, bool prefix_static = false)
 {
     const int G = Hq / Hkv;
     const int GS = G * S;
     const long long units = static_cast<long long>(B) * Hkv;
     const long long grid = units * pl.row_blocks * pl.splits;
     if (grid > 0x7fffffffLL) return DM05_ERR_SHAPE;  // more CTAs than one launch can name
-    if (pl.splits != 1 && pl.splits != 2 && pl.splits != 4 && pl.splits != 8 && pl.splits != 16)
-        return DM05_ERR_SHAPE;  // the kernel merges only these cluster sizes
+    if (pl.splits < 1 || pl.splits > dm05::kMaxSplits) return DM05_ERR_SHAPE;  // the kernel merges only these
 
     // ---- TMA descriptors (the tensor maps travel as kernel parameters)
     CUtensorMap tm_q, tm_kp, tm_vp, tm_ks, tm_vs;
@@ -489,6 +489,7 @@ int launch_attention(const void *q, const void *k_prefix, const void *v_prefix, 
     kp.splits = pl.splits;
     kp.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
     kp.causal = causal ? 1 : 0;
+    kp.prefix_static = prefix_static ? 1 : 0;
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
@@ -545,9 +546,7 @@ size_t dm05_suffix_attn_workspace_bytes(int B, int Hq, int Hkv, int P, int S, in
 
 int dm05_set_split_override(int splits_per_head)
 {
-    if (splits_per_head != 0 && splits_per_head != 1 && splits_per_head != 2 && splits_per_head != 4 &&
-        splits_per_head != 8 && splits_per_head != 16)
-        return DM05_ERR_SHAPE;
+    if (splits_per_head < 0 || splits_per_head > dm05::kMaxSplits) return DM05_ERR_SHAPE;
     std::lock_guard<std::mutex> lk(g_mu);
     g_split_override = splits_per_head;
     return DM05_OK;
@@ -555,9 +554,7 @@ int dm05_set_split_override(int splits_per_head)
 
 int dm05_set_row_block_override(int row_blocks)
 {
-    if (row_blocks != 0 && row_blocks != 1 && row_blocks != 2 && row_blocks != 4 && row_blocks != 8 &&
-        row_blocks != 16)
-        return DM05_ERR_SHAPE;
+    if (row_blocks < 0 || row_blocks > 16) return DM05_ERR_SHAPE;
     std::lock_guard<std::mutex> lk(g_mu);
     g_row_block_override = row_blocks;
     return DM05_OK;
@@ -600,6 +597,16 @@ int dm05_suffix_attn(const void *q, const void *k_prefix, const void *v_prefix, 
                      const uint8_t *prefix_mask, const void *k_suffix, const void *v_suffix, void *out, float *lse,
                      int B, int Hq, int Hkv, int P, int S, int D, cudaStream_t stream)
 {
+    return dm05_suffix_attn_ex(q, k_prefix, v_prefix, prefix_valid_len, prefix_mask, k_suffix, v_suffix, out, lse,
+                               B, Hq, Hkv, P, S, D, 0u, stream);
+}
+
+int dm05_suffix_attn_ex(const void *q, const void *k_prefix, const void *v_prefix, const int32_t *prefix_valid_len,
+                        const uint8_t *prefix_mask, const void *k_suffix, const void *v_suffix, void *out,
+                        float *lse, int B, int Hq, int Hkv, int P, int S, int D, unsigned flags,
+                        cudaStream_t stream)
+{
+    if ((flags & ~static_cast<unsigned>(DM05_FLAG_PREFIX_STATIC)) != 0) return DM05_ERR_SHAPE;
     // ---- host-side checks; nothing is launched on failure
     if (!q || !k_suffix || !v_suffix || !out) return DM05_ERR_NULL;
     if (P > 0 && (!k_prefix || !v_prefix)) return DM05_ERR_NULL;
@@ -636,7 +643,8 @@ int dm05_suffix_attn(const void *q, const void *k_prefix, const void *v_prefix, 
     }
 
     return launch_attention(q, k_prefix, v_prefix, prefix_valid_len, prefix_mask, k_suffix, v_suffix, out, lse, B,
-                            Hq, Hkv, P, S, D, pl, err_word, part_ws, stream);
+                            Hq, Hkv, P, S, D, pl, err_word, part_ws, stream, false,
+                            (flags & DM05_FLAG_PREFIX_STATIC) != 0);
 }
 
 int dm05_prefix_prefill_attn(const void *q, const void *k, const void *v, const int32_t *valid_len, void *out,

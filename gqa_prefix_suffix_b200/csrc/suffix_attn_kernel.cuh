@@ -65,6 +65,7 @@ namespace dm05 {
 // for the first and last slot, the global timer) of one CTA's phase boundary.
 #ifdef DM05_TRACE
 __device__ unsigned long long g_dm05_trace[4096][16];
+__device__ unsigned long long g_dm05_tile_trace[4096][4][24];  // per tile: K full, QK issued, S seen, P ready
 #define DM05_TRACE_CLOCK(slot)                                                      \
     do {                                                                            \
         if (blockIdx.x < 4096) g_dm05_trace[blockIdx.x][slot] = clock64();          \
@@ -73,11 +74,18 @@ __device__ unsigned long long g_dm05_trace[4096][16];
     do {                                                                            \
         if (blockIdx.x < 4096) g_dm05_trace[blockIdx.x][slot] = ptx::globaltimer_ns(); \
     } while (0)
+#define DM05_TRACE_TILE(ev, t)                                                              \
+    do {                                                                                    \
+        if (blockIdx.x < 4096 && (t) < 24) g_dm05_tile_trace[blockIdx.x][ev][t] = clock64(); \
+    } while (0)
 #else
 #define DM05_TRACE_CLOCK(slot) \
     do {                       \
     } while (0)
 #define DM05_TRACE_GTIME(slot) \
+    do {                       \
+    } while (0)
+#define DM05_TRACE_TILE(ev, t) \
     do {                       \
     } while (0)
 #endif
@@ -95,6 +103,7 @@ constexpr uint32_t kTmemO = 0;                    // O: columns [0, 256)
 constexpr uint32_t kTmemQ = 256;                  // Q as bf16 pairs: columns [256, 384)
 constexpr uint32_t kTmemS = 384;                  // S/P buffers: [384, 384 + kSBufs*NT)
 constexpr int kSBufs = 2;                         // S/P TMEM buffers in flight
+constexpr int kMaxSplits = 16;                    // CTAs per split cluster (the hardware's largest cluster)
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait
 constexpr float kRescaleThreshold = 8.0f;         // log2 units: p <= 2^8 between rescales
 constexpr uint32_t kEwClamped = 0x1u;
@@ -114,6 +123,8 @@ struct KernelParams {
     int SQ;                    // queries per head per block (S when row_blocks == 1)
     int splits;                // CTAs per (unit, query block): the cluster size
     float scale_log2;          // log2(e) / sqrt(D)
+    int prefix_static;         // 1: the preceding grid writes neither the prefix K/V, valid_len nor
+                               // the mask, so they may be read before it completes
     int causal;                // 0: suffix attention; 1: prefix prefill (queries are the P prefix
                                // positions, S == P, no suffix keys, key j visible to query i iff j <= i)
 };
@@ -207,56 +218,79 @@ __device__ __forceinline__ size_t block_out_row(size_t unit_row0, int k, int nq,
     return unit_row0 + static_cast<size_t>(h) * S + q0 + (k - h * nq);
 }
 
-// Combines the nr partial rows this CTA owns (rows whose query index within
-// the block is jlim or more are not written): partial c's row rr sits at
-// recv + (c * nr + rr) * kStageStride (D fp32 of unnormalised O, then
-// {m, l, l_hat, 0}).  One item per (row, 4-column quad); every item derives
-// its row's weights from the C statistics (a shared-memory broadcast within
-// the warp):
+// Merge of the nr partial rows this CTA owns (rows whose query index within
+// the block is jlim or more are not written).  Partial c's row rr sits at
+// recv + (c * nr + rr) * kStageStride: D fp32 of unnormalised O, then
+// {m, l, l_hat, 0}.  By the log-sum-exp rule
 //   M = max_c m_c,  w_c = 2^(m_c - M),  LH = sum_c l_hat_c w_c,  L = sum_c l_c w_c,
-//   out = sum_c w_c O_c / LH,  lse = (M + log2 L) ln 2.
-// A partial without visible keys (l_hat == 0) holds no O and gets no weight.
-template <int C, class L>
-__device__ __forceinline__ void merge_rows(const uint8_t *recv, int nr, __nv_bfloat16 *out, float *lse,
+//   out = sum_c (w_c / LH) O_c,  lse = (M + log2 L) ln 2,
+// where a partial without visible keys (l_hat == 0) gets no weight.
+// Pass 1 (merge_weights): one warp per row, lane c holds partial c's
+// statistics; the row's normalised weights w_c / LH replace the unused
+// fourth statistic of each partial row, and the LSE is written.
+template <class L>
+__device__ __forceinline__ void merge_weights(uint8_t *recv, int C, int nr, float *lse, size_t unit_row0, int k_lo,
+                                              int nq, int S, int q0, int jlim)
+{
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const size_t cstride = static_cast<size_t>(nr) * L::kStageStride;
+    for (int rr = warp; rr < nr; rr += kThreads / 32) {
+        float4 st = make_float4(-INFINITY, 0.f, 0.f, 0.f);
+        float *slot = nullptr;
+        if (lane < C) {
+            slot = reinterpret_cast<float *>(recv + lane * cstride + rr * L::kStageStride + kHeadDim * 4);
+            st = *reinterpret_cast<const float4 *>(slot);
+        }
+        const bool has = st.z > 0.0f;
+        float M = has ? st.x : -INFINITY;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+        const float w = has ? ptx::ex2(st.x - M) : 0.0f;
+        float LH = st.z * w, Ls = st.y * w;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            LH += __shfl_xor_sync(0xffffffffu, LH, o);
+            Ls += __shfl_xor_sync(0xffffffffu, Ls, o);
+        }
+        if (lane < C) slot[3] = w / LH;
+        if (lane == 0 && lse != nullptr && (k_lo + rr) % nq < jlim)
+            lse[block_out_row(unit_row0, k_lo + rr, nq, S, q0)] = (M + ptx::lg2(Ls)) * 0.69314718055994531f;
+    }
+}
+
+// Pass 2 (after a CTA barrier): one item per (row, 4-column quad):
+// out = sum_c wn_c O_c with all C loads independent.
+template <class L>
+__device__ __forceinline__ void merge_rows(const uint8_t *recv, int C, int nr, __nv_bfloat16 *out,
                                            size_t unit_row0, int k_lo, int nq, int S, int q0, int jlim)
 {
     const int items = nr * (kHeadDim / 4);
+    const size_t cstride = static_cast<size_t>(nr) * L::kStageStride;
     for (int i = threadIdx.x; i < items; i += kThreads) {
         const int rr = i / (kHeadDim / 4), ch = i - rr * (kHeadDim / 4);
         // only the queries [0, jlim) of each head of the block are written
         if ((k_lo + rr) % nq >= jlim) continue;
-        float4 st[C], v[C];
-#pragma unroll
-        for (int c = 0; c < C; ++c) {
-            const uint8_t *row = recv + (c * nr + rr) * L::kStageStride;
-            st[c] = *reinterpret_cast<const float4 *>(row + kHeadDim * 4);
-            v[c] = *reinterpret_cast<const float4 *>(row + ch * 16);
-        }
-        float M = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < C; ++c)
-            if (st[c].z > 0.0f) M = fmaxf(M, st[c].x);
-        float Ls = 0.0f, LHs = 0.0f;
+        const uint8_t *row0 = recv + rr * L::kStageStride;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-        for (int c = 0; c < C; ++c) {
-            if (st[c].z > 0.0f) {
-                const float w = ptx::ex2(st[c].x - M);
-                Ls += st[c].y * w;
-                LHs += st[c].z * w;
-                acc.x += w * v[c].x;
-                acc.y += w * v[c].y;
-                acc.z += w * v[c].z;
-                acc.w += w * v[c].w;
+        for (int c = 0; c < kMaxSplits; ++c) {
+            if (c < C) {
+                const uint8_t *row = row0 + c * cstride;
+                const float wn = *reinterpret_cast<const float *>(row + kHeadDim * 4 + 12);
+                const float4 v = *reinterpret_cast<const float4 *>(row + ch * 16);
+                if (wn != 0.0f) {  // a partial without keys may hold anything
+                    acc.x = fmaf(wn, v.x, acc.x);
+                    acc.y = fmaf(wn, v.y, acc.y);
+                    acc.z = fmaf(wn, v.z, acc.z);
+                    acc.w = fmaf(wn, v.w, acc.w);
+                }
             }
         }
-        const float inv = 1.0f / LHs;
-        __nv_bfloat162 h0 = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
-        __nv_bfloat162 h1 = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+        __nv_bfloat162 h0 = __floats2bfloat162_rn(acc.x, acc.y);
+        __nv_bfloat162 h1 = __floats2bfloat162_rn(acc.z, acc.w);
         const size_t orow = block_out_row(unit_row0, k_lo + rr, nq, S, q0);
         *reinterpret_cast<uint2 *>(out + orow * kHeadDim + ch * 4) =
             make_uint2(*reinterpret_cast<uint32_t *>(&h0), *reinterpret_cast<uint32_t *>(&h1));
-        if (ch == 0 && lse != nullptr) lse[orow] = (M + ptx::lg2(Ls)) * 0.69314718055994531f;
     }
 }
 
@@ -329,8 +363,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::tc_fence_after_sync();
     const uint32_t tmem = *tmem_slot;
 
-    // ---- from here on inputs are read: wait for the preceding grid
-    ptx::griddep_wait();
+    // ---- from here on inputs are read: wait for the preceding grid.  With
+    // a static prefix the TMA producer first requests the prefix tiles of its
+    // first ring slots (the preceding grid does not write them), and waits
+    // just before it needs Q or a suffix tile.
+    const bool early = p.prefix_static && warp == kProducerWarp && lane == 0;
+    if (!early) ptx::griddep_wait();
     if (threadIdx.x == 0) DM05_TRACE_CLOCK(2);
 
     uint8_t *sQ = smem + L::kQOff;
@@ -348,10 +386,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto key_limit = [&](int v) { return p.causal ? (q0 >= v ? 0 : min(v, q0 + nq)) : v; };
     const int t_bucket = TS + (key_limit(p.P) + NT - 1) / NT;
     const int g_spec = static_cast<int>((static_cast<long long>(t_bucket) * rank) / C);
-    const bool spec = g_spec < static_cast<int>((static_cast<long long>(t_bucket) * (rank + 1)) / C);
+    const bool spec =
+        !p.prefix_static && g_spec < static_cast<int>((static_cast<long long>(t_bucket) * (rank + 1)) / C);
     uint64_t pol = 0;
-    if (warp == kProducerWarp && lane == 0) {
-        pol = ptx::policy_evict_first();
+    auto issue_q = [&]() {
         if (p.row_blocks == 1) {
             // both heads' S queries are contiguous: one 128-row box per chunk
             // (4-D view [units][rows][4 chunks][64]: one request lands all
@@ -366,6 +404,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ptx::tma_load_3d(sQ + c * L::kQChunkBytes + h * rph * 128, &tm_q, &bars[L::kBarQFull],
                                      c * kChunkElems, h * p.S + q0, unit);
         }
+    };
+    if (warp == kProducerWarp && lane == 0) {
+        pol = ptx::policy_evict_first();
+        if (!p.prefix_static) issue_q();
         if (spec) {
             const TileInfo ti = tile_of<NT>(g_spec, TS, key_limit(p.P), p.S);
             const CUtensorMap *mk = ti.prefix ? &tm_kp : &tm_ks;
@@ -401,6 +443,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ================================================== TMA producer
         if (lane == 0) {
             int slots = spec ? 1 : 0;  // ring slots requested so far
+            bool q_issued = !p.prefix_static;
             if (shift == 1) {
                 // the early request is not one of this CTA's tiles: let it
                 // land, then release its slot as its consumer would
@@ -417,6 +460,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const TileInfo ti = tile_of<NT>(t_begin + t, TS, klim, p.S);
                 const CUtensorMap *mk = ti.prefix ? &tm_kp : &tm_ks;
                 const CUtensorMap *mv = ti.prefix ? &tm_vp : &tm_vs;
+                if (!q_issued && (!ti.prefix || slot >= STAGES - 1)) {
+                    // Q and the suffix tensors may come from the preceding grid
+                    ptx::griddep_wait();
+                    issue_q();
+                    q_issued = true;
+                }
                 if (n > 0 && !ptx::mbar_wait(&bars[L::kBarKEmpty + s], (n - 1) & 1, kWaitLimitNs)) {
                     failed = true;
                     break;
@@ -436,6 +485,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ptx::mbar_arrive_expect_tx(&bars[L::kBarVFull + s], L::kTileBytes);
                 ptx::tma_load_4d_hint(sV(s), mv, &bars[L::kBarVFull + s], 0, ti.row0, 0, unit, pol);
                 v_issued = slot + 1;
+            }
+            if (!q_issued) {
+                ptx::griddep_wait();
+                issue_q();
             }
             // Drain: every copy this thread issued must have landed before the
             // CTA may exit (normally all phases are long complete here).
@@ -498,6 +551,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     break;
                 }
                 if (t == 0) DM05_TRACE_CLOCK(14);
+                DM05_TRACE_TILE(0, t);
                 // S(t) overwrites the TMEM columns that held P(t - kSBufs): the
                 // PV MMA reading them must have completed (issue order alone
                 // does not order one MMA's operand reads before a later MMA's
@@ -523,6 +577,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 ptx::mma_commit(&bars[L::kBarKEmpty + s]);
                 ptx::mma_commit(&bars[L::kBarSFull + sb]);
+                DM05_TRACE_TILE(1, t);
                 if (t > 0 && !issue_pv(t - 1)) {
                     ok = false;
                     break;
@@ -592,6 +647,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             }
             if (t == 0 && threadIdx.x == 0) DM05_TRACE_CLOCK(15);
+            if (threadIdx.x == 0) DM05_TRACE_TILE(2, t);
             ptx::tc_fence_after_sync();
             const uint32_t scol = tmem + lane_base + kTmemS + sb * NT;
             uint32_t raw[NH / 16][16];
@@ -726,6 +782,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             ptx::tc_fence_before_sync();
             ptx::mbar_arrive(&bars[L::kBarPReady + sb]);
+            if (threadIdx.x == 0) DM05_TRACE_TILE(3, t);
         }
 
         if (T == 0) {
@@ -757,21 +814,27 @@ __global__ void __launch_bounds__(kThreads, 1)
             // ---------------------------------------- single CTA: normalise and store this half
             const float inv_l = 1.0f / lh_row;
 #pragma unroll 1
-            for (int j = 0; j < kHeadDim / 32; ++j) {
-                uint32_t o[16];
-                ptx::tmem_ld16(tmem + lane_base + kTmemO + hf * (kHeadDim / 2) + j * 16, o);
+            for (int j = 0; j < kHeadDim / 128; ++j) {
+                uint32_t o[4][16];
+#pragma unroll
+                for (int qq = 0; qq < 4; ++qq)
+                    ptx::tmem_ld16(tmem + lane_base + kTmemO + hf * (kHeadDim / 2) + j * 64 + qq * 16, o[qq]);
                 ptx::tmem_ld_wait();
                 if (row_valid) {
-                    uint32_t w[8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(o[2 * e]) * inv_l,
-                                                                 __uint_as_float(o[2 * e + 1]) * inv_l);
-                        w[e] = *reinterpret_cast<uint32_t *>(&h);
+                    for (int qq = 0; qq < 4; ++qq) {
+                        uint32_t w[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(o[qq][2 * e]) * inv_l,
+                                                                     __uint_as_float(o[qq][2 * e + 1]) * inv_l);
+                            w[e] = *reinterpret_cast<uint32_t *>(&h);
+                        }
+                        uint4 *dst = reinterpret_cast<uint4 *>(p.out + out_row * kHeadDim + hf * (kHeadDim / 2) +
+                                                               j * 64 + qq * 16);
+                        dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                        dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
                     }
-                    uint4 *dst = reinterpret_cast<uint4 *>(p.out + out_row * kHeadDim + hf * (kHeadDim / 2) + j * 16);
-                    dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-                    dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
                 }
             }
             if (hf == 0 && row_valid && p.lse != nullptr)
@@ -786,16 +849,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool write_o = T > 0 && !failed;
             if (write_o) {
 #pragma unroll 1
-                for (int j = 0; j < kHeadDim / 64; ++j) {
-                    uint32_t o[2][16];
+                for (int j = 0; j < kHeadDim / 128; ++j) {
+                    uint32_t o[4][16];
 #pragma unroll
-                    for (int qq = 0; qq < 2; ++qq)
-                        ptx::tmem_ld16(tmem + lane_base + kTmemO + hf * (kHeadDim / 2) + j * 32 + qq * 16, o[qq]);
+                    for (int qq = 0; qq < 4; ++qq)
+                        ptx::tmem_ld16(tmem + lane_base + kTmemO + hf * (kHeadDim / 2) + j * 64 + qq * 16, o[qq]);
                     ptx::tmem_ld_wait();
                     if (row_valid) {
 #pragma unroll
-                        for (int qq = 0; qq < 2; ++qq) {
-                            uint4 *d = reinterpret_cast<uint4 *>(srow + (hf * (kHeadDim / 2) + j * 32 + qq * 16) * 4);
+                        for (int qq = 0; qq < 4; ++qq) {
+                            uint4 *d = reinterpret_cast<uint4 *>(srow + (hf * (kHeadDim / 2) + j * 64 + qq * 16) * 4);
                             d[0] = make_uint4(o[qq][0], o[qq][1], o[qq][2], o[qq][3]);
                             d[1] = make_uint4(o[qq][4], o[qq][5], o[qq][6], o[qq][7]);
                             d[2] = make_uint4(o[qq][8], o[qq][9], o[qq][10], o[qq][11]);
@@ -812,6 +875,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             // both halves of the row staged
             if (!failed && !pair_sync()) failed = true;
+            if (threadIdx.x == 0) DM05_TRACE_TILE(3, 23);
             if (row_valid && hf == 0) {
                 ptx::bulk_store_s2g(reinterpret_cast<uint8_t *>(p.part) + prow * L::kStageStride, ptx::smem_addr(srow),
                                     L::kStageStride);
@@ -836,7 +900,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int r_lo = (NR * rank) / C;  // compact rows of this query block
         const int r_hi = (NR * (rank + 1)) / C;
         const int nr = r_hi - r_lo;
-        const uint8_t *recv = smem;  // [C][nr] rows of kStageStride bytes
+        uint8_t *recv = smem;  // [C][nr] rows of kStageStride bytes
         if (nr > 0 && warp == 0) {
             if (lane == 0) ptx::mbar_arrive_expect_tx(&bars[L::kBarMerge], static_cast<uint32_t>(C * nr * L::kStageStride));
             __syncwarp();
@@ -851,16 +915,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (nr > 0) {
             if (!warp_wait(&bars[L::kBarMerge], 0)) failed = true;
             if (threadIdx.x == 0) DM05_TRACE_CLOCK(11);
-            // the host launches only these cluster sizes; any other is
-            // reported and merges nothing
-            switch (C) {
-            case 2: merge_rows<2, L>(recv, nr, p.out, p.lse, unit_row0, r_lo, nq, p.S, q0, jlim); break;
-            case 4: merge_rows<4, L>(recv, nr, p.out, p.lse, unit_row0, r_lo, nq, p.S, q0, jlim); break;
-            case 8: merge_rows<8, L>(recv, nr, p.out, p.lse, unit_row0, r_lo, nq, p.S, q0, jlim); break;
-            case 16: merge_rows<16, L>(recv, nr, p.out, p.lse, unit_row0, r_lo, nq, p.S, q0, jlim); break;
-            default:
-                if (threadIdx.x == 0) atomicOr(p.err, kEwBadSplit);
-                break;
+            // the host launches clusters of 2..kMaxSplits CTAs; any other
+            // size is reported and merges nothing
+            if (C <= kMaxSplits) {
+                merge_weights<L>(recv, C, nr, p.lse, unit_row0, r_lo, nq, p.S, q0, jlim);
+                if (threadIdx.x == 0) DM05_TRACE_TILE(0, 23);
+                __syncthreads();
+                if (threadIdx.x == 0) DM05_TRACE_TILE(1, 23);
+                merge_rows<L>(recv, C, nr, p.out, unit_row0, r_lo, nq, p.S, q0, jlim);
+                if (threadIdx.x == 0) DM05_TRACE_TILE(2, 23);
+            } else if (threadIdx.x == 0) {
+                atomicOr(p.err, kEwBadSplit);
             }
         }
     }

@@ -101,6 +101,29 @@ int dm05_suffix_attn(const void *q, const void *k_prefix, const void *v_prefix,
                      int B, int Hq, int Hkv, int P, int S, int D,
                      cudaStream_t stream);
 
+/*
+ * dm05_suffix_attn_ex -- dm05_suffix_attn with option flags (0 gives exactly
+ * dm05_suffix_attn).  Unknown bits return DM05_ERR_SHAPE.
+ *
+ * DM05_FLAG_PREFIX_STATIC: the caller promises that the kernel launched
+ * right before this call on `stream` writes none of k_prefix, v_prefix,
+ * prefix_valid_len and prefix_mask (they were written earlier, as the pages'
+ * static, address-stable prefix KV cache is: page "TensorRT+Triton+
+ * FlexAttention: OpenDM VLA 快速推理加速栈深度剖析", section 3, where the cache
+ * is filled by the prefix graph and then read, unchanged, by every suffix
+ * step).  The call may then start reading them while that kernel is still
+ * running (programmatic dependent launch); q, k_suffix, v_suffix and the
+ * outputs are still ordered after it.  Breaking the promise gives wrong
+ * results.
+ */
+#define DM05_FLAG_PREFIX_STATIC 0x1u
+int dm05_suffix_attn_ex(const void *q, const void *k_prefix, const void *v_prefix,
+                        const int32_t *prefix_valid_len, const uint8_t *prefix_mask,
+                        const void *k_suffix, const void *v_suffix,
+                        void *out, float *lse,
+                        int B, int Hq, int Hkv, int P, int S, int D, unsigned flags,
+                        cudaStream_t stream);
+
 /* Upper bound of the device workspace dm05_suffix_attn uses for these sizes:
  * the error word plus the partial results of the largest split (16 CTAs per
  * (sample, KV head)).  0 if the sizes are invalid.
@@ -130,15 +153,16 @@ int dm05_suffix_attn_plan(int B, int Hq, int Hkv, int P, int S, int D,
                           int *splits_per_head, int *tile_rows, int *row_blocks);
 
 /* Forces the number of CTAs per (sample, KV head) for later calls on this
- * process: 1, 2, 4, 8 or 16; 0 restores the automatic choice.  For tuning
- * and tests.  Returns DM05_ERR_SHAPE for any other value. */
+ * process: 1 to 16; 0 restores the automatic choice.  For tuning and tests.
+ * Returns DM05_ERR_SHAPE for any other value. */
 int dm05_set_split_override(int splits_per_head);
 
 /* Forces the number of query blocks each (sample, KV head)'s S queries are
- * cut into, for later split calls on this process: 1, 2, 4, 8 or 16; 0
- * restores the automatic choice.  A block holds at least 8 queries per head
- * and (Hq/Hkv) * (block rounded up to 8) <= 128 rows, so a count that breaks
- * this (or a call that runs unsplit) uses one block; dm05_suffix_attn_plan
+ * cut into, for later split calls on this process: 1 to 16; 0 restores the
+ * automatic choice.  Blocks hold ceil(S / row_blocks) queries per head (the
+ * last one fewer), at least 8, and (Hq/Hkv) * (block rounded up to 8) <= 128
+ * rows; a count that breaks this, that another count already gives the same
+ * blocks, or a call that runs unsplit, uses one block.  dm05_suffix_attn_plan
  * reports what a call will use.  For tuning and tests.  Returns
  * DM05_ERR_SHAPE for any other value. */
 int dm05_set_row_block_override(int row_blocks);

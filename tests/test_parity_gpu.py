@@ -430,3 +430,58 @@ def test_wait_timeout_is_reported_and_the_context_stays_usable():
     out, lse, word = run_gpu(inp)
     assert word == 0
     check_close(out, lse, *ref(inp), what="after a wait time-out")
+
+
+# ---------------------------------------------------------------- static prefix (DM05_FLAG_PREFIX_STATIC)
+
+@pytest.mark.parametrize("case", ["base_chunk", "libero_tiny", "batched_mask"])
+def test_prefix_static_flag_gives_the_same_bits(case):
+    # the flag only lets the prefix tiles be requested earlier: the result is
+    # bit-identical to the default call, for every split count that the
+    # automatic plan or the override gives
+    inp = gen.WORKLOADS[case]()
+    d = inp.to("cuda")
+    for splits in (0, 1, 3):
+        assert bd.dm05_set_split_override(splits) == 0
+        try:
+            a = bd.suffix_attn(d.q, d.k_prefix, d.v_prefix, d.k_suffix, d.v_suffix,
+                               prefix_valid_len=d.prefix_valid_len, prefix_mask=d.prefix_mask)
+            b = bd.suffix_attn(d.q, d.k_prefix, d.v_prefix, d.k_suffix, d.v_suffix,
+                               prefix_valid_len=d.prefix_valid_len, prefix_mask=d.prefix_mask, prefix_static=True)
+            torch.cuda.synchronize()
+        finally:
+            bd.dm05_set_split_override(0)
+        assert torch.equal(a[0].view(torch.int16), b[0].view(torch.int16)), f"splits={splits}"
+        assert torch.equal(a[1], b[1])
+    o_ref, l_ref = ref(inp)
+    check_close(b[0].cpu(), b[1].cpu(), o_ref, l_ref, f"{case} prefix_static")
+
+
+def test_prefix_static_still_waits_for_q_and_the_suffix():
+    # q, k_suffix and v_suffix are rewritten by torch kernels right before
+    # each call; with the static-prefix flag the call must still see them
+    inp = gen.base_chunk()
+    d = inp.to("cuda")
+    q2, ks2, vs2 = torch.empty_like(d.q), torch.empty_like(d.k_suffix), torch.empty_like(d.v_suffix)
+    out = torch.empty_like(d.q)
+    lse = torch.empty(d.q.shape[:3], dtype=torch.float32, device="cuda")
+    for _ in range(3):
+        torch.mul(d.q, -1.0, out=q2)
+        torch.mul(d.k_suffix, 2.0, out=ks2)
+        torch.mul(d.v_suffix, -0.5, out=vs2)
+        bd.suffix_attn(q2, d.k_prefix, d.v_prefix, ks2, vs2, prefix_valid_len=d.prefix_valid_len, out=out,
+                       lse=lse, prefix_static=True)
+    torch.cuda.synchronize()
+    inp2 = gen.base_chunk()
+    inp2.q = -inp2.q
+    inp2.k_suffix = (inp2.k_suffix.float() * 2.0).to(torch.bfloat16)
+    inp2.v_suffix = (inp2.v_suffix.float() * -0.5).to(torch.bfloat16)
+    o_ref, l_ref = ref(inp2)
+    check_close(out.cpu(), lse.cpu(), o_ref, l_ref, "static prefix after producers")
+
+
+def test_prefix_static_rejects_unknown_flags():
+    fake = 0x7f0000001000
+    rc = bd.dm05_suffix_attn_ex(fake, fake, fake, None, None, fake, fake, fake, None, 1, 8, 4, 64, 10, 256,
+                                0x80, None)
+    assert rc == bd.DM05_ERR_SHAPE

@@ -232,6 +232,27 @@ def cpu_model():
     return "unknown"
 
 
+def warm_graphs(graphs, stream, min_passes=3, min_ms=200.0):
+    """Untimed replays of the captured graphs before the timed pass: at least
+    `min_passes` passes over all of them and at least `min_ms` of GPU time
+    (the first replays after capture run measurably slower)."""
+    import torch
+    spent, passes = 0.0, 0
+    while passes < min_passes or spent < min_ms:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for g in graphs:
+                g.replay()
+            e1.record(stream)
+        stream.synchronize()
+        spent += e0.elapsed_time(e1)
+        passes += 1
+        if passes > 1000:
+            break
+    return passes
+
+
 def time_calls(calls, K, W, dev, stream, bd, l2, rotate=True):
     """Device time per call of K dm05_suffix_attn calls that cycle through
     `calls` (a list of input sets, one call each), captured as CUDA graphs of
@@ -297,9 +318,7 @@ def time_calls(calls, K, W, dev, stream, bd, l2, rotate=True):
                 call(sets[(done + i) % n])
         graphs.append((g, m))
         done += m
-    for g, _ in graphs:
-        g.replay()
-    stream.synchronize()
+    warm_graphs([g for g, _ in graphs], stream)
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(graphs) + 1)]
     with torch.cuda.stream(stream):
         evs[0].record(stream)
@@ -361,9 +380,7 @@ def time_prefill(inp, K, W, dev, stream, bd, l2):
                 call(sets[(done + i) % copies])
         graphs.append(g)
         done += m
-    for g in graphs:
-        g.replay()
-    stream.synchronize()
+    warm_graphs(graphs, stream)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         e0.record(stream)
@@ -586,12 +603,9 @@ def main():
 
     g_full = capture(chunk, 0) if n_full else None
     g_rem = capture(rem, n_full * chunk) if rem else None
-    # one untimed replay of each graph
-    if g_full is not None:
-        g_full.replay()
-    if g_rem is not None:
-        g_rem.replay()
-    stream.synchronize()
+    # untimed replays of each graph (part of the warm-up: the first replays
+    # after capture run slower)
+    warm_graphs([g for g in (g_full, g_rem) if g is not None], stream)
 
     # one event between consecutive replays: the total spans all K calls, and
     # each replay gives one sample of the per-call time for the spread

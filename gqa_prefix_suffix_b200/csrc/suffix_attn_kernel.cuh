@@ -65,7 +65,7 @@ namespace dm05 {
 // for the first and last slot, the global timer) of one CTA's phase boundary.
 #ifdef DM05_TRACE
 __device__ unsigned long long g_dm05_trace[4096][16];
-__device__ unsigned long long g_dm05_tile_trace[4096][4][24];  // per tile: K full, QK issued, S seen, P ready
+__device__ unsigned long long g_dm05_tile_trace[4096][6][24];  // per tile: K full, QK issued, S seen, P ready, K requested, PV issued
 #define DM05_TRACE_CLOCK(slot)                                                      \
     do {                                                                            \
         if (blockIdx.x < 4096) g_dm05_trace[blockIdx.x][slot] = clock64();          \
@@ -272,18 +272,27 @@ __device__ __forceinline__ void merge_rows(const uint8_t *recv, int C, int nr, _
         if ((k_lo + rr) % nq >= jlim) continue;
         const uint8_t *row0 = recv + rr * L::kStageStride;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        // four partials at a time: their eight shared-memory loads are
+        // independent and issue back to back (a partial past C reads partial
+        // C - 1 again with weight 0)
+        for (int c0 = 0; c0 < C; c0 += 4) {
+            float wn[4];
+            float4 v[4];
 #pragma unroll
-        for (int c = 0; c < kMaxSplits; ++c) {
-            if (c < C) {
-                const uint8_t *row = row0 + c * cstride;
-                const float wn = *reinterpret_cast<const float *>(row + kHeadDim * 4 + 12);
-                const float4 v = *reinterpret_cast<const float4 *>(row + ch * 16);
-                if (wn != 0.0f) {  // a partial without keys may hold anything
-                    acc.x = fmaf(wn, v.x, acc.x);
-                    acc.y = fmaf(wn, v.y, acc.y);
-                    acc.z = fmaf(wn, v.z, acc.z);
-                    acc.w = fmaf(wn, v.w, acc.w);
-                }
+            for (int k = 0; k < 4; ++k) {
+                const uint8_t *row = row0 + min(c0 + k, C - 1) * cstride;
+                wn[k] = *reinterpret_cast<const float *>(row + kHeadDim * 4 + 12);
+                v[k] = *reinterpret_cast<const float4 *>(row + ch * 16);
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                // a partial without keys (weight 0) may hold anything, NaN included
+                const bool use = c0 + k < C && wn[k] != 0.0f;
+                const float w = use ? wn[k] : 0.0f;
+                acc.x = fmaf(w, use ? v[k].x : 0.0f, acc.x);
+                acc.y = fmaf(w, use ? v[k].y : 0.0f, acc.y);
+                acc.z = fmaf(w, use ? v[k].z : 0.0f, acc.z);
+                acc.w = fmaf(w, use ? v[k].w : 0.0f, acc.w);
             }
         }
         __nv_bfloat162 h0 = __floats2bfloat162_rn(acc.x, acc.y);
@@ -477,6 +486,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 ptx::mbar_arrive_expect_tx(&bars[L::kBarKFull + s], L::kTileBytes);
                 ptx::tma_load_4d_hint(sK(s), mk, &bars[L::kBarKFull + s], 0, ti.row0, 0, unit, pol);
+                DM05_TRACE_TILE(4, t);
                 k_issued = slot + 1;
                 if (n > 0 && !ptx::mbar_wait(&bars[L::kBarVEmpty + s], (n - 1) & 1, kWaitLimitNs)) {
                     failed = true;
@@ -503,15 +513,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0 && T > 0) {
             constexpr uint32_t idesc_pv = ptx::idesc_bf16_f32(kMRows, kHeadDim, true);
             const uint32_t q_base = ptx::smem_addr(sQ);
-            const uint32_t k_base = ptx::smem_addr(sK(0));
-            const uint32_t v_base = ptx::smem_addr(sV(0));
+            // operand descriptors of ring slot 0 (K-major K tile, MN-major V
+            // tile); a slot or k-step offset is added to the start-address
+            // field, which holds (address >> 4) in 14 bits (shared memory is
+            // below 256 KB, so the sum never carries out of the field)
+            const uint64_t kdesc0 = ptx::sw128_desc(ptx::smem_addr(sK(0)), 16, 1024);
+            const uint64_t vdesc0 = ptx::sw128_desc(ptx::smem_addr(sV(0)), L::kTileChunkBytes, 1024);
             auto issue_pv = [&](int u) -> bool {
                 const int s = (u + shift) % STAGES;
                 const int pb = u % kSBufs;
                 if (!ptx::mbar_wait(&bars[L::kBarPReady + pb], (u / kSBufs) & 1, kWaitLimitNs)) return false;
                 if (!ptx::mbar_wait(&bars[L::kBarVFull + s], ((u + shift) / STAGES) & 1, kWaitLimitNs)) return false;
                 ptx::tc_fence_after_sync();
-                const uint32_t vb = v_base + s * L::kStageBytes;
+                // descriptor of V rows [0, 16) of this slot; each 16-row k-step
+                // adds 16 * 128 bytes (in the 16-byte units of the address field)
+                const uint64_t vdesc = vdesc0 + static_cast<uint64_t>((s * L::kStageBytes) >> 4);
                 const uint32_t p_tmem = tmem + kTmemS + pb * NT;
                 // only the 16-row k-steps that hold valid keys (a partial tile
                 // stops early; the rows after its last valid key up to the
@@ -523,11 +539,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // B = V rows [16kk, 16kk+16) of the tile, all 256 columns:
                     // 128-byte rows (16 B units), column chunks LBO apart,
                     // 8-row groups SBO apart.
-                    const uint64_t bdesc = ptx::sw128_desc(vb + kk * 16 * 128, L::kTileChunkBytes, 1024);
-                    ptx::mma_bf16_ts(tmem + kTmemO, p_tmem + kk * 8, bdesc, idesc_pv, (u > 0 || kk > 0) ? 1u : 0u);
+                    ptx::mma_bf16_ts(tmem + kTmemO, p_tmem + kk * 8, vdesc + static_cast<uint64_t>((kk * 16 * 128) >> 4),
+                                     idesc_pv, (u > 0 || kk > 0) ? 1u : 0u);
                 }
                 ptx::mma_commit(&bars[L::kBarVEmpty + s]);
                 ptx::mma_commit(&bars[L::kBarPFree + pb]);
+                DM05_TRACE_TILE(5, u);
                 return true;
             };
             bool ok = ptx::mbar_wait(&bars[L::kBarQFull], 0, kWaitLimitNs);
@@ -561,7 +578,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     break;
                 }
                 ptx::tc_fence_after_sync();
-                const uint32_t kb = k_base + s * L::kStageBytes;
+                const uint64_t kdesc = kdesc0 + static_cast<uint64_t>((s * L::kStageBytes) >> 4);
                 const uint32_t d = tmem + kTmemS + sb * NT;
                 // N = the valid keys of the tile rounded up to 16; the
                 // softmax masks every column past the valid ones anyway.
@@ -571,9 +588,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int kk = 0; kk < kHeadDim / 16; ++kk) {
                     // K-major, 128-byte swizzle: 16 elements = 32 bytes along
                     // the row; chunk kk/4 holds columns [64(kk/4), 64(kk/4)+64).
-                    const uint32_t koff = (kk & 3) * 32;
-                    const uint64_t bdesc = ptx::sw128_desc(kb + (kk >> 2) * L::kTileChunkBytes + koff, 16, 1024);
-                    ptx::mma_bf16_ts(d, tmem + kTmemQ + kk * 8, bdesc, idesc_qk, kk > 0 ? 1u : 0u);
+                    const uint32_t koff = ((kk >> 2) * L::kTileChunkBytes + (kk & 3) * 32) >> 4;
+                    ptx::mma_bf16_ts(d, tmem + kTmemQ + kk * 8, kdesc + koff, idesc_qk, kk > 0 ? 1u : 0u);
                 }
                 ptx::mma_commit(&bars[L::kBarKEmpty + s]);
                 ptx::mma_commit(&bars[L::kBarSFull + sb]);

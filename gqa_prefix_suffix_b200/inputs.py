@@ -242,6 +242,65 @@ def prefill_history() -> PrefillInputs:
     return make_prefill_inputs(1, HQ, HKV, 2048, HEAD_DIM, 5002, valid_len=1900, name="prefill_b1_p2048_v1900")
 
 
+# --- suffix prologue (QKV projection + QK-Norm + RoPE) -----------------------
+
+@dataclass
+class PrologueInputs:
+    """One suffix-prologue call: the action tokens' hidden states, the QKV
+    weight and the QK-Norm weights, and each token's position."""
+    name: str
+    B: int
+    S: int
+    H: int
+    Hq: int
+    Hkv: int
+    D: int
+    x: torch.Tensor        # bf16 [B*S, H]
+    w: torch.Tensor        # bf16 [(Hq + 2*Hkv)*D, H]: query heads, key heads, value heads
+    qw: torch.Tensor       # bf16 [D]
+    kw: torch.Tensor       # bf16 [D]
+    pos: torch.Tensor      # int32 [B*S]
+
+    def to(self, device):
+        return PrologueInputs(self.name, self.B, self.S, self.H, self.Hq, self.Hkv, self.D, self.x.to(device),
+                              self.w.to(device), self.qw.to(device), self.kw.to(device), self.pos.to(device))
+
+    def tensors(self):
+        return dict(x=self.x, w=self.w, qw=self.qw, kw=self.kw, pos=self.pos)
+
+
+def make_prologue_inputs(B: int, S: int, seed: int, *, H: int = 1024, Hq: int = HQ, Hkv: int = HKV,
+                         D: int = HEAD_DIM, pos0=0, name: str = "prologue") -> PrologueInputs:
+    """Seeded prologue inputs: fp32 N(0,1) hidden states x [B*S, H]; the QKV
+    weight N(0,1) / sqrt(H) (so projections are O(1)); QK-Norm weights
+    1 + 0.1 N(0,1); all rounded once to bf16.  Token i of sample b sits at
+    position pos0[b] + i (pos0 an int or a list of B ints: the suffix follows
+    the prefix)."""
+    gen = torch.Generator().manual_seed(int(seed))
+    bf = torch.bfloat16
+    x = _randn(gen, (B * S, H)).to(bf)
+    w = (_randn(gen, ((Hq + 2 * Hkv) * D, H)) / (H ** 0.5)).to(bf)
+    qw = (1.0 + 0.1 * _randn(gen, (D,))).to(bf)
+    kw = (1.0 + 0.1 * _randn(gen, (D,))).to(bf)
+    p0 = [pos0] * B if isinstance(pos0, int) else list(pos0)
+    pos = torch.tensor([p0[b] + i for b in range(B) for i in range(S)], dtype=torch.int32)
+    return PrologueInputs(name, B, S, H, Hq, Hkv, D, x, w, qw, kw, pos)
+
+
+def prologue_base() -> PrologueInputs:
+    """The base-model chunk's prologue: B=1, S=50 action tokens after a
+    900-token prefix, hidden 1024, 8/4 heads, D=256 (the action expert's
+    shape)."""
+    return make_prologue_inputs(1, 50, 6001, pos0=900, name="prologue_b1_s50_h1024")
+
+
+def prologue_batched() -> PrologueInputs:
+    """The batched workload's prologue: B=32 chunks of S=50 tokens."""
+    gen = torch.Generator().manual_seed(6002)
+    starts = torch.randint(576, 1025, (32,), generator=gen).tolist()
+    return make_prologue_inputs(32, 50, 6003, pos0=starts, name="prologue_b32_s50_h1024")
+
+
 WORKLOADS = {
     "libero_tiny": libero_tiny,
     "base_chunk": base_chunk,

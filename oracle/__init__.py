@@ -73,6 +73,8 @@ class Oracle:
         lib.oracle_merge_parts.restype = i
         lib.oracle_prefix_causal_attn.argtypes = [p] * 6 + [i] * 6
         lib.oracle_prefix_causal_attn.restype = i
+        lib.oracle_qkv_prologue.argtypes = [p] * 5 + [ctypes.c_double] * 2 + [p] * 3 + [i] * 7
+        lib.oracle_qkv_prologue.restype = i
         lib.oracle_max_threads.argtypes = []
         lib.oracle_max_threads.restype = i
         self.lib = lib
@@ -150,6 +152,26 @@ class Oracle:
             raise ValueError(f"oracle_prefix_causal_attn failed with status {rc}")
         return out, lse
 
+    def qkv_prologue(self, x, w, qw, kw, pos, B, S, H, Hq, Hkv, D, eps=1e-6, theta=10000.0, nthreads: int = 1):
+        """QKV projection + QK-Norm + RoPE of the suffix tokens.
+
+        x [B*S, H], w [(Hq+2Hkv)*D, H], qw/kw [D] (bf16 tensors or uint16 bit
+        patterns), pos int32 [B*S].  Returns float64 (q [B,Hq,S,D],
+        k [B,Hkv,S,D], v [B,Hkv,S,D])."""
+        xb, wb, qwb, kwb = _bits(x), _bits(w), _bits(qw), _bits(kw)
+        if xb.size != B * S * H or wb.size != (Hq + 2 * Hkv) * D * H or qwb.size != D or kwb.size != D:
+            raise ValueError("x/w/qw/kw size does not match the dims")
+        pb = np.ascontiguousarray(np.asarray(pos, dtype=np.int32).reshape(B * S))
+        q = np.zeros((B, Hq, S, D), dtype=np.float64)
+        k = np.zeros((B, Hkv, S, D), dtype=np.float64)
+        v = np.zeros((B, Hkv, S, D), dtype=np.float64)
+        rc = self.lib.oracle_qkv_prologue(_ptr(xb), _ptr(wb), _ptr(qwb), _ptr(kwb), _ptr(pb), float(eps),
+                                          float(theta), _ptr(q), _ptr(k), _ptr(v), B, S, H, Hq, Hkv, D,
+                                          int(nthreads))
+        if rc != 0:
+            raise ValueError(f"oracle_qkv_prologue failed with status {rc}")
+        return q, k, v
+
     def inputs_call(self, inp, nthreads: int = 1, key_range=None, row_range=None):
         """Run on an object with the attributes of a SuffixAttnInputs."""
         return self.suffix_attn(inp.q, inp.k_prefix, inp.v_prefix, inp.prefix_valid_len,
@@ -179,6 +201,11 @@ def suffix_attn(*args, **kwargs):
 def merge_parts(o_parts, lse_parts):
     """Oracle.merge_parts on the default build."""
     return default().merge_parts(o_parts, lse_parts)
+
+
+def qkv_prologue(*args, **kwargs):
+    """Oracle.qkv_prologue on the default build."""
+    return default().qkv_prologue(*args, **kwargs)
 
 
 def prefix_causal_attn(*args, **kwargs):

@@ -332,6 +332,93 @@ int oracle_prefix_causal_attn(const uint16_t *q, const uint16_t *k, const uint16
     return failed ? -7 : 0;
 }
 
+/*
+ * Suffix attention prologue: QKV projection, QK-Norm and RoPE in one step
+ * (page "TensorRT+Triton+FlexAttention: OpenDM VLA 快速推理加速栈深度剖析",
+ * section 2.2, lists "QKV projection + QK-Norm + RoPE done at once" among
+ * the fused steps; the action expert's shape table gives hidden 1024,
+ * head_dim 256 and 8 / 4 heads).  It produces the suffix queries and keys
+ * and values in the layout the suffix attention reads.
+ *
+ * Readings where the page is silent (listed in the design notes):
+ *   - one weight matrix w [(Hq + 2 Hkv) * D, H] (rows: the Hq query heads,
+ *     then the Hkv key heads, then the Hkv value heads), no bias;
+ *   - QK-Norm is an RMS norm over each head's D features with a learned
+ *     per-feature weight shared by all heads of its kind (qw for queries, kw
+ *     for keys): y_d = x_d / sqrt(mean_d x_d^2 + eps) * w_d; values are not
+ *     normalised;
+ *   - RoPE rotates the normalised query and key features in the
+ *     "rotate-half" pairing (d, d + D/2) by the angle pos * theta^(-2d/D),
+ *     pos the token's position (an input per token);
+ *   - everything in double from bf16 inputs widened exactly.
+ *
+ * Layouts: x [B*S, H] bf16 bits (token t = b*S + i), w [(Hq+2Hkv)*D, H] bf16
+ * bits, qw / kw [D] bf16 bits, pos int32 [B*S]; outputs double
+ * q [B,Hq,S,D], k [B,Hkv,S,D], v [B,Hkv,S,D].
+ * Returns 0, -1 for a NULL pointer, -2 for a bad shape, -7 for no memory.
+ */
+int oracle_qkv_prologue(const uint16_t *x, const uint16_t *w, const uint16_t *qw, const uint16_t *kw,
+                        const int32_t *pos, double eps, double theta, double *q, double *k, double *v,
+                        int B, int S, int H, int Hq, int Hkv, int D, int nthreads)
+{
+    if (!x || !w || !qw || !kw || !pos || !q || !k || !v) return -1;
+    if (B < 1 || S < 1 || H < 1 || Hq < 1 || Hkv < 1 || D < 2 || D % 2 != 0) return -2;
+    const int n_heads = Hq + 2 * Hkv;
+    const long n_items = (long)B * S * n_heads; /* (token, head) pairs */
+    int failed = 0;
+    if (nthreads < 1) nthreads = 1;
+
+#pragma omp parallel num_threads(nthreads) reduction(| : failed)
+    {
+        double *feat = (double *)malloc(sizeof(double) * (size_t)D);
+        if (!feat) {
+            failed = 1;
+        } else {
+#pragma omp for schedule(static)
+            for (long it = 0; it < n_items; ++it) {
+                const long t = it / n_heads;           /* token b*S + i */
+                const int hd = (int)(it % n_heads);    /* head in projection order */
+                const int b = (int)(t / S), i = (int)(t % S);
+                /* projection: feature f of this head = <w row, x_t> */
+                for (int d = 0; d < D; ++d) {
+                    const uint16_t *w_row = w + ((size_t)hd * D + d) * (size_t)H;
+                    const uint16_t *x_row = x + (size_t)t * H;
+                    double acc = 0.0;
+                    for (int c = 0; c < H; ++c) acc += bf16_bits_to_double(w_row[c]) * bf16_bits_to_double(x_row[c]);
+                    feat[d] = acc;
+                }
+                double *dst;
+                if (hd >= Hq + Hkv) { /* value head: projection only */
+                    dst = v + (((size_t)b * Hkv + (hd - Hq - Hkv)) * S + i) * (size_t)D;
+                    for (int d = 0; d < D; ++d) dst[d] = feat[d];
+                    continue;
+                }
+                const int is_q = hd < Hq;
+                const uint16_t *nw = is_q ? qw : kw;
+                dst = is_q ? q + (((size_t)b * Hq + hd) * S + i) * (size_t)D
+                           : k + (((size_t)b * Hkv + (hd - Hq)) * S + i) * (size_t)D;
+                /* QK-Norm: RMS over the head's features, then the weight */
+                double ms = 0.0;
+                for (int d = 0; d < D; ++d) ms += feat[d] * feat[d];
+                const double inv_rms = 1.0 / sqrt(ms / (double)D + eps);
+                for (int d = 0; d < D; ++d) feat[d] = feat[d] * inv_rms * bf16_bits_to_double(nw[d]);
+                /* RoPE, rotate-half pairing: (d, d + D/2) turned by pos * theta^(-2d/D) */
+                const int half = D / 2;
+                const double p = (double)pos[t];
+                for (int d = 0; d < half; ++d) {
+                    const double ang = p * pow(theta, -2.0 * (double)d / (double)D);
+                    const double c = cos(ang), s = sin(ang);
+                    const double a = feat[d], e = feat[d + half];
+                    dst[d] = a * c - e * s;
+                    dst[d + half] = a * s + e * c;
+                }
+            }
+            free(feat);
+        }
+    }
+    return failed ? -7 : 0;
+}
+
 /* Number of OpenMP threads this build can use (1 without OpenMP). */
 int oracle_max_threads(void)
 {

@@ -411,8 +411,138 @@ def pin_prefill_decimal_bruteforce(orc):
             assert abs(float(z.ln()) - lse[0, h, i]) < 1e-14
 
 
+# --------------------------------------------------------------------------
+# Suffix prologue: QKV projection + QK-Norm + RoPE (page "TensorRT+Triton+
+# FlexAttention: OpenDM VLA 快速推理加速栈深度剖析", section 2.2).  Readings:
+# one weight matrix (query heads, then key heads, then value heads), RMS
+# norm over each head's features with a learned weight (eps 1e-6), rotate-half
+# RoPE with theta 10000 on the normalised queries and keys.
+
+def prologue_case(seed, B=1, S=3, H=32, Hq=4, Hkv=2, D=16, pos0=0):
+    gen = torch.Generator().manual_seed(seed)
+    x = bf16_rand(gen, (B * S, H))
+    w = bf16_rand(gen, ((Hq + 2 * Hkv) * D, H), mult=0.2)
+    qw = (1.0 + 0.1 * torch.randn(D, generator=gen)).to(BF)
+    kw = (1.0 + 0.1 * torch.randn(D, generator=gen)).to(BF)
+    pos = torch.arange(B * S, dtype=torch.int32) % S + pos0
+    return dict(x=x, w=w, qw=qw, kw=kw, pos=pos, B=B, S=S, H=H, Hq=Hq, Hkv=Hkv, D=D)
+
+
+def run_prologue(orc, c, **kw):
+    return orc.qkv_prologue(c["x"], c["w"], c["qw"], c["kw"], c["pos"], c["B"], c["S"], c["H"], c["Hq"], c["Hkv"],
+                            c["D"], **kw)
+
+
+def prologue_library_reference(c, eps=1e-6, theta=10000.0):
+    """float64 library routines: linear, rms_norm, and the rotation done as a
+    complex multiplication of the pairs (d, d + D/2) by exp(i * angle)."""
+    B, S, H, Hq, Hkv, D = (c[k] for k in ("B", "S", "H", "Hq", "Hkv", "D"))
+    f = lambda t: t.to(torch.float64)
+    proj = torch.nn.functional.linear(f(c["x"]), f(c["w"]))                  # [B*S, (Hq+2Hkv)*D]
+    heads = proj.view(B * S, Hq + 2 * Hkv, D)
+    q = torch.nn.functional.rms_norm(heads[:, :Hq], (D,), weight=f(c["qw"]), eps=eps)
+    k = torch.nn.functional.rms_norm(heads[:, Hq:Hq + Hkv], (D,), weight=f(c["kw"]), eps=eps)
+    v = heads[:, Hq + Hkv:]
+    half = D // 2
+    inv = theta ** (-2.0 * torch.arange(half, dtype=torch.float64) / D)
+    ang = c["pos"].to(torch.float64)[:, None] * inv[None, :]                 # [B*S, half]
+    rot = torch.polar(torch.ones_like(ang), ang)[:, None, :]
+
+    def rope(t):
+        z = torch.complex(t[..., :half], t[..., half:]) * rot
+        return torch.cat([z.real, z.imag], dim=-1)
+
+    def lay(t, n):
+        return t.view(B, S, n, D).permute(0, 2, 1, 3).numpy()
+    return lay(rope(q), Hq), lay(rope(k), Hkv), lay(v, Hkv)
+
+
+def pin_prologue_library_float64(orc):
+    """Equal to float64 library projection, RMS norm and complex rotation."""
+    for seed, B, S, pos0 in ((51, 1, 3, 0), (52, 2, 5, 900), (53, 1, 4, 1900)):
+        c = prologue_case(seed, B=B, S=S, pos0=pos0)
+        got = run_prologue(orc, c)
+        want = prologue_library_reference(c)
+        for g, w_, name in zip(got, want, "qkv"):
+            np.testing.assert_allclose(g, w_, rtol=0, atol=1e-11, err_msg=f"prologue {name}, seed {seed}")
+
+
+def pin_prologue_position_zero_and_norm(orc):
+    """At position 0 the rotation is the identity; with unit norm weights
+    every normalised query and key row has squared length D * ms / (ms + eps)
+    (a rotation keeps lengths); values are the plain projection."""
+    c = prologue_case(54, B=1, S=4, pos0=0)
+    c["pos"] = torch.zeros_like(c["pos"])
+    c["qw"] = torch.ones_like(c["qw"])
+    c["kw"] = torch.ones_like(c["kw"])
+    q, k, v = run_prologue(orc, c)
+    proj = c["x"].to(torch.float64) @ c["w"].to(torch.float64).T
+    D, Hq, Hkv = c["D"], c["Hq"], c["Hkv"]
+    for t in range(4):
+        for h in range(Hq + 2 * Hkv):
+            y = proj[t, h * D:(h + 1) * D].numpy()
+            ms = float((y * y).mean())
+            if h < Hq:
+                got = q[0, h, t]
+            elif h < Hq + Hkv:
+                got = k[0, h - Hq, t]
+            else:
+                np.testing.assert_allclose(v[0, h - Hq - Hkv, t], y, rtol=0, atol=1e-12)
+                continue
+            np.testing.assert_allclose(got, y / math.sqrt(ms + 1e-6), rtol=0, atol=1e-12)
+    c["pos"] = torch.arange(4, dtype=torch.int32) * 37
+    q2, k2, _ = run_prologue(orc, c)
+    for t in range(4):
+        for h in range(Hq):
+            assert abs(float((q2[0, h, t] ** 2).sum()) - float((q[0, h, t] ** 2).sum())) < 1e-10
+
+
+def pin_prologue_relative_position(orc):
+    """<q at position m, k at position n> depends only on m - n: shifting
+    every position by the same amount leaves all query-key dot products
+    unchanged (pins the rotation's pairing, sign and shared angles)."""
+    c = prologue_case(55, B=1, S=5, pos0=3)
+    q0, k0, _ = run_prologue(orc, c)
+    c2 = dict(c, pos=c["pos"] + 250)
+    q1, k1, _ = run_prologue(orc, c2)
+    d0 = np.einsum("bhid,bgjd->bhgij", q0, k0)
+    d1 = np.einsum("bhid,bgjd->bhgij", q1, k1)
+    np.testing.assert_allclose(d1, d0, rtol=0, atol=1e-9)
+    assert not np.allclose(q1, q0)
+
+
+def pin_prologue_decimal_bruteforce(orc):
+    """60-digit decimal projection and RMS norm at position 0 (no trigonometry
+    needed there) on a tiny case."""
+    decimal.getcontext().prec = 60
+    c = prologue_case(56, B=1, S=2, H=8, Hq=2, Hkv=1, D=4)
+    c["pos"] = torch.zeros_like(c["pos"])
+    q, k, v = run_prologue(orc, c)
+    X = _dec_bf16(c["x"])
+    W = _dec_bf16(c["w"])
+    QW, KW = _dec_bf16(c["qw"]), _dec_bf16(c["kw"])
+    H, D = 8, 4
+    eps = decimal.Decimal("1e-6")
+    for t in range(2):
+        for h in range(4):
+            y = [sum(W[(h * D + d) * H + cc] * X[t * H + cc] for cc in range(H)) for d in range(D)]
+            if h == 3:
+                for d in range(D):
+                    assert abs(float(y[d]) - v[0, 0, t, d]) < 1e-14
+                continue
+            ms = sum(e * e for e in y) / D
+            r = (ms + eps).sqrt()
+            nw = QW if h < 2 else KW
+            for d in range(D):
+                want = float(y[d] / r * nw[d])
+                got = q[0, h, t, d] if h < 2 else k[0, 0, t, d]
+                assert abs(want - got) < 1e-13
+
+
 ALL_PINS = [pin_sdpa_float64, pin_uniform_logits, pin_constant_v_gqa, pin_masked_rows_ignored,
             pin_single_suffix_key, pin_dominant_key, pin_prefix_permutation, pin_split_merge,
             pin_decimal_bruteforce, pin_valid_len_clamp_and_boundary,
             pin_prefill_sdpa_float64, pin_prefill_first_row_and_uniform, pin_prefill_future_keys_ignored,
-            pin_prefill_decimal_bruteforce]
+            pin_prefill_decimal_bruteforce,
+            pin_prologue_library_float64, pin_prologue_position_zero_and_norm, pin_prologue_relative_position,
+            pin_prologue_decimal_bruteforce]

@@ -49,6 +49,18 @@ MUTATIONS = {
     "prefill_lse_without_max": ("const double l = m + log(z);", "const double l = log(z);"),
     "prefill_k_used_as_v": ("const uint16_t *v_row = v + kv_off + (size_t)j * D;",
                             "const uint16_t *v_row = k + kv_off + (size_t)j * D;"),
+    # suffix prologue: QKV projection + QK-Norm + RoPE
+    "prologue_rope_sign": ("dst[d] = a * c - e * s;", "dst[d] = a * c + e * s;"),
+    "prologue_rope_interleaved_pairs": ("const double a = feat[d], e = feat[d + half];",
+                                        "const double a = feat[(2 * d) % D], e = feat[(2 * d + 1) % D];"),
+    "prologue_rope_angle_exponent": ("pow(theta, -2.0 * (double)d / (double)D)", "pow(theta, -1.0 * (double)d / (double)D)"),
+    "prologue_norm_without_mean": ("const double inv_rms = 1.0 / sqrt(ms / (double)D + eps);",
+                                   "const double inv_rms = 1.0 / sqrt(ms + eps);"),
+    "prologue_key_uses_query_weight": ("const uint16_t *nw = is_q ? qw : kw;", "const uint16_t *nw = qw;"),
+    "prologue_values_scaled_by_key_weight": ("for (int d = 0; d < D; ++d) dst[d] = feat[d];\n                    continue;",
+                                             "for (int d = 0; d < D; ++d) dst[d] = feat[d] * bf16_bits_to_double(kw[d]);\n                    continue;"),
+    "prologue_weight_row_of_next_head": ("const uint16_t *w_row = w + ((size_t)hd * D + d) * (size_t)H;",
+                                         "const uint16_t *w_row = w + ((size_t)((hd + 1) % n_heads) * D + d) * (size_t)H;"),
 }
 
 

@@ -50,6 +50,8 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU-baseline sample budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-workloads", action="store_true", help="skip the per-workload table")
+    ap.add_argument("--prefix-static", action="store_true",
+                    help="declare the prefix cache static (DM05_FLAG_PREFIX_STATIC) in the timed calls")
     return ap.parse_args()
 
 
@@ -575,11 +577,13 @@ def main():
         raise bd.Dm05Error(rc, "reserve")
     rc, splits, tile_rows, row_blocks = bd.dm05_suffix_attn_plan(B, Hq, Hkv, P, S, D)
 
+    flags = bd.DM05_FLAG_PREFIX_STATIC if args.prefix_static else 0
+
     def call(t, s=sh):
         ptr = lambda x: None if x is None else x.data_ptr()
-        rc = bd.dm05_suffix_attn(ptr(t["q"]), ptr(t["k_prefix"]), ptr(t["v_prefix"]), ptr(t["prefix_valid_len"]),
-                                 ptr(t["prefix_mask"]), ptr(t["k_suffix"]), ptr(t["v_suffix"]), ptr(t["out"]),
-                                 ptr(t["lse"]), B, Hq, Hkv, P, S, D, s)
+        rc = bd.dm05_suffix_attn_ex(ptr(t["q"]), ptr(t["k_prefix"]), ptr(t["v_prefix"]), ptr(t["prefix_valid_len"]),
+                                    ptr(t["prefix_mask"]), ptr(t["k_suffix"]), ptr(t["v_suffix"]), ptr(t["out"]),
+                                    ptr(t["lse"]), B, Hq, Hkv, P, S, D, flags, s)
         if rc != 0:
             raise bd.Dm05Error(rc, "dm05_suffix_attn")
 
@@ -744,7 +748,7 @@ def main():
                 "splits_per_head": splits, "row_blocks": row_blocks, "tile_rows": tile_rows,
                 "parallelism": f"replicas x{world}",
                 "l2": f"{R} rotating input sets, {R * set_bytes / 1e6:.0f} MB > 2 x L2 ({l2 / 1e6:.0f} MB)",
-                "graph_calls": chunk}),
+                "graph_calls": chunk, "prefix_static": bool(args.prefix_static)}),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": profiled_traffic(args.workload, (splits, row_blocks, tile_rows)),
                          "peak_source": peak_kind, "algorithmic_bytes": kv_bytes,

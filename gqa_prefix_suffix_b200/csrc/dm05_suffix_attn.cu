@@ -104,12 +104,15 @@ Plan make_plan(int B, int Hq, int Hkv, int P, int S, const DeviceState &ds)
         return units * blocks * c <= ds.num_sms && units * blocks <= ds.active[c];
     };
     // Estimated cost in microseconds, fitted on B200 measurements of this
-    // kernel: ~1.2 per key tile a CTA streams, and for a split unit a fixed
-    // ~2 for the merge plus ~0.04 per partial row a CTA publishes.
+    // kernel (base-model chunk, every plan of 1-16 CTAs x 1-5 query blocks,
+    // rotating inputs): a split unit costs ~6.4 fixed (launch, first data,
+    // merge latency chain), ~1.3 per key tile its slowest CTA streams and
+    // ~0.04 per partial row a CTA publishes; an unsplit unit has no merge.
+    // Cluster sizes that are not powers of two measured ~1-1.5 slower than
+    // the model and are not used.
     auto cost = [&](int c, int sq) {
-        double t = 1.2 * ((tiles + c - 1) / c);
-        if (c > 1) t += 2.0 + 0.04 * G * sq;
-        return t;
+        const double per_tile = 1.31 * ((tiles + c - 1) / c);
+        return c > 1 ? 6.4 + per_tile + 0.04 * G * sq : 3.0 + per_tile;
     };
     const int want_rb = g_row_block_override;
     Plan best;
@@ -117,7 +120,7 @@ Plan make_plan(int B, int Hq, int Hkv, int P, int S, const DeviceState &ds)
     double best_cost = 1e30;
     for (int c = 1; c <= dm05::kMaxSplits; ++c) {
         if (g_split_override > 0 && c != g_split_override) continue;
-        if (g_split_override == 0 && (c > ds.max_cluster || !fits(c, 1))) continue;
+        if (g_split_override == 0 && ((c & (c - 1)) != 0 || c > ds.max_cluster || !fits(c, 1))) continue;
         for (int r = 1; r <= 16; ++r) {
             if (c == 1 && r > 1) break;
             const int sq = (S + r - 1) / r;

@@ -1,0 +1,261 @@
+// qkv_prologue_kernel.cuh -- sm_100a kernel of the suffix attention's
+// prologue: QKV projection, QK-Norm and RoPE in one pass.
+//
+// What it computes (page "TensorRT+Triton+FlexAttention: OpenDM VLA
+// 快速推理加速栈深度剖析", section 2.2 lists "QKV projection + QK-Norm + RoPE
+// done at once" among the fused steps; the action expert's shape table gives
+// hidden 1024, head_dim 256, 8 / 4 heads): for token t (= b * S + i) and
+// head hd of the weight's row order (Hq query heads, Hkv key heads, Hkv value
+// heads),
+//   y      = w[hd * D : (hd + 1) * D, :] x_t                    (projection)
+//   y'     = y / sqrt(mean(y^2) + eps) * nw                     (query / key heads)
+//   out_d  = y'_d cos(a_d) - y'_{d+D/2} sin(a_d),               d < D/2,
+//   out_{d+D/2} = y'_d sin(a_d) + y'_{d+D/2} cos(a_d),  a_d = pos_t theta^(-2d/D)
+// value heads are the plain projection.  Outputs go to q [B,Hq,S,D],
+// k [B,Hkv,S,D], v [B,Hkv,S,D], the layout the suffix attention reads.
+//
+// Design (one CTA = one head half x one tile of NT tokens):
+//   * Swapped GEMM on tcgen05: D^T[features, tokens] = W_rows x X^T with
+//     M = 128 feature rows (A, K-major from the weight) and N = NT tokens
+//     (B, K-major from the hidden states), K = H in 64-column chunks staged by
+//     TMA (128-byte swizzle) in a ring.  The accumulator lives in TMEM.
+//   * A CTA's 128 feature rows are the two rotation partners of 64 pairs:
+//     features 64c + j (lanes j) and 64c + 128 + j (lanes 64 + j) of its head,
+//     so RoPE needs no data from another CTA.  The two halves of a head form a
+//     cluster of 2 and exchange their per-token sums of squares through
+//     distributed shared memory for the RMS norm.
+//   * Epilogue: TMEM -> shared memory [128][NT] fp32, per-token sums of
+//     squares, the exchange, then each thread produces rotated pairs and
+//     stores bf16 rows (consecutive threads write consecutive features).
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "sm100_ptx.cuh"
+
+namespace dm05 {
+namespace prologue {
+
+constexpr int kThreads = 128;
+constexpr int kStages = 4;
+constexpr int kChunk = 64;                 // K columns per stage (128 bytes of bf16)
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+constexpr uint32_t kEwTimeout = 0x2u;
+
+struct Params {
+    const __nv_bfloat16 *qw;   // [D] query-norm weight
+    const __nv_bfloat16 *kw;   // [D] key-norm weight
+    const int32_t *pos;        // [T] positions
+    __nv_bfloat16 *q, *k, *v;  // outputs
+    uint32_t *err;
+    int T, S, H, Hq, Hkv, D;   // tokens (B * S), tokens per sample, hidden, heads, head dim
+    float eps;
+    float log2_theta;          // log2(theta)
+};
+
+template <int NT>
+struct Smem {
+    static constexpr int kABytes = 128 * kChunk * 2;     // 16 KB: 128 feature rows
+    static constexpr int kBBytes = NT * kChunk * 2;      // NT token rows
+    static constexpr int kStageBytes = kABytes + kBBytes;
+    static constexpr int kRingBytes = kStages * kStageBytes;
+    static constexpr int kYStride = NT + 4;              // fp32 per feature row (padded)
+    static constexpr int kYBytes = 128 * kYStride * 4;
+    static_assert(kRingBytes >= kYBytes, "the epilogue tile reuses the ring");
+    static constexpr int kBarOff = kRingBytes;
+    static constexpr int kNumBars = 2 * kStages + 1;     // full[s], empty[s], mma done
+    static constexpr int kSsOff = kBarOff + kNumBars * 8 + 8;   // own sums [NT], partner's sums [NT]
+    static constexpr int kTmemSlotOff = kSsOff + 2 * NT * 4;
+    static constexpr int kEnd = kTmemSlotOff + 16;
+    static constexpr int kAllocBytes = kEnd + 1024;
+};
+
+template <int NT>
+__global__ void __launch_bounds__(kThreads, 1)
+    qkv_prologue_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
+                        const Params p)
+{
+    using L = Smem<NT>;
+    static_assert(NT % 16 == 0 && NT >= 16 && NT <= 256, "N of an M=128 MMA");
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kBarOff);
+    uint64_t *full = bars, *empty = bars + kStages, *mma_done = bars + 2 * kStages;
+    float *ss_own = reinterpret_cast<float *>(smem + L::kSsOff);
+    float *ss_peer = ss_own + NT;  // written by the other half of the head
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kTmemSlotOff);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // blockIdx.x = (head * 2 + half); blockIdx.y = token tile.  The two
+    // halves of a head are one cluster of 2.
+    const int half = blockIdx.x & 1;
+    const int hd = blockIdx.x >> 1;
+    const int t0 = blockIdx.y * NT;
+    const int D = p.D;
+    const int n_chunks = p.H / kChunk;
+    const bool is_v = hd >= p.Hq + p.Hkv;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            ptx::mbar_init(&full[s], 1);
+            ptx::mbar_init(&empty[s], 1);
+        }
+        ptx::mbar_init(mma_done, 1);
+        ptx::fence_mbar_init();
+        ptx::prefetch_tensormap(&tm_w);
+        ptx::prefetch_tensormap(&tm_x);
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc(tmem_slot, NT <= 32 ? 32 : NT <= 64 ? 64 : NT <= 128 ? 128 : 256);
+        ptx::tmem_relinquish();
+    }
+    ptx::griddep_launch_dependents();
+    ptx::tc_fence_before_sync();
+    __syncthreads();
+    ptx::tc_fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    ptx::griddep_wait();
+
+    bool failed = false;
+    // feature rows of this CTA: the head's rows [64*half, +64) then [64*half + 128, +64)
+    const int row_a = hd * D + 64 * half;
+    if (warp == 0 && lane == 0) {
+        // ------------------------------------------------ TMA producer
+        for (int c = 0; c < n_chunks; ++c) {
+            const int s = c % kStages, n = c / kStages;
+            if (n > 0 && !ptx::mbar_wait(&empty[s], (n - 1) & 1, kWaitLimitNs)) {
+                failed = true;
+                break;
+            }
+            uint8_t *a = smem + s * L::kStageBytes;
+            ptx::mbar_arrive_expect_tx(&full[s], L::kStageBytes);
+            ptx::tma_load_2d(a, &tm_w, &full[s], c * kChunk, row_a);
+            ptx::tma_load_2d(a + 64 * 128, &tm_w, &full[s], c * kChunk, row_a + 128);
+            ptx::tma_load_2d(a + L::kABytes, &tm_x, &full[s], c * kChunk, t0);
+        }
+        // drain: every issued copy has landed before the CTA may exit
+        for (int c = (n_chunks > kStages ? n_chunks - kStages : 0); c < n_chunks && !failed; ++c)
+            if (!ptx::mbar_wait(&full[c % kStages], (c / kStages) & 1, kWaitLimitNs)) failed = true;
+    } else if (warp == 1 && lane == 0) {
+        // ------------------------------------------------ MMA issuer
+        constexpr uint32_t idesc = ptx::idesc_bf16_f32(128, NT, false);
+        const uint64_t adesc0 = ptx::sw128_desc(ptx::smem_addr(smem), 16, 1024);
+        const uint64_t bdesc0 = ptx::sw128_desc(ptx::smem_addr(smem + L::kABytes), 16, 1024);
+        bool ok = true;
+        for (int c = 0; c < n_chunks; ++c) {
+            const int s = c % kStages;
+            if (!ptx::mbar_wait(&full[s], (c / kStages) & 1, kWaitLimitNs)) {
+                ok = false;
+                break;
+            }
+            ptx::tc_fence_after_sync();
+            const uint64_t so = static_cast<uint64_t>((s * L::kStageBytes) >> 4);
+#pragma unroll
+            for (int kk = 0; kk < kChunk / 16; ++kk)
+                ptx::mma_bf16_ss(tmem, adesc0 + so + static_cast<uint64_t>((kk * 32) >> 4),
+                                 bdesc0 + so + static_cast<uint64_t>((kk * 32) >> 4), idesc,
+                                 (c > 0 || kk > 0) ? 1u : 0u);
+            ptx::mma_commit(&empty[s]);
+        }
+        ptx::mma_commit(mma_done);
+        if (!ok) failed = true;
+    }
+    __syncwarp();
+
+    // ---------------------------------------------------- epilogue
+    // all MMAs (and so every stage's copies) complete
+    if (!ptx::mbar_wait(mma_done, 0, kWaitLimitNs)) failed = true;
+    ptx::tc_fence_after_sync();
+    // TMEM lane = this thread's feature row, columns = tokens
+    float *Y = reinterpret_cast<float *>(smem);  // [128][kYStride]
+    const int r = threadIdx.x;
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+#pragma unroll
+    for (int j = 0; j < NT / 16; ++j) {
+        uint32_t o[16];
+        ptx::tmem_ld16(tmem + lane_base + j * 16, o);
+        ptx::tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) Y[r * L::kYStride + j * 16 + e] = __uint_as_float(o[e]);
+    }
+    __syncthreads();
+    if (!is_v) {
+        // per-token sum of squares over this CTA's 128 features, then the
+        // other half's through its shared memory (cluster of 2)
+        for (int t = threadIdx.x; t < NT; t += kThreads) {
+            float acc = 0.0f;
+            for (int f = 0; f < 128; ++f) {
+                const float y = Y[f * L::kYStride + t];
+                acc = fmaf(y, y, acc);
+            }
+            ss_own[t] = acc;
+            ptx::st_dsmem_f32(ptx::mapa(ptx::smem_addr(ss_peer + t), static_cast<uint32_t>(half ^ 1)), acc);
+        }
+    }
+    ptx::cluster_sync();  // both halves' sums are in place (and no one still writes)
+
+    // each thread: feature pair j = threadIdx.x % 64 for tokens of one parity
+    const int j = threadIdx.x & 63;
+    const int fa = 64 * half + j;          // feature index within the head (first of the pair)
+    const int fb = fa + D / 2;
+    __nv_bfloat16 *dst_base;
+    int heads, h;
+    if (hd < p.Hq) {
+        dst_base = p.q;
+        heads = p.Hq;
+        h = hd;
+    } else if (!is_v) {
+        dst_base = p.k;
+        heads = p.Hkv;
+        h = hd - p.Hq;
+    } else {
+        dst_base = p.v;
+        heads = p.Hkv;
+        h = hd - p.Hq - p.Hkv;
+    }
+    float wa = 1.0f, wb = 1.0f;
+    double inv_freq = 0.0;
+    if (!is_v) {
+        const __nv_bfloat16 *nw = hd < p.Hq ? p.qw : p.kw;
+        wa = __bfloat162float(nw[fa]);
+        wb = __bfloat162float(nw[fb]);
+        // theta^(-2 fa / D), in double: positions reach thousands of radians
+        inv_freq = exp2(-2.0 * static_cast<double>(fa) / static_cast<double>(D) * static_cast<double>(p.log2_theta));
+    }
+    for (int t = (threadIdx.x >> 6); t < NT; t += kThreads / 64) {
+        const int tok = t0 + t;
+        if (tok >= p.T) break;
+        const float ya = Y[j * L::kYStride + t], yb = Y[(64 + j) * L::kYStride + t];
+        float oa = ya, ob = yb;
+        if (!is_v) {
+            const float ms = (ss_own[t] + ss_peer[t]) / static_cast<float>(D);
+            const float inv_rms = rsqrtf(ms + p.eps);
+            const float a = ya * inv_rms * wa, b = yb * inv_rms * wb;
+            // the angle reduced to [-pi, pi] in double, then its sine and cosine
+            const double two_pi = 6.283185307179586;
+            double ang = static_cast<double>(p.pos[tok]) * inv_freq;
+            ang -= two_pi * rint(ang / two_pi);
+            float sn, cs;
+            sincosf(static_cast<float>(ang), &sn, &cs);
+            oa = a * cs - b * sn;
+            ob = a * sn + b * cs;
+        }
+        const int bi = tok / p.S, i = tok - bi * p.S;
+        __nv_bfloat16 *row = dst_base + ((static_cast<size_t>(bi) * heads + h) * p.S + i) * D;
+        row[fa] = __float2bfloat16_rn(oa);
+        row[fb] = __float2bfloat16_rn(ob);
+    }
+
+    if (failed && lane == 0) atomicOr(p.err, kEwTimeout);
+    ptx::tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        ptx::tc_fence_after_sync();
+        ptx::tmem_dealloc(tmem, NT <= 32 ? 32 : NT <= 64 ? 64 : NT <= 128 ? 128 : 256);
+    }
+}
+
+}  // namespace prologue
+}  // namespace dm05

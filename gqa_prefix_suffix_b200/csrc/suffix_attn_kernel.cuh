@@ -266,8 +266,11 @@ __device__ __forceinline__ void merge_rows(const uint8_t *recv, int C, int nr, _
 {
     const int items = nr * (kHeadDim / 4);
     const size_t cstride = static_cast<size_t>(nr) * L::kStageStride;
+    int trace_n = 0;
     for (int i = threadIdx.x; i < items; i += kThreads) {
         const int rr = i / (kHeadDim / 4), ch = i - rr * (kHeadDim / 4);
+        if (threadIdx.x == 0 && trace_n < 2) DM05_TRACE_TILE(4 + trace_n, 22);
+        ++trace_n;
         // only the queries [0, jlim) of each head of the block are written
         if ((k_lo + rr) % nq >= jlim) continue;
         const uint8_t *row0 = recv + rr * L::kStageStride;

@@ -395,6 +395,111 @@ def time_prefill(inp, K, W, dev, stream, bd, l2):
     return us, copies
 
 
+def time_prologue(inp, K, W, dev, stream, bd, l2):
+    """Device time per dm05_suffix_qkv_prologue call: rotating on-device copies
+    of the inputs over 2 x L2, graphs of up to 1000 calls, CUDA events."""
+    import torch
+    one = sum(t.numel() * t.element_size() for t in inp.tensors().values())
+    copies = max(2, int(2 * l2 // max(1, one)) + 2)
+    d0 = inp.to(dev)
+    sets = []
+    for _ in range(copies):
+        sets.append(dict(x=d0.x.clone(), w=d0.w.clone(), qw=d0.qw.clone(), kw=d0.kw.clone(), pos=d0.pos.clone(),
+                         q=torch.empty((inp.B, inp.Hq, inp.S, inp.D), dtype=torch.bfloat16, device=dev),
+                         k=torch.empty((inp.B, inp.Hkv, inp.S, inp.D), dtype=torch.bfloat16, device=dev),
+                         v=torch.empty((inp.B, inp.Hkv, inp.S, inp.D), dtype=torch.bfloat16, device=dev)))
+
+    def call(t):
+        rc = bd.dm05_suffix_qkv_prologue(t["x"].data_ptr(), t["w"].data_ptr(), t["qw"].data_ptr(),
+                                         t["kw"].data_ptr(), t["pos"].data_ptr(), t["q"].data_ptr(),
+                                         t["k"].data_ptr(), t["v"].data_ptr(), inp.B, inp.S, inp.H, inp.Hq,
+                                         inp.Hkv, inp.D, 1e-6, 10000.0, stream.cuda_stream)
+        if rc != 0:
+            raise bd.Dm05Error(rc, "dm05_suffix_qkv_prologue")
+
+    with torch.cuda.stream(stream):
+        for i in range(max(3, W)):
+            call(sets[i % copies])
+    stream.synchronize()
+    graphs, done = [], 0
+    while done < K:
+        m = min(1000, K - done)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(m):
+                call(sets[(done + i) % copies])
+        graphs.append(g)
+        done += m
+    warm_graphs(graphs, stream)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for g in graphs:
+            g.replay()
+        e1.record(stream)
+    stream.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / K
+    del graphs, sets
+    return us, copies
+
+
+def history_steps(calls, K, dev, stream, bd):
+    """The 10 denoising-step calls of the history loop over one prefix cache:
+    (a) one dm05_suffix_attn_steps launch of the 10 calls (a graph the library
+    captured once, static-prefix flag set), (b) the same 10 calls issued one by
+    one with dm05_suffix_attn (no graph).  Both time whole 10-step loops with
+    CUDA events on the launching stream (the prefix stays warm across steps,
+    as specified)."""
+    import torch
+    ds = [c.to(dev) for c in calls]
+    d0 = ds[0]
+    outs = [torch.empty_like(d.q) for d in ds]
+    lses = [torch.empty(d.q.shape[:3], dtype=torch.float32, device=dev) for d in ds]
+    ptr = lambda x: None if x is None else x.data_ptr()
+    steps = [(ptr(d.q), ptr(d.k_suffix), ptr(d.v_suffix), ptr(o), ptr(l)) for d, o, l in zip(ds, outs, lses)]
+    B, Hq, Hkv, P, S, D = d0.B, d0.Hq, d0.Hkv, d0.P, d0.S, d0.D
+    rc, h = bd.dm05_suffix_attn_steps_create(steps, ptr(d0.k_prefix), ptr(d0.v_prefix), ptr(d0.prefix_valid_len),
+                                             None, B, Hq, Hkv, P, S, D, bd.DM05_FLAG_PREFIX_STATIC)
+    if rc != 0:
+        raise bd.Dm05Error(rc, "dm05_suffix_attn_steps_create")
+    loops = max(20, K // 10)
+
+    def timed(fn, n):
+        for _ in range(max(3, n // 10)):
+            fn()
+        stream.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(n):
+                fn()
+            e1.record(stream)
+        stream.synchronize()
+        return e0.elapsed_time(e1) * 1e3 / n
+
+    def one_launch():
+        if bd.dm05_suffix_attn_steps_launch(h, stream.cuda_stream) != 0:
+            raise RuntimeError("dm05_suffix_attn_steps_launch failed")
+
+    def separate():
+        for d, o, l in zip(ds, outs, lses):
+            if bd.dm05_suffix_attn(ptr(d.q), ptr(d0.k_prefix), ptr(d0.v_prefix), ptr(d0.prefix_valid_len), None,
+                                   ptr(d.k_suffix), ptr(d.v_suffix), ptr(o), ptr(l), B, Hq, Hkv, P, S, D,
+                                   stream.cuda_stream) != 0:
+                raise RuntimeError("dm05_suffix_attn failed")
+
+    try:
+        t_steps = timed(one_launch, loops)
+        t_sep = timed(separate, loops)
+    finally:
+        bd.dm05_suffix_attn_steps_destroy(h)
+    n = len(calls)
+    return {"steps_one_launch": {"per_10_steps": t_steps * 10 / n, "us_per_call": t_steps / n, "loops": loops,
+                                 "api": "dm05_suffix_attn_steps_launch (captured once, static-prefix flag)"},
+            "separate_calls": {"per_10_steps": t_sep * 10 / n, "us_per_call": t_sep / n, "loops": loops,
+                               "api": "10 x dm05_suffix_attn, no graph"}}
+
+
 def measured_tensor_peak():
     """Dense bf16 tensor peak in TFLOP/s: the measured burst figure when the
     driver's MEASURED_PEAKS.json is present, else the recipe's fallback."""
@@ -439,7 +544,7 @@ def workload_table(args, dev, stream, bd, l2, peak):
     warm = row(hist, rotate=False, note="one prefix cache, 10 fresh suffix sets per 10 steps (warm, as specified)")
     cold["per_10_steps"] = 10 * cold["us_per_call"]
     warm["per_10_steps"] = 10 * warm["us_per_call"]
-    out["history_loop"] = {"cold": cold, "warm": warm}
+    out["history_loop"] = {"cold": cold, "warm": warm, **history_steps(hist, K, dev, stream, bd)}
     out["batched_mask"] = row([gen.batched_mask()])
     # the prefix-prefill attention (prefix-causal mask) on the base chunk's and
     # the history demo's prefixes: a dense contraction, bound by the tensor cores
@@ -453,6 +558,23 @@ def workload_table(args, dev, stream, bd, l2, peak):
                          "roofline": {"bound": "tensor", "peak": tpeak, "peak_source": tkind, "frac": tf / tpeak},
                          "plan": {"splits_per_head": sp, "query_block": qb, "row_blocks": rb}, "calls": K,
                          "l2": f"{copies} rotating copies"}
+    # the suffix prologue (QKV projection + QK-Norm + RoPE): the weight stream
+    # bounds it at B = 1, the tensor cores at B = 32
+    for inp in (gen.prologue_base(), gen.prologue_batched()):
+        us, copies = time_prologue(inp, K, W, dev, stream, bd, l2)
+        F = (inp.Hq + 2 * inp.Hkv) * inp.D
+        T = inp.B * inp.S
+        nbytes = 2 * (F * inp.H + T * inp.H + T * F) + 4 * T
+        fl = 2 * T * F * inp.H
+        gbs, tf = nbytes / (us * 1e-6) / 1e9, fl / (us * 1e-6) / 1e12
+        t_hbm, t_tc = nbytes / (peak * 1e9), fl / (tpeak * 1e12)
+        bound = "hbm" if t_hbm >= t_tc else "tensor"
+        out[inp.name] = {"us_per_call": us, "algorithmic_bytes": nbytes, "algorithmic_flops": fl,
+                         "achieved_gbs": gbs, "achieved_tflops": tf,
+                         "roofline": {"bound": bound, "frac": (t_hbm if bound == "hbm" else t_tc) / (us * 1e-6),
+                                      "peak": peak if bound == "hbm" else tpeak,
+                                      "unit": "GB/s" if bound == "hbm" else "TFLOP/s"},
+                         "calls": K, "l2": f"{copies} rotating copies"}
     return out
 
 

@@ -31,10 +31,17 @@ EXPORTS = ("dm05_suffix_attn", "dm05_suffix_attn_ex", "dm05_suffix_attn_workspac
            "dm05_get_error_word",
            "dm05_status_string", "dm05_release", "dm05_suffix_attn_noalloc", "dm05_suffix_attn_host",
            "dm05_suffix_attn_host_copy_bytes", "dm05_selftest_wait_timeout", "dm05_prefix_prefill_attn",
-           "dm05_prefix_prefill_reserve", "dm05_prefix_prefill_plan")
+           "dm05_prefix_prefill_reserve", "dm05_prefix_prefill_plan", "dm05_suffix_qkv_prologue",
+           "dm05_suffix_attn_steps_create", "dm05_suffix_attn_steps_launch", "dm05_suffix_attn_steps_destroy")
 
 _lock = threading.Lock()
 _lib = None
+
+
+class Dm05Step(ctypes.Structure):
+    """dm05_step: one call's own tensors (device addresses)."""
+    _fields_ = [("q", ctypes.c_void_p), ("k_suffix", ctypes.c_void_p), ("v_suffix", ctypes.c_void_p),
+                ("out", ctypes.c_void_p), ("lse", ctypes.c_void_p)]
 
 
 class Dm05Error(RuntimeError):
@@ -88,6 +95,15 @@ def lib() -> ctypes.CDLL:
             L.dm05_prefix_prefill_reserve.restype = i
             L.dm05_prefix_prefill_plan.argtypes = [i] * 5 + [ctypes.POINTER(i)] * 3
             L.dm05_prefix_prefill_plan.restype = i
+            L.dm05_suffix_qkv_prologue.argtypes = [p] * 8 + [i] * 6 + [ctypes.c_float] * 2 + [p]
+            L.dm05_suffix_qkv_prologue.restype = i
+            L.dm05_suffix_attn_steps_create.argtypes = [ctypes.POINTER(Dm05Step), i] + [p] * 4 + [i] * 6 + \
+                [ctypes.c_uint, ctypes.POINTER(p)]
+            L.dm05_suffix_attn_steps_create.restype = i
+            L.dm05_suffix_attn_steps_launch.argtypes = [p, p]
+            L.dm05_suffix_attn_steps_launch.restype = i
+            L.dm05_suffix_attn_steps_destroy.argtypes = [p]
+            L.dm05_suffix_attn_steps_destroy.restype = i
             _lib = L
     return _lib
 
@@ -145,6 +161,32 @@ def dm05_prefix_prefill_plan(B, Hq, Hkv, P, D):
     sp, qb, rb = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int(0)
     rc = lib().dm05_prefix_prefill_plan(B, Hq, Hkv, P, D, ctypes.byref(sp), ctypes.byref(qb), ctypes.byref(rb))
     return rc, sp.value, qb.value, rb.value
+
+
+def dm05_suffix_qkv_prologue(x, w, q_norm_w, k_norm_w, positions, q, k, v, B, S, H, Hq, Hkv, D, eps, theta,
+                             stream) -> int:
+    """QKV projection + QK-Norm + RoPE of the suffix tokens."""
+    return lib().dm05_suffix_qkv_prologue(x, w, q_norm_w, k_norm_w, positions, q, k, v, B, S, H, Hq, Hkv, D,
+                                          float(eps), float(theta), stream)
+
+
+def dm05_suffix_attn_steps_create(steps, k_prefix, v_prefix, prefix_valid_len, prefix_mask, B, Hq, Hkv, P, S, D,
+                                  flags=0):
+    """steps: a list of (q, k_suffix, v_suffix, out, lse) device addresses.
+    Returns (status, handle)."""
+    arr = (Dm05Step * len(steps))(*[Dm05Step(*st) for st in steps])
+    h = ctypes.c_void_p(0)
+    rc = lib().dm05_suffix_attn_steps_create(arr, len(steps), k_prefix, v_prefix, prefix_valid_len, prefix_mask,
+                                             B, Hq, Hkv, P, S, D, flags, ctypes.byref(h))
+    return rc, h.value
+
+
+def dm05_suffix_attn_steps_launch(handle, stream) -> int:
+    return lib().dm05_suffix_attn_steps_launch(handle, stream)
+
+
+def dm05_suffix_attn_steps_destroy(handle) -> int:
+    return lib().dm05_suffix_attn_steps_destroy(handle)
 
 
 def dm05_suffix_attn_workspace_bytes(B, Hq, Hkv, P, S, D) -> int:
@@ -325,6 +367,35 @@ def prefix_prefill_attn(q, k, v, valid_len=None, out=None, lse=None, want_lse: b
     if rc != DM05_OK:
         raise Dm05Error(rc, "dm05_prefix_prefill_attn")
     return out, lse
+
+
+def suffix_qkv_prologue(x, w, q_norm_w, k_norm_w, positions, B, S, Hq=8, Hkv=4, D=256, eps=1e-6, theta=10000.0,
+                        q=None, k=None, v=None, stream=None):
+    """QKV projection + QK-Norm + RoPE on CUDA torch tensors; returns (q, k, v)
+    in the suffix attention's layout.  x [B*S, H] bf16, w [(Hq+2Hkv)*D, H]
+    bf16, norm weights [D] bf16, positions int32 [B*S]."""
+    import torch
+    H = x.shape[1]
+    for name, t, shape, dt in (("x", x, (B * S, H), torch.bfloat16), ("w", w, ((Hq + 2 * Hkv) * D, H), torch.bfloat16),
+                               ("q_norm_w", q_norm_w, (D,), torch.bfloat16), ("k_norm_w", k_norm_w, (D,), torch.bfloat16),
+                               ("positions", positions, (B * S,), torch.int32)):
+        if not t.is_cuda or t.dtype != dt or tuple(t.shape) != shape or not t.is_contiguous() or t.device != x.device:
+            raise ValueError(f"{name} must be a contiguous CUDA {dt} tensor {list(shape)} on {x.device}")
+    if q is None:
+        q = torch.empty((B, Hq, S, D), dtype=torch.bfloat16, device=x.device)
+    if k is None:
+        k = torch.empty((B, Hkv, S, D), dtype=torch.bfloat16, device=x.device)
+    if v is None:
+        v = torch.empty((B, Hkv, S, D), dtype=torch.bfloat16, device=x.device)
+    for name, t, shape in (("q", q, (B, Hq, S, D)), ("k", k, (B, Hkv, S, D)), ("v", v, (B, Hkv, S, D))):
+        if not t.is_cuda or t.dtype != torch.bfloat16 or tuple(t.shape) != shape or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA bfloat16 tensor {list(shape)}")
+    rc = dm05_suffix_qkv_prologue(x.data_ptr(), w.data_ptr(), q_norm_w.data_ptr(), k_norm_w.data_ptr(),
+                                  positions.data_ptr(), q.data_ptr(), k.data_ptr(), v.data_ptr(), B, S, H, Hq, Hkv, D,
+                                  eps, theta, _stream_handle(stream))
+    if rc != DM05_OK:
+        raise Dm05Error(rc, "dm05_suffix_qkv_prologue")
+    return q, k, v
 
 
 def reserve_for(q, k_prefix, stream=None) -> None:

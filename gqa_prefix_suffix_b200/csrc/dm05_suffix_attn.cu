@@ -16,6 +16,7 @@
 #include <thread>
 #include <vector>
 
+#include "qkv_prologue_kernel.cuh"
 #include "suffix_attn_kernel.cuh"
 
 namespace {
@@ -31,6 +32,7 @@ constexpr int kMaxPrefix = 1 << 24;      // P
 struct DeviceState {
     uint32_t *err = nullptr;   // device error word
     bool attrs_set = false;
+    bool prologue_attrs_set = false;
     int num_sms = 0;
     int max_cluster = 0;       // largest cluster size (<= 16) that can be resident
     int active[17] = {};       // active[c]: clusters of c CTAs the device holds at once (0: not allowed)
@@ -61,6 +63,8 @@ int g_row_block_override = 0;
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
 auto *kKernel = &dm05::suffix_attn_kernel<kTileRows, kStages>;
+auto *kPrologue64 = &dm05::prologue::qkv_prologue_kernel<64>;
+auto *kPrologue128 = &dm05::prologue::qkv_prologue_kernel<128>;
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -438,6 +442,20 @@ int encode_3d(CUtensorMap *map, const void *base, uint64_t d1, uint64_t d2, uint
 }
 
 
+// bf16 matrix [rows][cols] (cols contiguous) loaded in boxes of 64 columns x
+// box_rows rows with 128-byte swizzle; rows past the end read as zero.
+int encode_2d(CUtensorMap *map, const void *base, uint64_t cols, uint64_t rows, uint32_t box_rows)
+{
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {64, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? DM05_OK : DM05_ERR_CUDA;
+}
+
 // Encodes the tensor maps and launches the kernel with plan `pl` on
 // `stream`; `err` is the device error word, `part` the partial-result area
 // (unused when pl.splits == 1).  Sizes and pointers are already checked.
@@ -720,6 +738,194 @@ int dm05_prefix_prefill_plan(int B, int Hq, int Hkv, int P, int D, int *splits_p
     if (splits_per_head) *splits_per_head = pl.splits;
     if (query_block) *query_block = pl.SQ;
     if (row_blocks) *row_blocks = pl.row_blocks;
+    return DM05_OK;
+}
+
+int dm05_suffix_qkv_prologue(const void *x, const void *w, const void *q_norm_w, const void *k_norm_w,
+                             const int32_t *positions, void *q, void *k, void *v, int B, int S, int H, int Hq,
+                             int Hkv, int D, float eps, float theta, cudaStream_t stream)
+{
+    if (!x || !w || !q_norm_w || !k_norm_w || !positions || !q || !k || !v) return DM05_ERR_NULL;
+    if (B < 1 || S < 1 || H < 1 || Hq < 1 || Hkv < 1) return DM05_ERR_SHAPE;
+    const long long T = static_cast<long long>(B) * S;
+    if (T > (1LL << 24) || H > (1 << 20) || static_cast<long long>(Hq + 2 * Hkv) * D > (1LL << 24))
+        return DM05_ERR_SHAPE;
+    if (!(eps > 0.0f) || !(theta > 1.0f)) return DM05_ERR_SHAPE;
+    if (D != dm05::kHeadDim || H % dm05::prologue::kChunk != 0) return DM05_ERR_UNSUPPORTED;
+    if (!aligned16(x) || !aligned16(w) || !aligned16(q) || !aligned16(k) || !aligned16(v) ||
+        (reinterpret_cast<uintptr_t>(q_norm_w) & 1u) || (reinterpret_cast<uintptr_t>(k_norm_w) & 1u) ||
+        (reinterpret_cast<uintptr_t>(positions) & 3u))
+        return DM05_ERR_ALIGN;
+    const bool small = T <= 64;
+    uint32_t *err = nullptr;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (get_encoder() != DM05_OK) return DM05_ERR_CUDA;
+        DeviceState *ds = nullptr;
+        int rc = device_state(false, &ds);
+        if (rc != DM05_OK) return rc;
+        if (ds->err == nullptr || !ds->prologue_attrs_set) {
+            cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+            if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) return DM05_ERR_CUDA;
+            if (cs != cudaStreamCaptureStatusNone) return DM05_ERR_WORKSPACE;
+            rc = device_state(true, &ds, stream);
+            if (rc != DM05_OK) return rc;
+            if (cudaFuncSetAttribute(kPrologue64, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     dm05::prologue::Smem<64>::kAllocBytes) != cudaSuccess ||
+                cudaFuncSetAttribute(kPrologue128, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     dm05::prologue::Smem<128>::kAllocBytes) != cudaSuccess)
+                return DM05_ERR_CUDA;
+            ds->prologue_attrs_set = true;
+        }
+        err = ds->err;
+    }
+    const int NT = small ? 64 : 128;
+    CUtensorMap tm_w, tm_x;
+    if (encode_2d(&tm_w, w, static_cast<uint64_t>(H), static_cast<uint64_t>(Hq + 2 * Hkv) * D, 64) != DM05_OK ||
+        encode_2d(&tm_x, x, static_cast<uint64_t>(H), static_cast<uint64_t>(T), static_cast<uint32_t>(NT)) != DM05_OK)
+        return DM05_ERR_CUDA;
+    dm05::prologue::Params pp;
+    pp.qw = static_cast<const __nv_bfloat16 *>(q_norm_w);
+    pp.kw = static_cast<const __nv_bfloat16 *>(k_norm_w);
+    pp.pos = positions;
+    pp.q = static_cast<__nv_bfloat16 *>(q);
+    pp.k = static_cast<__nv_bfloat16 *>(k);
+    pp.v = static_cast<__nv_bfloat16 *>(v);
+    pp.err = err;
+    pp.T = static_cast<int>(T);
+    pp.S = S;
+    pp.H = H;
+    pp.Hq = Hq;
+    pp.Hkv = Hkv;
+    pp.D = D;
+    pp.eps = eps;
+    pp.log2_theta = std::log2(theta);
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * (Hq + 2 * Hkv)), static_cast<unsigned>((T + NT - 1) / NT), 1);
+    cfg.blockDim = dim3(dm05::prologue::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = small ? dm05::prologue::Smem<64>::kAllocBytes : dm05::prologue::Smem<128>::kAllocBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute at[2];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    at[1].id = cudaLaunchAttributeClusterDimension;
+    at[1].val.clusterDim.x = 2;  // the two halves of a head
+    at[1].val.clusterDim.y = 1;
+    at[1].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 2;
+    const cudaError_t e = small ? cudaLaunchKernelEx(&cfg, kPrologue64, tm_w, tm_x, pp)
+                                : cudaLaunchKernelEx(&cfg, kPrologue128, tm_w, tm_x, pp);
+    return e == cudaSuccess ? DM05_OK : DM05_ERR_CUDA;
+}
+
+
+// ---------------------------------------------------------------------------
+// Multi-step calls: N suffix-attention calls over one prefix cache captured
+// once into a CUDA graph the library owns, then replayed with one launch.
+struct dm05_steps_s {
+    int dev = -1;
+    cudaGraphExec_t exec = nullptr;
+    void *workspace = nullptr;  // partial results of split calls, owned by the handle
+    int n_steps = 0;
+};
+
+int dm05_suffix_attn_steps_create(const dm05_step *steps, int n_steps, const void *k_prefix, const void *v_prefix,
+                                  const int32_t *prefix_valid_len, const uint8_t *prefix_mask, int B, int Hq,
+                                  int Hkv, int P, int S, int D, unsigned flags, dm05_steps_handle *handle)
+{
+    if (!handle) return DM05_ERR_NULL;
+    *handle = nullptr;
+    if (!steps || n_steps < 1 || n_steps > 4096) return n_steps < 1 || n_steps > 4096 ? DM05_ERR_SHAPE : DM05_ERR_NULL;
+    if ((flags & ~static_cast<unsigned>(DM05_FLAG_PREFIX_STATIC)) != 0) return DM05_ERR_SHAPE;
+    if (P > 0 && (!k_prefix || !v_prefix)) return DM05_ERR_NULL;
+    int rc = check_sizes(B, Hq, Hkv, P, S, D);
+    if (rc != DM05_OK) return rc;
+    if (P > 0 && (!aligned16(k_prefix) || !aligned16(v_prefix))) return DM05_ERR_ALIGN;
+    for (int t = 0; t < n_steps; ++t) {
+        const dm05_step &st = steps[t];
+        if (!st.q || !st.k_suffix || !st.v_suffix || !st.out) return DM05_ERR_NULL;
+        if (!aligned16(st.q) || !aligned16(st.k_suffix) || !aligned16(st.v_suffix) || !aligned16(st.out) ||
+            (st.lse != nullptr && (reinterpret_cast<uintptr_t>(st.lse) & 3u) != 0))
+            return DM05_ERR_ALIGN;
+    }
+    const int G = Hq / Hkv;
+    const int units = B * Hkv;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return DM05_ERR_CUDA;
+    uint32_t *err_word = nullptr;
+    Plan pl;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (get_encoder() != DM05_OK) return DM05_ERR_CUDA;
+        DeviceState *ds = nullptr;
+        rc = device_state(true, &ds, nullptr);
+        if (rc != DM05_OK) return rc;
+        pl = make_plan(B, Hq, Hkv, P, S, *ds);
+        err_word = ds->err;
+    }
+    dm05_steps_s *h = new dm05_steps_s();
+    h->dev = dev;
+    h->n_steps = n_steps;
+    const size_t ws_bytes = partial_bytes(units, pl, G);
+    if (ws_bytes > 0 && cudaMalloc(&h->workspace, ws_bytes) != cudaSuccess) {
+        delete h;
+        return DM05_ERR_CUDA;
+    }
+    // capture the calls, in order, on a private stream
+    cudaStream_t cs = nullptr;
+    cudaGraph_t graph = nullptr;
+    bool ok = cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal) == cudaSuccess;
+    int launch_rc = DM05_OK;
+    for (int t = 0; ok && t < n_steps && launch_rc == DM05_OK; ++t) {
+        const dm05_step &st = steps[t];
+        launch_rc = launch_attention(st.q, k_prefix, v_prefix, prefix_valid_len, prefix_mask, st.k_suffix,
+                                     st.v_suffix, st.out, st.lse, B, Hq, Hkv, P, S, D, pl, err_word, h->workspace,
+                                     cs, false, (flags & DM05_FLAG_PREFIX_STATIC) != 0);
+    }
+    if (cs != nullptr) {
+        cudaStreamCaptureStatus st = cudaStreamCaptureStatusNone;
+        if (cudaStreamIsCapturing(cs, &st) == cudaSuccess && st != cudaStreamCaptureStatusNone)
+            ok = cudaStreamEndCapture(cs, &graph) == cudaSuccess && ok;
+        cudaStreamDestroy(cs);
+    }
+    if (ok && launch_rc == DM05_OK && graph != nullptr)
+        ok = cudaGraphInstantiate(&h->exec, graph, 0) == cudaSuccess;
+    if (graph != nullptr) cudaGraphDestroy(graph);
+    if (!ok || launch_rc != DM05_OK || h->exec == nullptr) {
+        cudaGetLastError();
+        if (h->exec) cudaGraphExecDestroy(h->exec);
+        if (h->workspace) cudaFree(h->workspace);
+        delete h;
+        return launch_rc != DM05_OK ? launch_rc : DM05_ERR_CUDA;
+    }
+    *handle = h;
+    return DM05_OK;
+}
+
+int dm05_suffix_attn_steps_launch(dm05_steps_handle handle, cudaStream_t stream)
+{
+    if (!handle) return DM05_ERR_NULL;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return DM05_ERR_CUDA;
+    if (dev != handle->dev) return DM05_ERR_SHAPE;
+    return cudaGraphLaunch(handle->exec, stream) == cudaSuccess ? DM05_OK : DM05_ERR_CUDA;
+}
+
+int dm05_suffix_attn_steps_destroy(dm05_steps_handle handle)
+{
+    if (!handle) return DM05_OK;
+    int cur = 0;
+    const bool have_cur = cudaGetDevice(&cur) == cudaSuccess;
+    if (cudaSetDevice(handle->dev) != cudaSuccess) return DM05_ERR_CUDA;
+    // no launch of the graph may still be running: wait for the device
+    cudaDeviceSynchronize();
+    if (handle->exec) cudaGraphExecDestroy(handle->exec);
+    if (handle->workspace) cudaFree(handle->workspace);
+    delete handle;
+    if (have_cur) cudaSetDevice(cur);
     return DM05_OK;
 }
 

@@ -63,7 +63,8 @@ struct Smem {
     static constexpr int kRingBytes = kStages * kStageBytes;
     static constexpr int kYStride = NT + 4;              // fp32 per feature row (padded)
     static constexpr int kYBytes = 128 * kYStride * 4;
-    static_assert(kRingBytes >= kYBytes, "the epilogue tile reuses the ring");
+    // the epilogue tile and the per-group sums of squares reuse the ring
+    static_assert(kRingBytes >= kYBytes + kThreads * 4 * 4, "the epilogue tile reuses the ring");
     static constexpr int kBarOff = kRingBytes;
     static constexpr int kNumBars = 2 * kStages + 1;     // full[s], empty[s], mma done
     static constexpr int kSsOff = kBarOff + kNumBars * 8 + 8;   // own sums [NT], partner's sums [NT]
@@ -182,14 +183,32 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncthreads();
     if (!is_v) {
-        // per-token sum of squares over this CTA's 128 features, then the
-        // other half's through its shared memory (cluster of 2)
+        // per-token sum of squares over this CTA's 128 features: thread
+        // (token t, feature group g) sums 128 / kGroups features with four
+        // independent chains; the groups' sums meet in shared memory, and the
+        // token's total goes to the other half of the head too (cluster of 2)
+        constexpr int kGroups = kThreads / NT > 0 ? kThreads / NT : 1;
+        constexpr int kPer = 128 / kGroups;
+        float *part = reinterpret_cast<float *>(smem + L::kYBytes);  // [kGroups][NT], after the tile
+        for (int idx = threadIdx.x; idx < NT * kGroups; idx += kThreads) {
+            const int t = idx % NT, g = idx / NT;
+            float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+            const float *col = Y + (g * kPer) * L::kYStride + t;
+#pragma unroll 4
+            for (int f = 0; f < kPer; f += 4) {
+                const float y0 = col[(f + 0) * L::kYStride], y1 = col[(f + 1) * L::kYStride];
+                const float y2 = col[(f + 2) * L::kYStride], y3 = col[(f + 3) * L::kYStride];
+                a0 = fmaf(y0, y0, a0);
+                a1 = fmaf(y1, y1, a1);
+                a2 = fmaf(y2, y2, a2);
+                a3 = fmaf(y3, y3, a3);
+            }
+            part[g * NT + t] = (a0 + a1) + (a2 + a3);
+        }
+        __syncthreads();
         for (int t = threadIdx.x; t < NT; t += kThreads) {
             float acc = 0.0f;
-            for (int f = 0; f < 128; ++f) {
-                const float y = Y[f * L::kYStride + t];
-                acc = fmaf(y, y, acc);
-            }
+            for (int g = 0; g < kGroups; ++g) acc += part[g * NT + t];
             ss_own[t] = acc;
             ptx::st_dsmem_f32(ptx::mapa(ptx::smem_addr(ss_peer + t), static_cast<uint32_t>(half ^ 1)), acc);
         }
@@ -234,9 +253,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float inv_rms = rsqrtf(ms + p.eps);
             const float a = ya * inv_rms * wa, b = yb * inv_rms * wb;
             // the angle reduced to [-pi, pi] in double, then its sine and cosine
-            const double two_pi = 6.283185307179586;
+            const double two_pi = 6.283185307179586, inv_two_pi = 0.15915494309189535;
             double ang = static_cast<double>(p.pos[tok]) * inv_freq;
-            ang -= two_pi * rint(ang / two_pi);
+            ang = fma(-two_pi, rint(ang * inv_two_pi), ang);
             float sn, cs;
             sincosf(static_cast<float>(ang), &sn, &cs);
             oa = a * cs - b * sn;

@@ -301,6 +301,66 @@ def prologue_batched() -> PrologueInputs:
     return make_prologue_inputs(32, 50, 6003, pos0=starts, name="prologue_b32_s50_h1024")
 
 
+# --- post-attention block (output projection, Adarms, GEGLU, MLP down) -------
+
+@dataclass
+class PostAttnInputs:
+    """One post-attention block call of an action-expert layer."""
+    name: str
+    B: int
+    S: int
+    Hq: int
+    D: int
+    Hd: int
+    F: int
+    attn: torch.Tensor    # bf16 [B, Hq, S, D]: the suffix attention's output
+    h: torch.Tensor       # bf16 [B*S, Hd]: residual stream entering the layer
+    scale: torch.Tensor   # bf16 [B, Hd]: time modulation (per sample)
+    shift: torch.Tensor   # bf16 [B, Hd]
+    gate: torch.Tensor    # bf16 [B, Hd]
+    wo: torch.Tensor      # bf16 [Hd, Hq*D]
+    wgu: torch.Tensor     # bf16 [2F, Hd]: gate rows, then up rows
+    wd: torch.Tensor      # bf16 [Hd, F]
+
+    def to(self, device):
+        f = {k: getattr(self, k).to(device) for k in self.tensors()}
+        return PostAttnInputs(self.name, self.B, self.S, self.Hq, self.D, self.Hd, self.F, **f)
+
+    def tensors(self):
+        return dict(attn=self.attn, h=self.h, scale=self.scale, shift=self.shift, gate=self.gate, wo=self.wo,
+                    wgu=self.wgu, wd=self.wd)
+
+
+def make_post_inputs(B: int, S: int, seed: int, *, Hq: int = HQ, D: int = HEAD_DIM, Hd: int = 1024,
+                     F: int = 4096, name: str = "post") -> PostAttnInputs:
+    """Seeded post-attention inputs, drawn in this order as fp32 N(0,1) and
+    rounded once to bf16: attention output, residual, then the time
+    modulation scale and shift (x 0.1) and gate (x 0.5), then the weights
+    scaled by 1/sqrt(fan-in) so every projection is O(1)."""
+    gen = torch.Generator().manual_seed(int(seed))
+    bf = torch.bfloat16
+    attn = _randn(gen, (B, Hq, S, D)).to(bf)
+    h = _randn(gen, (B * S, Hd)).to(bf)
+    scale = (0.1 * _randn(gen, (B, Hd))).to(bf)
+    shift = (0.1 * _randn(gen, (B, Hd))).to(bf)
+    gate = (0.5 * _randn(gen, (B, Hd))).to(bf)
+    wo = (_randn(gen, (Hd, Hq * D)) / (Hq * D) ** 0.5).to(bf)
+    wgu = (_randn(gen, (2 * F, Hd)) / Hd ** 0.5).to(bf)
+    wd = (_randn(gen, (Hd, F)) / F ** 0.5).to(bf)
+    return PostAttnInputs(name, B, S, Hq, D, Hd, F, attn, h, scale, shift, gate, wo, wgu, wd)
+
+
+def post_base() -> PostAttnInputs:
+    """The base-model chunk's post-attention block: B=1, S=50, hidden 1024,
+    intermediate 4096, 8 heads of 256."""
+    return make_post_inputs(1, 50, 8001, name="post_b1_s50_h1024_f4096")
+
+
+def post_batched() -> PostAttnInputs:
+    """The batched workload's post-attention block: B=32, S=50."""
+    return make_post_inputs(32, 50, 8002, name="post_b32_s50_h1024_f4096")
+
+
 WORKLOADS = {
     "libero_tiny": libero_tiny,
     "base_chunk": base_chunk,

@@ -124,6 +124,48 @@ int dm05_suffix_attn_ex(const void *q, const void *k_prefix, const void *v_prefi
                         int B, int Hq, int Hkv, int P, int S, int D, unsigned flags,
                         cudaStream_t stream);
 
+/*
+ * Multi-step calls -- N suffix-attention calls over one prefix cache, run by
+ * one launch.  The pages' runtime captures the suffix-decode step of every
+ * prefix-length bucket into a CUDA graph at start-up and replays it per
+ * request, for the diffusion_steps denoising steps (page "TensorRT+Triton+
+ * FlexAttention: OpenDM VLA 快速推理加速栈深度剖析", section 3; page "DM05
+ * 推理指南", section 6: diffusion_steps defaults to 10 and is fixed after
+ * capture); every step reads the same, unchanged prefix cache.
+ *
+ * dm05_suffix_attn_steps_create captures n_steps calls, in order, each one
+ * exactly a dm05_suffix_attn_ex call with the shared prefix arguments and its
+ * own dm05_step, into a CUDA graph owned by the returned handle (with its own
+ * workspace for split partial results).  Consecutive calls are ordered as on
+ * one stream: call t + 1 reads its inputs only after call t has written its
+ * outputs, so a step's q may be an earlier step's out.  With
+ * DM05_FLAG_PREFIX_STATIC every call may request its prefix tiles while the
+ * previous call finishes (the prefix arguments must not be written by any
+ * step).  The pointers are baked into the graph: every launch reads and
+ * writes the same buffers.  Create outside any stream capture; the device
+ * current at creation must be current at every launch.
+ *
+ * dm05_suffix_attn_steps_launch enqueues all n_steps calls on `stream` with
+ * one graph launch (asynchronous).  Launches of one handle must not overlap
+ * on the GPU (they share its workspace).
+ *
+ * dm05_suffix_attn_steps_destroy waits for the device and frees the handle.
+ */
+typedef struct {
+    const void *q;        /* bf16 [B, Hq, S, D] */
+    const void *k_suffix; /* bf16 [B, Hkv, S, D] */
+    const void *v_suffix; /* bf16 [B, Hkv, S, D] */
+    void *out;            /* bf16 [B, Hq, S, D] */
+    float *lse;           /* fp32 [B, Hq, S] or NULL */
+} dm05_step;
+typedef struct dm05_steps_s *dm05_steps_handle;
+int dm05_suffix_attn_steps_create(const dm05_step *steps, int n_steps, const void *k_prefix, const void *v_prefix,
+                                  const int32_t *prefix_valid_len, const uint8_t *prefix_mask,
+                                  int B, int Hq, int Hkv, int P, int S, int D, unsigned flags,
+                                  dm05_steps_handle *handle);
+int dm05_suffix_attn_steps_launch(dm05_steps_handle handle, cudaStream_t stream);
+int dm05_suffix_attn_steps_destroy(dm05_steps_handle handle);
+
 /* Upper bound of the device workspace dm05_suffix_attn uses for these sizes:
  * the error word plus the partial results of the largest split (16 CTAs per
  * (sample, KV head)).  0 if the sizes are invalid.
@@ -213,6 +255,42 @@ int dm05_prefix_prefill_reserve(int B, int Hq, int Hkv, int P, int D, cudaStream
  * the number of blocks.  Any output pointer may be NULL. */
 int dm05_prefix_prefill_plan(int B, int Hq, int Hkv, int P, int D, int *splits_per_head, int *query_block,
                              int *row_blocks);
+
+/*
+ * dm05_suffix_qkv_prologue -- the step right before the suffix attention:
+ * QKV projection, QK-Norm and RoPE of the action tokens in one kernel,
+ * asynchronous on `stream`.
+ *
+ * The operation (page "TensorRT+Triton+FlexAttention: OpenDM VLA
+ * 快速推理加速栈深度剖析", section 2.2: "QKV projection + QK-Norm + RoPE done
+ * at once" is one of the fused steps; the action expert's shape table gives
+ * hidden 1024, head_dim 256, 8 / 4 heads).  For token t = b * S + i and head
+ * hd of w's row order (Hq query heads, then Hkv key heads, then Hkv value
+ * heads):
+ *   y        = w[hd*D : (hd+1)*D, :] x[t, :]                         (fp32 accumulation)
+ *   query / key heads: y' = y / sqrt(mean(y^2) + eps) * nw  (nw = q_norm_w or k_norm_w),
+ *                      then RoPE in the rotate-half pairing (d, d + D/2) by the
+ *                      angle positions[t] * theta^(-2d/D);
+ *   value heads: the projection y unchanged;
+ * written (rounded once to bf16) to q [B,Hq,S,D], k [B,Hkv,S,D], v [B,Hkv,S,D]:
+ * exactly the q / k_suffix / v_suffix layout dm05_suffix_attn reads.
+ *
+ *   x          bf16  [B*S, H]                  hidden states of the action tokens
+ *   w          bf16  [(Hq + 2*Hkv) * D, H]     QKV weight (row-major)
+ *   q_norm_w, k_norm_w  bf16 [D]               QK-Norm weights
+ *   positions  int32 [B*S]                     RoPE position of each token
+ *   q, k, v    bf16  outputs as above
+ *   eps > 0, theta > 1                          norm epsilon and RoPE base
+ *
+ * Supported: D == 256, H a multiple of 64.  x, w, q, k, v 16-byte aligned,
+ * the norm weights 2-byte and positions 4-byte aligned.  Errors, capture
+ * and determinism as dm05_suffix_attn (the first call on a device creates
+ * the error word and must run outside stream capture).
+ */
+int dm05_suffix_qkv_prologue(const void *x, const void *w, const void *q_norm_w, const void *k_norm_w,
+                             const int32_t *positions, void *q, void *k, void *v,
+                             int B, int S, int H, int Hq, int Hkv, int D, float eps, float theta,
+                             cudaStream_t stream);
 
 /*
  * dm05_suffix_attn_noalloc -- the same attention as dm05_suffix_attn, for

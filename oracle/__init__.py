@@ -75,6 +75,8 @@ class Oracle:
         lib.oracle_prefix_causal_attn.restype = i
         lib.oracle_qkv_prologue.argtypes = [p] * 5 + [ctypes.c_double] * 2 + [p] * 3 + [i] * 7
         lib.oracle_qkv_prologue.restype = i
+        lib.oracle_post_attention.argtypes = [p] * 8 + [ctypes.c_double, p] + [i] * 7
+        lib.oracle_post_attention.restype = i
         lib.oracle_max_threads.argtypes = []
         lib.oracle_max_threads.restype = i
         self.lib = lib
@@ -172,6 +174,23 @@ class Oracle:
             raise ValueError(f"oracle_qkv_prologue failed with status {rc}")
         return q, k, v
 
+    def post_attention(self, attn, h, scale, shift, gate, wo, wgu, wd, B, S, Hq, D, Hd, F, eps=1e-6,
+                       nthreads: int = 1):
+        """Output projection + residual, Adarms, GEGLU, MLP down and gated
+        residual.  attn [B,Hq,S,D], h [B*S,Hd], scale/shift/gate [B,Hd],
+        wo [Hd,Hq*D], wgu [2F,Hd], wd [Hd,F] (bf16 tensors or uint16 bit
+        patterns).  Returns float64 out [B*S, Hd]."""
+        arrs = [_bits(a) for a in (attn, h, scale, shift, gate, wo, wgu, wd)]
+        sizes = [B * Hq * S * D, B * S * Hd, B * Hd, B * Hd, B * Hd, Hd * Hq * D, 2 * F * Hd, Hd * F]
+        if any(a.size != n for a, n in zip(arrs, sizes)):
+            raise ValueError("an input's size does not match the dims")
+        out = np.zeros((B * S, Hd), dtype=np.float64)
+        rc = self.lib.oracle_post_attention(*[_ptr(a) for a in arrs], float(eps), _ptr(out), B, S, Hq, D, Hd, F,
+                                            int(nthreads))
+        if rc != 0:
+            raise ValueError(f"oracle_post_attention failed with status {rc}")
+        return out
+
     def inputs_call(self, inp, nthreads: int = 1, key_range=None, row_range=None):
         """Run on an object with the attributes of a SuffixAttnInputs."""
         return self.suffix_attn(inp.q, inp.k_prefix, inp.v_prefix, inp.prefix_valid_len,
@@ -201,6 +220,11 @@ def suffix_attn(*args, **kwargs):
 def merge_parts(o_parts, lse_parts):
     """Oracle.merge_parts on the default build."""
     return default().merge_parts(o_parts, lse_parts)
+
+
+def post_attention(*args, **kwargs):
+    """Oracle.post_attention on the default build."""
+    return default().post_attention(*args, **kwargs)
 
 
 def qkv_prologue(*args, **kwargs):

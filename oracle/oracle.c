@@ -33,6 +33,7 @@
  * logits, constant V, one visible key), invariants (masked rows ignored,
  * prefix permutation), and an arbitrary-precision brute force.
  */
+#define _GNU_SOURCE
 #include <math.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -415,6 +416,97 @@ int oracle_qkv_prologue(const uint16_t *x, const uint16_t *w, const uint16_t *qw
             }
             free(feat);
         }
+    }
+    return failed ? -7 : 0;
+}
+
+/*
+ * Post-attention block of an action-expert layer (page "TensorRT+Triton+
+ * FlexAttention: OpenDM VLA 快速推理加速栈深度剖析", section 2.2: after the
+ * three attention stages the suffix path chains the time modulation Adarms,
+ * the GEGLU gate-up and the MLP down; the action expert's shape table gives
+ * hidden 1024 and intermediate 4096).
+ *
+ * Readings where the page is silent (listed in the design notes), for token
+ * t = b * S + i of sample b:
+ *   a_t   = the attention output of the token, its Hq heads' D features
+ *           concatenated (head-major) into Hq * D values;
+ *   h1    = h_t + Wo a_t                          (output projection, residual)
+ *   u     = h1 / sqrt(mean(h1^2) + eps) * (1 + scale_b) + shift_b   (Adarms:
+ *           an RMS norm whose weight and bias come from the time embedding,
+ *           one (scale, shift, gate) triple per sample)
+ *   m     = gelu_tanh(Wg u) * (Wu u)              (GEGLU, gate and up rows of Wgu)
+ *   out_t = h1 + gate_b * (Wd m)                  (MLP down, gated residual)
+ * with gelu_tanh(z) = z / 2 * (1 + tanh(sqrt(2/pi) (z + 0.044715 z^3))).
+ *
+ * Layouts: attn [B,Hq,S,D] bf16 bits; h [B*S, Hd] bf16 bits; scale, shift,
+ * gate [B, Hd] bf16 bits; wo [Hd, Hq*D], wgu [2*F, Hd] (gate rows then up
+ * rows), wd [Hd, F] bf16 bits; out double [B*S, Hd].
+ * Returns 0, -1 for a NULL pointer, -2 for a bad shape, -7 for no memory.
+ */
+int oracle_post_attention(const uint16_t *attn, const uint16_t *h, const uint16_t *scale, const uint16_t *shift,
+                          const uint16_t *gate, const uint16_t *wo, const uint16_t *wgu, const uint16_t *wd,
+                          double eps, double *out, int B, int S, int Hq, int D, int Hd, int F, int nthreads)
+{
+    if (!attn || !h || !scale || !shift || !gate || !wo || !wgu || !wd || !out) return -1;
+    if (B < 1 || S < 1 || Hq < 1 || D < 1 || Hd < 1 || F < 1) return -2;
+    const long T = (long)B * S;
+    const int A = Hq * D;
+    int failed = 0;
+    if (nthreads < 1) nthreads = 1;
+
+#pragma omp parallel num_threads(nthreads) reduction(| : failed)
+    {
+        double *av = (double *)malloc(sizeof(double) * (size_t)A);
+        double *h1 = (double *)malloc(sizeof(double) * (size_t)Hd);
+        double *u = (double *)malloc(sizeof(double) * (size_t)Hd);
+        double *m = (double *)malloc(sizeof(double) * (size_t)F);
+        if (!av || !h1 || !u || !m) {
+            failed = 1;
+        } else {
+#pragma omp for schedule(static)
+            for (long t = 0; t < T; ++t) {
+                const int b = (int)(t / S), i = (int)(t % S);
+                /* the token's attention output, heads concatenated */
+                for (int hh = 0; hh < Hq; ++hh)
+                    for (int d = 0; d < D; ++d)
+                        av[hh * D + d] = bf16_bits_to_double(attn[(((size_t)b * Hq + hh) * S + i) * D + d]);
+                /* output projection and residual */
+                for (int o = 0; o < Hd; ++o) {
+                    double acc = 0.0;
+                    for (int c = 0; c < A; ++c) acc += bf16_bits_to_double(wo[(size_t)o * A + c]) * av[c];
+                    h1[o] = bf16_bits_to_double(h[(size_t)t * Hd + o]) + acc;
+                }
+                /* Adarms: RMS norm with the time modulation as weight and bias */
+                double ms = 0.0;
+                for (int o = 0; o < Hd; ++o) ms += h1[o] * h1[o];
+                const double inv_rms = 1.0 / sqrt(ms / (double)Hd + eps);
+                for (int o = 0; o < Hd; ++o)
+                    u[o] = h1[o] * inv_rms * (1.0 + bf16_bits_to_double(scale[(size_t)b * Hd + o])) +
+                           bf16_bits_to_double(shift[(size_t)b * Hd + o]);
+                /* GEGLU: gelu(gate projection) times up projection */
+                for (int f = 0; f < F; ++f) {
+                    double g = 0.0, up = 0.0;
+                    for (int c = 0; c < Hd; ++c) {
+                        g += bf16_bits_to_double(wgu[(size_t)f * Hd + c]) * u[c];
+                        up += bf16_bits_to_double(wgu[((size_t)F + f) * Hd + c]) * u[c];
+                    }
+                    const double z = g;
+                    const double gelu = 0.5 * z * (1.0 + tanh(sqrt(2.0 / M_PI) * (z + 0.044715 * z * z * z)));
+                    m[f] = gelu * up;
+                }
+                /* MLP down and the gated residual */
+                for (int o = 0; o < Hd; ++o) {
+                    double acc = 0.0;
+                    for (int f = 0; f < F; ++f) acc += bf16_bits_to_double(wd[(size_t)o * F + f]) * m[f];
+                    out[(size_t)t * Hd + o] = h1[o] + bf16_bits_to_double(gate[(size_t)b * Hd + o]) * acc;
+                }
+            }
+        }
+        free(av);
+        free(h1);
+        free(u);
+        free(m);
     }
     return failed ? -7 : 0;
 }

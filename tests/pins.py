@@ -539,10 +539,119 @@ def pin_prologue_decimal_bruteforce(orc):
                 assert abs(want - got) < 1e-13
 
 
+# --------------------------------------------------------------------------
+# Post-attention block (page "TensorRT+Triton+FlexAttention: OpenDM VLA
+# 快速推理加速栈深度剖析", section 2.2: Adarms time modulation, GEGLU gate-up,
+# MLP down).  Readings: output projection + residual, an RMS norm whose
+# weight (1 + scale) and bias (shift) come from the time embedding, GEGLU with
+# the tanh GELU, MLP down, and a residual gated by the time embedding's gate.
+
+def post_case(seed, B=2, S=3, Hq=2, D=8, Hd=16, F=24, wscale=0.3):
+    gen = torch.Generator().manual_seed(seed)
+    return dict(attn=bf16_rand(gen, (B, Hq, S, D)), h=bf16_rand(gen, (B * S, Hd)),
+                scale=bf16_rand(gen, (B, Hd), 0.2), shift=bf16_rand(gen, (B, Hd), 0.2),
+                gate=bf16_rand(gen, (B, Hd), 0.5), wo=bf16_rand(gen, (Hd, Hq * D), wscale),
+                wgu=bf16_rand(gen, (2 * F, Hd), wscale), wd=bf16_rand(gen, (Hd, F), wscale),
+                B=B, S=S, Hq=Hq, D=D, Hd=Hd, F=F)
+
+
+def run_post(orc, c, **kw):
+    return orc.post_attention(c["attn"], c["h"], c["scale"], c["shift"], c["gate"], c["wo"], c["wgu"], c["wd"],
+                              c["B"], c["S"], c["Hq"], c["D"], c["Hd"], c["F"], **kw)
+
+
+def post_library_reference(c, eps=1e-6):
+    """float64 library routines: linear, rms_norm, gelu (tanh approximation)."""
+    B, S, Hq, D, Hd, F = (c[k] for k in ("B", "S", "Hq", "D", "Hd", "F"))
+    f = lambda t: t.to(torch.float64)
+    a = f(c["attn"]).permute(0, 2, 1, 3).reshape(B * S, Hq * D)
+    h1 = f(c["h"]) + torch.nn.functional.linear(a, f(c["wo"]))
+    per_tok = lambda t: f(t).repeat_interleave(S, dim=0)               # [B*S, Hd]
+    u = torch.nn.functional.rms_norm(h1, (Hd,), eps=eps) * (1.0 + per_tok(c["scale"])) + per_tok(c["shift"])
+    gu = torch.nn.functional.linear(u, f(c["wgu"]))
+    m = torch.nn.functional.gelu(gu[:, :F], approximate="tanh") * gu[:, F:]
+    return (h1 + per_tok(c["gate"]) * torch.nn.functional.linear(m, f(c["wd"]))).numpy()
+
+
+def pin_post_library_float64(orc):
+    """Equal to float64 library linear, rms_norm and tanh-GELU on tiny shapes."""
+    for seed in (61, 62, 63):
+        c = post_case(seed)
+        np.testing.assert_allclose(run_post(orc, c), post_library_reference(c), rtol=0, atol=1e-11,
+                                   err_msg=f"post-attention block vs float64 library, seed {seed}")
+
+
+def pin_post_closed_forms(orc):
+    """A zero gate leaves out = h + Wo a (the residual after the projection);
+    scale = -1 and shift = 0 make the MLP input zero, so out = h + Wo a too;
+    zero projections leave out = h."""
+    c = post_case(64)
+    B, S, Hq, D = c["B"], c["S"], c["Hq"], c["D"]
+    a = c["attn"].to(torch.float64).permute(0, 2, 1, 3).reshape(B * S, Hq * D)
+    h1 = (c["h"].to(torch.float64) + a @ c["wo"].to(torch.float64).T).numpy()
+    np.testing.assert_allclose(run_post(orc, dict(c, gate=torch.zeros_like(c["gate"]))), h1, rtol=0, atol=1e-12)
+    c2 = dict(c, scale=torch.full_like(c["scale"], -1.0), shift=torch.zeros_like(c["shift"]))
+    np.testing.assert_allclose(run_post(orc, c2), h1, rtol=0, atol=1e-12)
+    c3 = dict(c, wo=torch.zeros_like(c["wo"]), wd=torch.zeros_like(c["wd"]))
+    np.testing.assert_allclose(run_post(orc, c3), c["h"].to(torch.float64).numpy(), rtol=0, atol=0)
+
+
+def pin_post_gelu_value(orc):
+    """One token, one intermediate feature: u_0 = 1 exactly (shift 1, scale
+    -1 so the norm term vanishes), gate row picks u_0, up row picks u_0, down
+    weight 1 and gate 1: out - h1 = gelu_tanh(1) * 1, the textbook value
+    0.5 * (1 + tanh(sqrt(2/pi) * 1.044715))."""
+    c = post_case(65, B=1, S=1, Hq=1, D=4, Hd=4, F=1)
+    c["scale"] = torch.full_like(c["scale"], -1.0)
+    c["shift"] = torch.tensor([[1.0, 0.0, 0.0, 0.0]], dtype=BF)
+    c["gate"] = torch.ones_like(c["gate"])
+    c["wgu"] = torch.tensor([[1.0, 0.0, 0.0, 0.0], [1.0, 0.0, 0.0, 0.0]], dtype=BF)
+    c["wd"] = torch.tensor([[1.0], [0.0], [0.0], [0.0]], dtype=BF)
+    out = run_post(orc, c)
+    h1 = (c["h"].to(torch.float64) + c["attn"].to(torch.float64).reshape(1, 4) @ c["wo"].to(torch.float64).T).numpy()
+    want = 0.5 * (1.0 + math.tanh(math.sqrt(2.0 / math.pi) * 1.044715))
+    assert abs((out - h1)[0, 0] - want) < 1e-15 and abs(want - 0.8411919906082768) < 1e-15
+    np.testing.assert_allclose((out - h1)[0, 1:], 0.0, atol=0)
+
+
+def pin_post_decimal_bruteforce(orc):
+    """60-digit decimal evaluation of the whole block on a tiny case (tanh from
+    the decimal exponential)."""
+    decimal.getcontext().prec = 60
+    c = post_case(66, B=1, S=2, Hq=1, D=4, Hd=4, F=3)
+    out = run_post(orc, c)
+    Dc = decimal.Decimal
+    A = _dec_bf16(c["attn"])
+    Hh = _dec_bf16(c["h"])
+    SC, SH, GT = _dec_bf16(c["scale"]), _dec_bf16(c["shift"]), _dec_bf16(c["gate"])
+    WO, WGU, WD = _dec_bf16(c["wo"]), _dec_bf16(c["wgu"]), _dec_bf16(c["wd"])
+    Hd, F = 4, 3
+    k = (Dc(2) / Dc("3.14159265358979323846264338327950288419716939937510")).sqrt()
+
+    def tanh(x):
+        e = (2 * x).exp()
+        return (e - 1) / (e + 1)
+
+    for t in range(2):
+        a = [A[t * 4 + d] for d in range(4)]          # attn [1, 1, S=2, D=4]: query t, feature d
+        h1 = [Hh[t * Hd + o] + sum(WO[o * 4 + cc] * a[cc] for cc in range(4)) for o in range(Hd)]
+        r = (sum(x * x for x in h1) / Hd + Dc("1e-6")).sqrt()
+        u = [h1[o] / r * (1 + SC[o]) + SH[o] for o in range(Hd)]
+        m = []
+        for f in range(F):
+            g = sum(WGU[f * Hd + cc] * u[cc] for cc in range(Hd))
+            up = sum(WGU[(F + f) * Hd + cc] * u[cc] for cc in range(Hd))
+            m.append(g / 2 * (1 + tanh(k * (g + Dc("0.044715") * g * g * g))) * up)
+        for o in range(Hd):
+            want = h1[o] + GT[o] * sum(WD[o * F + f] * m[f] for f in range(F))
+            assert abs(float(want) - out[t, o]) < 1e-13
+
+
 ALL_PINS = [pin_sdpa_float64, pin_uniform_logits, pin_constant_v_gqa, pin_masked_rows_ignored,
             pin_single_suffix_key, pin_dominant_key, pin_prefix_permutation, pin_split_merge,
             pin_decimal_bruteforce, pin_valid_len_clamp_and_boundary,
             pin_prefill_sdpa_float64, pin_prefill_first_row_and_uniform, pin_prefill_future_keys_ignored,
             pin_prefill_decimal_bruteforce,
             pin_prologue_library_float64, pin_prologue_position_zero_and_norm, pin_prologue_relative_position,
-            pin_prologue_decimal_bruteforce]
+            pin_prologue_decimal_bruteforce,
+            pin_post_library_float64, pin_post_closed_forms, pin_post_gelu_value, pin_post_decimal_bruteforce]

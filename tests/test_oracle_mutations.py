@@ -61,6 +61,21 @@ MUTATIONS = {
                                              "for (int d = 0; d < D; ++d) dst[d] = feat[d] * bf16_bits_to_double(kw[d]);\n                    continue;"),
     "prologue_weight_row_of_next_head": ("const uint16_t *w_row = w + ((size_t)hd * D + d) * (size_t)H;",
                                          "const uint16_t *w_row = w + ((size_t)((hd + 1) % n_heads) * D + d) * (size_t)H;"),
+    # post-attention block
+    "post_residual_dropped": ("h1[o] = bf16_bits_to_double(h[(size_t)t * Hd + o]) + acc;", "h1[o] = acc;"),
+    "post_scale_without_one": ("* (1.0 + bf16_bits_to_double(scale[(size_t)b * Hd + o])) +",
+                               "* (bf16_bits_to_double(scale[(size_t)b * Hd + o])) +"),
+    "post_shift_dropped": ("+\n                           bf16_bits_to_double(shift[(size_t)b * Hd + o]);",
+                           "+\n                           0.0 * bf16_bits_to_double(shift[(size_t)b * Hd + o]);"),
+    "post_gelu_cube_dropped": ("(z + 0.044715 * z * z * z)", "(z)"),
+    "post_gate_ignored": ("out[(size_t)t * Hd + o] = h1[o] + bf16_bits_to_double(gate[(size_t)b * Hd + o]) * acc;",
+                          "out[(size_t)t * Hd + o] = h1[o] + acc;"),
+    "post_up_rows_are_gate_rows": ("up += bf16_bits_to_double(wgu[((size_t)F + f) * Hd + c]) * u[c];",
+                                   "up += bf16_bits_to_double(wgu[(size_t)f * Hd + c]) * u[c];"),
+    "post_norm_without_mean": ("const double inv_rms = 1.0 / sqrt(ms / (double)Hd + eps);",
+                               "const double inv_rms = 1.0 / sqrt(ms + eps);"),
+    "post_heads_token_major": ("av[hh * D + d] = bf16_bits_to_double(attn[(((size_t)b * Hq + hh) * S + i) * D + d]);",
+                               "av[hh * D + d] = bf16_bits_to_double(attn[(((size_t)b * S + i) * Hq + hh) * D + d]);"),
 }
 
 

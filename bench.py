@@ -458,10 +458,13 @@ def history_steps(calls, K, dev, stream, bd):
     ptr = lambda x: None if x is None else x.data_ptr()
     steps = [(ptr(d.q), ptr(d.k_suffix), ptr(d.v_suffix), ptr(o), ptr(l)) for d, o, l in zip(ds, outs, lses)]
     B, Hq, Hkv, P, S, D = d0.B, d0.Hq, d0.Hkv, d0.P, d0.S, d0.D
-    rc, h = bd.dm05_suffix_attn_steps_create(steps, ptr(d0.k_prefix), ptr(d0.v_prefix), ptr(d0.prefix_valid_len),
-                                             None, B, Hq, Hkv, P, S, D, bd.DM05_FLAG_PREFIX_STATIC)
-    if rc != 0:
-        raise bd.Dm05Error(rc, "dm05_suffix_attn_steps_create")
+    handles = {}
+    for name, flags in (("steps_one_launch", 0), ("steps_one_launch_static_prefix", bd.DM05_FLAG_PREFIX_STATIC)):
+        rc, h = bd.dm05_suffix_attn_steps_create(steps, ptr(d0.k_prefix), ptr(d0.v_prefix),
+                                                 ptr(d0.prefix_valid_len), None, B, Hq, Hkv, P, S, D, flags)
+        if rc != 0:
+            raise bd.Dm05Error(rc, "dm05_suffix_attn_steps_create")
+        handles[name] = h
     loops = max(20, K // 10)
 
     def timed(fn, n):
@@ -477,9 +480,11 @@ def history_steps(calls, K, dev, stream, bd):
         stream.synchronize()
         return e0.elapsed_time(e1) * 1e3 / n
 
-    def one_launch():
-        if bd.dm05_suffix_attn_steps_launch(h, stream.cuda_stream) != 0:
-            raise RuntimeError("dm05_suffix_attn_steps_launch failed")
+    def one_launch(h):
+        def go():
+            if bd.dm05_suffix_attn_steps_launch(h, stream.cuda_stream) != 0:
+                raise RuntimeError("dm05_suffix_attn_steps_launch failed")
+        return go
 
     def separate():
         for d, o, l in zip(ds, outs, lses):
@@ -488,16 +493,69 @@ def history_steps(calls, K, dev, stream, bd):
                                    stream.cuda_stream) != 0:
                 raise RuntimeError("dm05_suffix_attn failed")
 
+    n = len(calls)
+    res = {}
     try:
-        t_steps = timed(one_launch, loops)
+        for name, h in handles.items():
+            t = timed(one_launch(h), loops)
+            res[name] = {"per_10_steps": t * 10 / n, "us_per_call": t / n, "loops": loops,
+                         "api": "dm05_suffix_attn_steps_launch (the 10 calls captured once)"
+                                + (", DM05_FLAG_PREFIX_STATIC" if "static" in name else "")}
         t_sep = timed(separate, loops)
     finally:
-        bd.dm05_suffix_attn_steps_destroy(h)
-    n = len(calls)
-    return {"steps_one_launch": {"per_10_steps": t_steps * 10 / n, "us_per_call": t_steps / n, "loops": loops,
-                                 "api": "dm05_suffix_attn_steps_launch (captured once, static-prefix flag)"},
-            "separate_calls": {"per_10_steps": t_sep * 10 / n, "us_per_call": t_sep / n, "loops": loops,
-                               "api": "10 x dm05_suffix_attn, no graph"}}
+        for h in handles.values():
+            bd.dm05_suffix_attn_steps_destroy(h)
+    res["separate_calls"] = {"per_10_steps": t_sep * 10 / n, "us_per_call": t_sep / n, "loops": loops,
+                             "api": "10 x dm05_suffix_attn, no graph"}
+    return res
+
+
+def time_post(inp, K, W, dev, stream, bd, l2):
+    """Device time per dm05_post_attention call (five launches), the same
+    rotating-copy and graph protocol as the other workloads."""
+    import torch
+    one = sum(t.numel() * t.element_size() for t in inp.tensors().values())
+    copies = max(2, int(2 * l2 // max(1, one)) + 2)
+    d0 = inp.to(dev)
+    sets = [dict({k: v.clone() for k, v in d0.tensors().items()},
+                 out=torch.empty((inp.B * inp.S, inp.Hd), dtype=torch.bfloat16, device=dev)) for _ in range(copies)]
+    rc = bd.dm05_post_attention_reserve(inp.B, inp.S, inp.Hq, inp.D, inp.Hd, inp.F, stream.cuda_stream)
+    if rc != 0:
+        raise bd.Dm05Error(rc, "dm05_post_attention_reserve")
+
+    def call(t):
+        rc = bd.dm05_post_attention(t["attn"].data_ptr(), t["h"].data_ptr(), t["scale"].data_ptr(),
+                                    t["shift"].data_ptr(), t["gate"].data_ptr(), t["wo"].data_ptr(),
+                                    t["wgu"].data_ptr(), t["wd"].data_ptr(), t["out"].data_ptr(), inp.B, inp.S,
+                                    inp.Hq, inp.D, inp.Hd, inp.F, 1e-6, stream.cuda_stream)
+        if rc != 0:
+            raise bd.Dm05Error(rc, "dm05_post_attention")
+
+    with torch.cuda.stream(stream):
+        for i in range(max(3, W)):
+            call(sets[i % copies])
+    stream.synchronize()
+    n = max(1, min(K, 400))
+    graphs, done = [], 0
+    while done < n:
+        m = min(200, n - done)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(m):
+                call(sets[(done + i) % copies])
+        graphs.append(g)
+        done += m
+    warm_graphs(graphs, stream)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for g in graphs:
+            g.replay()
+        e1.record(stream)
+    stream.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / n
+    del graphs, sets
+    return us, copies
 
 
 def measured_tensor_peak():
@@ -558,6 +616,20 @@ def workload_table(args, dev, stream, bd, l2, peak):
                          "roofline": {"bound": "tensor", "peak": tpeak, "peak_source": tkind, "frac": tf / tpeak},
                          "plan": {"splits_per_head": sp, "query_block": qb, "row_blocks": rb}, "calls": K,
                          "l2": f"{copies} rotating copies"}
+    # the post-attention block (output projection, Adarms, GEGLU, MLP down):
+    # weight-bound at B = 1, tensor-bound at B = 32
+    for inp in (gen.post_base(), gen.post_batched()):
+        us, copies = time_post(inp, K, W, dev, stream, bd, l2)
+        T = inp.B * inp.S
+        wbytes = 2 * (inp.Hd * inp.Hq * inp.D + 2 * inp.F * inp.Hd + inp.Hd * inp.F)
+        nbytes = wbytes + 2 * (T * inp.Hq * inp.D + 2 * T * inp.Hd) + 6 * inp.B * inp.Hd
+        fl = 2 * T * (inp.Hd * inp.Hq * inp.D + 2 * inp.F * inp.Hd + inp.Hd * inp.F)
+        t_hbm, t_tc = nbytes / (peak * 1e9), fl / (tpeak * 1e12)
+        bound = "hbm" if t_hbm >= t_tc else "tensor"
+        out[inp.name] = {"us_per_call": us, "algorithmic_bytes": nbytes, "algorithmic_flops": fl,
+                         "achieved_gbs": nbytes / (us * 1e-6) / 1e9, "achieved_tflops": fl / (us * 1e-6) / 1e12,
+                         "roofline": {"bound": bound, "frac": (t_hbm if bound == "hbm" else t_tc) / (us * 1e-6)},
+                         "calls": K, "l2": f"{copies} rotating copies", "launches_per_call": 5}
     # the suffix prologue (QKV projection + QK-Norm + RoPE): the weight stream
     # bounds it at B = 1, the tensor cores at B = 32
     for inp in (gen.prologue_base(), gen.prologue_batched()):

@@ -32,7 +32,8 @@ EXPORTS = ("dm05_suffix_attn", "dm05_suffix_attn_ex", "dm05_suffix_attn_workspac
            "dm05_status_string", "dm05_release", "dm05_suffix_attn_noalloc", "dm05_suffix_attn_host",
            "dm05_suffix_attn_host_copy_bytes", "dm05_selftest_wait_timeout", "dm05_prefix_prefill_attn",
            "dm05_prefix_prefill_reserve", "dm05_prefix_prefill_plan", "dm05_suffix_qkv_prologue",
-           "dm05_suffix_attn_steps_create", "dm05_suffix_attn_steps_launch", "dm05_suffix_attn_steps_destroy")
+           "dm05_suffix_attn_steps_create", "dm05_suffix_attn_steps_launch", "dm05_suffix_attn_steps_destroy",
+           "dm05_post_attention", "dm05_post_attention_reserve")
 
 _lock = threading.Lock()
 _lib = None
@@ -104,6 +105,10 @@ def lib() -> ctypes.CDLL:
             L.dm05_suffix_attn_steps_launch.restype = i
             L.dm05_suffix_attn_steps_destroy.argtypes = [p]
             L.dm05_suffix_attn_steps_destroy.restype = i
+            L.dm05_post_attention.argtypes = [p] * 9 + [i] * 6 + [ctypes.c_float, p]
+            L.dm05_post_attention.restype = i
+            L.dm05_post_attention_reserve.argtypes = [i] * 6 + [p]
+            L.dm05_post_attention_reserve.restype = i
             _lib = L
     return _lib
 
@@ -187,6 +192,40 @@ def dm05_suffix_attn_steps_launch(handle, stream) -> int:
 
 def dm05_suffix_attn_steps_destroy(handle) -> int:
     return lib().dm05_suffix_attn_steps_destroy(handle)
+
+
+def dm05_post_attention(attn, h, scale, shift, gate, wo, wgu, wd, out, B, S, Hq, D, Hd, F, eps, stream) -> int:
+    """Output projection + residual, Adarms, GEGLU, MLP down + gated residual."""
+    return lib().dm05_post_attention(attn, h, scale, shift, gate, wo, wgu, wd, out, B, S, Hq, D, Hd, F,
+                                     float(eps), stream)
+
+
+def dm05_post_attention_reserve(B, S, Hq, D, Hd, F, stream) -> int:
+    return lib().dm05_post_attention_reserve(B, S, Hq, D, Hd, F, stream)
+
+
+def post_attention(attn, h, scale, shift, gate, wo, wgu, wd, eps=1e-6, out=None, stream=None):
+    """The post-attention block on CUDA torch tensors; returns out [B*S, Hd] bf16."""
+    import torch
+    B, Hq, S, D = attn.shape
+    Hd = h.shape[1]
+    F = wgu.shape[0] // 2
+    for name, t, shape in (("attn", attn, (B, Hq, S, D)), ("h", h, (B * S, Hd)), ("scale", scale, (B, Hd)),
+                           ("shift", shift, (B, Hd)), ("gate", gate, (B, Hd)), ("wo", wo, (Hd, Hq * D)),
+                           ("wgu", wgu, (2 * F, Hd)), ("wd", wd, (Hd, F))):
+        if (not t.is_cuda or t.dtype != torch.bfloat16 or tuple(t.shape) != shape or not t.is_contiguous()
+                or t.device != attn.device):
+            raise ValueError(f"{name} must be a contiguous CUDA bfloat16 tensor {list(shape)} on {attn.device}")
+    if out is None:
+        out = torch.empty((B * S, Hd), dtype=torch.bfloat16, device=attn.device)
+    if (not out.is_cuda or out.dtype != torch.bfloat16 or tuple(out.shape) != (B * S, Hd) or not out.is_contiguous()):
+        raise ValueError(f"out must be a contiguous CUDA bfloat16 tensor {[B * S, Hd]}")
+    rc = dm05_post_attention(attn.data_ptr(), h.data_ptr(), scale.data_ptr(), shift.data_ptr(), gate.data_ptr(),
+                             wo.data_ptr(), wgu.data_ptr(), wd.data_ptr(), out.data_ptr(), B, S, Hq, D, Hd, F, eps,
+                             _stream_handle(stream))
+    if rc != DM05_OK:
+        raise Dm05Error(rc, "dm05_post_attention")
+    return out
 
 
 def dm05_suffix_attn_workspace_bytes(B, Hq, Hkv, P, S, D) -> int:

@@ -8,6 +8,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstdlib>
@@ -16,6 +17,7 @@
 #include <thread>
 #include <vector>
 
+#include "post_attn_kernels.cuh"
 #include "qkv_prologue_kernel.cuh"
 #include "suffix_attn_kernel.cuh"
 
@@ -33,6 +35,7 @@ struct DeviceState {
     uint32_t *err = nullptr;   // device error word
     bool attrs_set = false;
     bool prologue_attrs_set = false;
+    bool post_attrs_set = false;
     int num_sms = 0;
     int max_cluster = 0;       // largest cluster size (<= 16) that can be resident
     int active[17] = {};       // active[c]: clusters of c CTAs the device holds at once (0: not allowed)
@@ -291,6 +294,45 @@ int stream_workspace(cudaStream_t stream, size_t need, void **out)
         if (w->base != nullptr) {
             // cudaFree waits for the device, so no kernel still uses the old buffer
             cudaFree(w->base);
+            w->base = nullptr;
+            w->bytes = 0;
+        }
+        void *p = nullptr;
+        if (cudaMalloc(&p, need) != cudaSuccess) return DM05_ERR_CUDA;
+        w->base = p;
+        w->bytes = need;
+    }
+    *out = w->base;
+    return DM05_OK;
+}
+
+// A buffer of at least `need` bytes keyed by (current device, stream[, thread
+// for cudaStreamPerThread]) in `list`; grows only outside stream capture (a
+// smaller existing buffer during capture gives DM05_ERR_WORKSPACE).  Caller
+// holds g_mu.
+int keyed_buffer(std::vector<StreamWorkspace> &list, cudaStream_t stream, size_t need, void **out)
+{
+    *out = nullptr;
+    if (need == 0) return DM05_OK;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return DM05_ERR_CUDA;
+    const std::thread::id owner = stream_owner(stream);
+    StreamWorkspace *w = nullptr;
+    for (auto &e : list)
+        if (e.dev == dev && e.stream == stream && e.thread == owner) w = &e;
+    if (w == nullptr) {
+        list.push_back(StreamWorkspace{});
+        w = &list.back();
+        w->dev = dev;
+        w->stream = stream;
+        w->thread = owner;
+    }
+    if (w->bytes < need) {
+        cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+        if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) return DM05_ERR_CUDA;
+        if (cs != cudaStreamCaptureStatusNone) return DM05_ERR_WORKSPACE;
+        if (w->base != nullptr) {
+            cudaFree(w->base);  // waits for the device: no earlier call still uses it
             w->base = nullptr;
             w->bytes = 0;
         }
@@ -1161,6 +1203,8 @@ int dm05_get_error_word(cudaStream_t stream, uint32_t *host_word)
     return DM05_OK;
 }
 
+void release_post_buffers();
+
 void dm05_release(void)
 {
     std::lock_guard<std::mutex> lk(g_mu);
@@ -1180,7 +1224,273 @@ void dm05_release(void)
         if (w.base != nullptr && cudaSetDevice(w.dev) == cudaSuccess) cudaFree(w.base);
     }
     g_stage.clear();
+    release_post_buffers();
     if (have_cur) cudaSetDevice(cur);
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Post-attention block: output projection + residual, Adarms, GEGLU, MLP
+// down + gated residual (five launches on the caller's stream).
+namespace {
+
+struct PostPlan {
+    int NT = 64, tiles = 1, ks_o = 1, ks_d = 1;
+    size_t off_part_o = 0, off_h1 = 0, off_u = 0, off_m = 0, off_part_d = 0, total = 0;
+};
+
+// the largest divisor of `chunks` that is at most `want` (at least 1)
+int split_count(int chunks, int want)
+{
+    int best = 1;
+    for (int k = 1; k <= chunks && k <= want; ++k)
+        if (chunks % k == 0) best = k;
+    return best;
+}
+
+PostPlan post_plan(int B, int S, int Hq, int D, int Hd, int F, int num_sms)
+{
+    PostPlan pl;
+    pl.NT = S <= 64 ? 64 : 128;
+    pl.tiles = (S + pl.NT - 1) / pl.NT;
+    const long long T = static_cast<long long>(B) * S;
+    const long long tok_tiles = static_cast<long long>(B) * pl.tiles;
+    const long long row_tiles = Hd / 128;
+    // spread the two long-K projections over about one wave of CTAs
+    const long long want = std::max<long long>(1, num_sms / std::max<long long>(1, row_tiles * tok_tiles));
+    pl.ks_o = split_count(Hq * D / 64, static_cast<int>(std::min<long long>(want, 64)));
+    pl.ks_d = split_count(F / 64, static_cast<int>(std::min<long long>(want, 64)));
+    auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+    size_t o = 0;
+    pl.off_part_o = o; o += up(static_cast<size_t>(pl.ks_o) * T * Hd * 4);
+    pl.off_h1 = o;     o += up(static_cast<size_t>(T) * Hd * 4);
+    pl.off_u = o;      o += up(static_cast<size_t>(T) * Hd * 2);
+    pl.off_m = o;      o += up(static_cast<size_t>(T) * F * 2);
+    pl.off_part_d = o; o += up(static_cast<size_t>(pl.ks_d) * T * Hd * 4);
+    pl.total = o;
+    return pl;
+}
+
+std::vector<StreamWorkspace> g_post_ws;  // per (device, stream[, thread]) buffers of the post-attention block
+
+// activation viewed as 4-D [B][K / inner][S][inner]; boxes of 64 x NT x 1 x 1
+int encode_act(CUtensorMap *map, const void *base, int B, int S, int K, int inner, int NT)
+{
+    cuuint64_t dims[4] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(S),
+                          static_cast<cuuint64_t>(K / inner), static_cast<cuuint64_t>(B)};
+    cuuint64_t strides[3] = {static_cast<cuuint64_t>(inner) * 2, static_cast<cuuint64_t>(S) * inner * 2,
+                             static_cast<cuuint64_t>(K) * S * 2};
+    // [B][S][K] (inner == K): the rows of one sample are K apart, not inner
+    if (inner == K) strides[1] = static_cast<cuuint64_t>(S) * K * 2;
+    cuuint32_t box[4] = {64, static_cast<cuuint32_t>(NT), 1, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? DM05_OK : DM05_ERR_CUDA;
+}
+
+int post_check(const void *attn, const void *h, const void *scale, const void *shift, const void *gate,
+               const void *wo, const void *wgu, const void *wd, const void *out, int B, int S, int Hq, int D, int Hd,
+               int F)
+{
+    if (!attn || !h || !scale || !shift || !gate || !wo || !wgu || !wd || !out) return DM05_ERR_NULL;
+    if (B < 1 || S < 1 || Hq < 1 || D < 1 || Hd < 1 || F < 1) return DM05_ERR_SHAPE;
+    if (static_cast<long long>(B) * S > (1LL << 20) || static_cast<long long>(Hq) * D > (1 << 20) || Hd > (1 << 16) ||
+        F > (1 << 20))
+        return DM05_ERR_SHAPE;
+    if (D % 64 != 0 || Hd % 128 != 0 || F % 64 != 0) return DM05_ERR_UNSUPPORTED;
+    for (const void *ptr : {attn, h, wo, wgu, wd, out})
+        if (!aligned16(ptr)) return DM05_ERR_ALIGN;
+    for (const void *ptr : {scale, shift, gate})
+        if (reinterpret_cast<uintptr_t>(ptr) & 1u) return DM05_ERR_ALIGN;
+    return DM05_OK;
+}
+
+auto *kGemmPartial64 = &dm05::post::gemm_kernel<64, dm05::post::kPartial>;
+auto *kGemmPartial128 = &dm05::post::gemm_kernel<128, dm05::post::kPartial>;
+auto *kGemmGeglu64 = &dm05::post::gemm_kernel<64, dm05::post::kGeglu>;
+auto *kGemmGeglu128 = &dm05::post::gemm_kernel<128, dm05::post::kGeglu>;
+
+int launch_gemm(bool geglu, int NT, dim3 grid, const CUtensorMap &tw, const CUtensorMap &tx,
+                const dm05::post::GemmParams &gp, cudaStream_t stream)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(dm05::post::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = NT == 64 ? dm05::post::GemmSmem<64>::kAllocBytes : dm05::post::GemmSmem<128>::kAllocBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    cudaError_t e;
+    if (geglu)
+        e = NT == 64 ? cudaLaunchKernelEx(&cfg, kGemmGeglu64, tw, tx, gp) : cudaLaunchKernelEx(&cfg, kGemmGeglu128, tw, tx, gp);
+    else
+        e = NT == 64 ? cudaLaunchKernelEx(&cfg, kGemmPartial64, tw, tx, gp)
+                     : cudaLaunchKernelEx(&cfg, kGemmPartial128, tw, tx, gp);
+    return e == cudaSuccess ? DM05_OK : DM05_ERR_CUDA;
+}
+
+template <class K>
+int launch_rows(K kernel, int T, const dm05::post::RowParams &rp, cudaStream_t stream)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(T), 1, 1);
+    cfg.blockDim = dim3(256, 1, 1);
+    cfg.stream = stream;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, rp) == cudaSuccess ? DM05_OK : DM05_ERR_CUDA;
+}
+
+// Device state with the post-attention kernels' attributes set (once per
+// device) and the error word; outside capture only.  Caller holds g_mu.
+int post_device_state(cudaStream_t stream, DeviceState **out)
+{
+    DeviceState *ds = nullptr;
+    int rc = device_state(false, &ds);
+    if (rc != DM05_OK) return rc;
+    if (ds->err == nullptr || !ds->post_attrs_set) {
+        cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+        if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) return DM05_ERR_CUDA;
+        if (cs != cudaStreamCaptureStatusNone) return DM05_ERR_WORKSPACE;
+        rc = device_state(true, &ds, stream);
+        if (rc != DM05_OK) return rc;
+        const int s64 = dm05::post::GemmSmem<64>::kAllocBytes, s128 = dm05::post::GemmSmem<128>::kAllocBytes;
+        if (cudaFuncSetAttribute(kGemmPartial64, cudaFuncAttributeMaxDynamicSharedMemorySize, s64) != cudaSuccess ||
+            cudaFuncSetAttribute(kGemmPartial128, cudaFuncAttributeMaxDynamicSharedMemorySize, s128) != cudaSuccess ||
+            cudaFuncSetAttribute(kGemmGeglu64, cudaFuncAttributeMaxDynamicSharedMemorySize, s64) != cudaSuccess ||
+            cudaFuncSetAttribute(kGemmGeglu128, cudaFuncAttributeMaxDynamicSharedMemorySize, s128) != cudaSuccess)
+            return DM05_ERR_CUDA;
+        ds->post_attrs_set = true;
+    }
+    *out = ds;
+    return DM05_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int dm05_post_attention_reserve(int B, int S, int Hq, int D, int Hd, int F, cudaStream_t stream)
+{
+    if (B < 1 || S < 1 || Hq < 1 || D < 1 || Hd < 1 || F < 1) return DM05_ERR_SHAPE;
+    if (D % 64 != 0 || Hd % 128 != 0 || F % 64 != 0) return DM05_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (get_encoder() != DM05_OK) return DM05_ERR_CUDA;
+    DeviceState *ds = nullptr;
+    int rc = post_device_state(stream, &ds);
+    if (rc != DM05_OK) return rc;
+    const PostPlan pl = post_plan(B, S, Hq, D, Hd, F, ds->num_sms);
+    void *ws = nullptr;
+    return keyed_buffer(g_post_ws, stream, pl.total, &ws);
+}
+
+int dm05_post_attention(const void *attn, const void *h, const void *scale, const void *shift, const void *gate,
+                        const void *wo, const void *wgu, const void *wd, void *out, int B, int S, int Hq, int D,
+                        int Hd, int F, float eps, cudaStream_t stream)
+{
+    int rc = post_check(attn, h, scale, shift, gate, wo, wgu, wd, out, B, S, Hq, D, Hd, F);
+    if (rc != DM05_OK) return rc;
+    if (!(eps > 0.0f)) return DM05_ERR_SHAPE;
+    const int T = B * S;
+    PostPlan pl;
+    uint32_t *err = nullptr;
+    uint8_t *ws = nullptr;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (get_encoder() != DM05_OK) return DM05_ERR_CUDA;
+        DeviceState *ds = nullptr;
+        rc = post_device_state(stream, &ds);
+        if (rc != DM05_OK) return rc;
+        pl = post_plan(B, S, Hq, D, Hd, F, ds->num_sms);
+        err = ds->err;
+        void *p = nullptr;
+        rc = keyed_buffer(g_post_ws, stream, pl.total, &p);
+        if (rc != DM05_OK) return rc;
+        ws = static_cast<uint8_t *>(p);
+    }
+    float *part_o = reinterpret_cast<float *>(ws + pl.off_part_o);
+    float *h1 = reinterpret_cast<float *>(ws + pl.off_h1);
+    __nv_bfloat16 *u = reinterpret_cast<__nv_bfloat16 *>(ws + pl.off_u);
+    __nv_bfloat16 *m = reinterpret_cast<__nv_bfloat16 *>(ws + pl.off_m);
+    float *part_d = reinterpret_cast<float *>(ws + pl.off_part_d);
+
+    CUtensorMap tw_o, tw_gu, tw_d, tx_a, tx_u, tx_m;
+    const int A = Hq * D;
+    if (encode_2d(&tw_o, wo, static_cast<uint64_t>(A), static_cast<uint64_t>(Hd), 64) != DM05_OK ||
+        encode_2d(&tw_gu, wgu, static_cast<uint64_t>(Hd), static_cast<uint64_t>(2) * F, 64) != DM05_OK ||
+        encode_2d(&tw_d, wd, static_cast<uint64_t>(F), static_cast<uint64_t>(Hd), 64) != DM05_OK ||
+        encode_act(&tx_a, attn, B, S, A, D, pl.NT) != DM05_OK || encode_act(&tx_u, u, B, S, Hd, Hd, pl.NT) != DM05_OK ||
+        encode_act(&tx_m, m, B, S, F, F, pl.NT) != DM05_OK)
+        return DM05_ERR_CUDA;
+
+    dm05::post::GemmParams gp{};
+    gp.err = err;
+    gp.T = T;
+    gp.S = S;
+    gp.tiles_per_sample = pl.tiles;
+    const unsigned tok_tiles = static_cast<unsigned>(B * pl.tiles);
+    // 1. output projection: partial sums over ks_o K ranges
+    gp.part = part_o;
+    gp.N_rows = Hd;
+    gp.xk_inner = D;
+    gp.chunks_per_split = A / 64 / pl.ks_o;
+    rc = launch_gemm(false, pl.NT, dim3(Hd / 128, tok_tiles, pl.ks_o), tw_o, tx_a, gp, stream);
+    if (rc != DM05_OK) return rc;
+    // 2. residual, Adarms
+    dm05::post::RowParams rp{};
+    rp.part = part_o;
+    rp.splits = pl.ks_o;
+    rp.h = static_cast<const __nv_bfloat16 *>(h);
+    rp.scale = static_cast<const __nv_bfloat16 *>(scale);
+    rp.shift = static_cast<const __nv_bfloat16 *>(shift);
+    rp.gate = static_cast<const __nv_bfloat16 *>(gate);
+    rp.h1 = h1;
+    rp.u = u;
+    rp.out = static_cast<__nv_bfloat16 *>(out);
+    rp.T = T;
+    rp.S = S;
+    rp.Hd = Hd;
+    rp.eps = eps;
+    rc = launch_rows(dm05::post::adarms_rows, T, rp, stream);
+    if (rc != DM05_OK) return rc;
+    // 3. GEGLU gate-up
+    gp.part = nullptr;
+    gp.m = m;
+    gp.F = F;
+    gp.xk_inner = Hd;
+    gp.chunks_per_split = Hd / 64;
+    rc = launch_gemm(true, pl.NT, dim3(F / 64, tok_tiles, 1), tw_gu, tx_u, gp, stream);
+    if (rc != DM05_OK) return rc;
+    // 4. MLP down: partial sums over ks_d K ranges
+    gp.part = part_d;
+    gp.m = nullptr;
+    gp.N_rows = Hd;
+    gp.xk_inner = F;
+    gp.chunks_per_split = F / 64 / pl.ks_d;
+    rc = launch_gemm(false, pl.NT, dim3(Hd / 128, tok_tiles, pl.ks_d), tw_d, tx_m, gp, stream);
+    if (rc != DM05_OK) return rc;
+    // 5. gated residual
+    rp.part = part_d;
+    rp.splits = pl.ks_d;
+    return launch_rows(dm05::post::gated_residual_rows, T, rp, stream);
+}
+
+}  // extern "C"
+
+// Frees the post-attention block's buffers (called by dm05_release with g_mu held).
+void release_post_buffers()
+{
+    for (auto &w : g_post_ws) {
+        if (w.base != nullptr && cudaSetDevice(w.dev) == cudaSuccess) cudaFree(w.base);
+    }
+    g_post_ws.clear();
+}

@@ -39,7 +39,10 @@ namespace dm05 {
 namespace prologue {
 
 constexpr int kThreads = 128;
-constexpr int kStages = 4;
+// ring depth: as many 64-column K chunks in flight as fit in ~192 KB (a CTA
+// then has an SM to itself and keeps the weight stream's latency covered)
+template <int NT>
+constexpr int stages_for() { return (192 * 1024) / (128 * 128 + NT * 128) > 8 ? 8 : (192 * 1024) / (128 * 128 + NT * 128); }
 constexpr int kChunk = 64;                 // K columns per stage (128 bytes of bf16)
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr uint32_t kEwTimeout = 0x2u;
@@ -60,6 +63,7 @@ struct Smem {
     static constexpr int kABytes = 128 * kChunk * 2;     // 16 KB: 128 feature rows
     static constexpr int kBBytes = NT * kChunk * 2;      // NT token rows
     static constexpr int kStageBytes = kABytes + kBBytes;
+    static constexpr int kStages = stages_for<NT>();
     static constexpr int kRingBytes = kStages * kStageBytes;
     static constexpr int kYStride = NT + 4;              // fp32 per feature row (padded)
     static constexpr int kYBytes = 128 * kYStride * 4;
@@ -83,6 +87,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kBarOff);
+    constexpr int kStages = L::kStages;
     uint64_t *full = bars, *empty = bars + kStages, *mma_done = bars + 2 * kStages;
     float *ss_own = reinterpret_cast<float *>(smem + L::kSsOff);
     float *ss_peer = ss_own + NT;  // written by the other half of the head

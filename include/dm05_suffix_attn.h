@@ -293,6 +293,43 @@ int dm05_suffix_qkv_prologue(const void *x, const void *w, const void *q_norm_w,
                              cudaStream_t stream);
 
 /*
+ * dm05_post_attention -- the step right after the suffix attention in an
+ * action-expert layer: output projection + residual, Adarms time
+ * modulation, GEGLU gate-up, MLP down + gated residual; asynchronous on
+ * `stream` (five kernel launches).
+ *
+ * The operation (page "TensorRT+Triton+FlexAttention: OpenDM VLA
+ * 快速推理加速栈深度剖析", section 2.2: after the three attention stages the
+ * suffix path chains the time modulation Adarms, the GEGLU gate-up and the
+ * MLP down; hidden 1024, intermediate 4096).  For token t = b * S + i:
+ *   a_t  = the attention output of the token, its Hq heads concatenated (Hq * D)
+ *   h1   = h[t] + wo a_t
+ *   u    = h1 / sqrt(mean(h1^2) + eps) * (1 + scale[b]) + shift[b]
+ *   m    = gelu_tanh(wgu[0:F] u) * (wgu[F:2F] u)
+ *   out[t] = h1 + gate[b] * (wd m)              (rounded once to bf16)
+ * gelu_tanh(z) = z / 2 (1 + tanh(sqrt(2/pi) (z + 0.044715 z^3))).
+ *
+ *   attn   bf16 [B, Hq, S, D]   the suffix attention's output (its `out`)
+ *   h      bf16 [B*S, Hd]       residual stream entering the layer
+ *   scale, shift, gate  bf16 [B, Hd]   time modulation of each sample
+ *   wo     bf16 [Hd, Hq*D], wgu bf16 [2F, Hd] (gate rows, then up rows),
+ *   wd     bf16 [Hd, F]
+ *   out    bf16 [B*S, Hd]
+ *
+ * Supported: D and F multiples of 64, Hd a multiple of 128.  attn, h, the
+ * weights and out 16-byte aligned; scale, shift, gate 2-byte aligned.  The
+ * intermediates (h1 fp32, u and m bf16, and fp32 split-K partial sums) live
+ * in a library workspace per (device, stream), created by the first call
+ * outside stream capture or by dm05_post_attention_reserve (call it before
+ * capturing); results are deterministic (the split-K partial sums are added
+ * in a fixed order).  Errors as dm05_suffix_attn.
+ */
+int dm05_post_attention(const void *attn, const void *h, const void *scale, const void *shift, const void *gate,
+                        const void *wo, const void *wgu, const void *wd, void *out,
+                        int B, int S, int Hq, int D, int Hd, int F, float eps, cudaStream_t stream);
+int dm05_post_attention_reserve(int B, int S, int Hq, int D, int Hd, int F, cudaStream_t stream);
+
+/*
  * dm05_suffix_attn_noalloc -- the same attention as dm05_suffix_attn, for
  * callers that must not allocate device memory.  The source pages have no
  * counterpart of this entry point; it exists for embedding.

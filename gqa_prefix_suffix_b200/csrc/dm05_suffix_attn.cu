@@ -66,8 +66,25 @@ int g_row_block_override = 0;
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
 auto *kKernel = &dm05::suffix_attn_kernel<kTileRows, kStages>;
-auto *kPrologue64 = &dm05::prologue::qkv_prologue_kernel<64>;
-auto *kPrologue128 = &dm05::prologue::qkv_prologue_kernel<128>;
+
+// Prologue variants: token tile NT (64 or 128) x ring depth (deep: one CTA per
+// SM for grids of about one wave; shallow: two per SM for larger grids).
+using PrologueFn = void (*)(CUtensorMap, CUtensorMap, dm05::prologue::Params);
+struct PrologueVariant {
+    PrologueFn fn;
+    int smem;
+};
+template <int NT, int ST>
+PrologueVariant prologue_variant()
+{
+    return {&dm05::prologue::qkv_prologue_kernel<NT, ST>, dm05::prologue::Smem<NT, ST>::kAllocBytes};
+}
+const PrologueVariant kPrologueVariants[4] = {
+    prologue_variant<64, dm05::prologue::deep_stages<64>()>(),
+    prologue_variant<64, dm05::prologue::shallow_stages<64>()>(),
+    prologue_variant<128, dm05::prologue::deep_stages<128>()>(),
+    prologue_variant<128, dm05::prologue::shallow_stages<128>()>(),
+};
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -800,6 +817,7 @@ int dm05_suffix_qkv_prologue(const void *x, const void *w, const void *q_norm_w,
         return DM05_ERR_ALIGN;
     const bool small = T <= 64;
     uint32_t *err = nullptr;
+    int num_sms = 148;
     {
         std::lock_guard<std::mutex> lk(g_mu);
         if (get_encoder() != DM05_OK) return DM05_ERR_CUDA;
@@ -812,16 +830,17 @@ int dm05_suffix_qkv_prologue(const void *x, const void *w, const void *q_norm_w,
             if (cs != cudaStreamCaptureStatusNone) return DM05_ERR_WORKSPACE;
             rc = device_state(true, &ds, stream);
             if (rc != DM05_OK) return rc;
-            if (cudaFuncSetAttribute(kPrologue64, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     dm05::prologue::Smem<64>::kAllocBytes) != cudaSuccess ||
-                cudaFuncSetAttribute(kPrologue128, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     dm05::prologue::Smem<128>::kAllocBytes) != cudaSuccess)
-                return DM05_ERR_CUDA;
+            for (const PrologueVariant &pv : kPrologueVariants)
+                if (cudaFuncSetAttribute(pv.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, pv.smem) != cudaSuccess)
+                    return DM05_ERR_CUDA;
             ds->prologue_attrs_set = true;
         }
         err = ds->err;
+        num_sms = ds->num_sms;
     }
     const int NT = small ? 64 : 128;
+    const long long ctas = static_cast<long long>(2 * (Hq + 2 * Hkv)) * ((T + NT - 1) / NT);
+    const PrologueVariant &pv = kPrologueVariants[(small ? 0 : 2) + (ctas > 2LL * num_sms ? 1 : 0)];
     CUtensorMap tm_w, tm_x;
     if (encode_2d(&tm_w, w, static_cast<uint64_t>(H), static_cast<uint64_t>(Hq + 2 * Hkv) * D, 64) != DM05_OK ||
         encode_2d(&tm_x, x, static_cast<uint64_t>(H), static_cast<uint64_t>(T), static_cast<uint32_t>(NT)) != DM05_OK)
@@ -846,7 +865,7 @@ int dm05_suffix_qkv_prologue(const void *x, const void *w, const void *q_norm_w,
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(2 * (Hq + 2 * Hkv)), static_cast<unsigned>((T + NT - 1) / NT), 1);
     cfg.blockDim = dim3(dm05::prologue::kThreads, 1, 1);
-    cfg.dynamicSmemBytes = small ? dm05::prologue::Smem<64>::kAllocBytes : dm05::prologue::Smem<128>::kAllocBytes;
+    cfg.dynamicSmemBytes = static_cast<size_t>(pv.smem);
     cfg.stream = stream;
     cudaLaunchAttribute at[2];
     at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -857,8 +876,7 @@ int dm05_suffix_qkv_prologue(const void *x, const void *w, const void *q_norm_w,
     at[1].val.clusterDim.z = 1;
     cfg.attrs = at;
     cfg.numAttrs = 2;
-    const cudaError_t e = small ? cudaLaunchKernelEx(&cfg, kPrologue64, tm_w, tm_x, pp)
-                                : cudaLaunchKernelEx(&cfg, kPrologue128, tm_w, tm_x, pp);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, pv.fn, tm_w, tm_x, pp);
     return e == cudaSuccess ? DM05_OK : DM05_ERR_CUDA;
 }
 
@@ -1304,35 +1322,53 @@ int post_check(const void *attn, const void *h, const void *scale, const void *s
     for (const void *ptr : {attn, h, wo, wgu, wd, out})
         if (!aligned16(ptr)) return DM05_ERR_ALIGN;
     for (const void *ptr : {scale, shift, gate})
-        if (reinterpret_cast<uintptr_t>(ptr) & 1u) return DM05_ERR_ALIGN;
+        if (reinterpret_cast<uintptr_t>(ptr) & 7u) return DM05_ERR_ALIGN;  // four bf16 per load
     return DM05_OK;
 }
 
-auto *kGemmPartial64 = &dm05::post::gemm_kernel<64, dm05::post::kPartial>;
-auto *kGemmPartial128 = &dm05::post::gemm_kernel<128, dm05::post::kPartial>;
-auto *kGemmGeglu64 = &dm05::post::gemm_kernel<64, dm05::post::kGeglu>;
-auto *kGemmGeglu128 = &dm05::post::gemm_kernel<128, dm05::post::kGeglu>;
+// GEMM variants: epilogue x token tile NT (64 or 128) x ring depth (deep
+// for grids of at most one wave, shallow, two CTAs per SM, for larger ones).
+using GemmFn = void (*)(CUtensorMap, CUtensorMap, dm05::post::GemmParams);
+struct GemmVariant {
+    GemmFn fn;
+    int smem;
+};
+template <int NT, int EPI, int ST>
+GemmVariant gemm_variant()
+{
+    return {&dm05::post::gemm_kernel<NT, EPI, ST>, dm05::post::GemmSmem<NT, ST>::kAllocBytes};
+}
+template <int NT, int EPI>
+GemmVariant gemm_variant_depth(bool deep)
+{
+    return deep ? gemm_variant<NT, EPI, dm05::post::deep_stages<NT>()>()
+                : gemm_variant<NT, EPI, dm05::post::shallow_stages<NT>()>();
+}
+GemmVariant gemm_variant_for(bool geglu, int NT, bool deep)
+{
+    if (geglu)
+        return NT == 64 ? gemm_variant_depth<64, dm05::post::kGeglu>(deep)
+                        : gemm_variant_depth<128, dm05::post::kGeglu>(deep);
+    return NT == 64 ? gemm_variant_depth<64, dm05::post::kPartial>(deep)
+                    : gemm_variant_depth<128, dm05::post::kPartial>(deep);
+}
 
 int launch_gemm(bool geglu, int NT, dim3 grid, const CUtensorMap &tw, const CUtensorMap &tx,
-                const dm05::post::GemmParams &gp, cudaStream_t stream)
+                const dm05::post::GemmParams &gp, int num_sms, cudaStream_t stream)
 {
+    const long long ctas = static_cast<long long>(grid.x) * grid.y * grid.z;
+    const GemmVariant gv = gemm_variant_for(geglu, NT, ctas <= num_sms);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = dim3(dm05::post::kThreads, 1, 1);
-    cfg.dynamicSmemBytes = NT == 64 ? dm05::post::GemmSmem<64>::kAllocBytes : dm05::post::GemmSmem<128>::kAllocBytes;
+    cfg.dynamicSmemBytes = static_cast<size_t>(gv.smem);
     cfg.stream = stream;
     cudaLaunchAttribute at[1];
     at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     at[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = at;
     cfg.numAttrs = 1;
-    cudaError_t e;
-    if (geglu)
-        e = NT == 64 ? cudaLaunchKernelEx(&cfg, kGemmGeglu64, tw, tx, gp) : cudaLaunchKernelEx(&cfg, kGemmGeglu128, tw, tx, gp);
-    else
-        e = NT == 64 ? cudaLaunchKernelEx(&cfg, kGemmPartial64, tw, tx, gp)
-                     : cudaLaunchKernelEx(&cfg, kGemmPartial128, tw, tx, gp);
-    return e == cudaSuccess ? DM05_OK : DM05_ERR_CUDA;
+    return cudaLaunchKernelEx(&cfg, gv.fn, tw, tx, gp) == cudaSuccess ? DM05_OK : DM05_ERR_CUDA;
 }
 
 template <class K>
@@ -1340,7 +1376,7 @@ int launch_rows(K kernel, int T, const dm05::post::RowParams &rp, cudaStream_t s
 {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(T), 1, 1);
-    cfg.blockDim = dim3(256, 1, 1);
+    cfg.blockDim = dim3(dm05::post::kRowThreads, 1, 1);
     cfg.stream = stream;
     cudaLaunchAttribute at[1];
     at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -1363,12 +1399,11 @@ int post_device_state(cudaStream_t stream, DeviceState **out)
         if (cs != cudaStreamCaptureStatusNone) return DM05_ERR_WORKSPACE;
         rc = device_state(true, &ds, stream);
         if (rc != DM05_OK) return rc;
-        const int s64 = dm05::post::GemmSmem<64>::kAllocBytes, s128 = dm05::post::GemmSmem<128>::kAllocBytes;
-        if (cudaFuncSetAttribute(kGemmPartial64, cudaFuncAttributeMaxDynamicSharedMemorySize, s64) != cudaSuccess ||
-            cudaFuncSetAttribute(kGemmPartial128, cudaFuncAttributeMaxDynamicSharedMemorySize, s128) != cudaSuccess ||
-            cudaFuncSetAttribute(kGemmGeglu64, cudaFuncAttributeMaxDynamicSharedMemorySize, s64) != cudaSuccess ||
-            cudaFuncSetAttribute(kGemmGeglu128, cudaFuncAttributeMaxDynamicSharedMemorySize, s128) != cudaSuccess)
-            return DM05_ERR_CUDA;
+        for (int v = 0; v < 8; ++v) {
+            const GemmVariant gv = gemm_variant_for((v & 1) != 0, (v & 2) ? 128 : 64, (v & 4) != 0);
+            if (cudaFuncSetAttribute(gv.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, gv.smem) != cudaSuccess)
+                return DM05_ERR_CUDA;
+        }
         ds->post_attrs_set = true;
     }
     *out = ds;
@@ -1402,6 +1437,7 @@ int dm05_post_attention(const void *attn, const void *h, const void *scale, cons
     if (!(eps > 0.0f)) return DM05_ERR_SHAPE;
     const int T = B * S;
     PostPlan pl;
+    int num_sms = 148;
     uint32_t *err = nullptr;
     uint8_t *ws = nullptr;
     {
@@ -1411,6 +1447,7 @@ int dm05_post_attention(const void *attn, const void *h, const void *scale, cons
         rc = post_device_state(stream, &ds);
         if (rc != DM05_OK) return rc;
         pl = post_plan(B, S, Hq, D, Hd, F, ds->num_sms);
+        num_sms = ds->num_sms;
         err = ds->err;
         void *p = nullptr;
         rc = keyed_buffer(g_post_ws, stream, pl.total, &p);
@@ -1443,7 +1480,7 @@ int dm05_post_attention(const void *attn, const void *h, const void *scale, cons
     gp.N_rows = Hd;
     gp.xk_inner = D;
     gp.chunks_per_split = A / 64 / pl.ks_o;
-    rc = launch_gemm(false, pl.NT, dim3(Hd / 128, tok_tiles, pl.ks_o), tw_o, tx_a, gp, stream);
+    rc = launch_gemm(false, pl.NT, dim3(Hd / 128, tok_tiles, pl.ks_o), tw_o, tx_a, gp, num_sms, stream);
     if (rc != DM05_OK) return rc;
     // 2. residual, Adarms
     dm05::post::RowParams rp{};
@@ -1468,7 +1505,7 @@ int dm05_post_attention(const void *attn, const void *h, const void *scale, cons
     gp.F = F;
     gp.xk_inner = Hd;
     gp.chunks_per_split = Hd / 64;
-    rc = launch_gemm(true, pl.NT, dim3(F / 64, tok_tiles, 1), tw_gu, tx_u, gp, stream);
+    rc = launch_gemm(true, pl.NT, dim3(F / 64, tok_tiles, 1), tw_gu, tx_u, gp, num_sms, stream);
     if (rc != DM05_OK) return rc;
     // 4. MLP down: partial sums over ks_d K ranges
     gp.part = part_d;
@@ -1476,7 +1513,7 @@ int dm05_post_attention(const void *attn, const void *h, const void *scale, cons
     gp.N_rows = Hd;
     gp.xk_inner = F;
     gp.chunks_per_split = F / 64 / pl.ks_d;
-    rc = launch_gemm(false, pl.NT, dim3(Hd / 128, tok_tiles, pl.ks_d), tw_d, tx_m, gp, stream);
+    rc = launch_gemm(false, pl.NT, dim3(Hd / 128, tok_tiles, pl.ks_d), tw_d, tx_m, gp, num_sms, stream);
     if (rc != DM05_OK) return rc;
     // 5. gated residual
     rp.part = part_d;

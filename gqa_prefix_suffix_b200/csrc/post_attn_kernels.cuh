@@ -35,10 +35,15 @@ namespace dm05 {
 namespace post {
 
 constexpr int kThreads = 128;
-// ring depth: as many 64-column K chunks in flight as fit in ~192 KB (a CTA
-// then has an SM to itself and keeps the weight stream's latency covered)
+// Ring depth in 64-column K chunks: deep (about 192 KB, one CTA per SM)
+// when the grid is about one wave and each CTA must keep its own weight
+// stream's latency covered; shallow (about 96 KB, two CTAs per SM) when
+// the grid spans several waves, so that one CTA's copies overlap the
+// other's epilogue.
 template <int NT>
-constexpr int stages_for() { return (192 * 1024) / (128 * 128 + NT * 128) > 8 ? 8 : (192 * 1024) / (128 * 128 + NT * 128); }
+constexpr int deep_stages() { return (192 * 1024) / (128 * 128 + NT * 128) > 8 ? 8 : (192 * 1024) / (128 * 128 + NT * 128); }
+template <int NT>
+constexpr int shallow_stages() { return (96 * 1024) / (128 * 128 + NT * 128); }
 constexpr int kChunk = 64;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr uint32_t kEwTimeout = 0x2u;
@@ -61,12 +66,12 @@ struct GemmParams {
     int chunks_per_split;      // K chunks each split covers
 };
 
-template <int NT>
+template <int NT, int STAGES>
 struct GemmSmem {
     static constexpr int kABytes = 128 * kChunk * 2;
     static constexpr int kBBytes = NT * kChunk * 2;
     static constexpr int kStageBytes = kABytes + kBBytes;
-    static constexpr int kStages = stages_for<NT>();
+    static constexpr int kStages = STAGES;
     static constexpr int kRingBytes = kStages * kStageBytes;
     static constexpr int kBarOff = kRingBytes;
     static constexpr int kNumBars = 2 * kStages + 1;
@@ -90,12 +95,12 @@ __device__ __forceinline__ float gelu_tanh(float z)
 // (k % xk_inner, i, k / xk_inner, b), which covers both a [B*S][K] matrix
 // (xk_inner = K) and the attention output [B][Hq][S][D] read as the tokens'
 // heads concatenated (xk_inner = D).
-template <int NT, int EPI>
+template <int NT, int EPI, int STAGES>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
                 const GemmParams p)
 {
-    using L = GemmSmem<NT>;
+    using L = GemmSmem<NT, STAGES>;
     static_assert(NT % 16 == 0 && NT >= 16 && NT <= 256, "N of an M=128 MMA");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -201,38 +206,30 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     } else {
-        // lanes 0-63: gate rows, lanes 64-127: the matching up rows; pass the
-        // up values through shared memory (the ring is free now)
-        float *up_s = reinterpret_cast<float *>(smem);  // [64][NT + 1]
+        // lanes 0-63: gate rows, lanes 64-127: the matching up rows.  Every
+        // warp moves its rows to shared memory (the ring is free now); then
+        // each thread takes two adjacent features f, f + 1 (f = 64 x + 2 lane)
+        // for the tokens t = warp (mod 4): bf16x2 stores, 128 contiguous
+        // bytes per warp and token.
         constexpr int kUS = NT + 1;
-        if (warp >= 2) {
+        float *rows_s = reinterpret_cast<float *>(smem);  // [128][NT + 1]: gate rows, then up rows
+        static_assert(128 * kUS * 4 <= L::kRingBytes, "the gate/up tile reuses the ring");
 #pragma unroll
-            for (int j = 0; j < NT / 16; ++j) {
-                uint32_t o[16];
-                ptx::tmem_ld16(tmem + lane_base + j * 16, o);
-                ptx::tmem_ld_wait();
+        for (int j = 0; j < NT / 16; ++j) {
+            uint32_t o[16];
+            ptx::tmem_ld16(tmem + lane_base + j * 16, o);
+            ptx::tmem_ld_wait();
 #pragma unroll
-                for (int e = 0; e < 16; ++e) up_s[(threadIdx.x - 64) * kUS + j * 16 + e] = __uint_as_float(o[e]);
-            }
+            for (int e = 0; e < 16; ++e) rows_s[threadIdx.x * kUS + j * 16 + e] = __uint_as_float(o[e]);
         }
         __syncthreads();
-        if (warp < 2) {
-            const int f = 64 * blockIdx.x + threadIdx.x;
-#pragma unroll
-            for (int j = 0; j < NT / 16; ++j) {
-                uint32_t o[16];
-                ptx::tmem_ld16(tmem + lane_base + j * 16, o);
-                ptx::tmem_ld_wait();
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const int jj = j * 16 + e;
-                    if (jj < n_tok) {
-                        const float g = __uint_as_float(o[e]);
-                        const float up = up_s[threadIdx.x * kUS + jj];
-                        p.m[static_cast<size_t>(tok0 + jj) * p.F + f] = __float2bfloat16_rn(gelu_tanh(g) * up);
-                    }
-                }
-            }
+        const int fl = 2 * lane;
+        const int f = 64 * blockIdx.x + fl;
+        for (int t = warp; t < n_tok; t += kThreads / 32) {
+            const float g0 = rows_s[fl * kUS + t], g1 = rows_s[(fl + 1) * kUS + t];
+            const float u0 = rows_s[(64 + fl) * kUS + t], u1 = rows_s[(65 + fl) * kUS + t];
+            *reinterpret_cast<__nv_bfloat162 *>(p.m + static_cast<size_t>(tok0 + t) * p.F + f) =
+                __floats2bfloat162_rn(gelu_tanh(g0) * u0, gelu_tanh(g1) * u1);
         }
     }
 
@@ -259,48 +256,118 @@ struct RowParams {
     float eps;
 };
 
-// One CTA per token: h1 = h + sum of the partials (fixed order), the RMS over
-// Hd, then u = h1 / rms * (1 + scale) + shift.
-__global__ void __launch_bounds__(256) adarms_rows(const RowParams p)
+// Sum over the splits of four consecutive fp32 partials, in split order
+// (deterministic); the loads of eight splits are issued before any add.
+__device__ __forceinline__ float4 split_sum4(const float *__restrict__ part, int splits, size_t split_stride,
+                                             size_t off)
 {
-    __shared__ float red[8];
+    float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    int sp = 0;
+    for (; sp + 8 <= splits; sp += 8) {
+        float4 v[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) v[k] = *reinterpret_cast<const float4 *>(part + (sp + k) * split_stride + off);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            acc.x += v[k].x;
+            acc.y += v[k].y;
+            acc.z += v[k].z;
+            acc.w += v[k].w;
+        }
+    }
+    for (; sp < splits; ++sp) {
+        const float4 v = *reinterpret_cast<const float4 *>(part + sp * split_stride + off);
+        acc.x += v.x;
+        acc.y += v.y;
+        acc.z += v.z;
+        acc.w += v.w;
+    }
+    return acc;
+}
+
+__device__ __forceinline__ float4 ld_bf16x4(const __nv_bfloat16 *p)
+{
+    const uint2 u = *reinterpret_cast<const uint2 *>(p);
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
+    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
+    return make_float4(a.x, a.y, b.x, b.y);
+}
+
+__device__ __forceinline__ void st_bf16x4(__nv_bfloat16 *p, float a, float b, float c, float d)
+{
+    __nv_bfloat162 lo = __floats2bfloat162_rn(a, b), hi = __floats2bfloat162_rn(c, d);
+    *reinterpret_cast<uint2 *>(p) = make_uint2(*reinterpret_cast<uint32_t *>(&lo), *reinterpret_cast<uint32_t *>(&hi));
+}
+
+constexpr int kRowThreads = 256;
+constexpr int kRowVecs = 4;  // float4 per thread kept in registers between the two passes (Hd <= 4096)
+
+// One CTA per token: h1 = h + sum of the partials (fixed order), the RMS over
+// Hd, then u = h1 / rms * (1 + scale) + shift.  Each thread owns groups of
+// four consecutive features; Hd is a multiple of 128.
+__global__ void __launch_bounds__(kRowThreads) adarms_rows(const RowParams p)
+{
+    __shared__ float red[kRowThreads / 32];
     ptx::griddep_launch_dependents();
     ptx::griddep_wait();
     const int t = blockIdx.x, b = t / p.S;
+    const int n4 = p.Hd / 4;
+    const size_t stride = static_cast<size_t>(p.T) * p.Hd;
+    const size_t row = static_cast<size_t>(t) * p.Hd;
     float ss = 0.0f;
-    for (int o = threadIdx.x; o < p.Hd; o += blockDim.x) {
-        float acc = 0.0f;
-        for (int sp = 0; sp < p.splits; ++sp) acc += p.part[(static_cast<size_t>(sp) * p.T + t) * p.Hd + o];
-        const float x = __bfloat162float(p.h[static_cast<size_t>(t) * p.Hd + o]) + acc;
-        p.h1[static_cast<size_t>(t) * p.Hd + o] = x;
-        ss = fmaf(x, x, ss);
-    }
+    auto first = [&](int i) {
+        const float4 acc = split_sum4(p.part, p.splits, stride, row + 4 * i);
+        const float4 hv = ld_bf16x4(p.h + row + 4 * i);
+        const float4 x = make_float4(hv.x + acc.x, hv.y + acc.y, hv.z + acc.z, hv.w + acc.w);
+        *reinterpret_cast<float4 *>(p.h1 + row + 4 * i) = x;
+        ss = fmaf(x.x, x.x, ss);
+        ss = fmaf(x.y, x.y, ss);
+        ss = fmaf(x.z, x.z, ss);
+        ss = fmaf(x.w, x.w, ss);
+        return x;
+    };
+    float4 xr[kRowVecs];
+#pragma unroll
+    for (int v = 0; v < kRowVecs; ++v)
+        if (threadIdx.x + v * kRowThreads < n4) xr[v] = first(threadIdx.x + v * kRowThreads);
+    for (int i = threadIdx.x + kRowVecs * kRowThreads; i < n4; i += kRowThreads) first(i);
 #pragma unroll
     for (int k = 16; k > 0; k >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, k);
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
     __syncthreads();
     float tot = 0.0f;
-    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) tot += red[w];
+#pragma unroll
+    for (int w = 0; w < kRowThreads / 32; ++w) tot += red[w];
     const float inv_rms = rsqrtf(tot / static_cast<float>(p.Hd) + p.eps);
-    for (int o = threadIdx.x; o < p.Hd; o += blockDim.x) {
-        const float x = p.h1[static_cast<size_t>(t) * p.Hd + o];
-        const float sc = __bfloat162float(p.scale[static_cast<size_t>(b) * p.Hd + o]);
-        const float sh = __bfloat162float(p.shift[static_cast<size_t>(b) * p.Hd + o]);
-        p.u[static_cast<size_t>(t) * p.Hd + o] = __float2bfloat16_rn(fmaf(x * inv_rms, 1.0f + sc, sh));
-    }
+    const size_t brow = static_cast<size_t>(b) * p.Hd;
+    auto second = [&](int i, const float4 &x) {
+        const float4 sc = ld_bf16x4(p.scale + brow + 4 * i);
+        const float4 sh = ld_bf16x4(p.shift + brow + 4 * i);
+        st_bf16x4(p.u + row + 4 * i, fmaf(x.x * inv_rms, 1.0f + sc.x, sh.x), fmaf(x.y * inv_rms, 1.0f + sc.y, sh.y),
+                  fmaf(x.z * inv_rms, 1.0f + sc.z, sh.z), fmaf(x.w * inv_rms, 1.0f + sc.w, sh.w));
+    };
+#pragma unroll
+    for (int v = 0; v < kRowVecs; ++v)
+        if (threadIdx.x + v * kRowThreads < n4) second(threadIdx.x + v * kRowThreads, xr[v]);
+    for (int i = threadIdx.x + kRowVecs * kRowThreads; i < n4; i += kRowThreads)
+        second(i, *reinterpret_cast<const float4 *>(p.h1 + row + 4 * i));
 }
 
 // One CTA per token: out = h1 + gate * (sum of the partials).
-__global__ void __launch_bounds__(256) gated_residual_rows(const RowParams p)
+__global__ void __launch_bounds__(kRowThreads) gated_residual_rows(const RowParams p)
 {
     ptx::griddep_launch_dependents();
     ptx::griddep_wait();
     const int t = blockIdx.x, b = t / p.S;
-    for (int o = threadIdx.x; o < p.Hd; o += blockDim.x) {
-        float acc = 0.0f;
-        for (int sp = 0; sp < p.splits; ++sp) acc += p.part[(static_cast<size_t>(sp) * p.T + t) * p.Hd + o];
-        const float g = __bfloat162float(p.gate[static_cast<size_t>(b) * p.Hd + o]);
-        p.out[static_cast<size_t>(t) * p.Hd + o] = __float2bfloat16_rn(fmaf(g, acc, p.h1[static_cast<size_t>(t) * p.Hd + o]));
+    const int n4 = p.Hd / 4;
+    const size_t stride = static_cast<size_t>(p.T) * p.Hd;
+    const size_t row = static_cast<size_t>(t) * p.Hd, brow = static_cast<size_t>(b) * p.Hd;
+    for (int i = threadIdx.x; i < n4; i += kRowThreads) {
+        const float4 acc = split_sum4(p.part, p.splits, stride, row + 4 * i);
+        const float4 g = ld_bf16x4(p.gate + brow + 4 * i);
+        const float4 h1 = *reinterpret_cast<const float4 *>(p.h1 + row + 4 * i);
+        st_bf16x4(p.out + row + 4 * i, fmaf(g.x, acc.x, h1.x), fmaf(g.y, acc.y, h1.y), fmaf(g.z, acc.z, h1.z),
+                  fmaf(g.w, acc.w, h1.w));
     }
 }
 

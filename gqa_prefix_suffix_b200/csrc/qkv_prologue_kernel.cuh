@@ -39,10 +39,15 @@ namespace dm05 {
 namespace prologue {
 
 constexpr int kThreads = 128;
-// ring depth: as many 64-column K chunks in flight as fit in ~192 KB (a CTA
-// then has an SM to itself and keeps the weight stream's latency covered)
+// Ring depth in 64-column K chunks: deep (about 192 KB, one CTA per SM)
+// when the grid is about one wave and each CTA must keep its own weight
+// stream's latency covered; shallow (about 96 KB, two CTAs per SM) when
+// the grid spans several waves, so that one CTA's copies overlap the
+// other's epilogue.
 template <int NT>
-constexpr int stages_for() { return (192 * 1024) / (128 * 128 + NT * 128) > 8 ? 8 : (192 * 1024) / (128 * 128 + NT * 128); }
+constexpr int deep_stages() { return (192 * 1024) / (128 * 128 + NT * 128) > 8 ? 8 : (192 * 1024) / (128 * 128 + NT * 128); }
+template <int NT>
+constexpr int shallow_stages() { return (96 * 1024) / (128 * 128 + NT * 128); }
 constexpr int kChunk = 64;                 // K columns per stage (128 bytes of bf16)
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr uint32_t kEwTimeout = 0x2u;
@@ -58,31 +63,32 @@ struct Params {
     float log2_theta;          // log2(theta)
 };
 
-template <int NT>
+template <int NT, int STAGES>
 struct Smem {
     static constexpr int kABytes = 128 * kChunk * 2;     // 16 KB: 128 feature rows
     static constexpr int kBBytes = NT * kChunk * 2;      // NT token rows
     static constexpr int kStageBytes = kABytes + kBBytes;
-    static constexpr int kStages = stages_for<NT>();
+    static constexpr int kStages = STAGES;
     static constexpr int kRingBytes = kStages * kStageBytes;
-    static constexpr int kYStride = NT + 4;              // fp32 per feature row (padded)
+    static constexpr int kYStride = NT + 1;              // fp32 per feature row (odd: conflict-free row writes)
     static constexpr int kYBytes = 128 * kYStride * 4;
     // the epilogue tile and the per-group sums of squares reuse the ring
     static_assert(kRingBytes >= kYBytes + kThreads * 4 * 4, "the epilogue tile reuses the ring");
     static constexpr int kBarOff = kRingBytes;
     static constexpr int kNumBars = 2 * kStages + 1;     // full[s], empty[s], mma done
     static constexpr int kSsOff = kBarOff + kNumBars * 8 + 8;   // own sums [NT], partner's sums [NT]
-    static constexpr int kTmemSlotOff = kSsOff + 2 * NT * 4;
+    static constexpr int kPosOff = kSsOff + 2 * NT * 4;         // the tile's token positions [NT]
+    static constexpr int kTmemSlotOff = kPosOff + NT * 4;
     static constexpr int kEnd = kTmemSlotOff + 16;
     static constexpr int kAllocBytes = kEnd + 1024;
 };
 
-template <int NT>
+template <int NT, int STAGES>
 __global__ void __launch_bounds__(kThreads, 1)
     qkv_prologue_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
                         const Params p)
 {
-    using L = Smem<NT>;
+    using L = Smem<NT, STAGES>;
     static_assert(NT % 16 == 0 && NT >= 16 && NT <= 256, "N of an M=128 MMA");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -91,6 +97,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *full = bars, *empty = bars + kStages, *mma_done = bars + 2 * kStages;
     float *ss_own = reinterpret_cast<float *>(smem + L::kSsOff);
     float *ss_peer = ss_own + NT;  // written by the other half of the head
+    int *pos_s = reinterpret_cast<int *>(smem + L::kPosOff);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kTmemSlotOff);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -123,6 +130,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::tc_fence_after_sync();
     const uint32_t tmem = *tmem_slot;
     ptx::griddep_wait();
+    // warps 2-3 (idle until the epilogue) fetch the tile's positions now, so
+    // that the rotation loop below reads none from global memory
+    for (int i = threadIdx.x - 64; i >= 0 && i < NT; i += kThreads - 64) pos_s[i] = t0 + i < p.T ? p.pos[t0 + i] : 0;
 
     bool failed = false;
     // feature rows of this CTA: the head's rows [64*half, +64) then [64*half + 128, +64)
@@ -220,9 +230,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     ptx::cluster_sync();  // both halves' sums are in place (and no one still writes)
 
-    // each thread: feature pair j = threadIdx.x % 64 for tokens of one parity
-    const int j = threadIdx.x & 63;
-    const int fa = 64 * half + j;          // feature index within the head (first of the pair)
+    // each thread: the two adjacent rotation pairs (fa, fa + D/2) and
+    // (fa + 1, fa + 1 + D/2), fa = 64 * half + 2 * lane, for the tokens
+    // t = warp (mod 4): bf16x2 stores, 32 lanes covering 128 contiguous bytes
+    const int j0 = 2 * lane;
+    const int fa = 64 * half + j0;  // feature index within the head (first of the two pairs)
     const int fb = fa + D / 2;
     __nv_bfloat16 *dst_base;
     int heads, h;
@@ -239,37 +251,49 @@ __global__ void __launch_bounds__(kThreads, 1)
         heads = p.Hkv;
         h = hd - p.Hq - p.Hkv;
     }
-    float wa = 1.0f, wb = 1.0f;
-    double inv_freq = 0.0;
+    float wa0 = 1.0f, wa1 = 1.0f, wb0 = 1.0f, wb1 = 1.0f;
+    double inv_freq0 = 0.0, inv_freq1 = 0.0;
     if (!is_v) {
         const __nv_bfloat16 *nw = hd < p.Hq ? p.qw : p.kw;
-        wa = __bfloat162float(nw[fa]);
-        wb = __bfloat162float(nw[fb]);
-        // theta^(-2 fa / D), in double: positions reach thousands of radians
-        inv_freq = exp2(-2.0 * static_cast<double>(fa) / static_cast<double>(D) * static_cast<double>(p.log2_theta));
+        wa0 = __bfloat162float(nw[fa]);
+        wa1 = __bfloat162float(nw[fa + 1]);
+        wb0 = __bfloat162float(nw[fb]);
+        wb1 = __bfloat162float(nw[fb + 1]);
+        // theta^(-2 f / D), in double: positions reach thousands of radians
+        inv_freq0 = exp2(-2.0 * static_cast<double>(fa) / static_cast<double>(D) * static_cast<double>(p.log2_theta));
+        inv_freq1 = exp2(-2.0 * static_cast<double>(fa + 1) / static_cast<double>(D) * static_cast<double>(p.log2_theta));
     }
-    for (int t = (threadIdx.x >> 6); t < NT; t += kThreads / 64) {
+    // the angle reduced to [-pi, pi] in double, then its sine and cosine
+    auto rot = [](double ang, float &sn, float &cs) {
+        const double two_pi = 6.283185307179586, inv_two_pi = 0.15915494309189535;
+        ang = fma(-two_pi, rint(ang * inv_two_pi), ang);
+        sincosf(static_cast<float>(ang), &sn, &cs);
+    };
+    const int n_tok = min(NT, p.T - t0);
+#pragma unroll 2
+    for (int t = warp; t < n_tok; t += kThreads / 32) {
         const int tok = t0 + t;
-        if (tok >= p.T) break;
-        const float ya = Y[j * L::kYStride + t], yb = Y[(64 + j) * L::kYStride + t];
-        float oa = ya, ob = yb;
+        const float ya0 = Y[j0 * L::kYStride + t], ya1 = Y[(j0 + 1) * L::kYStride + t];
+        const float yb0 = Y[(64 + j0) * L::kYStride + t], yb1 = Y[(65 + j0) * L::kYStride + t];
+        float oa0 = ya0, oa1 = ya1, ob0 = yb0, ob1 = yb1;
         if (!is_v) {
             const float ms = (ss_own[t] + ss_peer[t]) / static_cast<float>(D);
             const float inv_rms = rsqrtf(ms + p.eps);
-            const float a = ya * inv_rms * wa, b = yb * inv_rms * wb;
-            // the angle reduced to [-pi, pi] in double, then its sine and cosine
-            const double two_pi = 6.283185307179586, inv_two_pi = 0.15915494309189535;
-            double ang = static_cast<double>(p.pos[tok]) * inv_freq;
-            ang = fma(-two_pi, rint(ang * inv_two_pi), ang);
-            float sn, cs;
-            sincosf(static_cast<float>(ang), &sn, &cs);
-            oa = a * cs - b * sn;
-            ob = a * sn + b * cs;
+            const float a0 = ya0 * inv_rms * wa0, a1 = ya1 * inv_rms * wa1;
+            const float b0 = yb0 * inv_rms * wb0, b1 = yb1 * inv_rms * wb1;
+            const double ps = static_cast<double>(pos_s[t]);
+            float sn0, cs0, sn1, cs1;
+            rot(ps * inv_freq0, sn0, cs0);
+            rot(ps * inv_freq1, sn1, cs1);
+            oa0 = a0 * cs0 - b0 * sn0;
+            ob0 = a0 * sn0 + b0 * cs0;
+            oa1 = a1 * cs1 - b1 * sn1;
+            ob1 = a1 * sn1 + b1 * cs1;
         }
         const int bi = tok / p.S, i = tok - bi * p.S;
         __nv_bfloat16 *row = dst_base + ((static_cast<size_t>(bi) * heads + h) * p.S + i) * D;
-        row[fa] = __float2bfloat16_rn(oa);
-        row[fb] = __float2bfloat16_rn(ob);
+        *reinterpret_cast<__nv_bfloat162 *>(row + fa) = __floats2bfloat162_rn(oa0, oa1);
+        *reinterpret_cast<__nv_bfloat162 *>(row + fb) = __floats2bfloat162_rn(ob0, ob1);
     }
 
     if (failed && lane == 0) atomicOr(p.err, kEwTimeout);

@@ -317,7 +317,7 @@ int dm05_suffix_qkv_prologue(const void *x, const void *w, const void *q_norm_w,
  *   out    bf16 [B*S, Hd]
  *
  * Supported: D and F multiples of 64, Hd a multiple of 128.  attn, h, the
- * weights and out 16-byte aligned; scale, shift, gate 2-byte aligned.  The
+ * weights and out 16-byte aligned; scale, shift, gate 8-byte aligned.  The
  * intermediates (h1 fp32, u and m bf16, and fp32 split-K partial sums) live
  * in a library workspace per (device, stream), created by the first call
  * outside stream capture or by dm05_post_attention_reserve (call it before

@@ -65,7 +65,7 @@ namespace dm05 {
 // for the first and last slot, the global timer) of one CTA's phase boundary.
 #ifdef DM05_TRACE
 __device__ unsigned long long g_dm05_trace[4096][16];
-__device__ unsigned long long g_dm05_tile_trace[4096][6][24];  // per tile: K full, QK issued, S seen, P ready, K requested, PV issued
+__device__ unsigned long long g_dm05_tile_trace[4096][8][24];  // per tile: K full, QK issued, S seen, P ready, K requested, PV issued, QK start, PV start
 #define DM05_TRACE_CLOCK(slot)                                                      \
     do {                                                                            \
         if (blockIdx.x < 4096) g_dm05_trace[blockIdx.x][slot] = clock64();          \
@@ -527,6 +527,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int pb = u % kSBufs;
                 if (!ptx::mbar_wait(&bars[L::kBarPReady + pb], (u / kSBufs) & 1, kWaitLimitNs)) return false;
                 if (!ptx::mbar_wait(&bars[L::kBarVFull + s], ((u + shift) / STAGES) & 1, kWaitLimitNs)) return false;
+                DM05_TRACE_TILE(7, u);
                 ptx::tc_fence_after_sync();
                 // descriptor of V rows [0, 16) of this slot; each 16-row k-step
                 // adds 16 * 128 bytes (in the 16-byte units of the address field)
@@ -580,6 +581,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ok = false;
                     break;
                 }
+                DM05_TRACE_TILE(6, t);
                 ptx::tc_fence_after_sync();
                 const uint64_t kdesc = kdesc0 + static_cast<uint64_t>((s * L::kStageBytes) >> 4);
                 const uint32_t d = tmem + kTmemS + sb * NT;

@@ -225,44 +225,57 @@ __device__ __forceinline__ size_t block_out_row(size_t unit_row0, int k, int nq,
 //   M = max_c m_c,  w_c = 2^(m_c - M),  LH = sum_c l_hat_c w_c,  L = sum_c l_c w_c,
 //   out = sum_c (w_c / LH) O_c,  lse = (M + log2 L) ln 2,
 // where a partial without visible keys (l_hat == 0) gets no weight.
-// Pass 1 (merge_weights): one warp per row, lane c holds partial c's
-// statistics; the row's normalised weights w_c / LH replace the unused
-// fourth statistic of each partial row, and the LSE is written.
+// Pass 1 (merge_weights): each row takes a segment of W lanes (W = C rounded
+// up to a power of two), lane c of the segment holding partial c's
+// statistics, so a warp reduces 32 / W rows at once with segment-wide
+// shuffles; the row's normalised weights w_c / LH replace the unused fourth
+// statistic of each partial row, the LSE is written, and orow[rr] receives
+// the row's output row (or -1 when the row is not written), so that pass 2
+// does no index arithmetic.
 template <class L>
 __device__ __forceinline__ void merge_weights(uint8_t *recv, int C, int nr, float *lse, size_t unit_row0, int k_lo,
-                                              int nq, int S, int q0, int jlim)
+                                              int nq, int S, int q0, int jlim, long long *orow)
 {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    int W = 1;
+    while (W < C) W <<= 1;  // C <= 16, so W <= 16
+    const int per_warp = 32 / W;
+    const int seg = lane / W, c = lane - seg * W;
     const size_t cstride = static_cast<size_t>(nr) * L::kStageStride;
-    for (int rr = warp; rr < nr; rr += kThreads / 32) {
+    // every lane of the warp runs the same number of rounds (shuffles need them all)
+    for (int base = warp * per_warp; base < nr; base += (kThreads / 32) * per_warp) {
+        const int rr = base + seg;
+        const bool row_ok = rr < nr;
         float4 st = make_float4(-INFINITY, 0.f, 0.f, 0.f);
         float *slot = nullptr;
-        if (lane < C) {
-            slot = reinterpret_cast<float *>(recv + lane * cstride + rr * L::kStageStride + kHeadDim * 4);
+        if (row_ok && c < C) {
+            slot = reinterpret_cast<float *>(recv + c * cstride + rr * L::kStageStride + kHeadDim * 4);
             st = *reinterpret_cast<const float4 *>(slot);
         }
         const bool has = st.z > 0.0f;
         float M = has ? st.x : -INFINITY;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+        for (int o = W >> 1; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o, W));
         const float w = has ? ptx::ex2(st.x - M) : 0.0f;
         float LH = st.z * w, Ls = st.y * w;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            LH += __shfl_xor_sync(0xffffffffu, LH, o);
-            Ls += __shfl_xor_sync(0xffffffffu, Ls, o);
+        for (int o = W >> 1; o > 0; o >>= 1) {
+            LH += __shfl_xor_sync(0xffffffffu, LH, o, W);
+            Ls += __shfl_xor_sync(0xffffffffu, Ls, o, W);
         }
-        if (lane < C) slot[3] = w / LH;
-        if (lane == 0 && lse != nullptr && (k_lo + rr) % nq < jlim)
-            lse[block_out_row(unit_row0, k_lo + rr, nq, S, q0)] = (M + ptx::lg2(Ls)) * 0.69314718055994531f;
+        if (slot != nullptr) slot[3] = w / LH;
+        if (row_ok && c == 0) {
+            const bool written = (k_lo + rr) % nq < jlim;
+            const size_t o = block_out_row(unit_row0, k_lo + rr, nq, S, q0);
+            orow[rr] = written ? static_cast<long long>(o) : -1;
+            if (written && lse != nullptr) lse[o] = (M + ptx::lg2(Ls)) * 0.69314718055994531f;
+        }
     }
 }
 
 // Pass 2 (after a CTA barrier): one item per (row, 4-column quad):
-// out = sum_c wn_c O_c with all C loads independent.
+// out = sum_c wn_c O_c, two partials' loads in flight at a time.
 template <class L>
 __device__ __forceinline__ void merge_rows(const uint8_t *recv, int C, int nr, __nv_bfloat16 *out,
-                                           size_t unit_row0, int k_lo, int nq, int S, int q0, int jlim)
+                                           const long long *orow)
 {
     const int items = nr * (kHeadDim / 4);
     const size_t cstride = static_cast<size_t>(nr) * L::kStageStride;
@@ -271,37 +284,36 @@ __device__ __forceinline__ void merge_rows(const uint8_t *recv, int C, int nr, _
         const int rr = i / (kHeadDim / 4), ch = i - rr * (kHeadDim / 4);
         if (threadIdx.x == 0 && trace_n < 2) DM05_TRACE_TILE(4 + trace_n, 22);
         ++trace_n;
-        // only the queries [0, jlim) of each head of the block are written
-        if ((k_lo + rr) % nq >= jlim) continue;
-        const uint8_t *row0 = recv + rr * L::kStageStride;
+        const long long o = orow[rr];
+        if (o < 0) continue;
+        const uint8_t *row = recv + rr * L::kStageStride;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        // four partials at a time: their eight shared-memory loads are
-        // independent and issue back to back (a partial past C reads partial
-        // C - 1 again with weight 0)
-        for (int c0 = 0; c0 < C; c0 += 4) {
-            float wn[4];
-            float4 v[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const uint8_t *row = row0 + min(c0 + k, C - 1) * cstride;
-                wn[k] = *reinterpret_cast<const float *>(row + kHeadDim * 4 + 12);
-                v[k] = *reinterpret_cast<const float4 *>(row + ch * 16);
-            }
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                // a partial without keys (weight 0) may hold anything, NaN included
-                const bool use = c0 + k < C && wn[k] != 0.0f;
-                const float w = use ? wn[k] : 0.0f;
-                acc.x = fmaf(w, use ? v[k].x : 0.0f, acc.x);
-                acc.y = fmaf(w, use ? v[k].y : 0.0f, acc.y);
-                acc.z = fmaf(w, use ? v[k].z : 0.0f, acc.z);
-                acc.w = fmaf(w, use ? v[k].w : 0.0f, acc.w);
-            }
+        // a partial without keys (weight 0) may hold anything, NaN included
+        auto add = [&](float w, const float4 &v) {
+            const bool use = w != 0.0f;
+            const float ww = use ? w : 0.0f;
+            acc.x = fmaf(ww, use ? v.x : 0.0f, acc.x);
+            acc.y = fmaf(ww, use ? v.y : 0.0f, acc.y);
+            acc.z = fmaf(ww, use ? v.z : 0.0f, acc.z);
+            acc.w = fmaf(ww, use ? v.w : 0.0f, acc.w);
+        };
+        int c = 0;
+        for (; c + 2 <= C; c += 2) {
+            const uint8_t *r0 = row + c * cstride, *r1 = r0 + cstride;
+            const float w0 = *reinterpret_cast<const float *>(r0 + kHeadDim * 4 + 12);
+            const float w1 = *reinterpret_cast<const float *>(r1 + kHeadDim * 4 + 12);
+            const float4 v0 = *reinterpret_cast<const float4 *>(r0 + ch * 16);
+            const float4 v1 = *reinterpret_cast<const float4 *>(r1 + ch * 16);
+            add(w0, v0);
+            add(w1, v1);
+        }
+        if (c < C) {
+            const uint8_t *r0 = row + c * cstride;
+            add(*reinterpret_cast<const float *>(r0 + kHeadDim * 4 + 12), *reinterpret_cast<const float4 *>(r0 + ch * 16));
         }
         __nv_bfloat162 h0 = __floats2bfloat162_rn(acc.x, acc.y);
         __nv_bfloat162 h1 = __floats2bfloat162_rn(acc.z, acc.w);
-        const size_t orow = block_out_row(unit_row0, k_lo + rr, nq, S, q0);
-        *reinterpret_cast<uint2 *>(out + orow * kHeadDim + ch * 4) =
+        *reinterpret_cast<uint2 *>(out + static_cast<size_t>(o) * kHeadDim + ch * 4) =
             make_uint2(*reinterpret_cast<uint32_t *>(&h0), *reinterpret_cast<uint32_t *>(&h1));
     }
 }
@@ -922,6 +934,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int r_hi = (NR * (rank + 1)) / C;
         const int nr = r_hi - r_lo;
         uint8_t *recv = smem;  // [C][nr] rows of kStageStride bytes
+        // output row of each merged row (the softmax exchange area is free now;
+        // nr <= NR <= 128 rows)
+        long long *orow_s = reinterpret_cast<long long *>(smem + L::kXchgOff);
         if (nr > 0 && warp == 0) {
             if (lane == 0) ptx::mbar_arrive_expect_tx(&bars[L::kBarMerge], static_cast<uint32_t>(C * nr * L::kStageStride));
             __syncwarp();
@@ -939,11 +954,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             // the host launches clusters of 2..kMaxSplits CTAs; any other
             // size is reported and merges nothing
             if (C <= kMaxSplits) {
-                merge_weights<L>(recv, C, nr, p.lse, unit_row0, r_lo, nq, p.S, q0, jlim);
+                merge_weights<L>(recv, C, nr, p.lse, unit_row0, r_lo, nq, p.S, q0, jlim, orow_s);
                 if (threadIdx.x == 0) DM05_TRACE_TILE(0, 23);
                 __syncthreads();
                 if (threadIdx.x == 0) DM05_TRACE_TILE(1, 23);
-                merge_rows<L>(recv, C, nr, p.out, unit_row0, r_lo, nq, p.S, q0, jlim);
+                merge_rows<L>(recv, C, nr, p.out, orow_s);
                 if (threadIdx.x == 0) DM05_TRACE_TILE(2, 23);
             } else if (threadIdx.x == 0) {
                 atomicOr(p.err, kEwBadSplit);

@@ -597,10 +597,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ptx::tc_fence_after_sync();
                 const uint64_t kdesc = kdesc0 + static_cast<uint64_t>((s * L::kStageBytes) >> 4);
                 const uint32_t d = tmem + kTmemS + sb * NT;
-                // N = the valid keys of the tile rounded up to 16; the
-                // softmax masks every column past the valid ones anyway.
-                const int nv16 = (tile_of<NT>(t_begin + t, TS, klim, p.S).n_valid + 15) / 16 * 16;
-                const uint32_t idesc_qk = ptx::idesc_bf16_f32(kMRows, nv16, false);
+                // N = the whole tile (a compile-time instruction descriptor issues
+                // faster than one built from the tile's valid keys); the softmax
+                // masks every column past the valid ones, NaN rows included
+                constexpr uint32_t idesc_qk = ptx::idesc_bf16_f32(kMRows, NT, false);
 #pragma unroll
                 for (int kk = 0; kk < kHeadDim / 16; ++kk) {
                     // K-major, 128-byte swizzle: 16 elements = 32 bytes along

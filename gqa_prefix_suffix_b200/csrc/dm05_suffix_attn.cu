@@ -1256,8 +1256,13 @@ void dm05_release(void)
 // down + gated residual (five launches on the caller's stream).
 namespace {
 
+// The output projection reads the attention output in place ([B][Hq][S][D]),
+// so its token tiles stay inside one sample (NT tokens of a sample, `tiles`
+// per sample).  u and m are plain [B*S][K] matrices: the GEGLU and the MLP
+// down run over flat tiles of NTf consecutive tokens that may span samples
+// (no padding rows per sample, and 128-token tiles once B*S > 64).
 struct PostPlan {
-    int NT = 64, tiles = 1, ks_o = 1, ks_d = 1;
+    int NT = 64, tiles = 1, NTf = 64, tiles_f = 1, ks_o = 1, ks_d = 1;
     size_t off_part_o = 0, off_h1 = 0, off_u = 0, off_m = 0, off_part_d = 0, total = 0;
 };
 
@@ -1277,11 +1282,14 @@ PostPlan post_plan(int B, int S, int Hq, int D, int Hd, int F, int num_sms)
     pl.tiles = (S + pl.NT - 1) / pl.NT;
     const long long T = static_cast<long long>(B) * S;
     const long long tok_tiles = static_cast<long long>(B) * pl.tiles;
+    pl.NTf = T <= 64 ? 64 : 128;
+    pl.tiles_f = static_cast<int>((T + pl.NTf - 1) / pl.NTf);
     const long long row_tiles = Hd / 128;
     // spread the two long-K projections over about one wave of CTAs
-    const long long want = std::max<long long>(1, num_sms / std::max<long long>(1, row_tiles * tok_tiles));
-    pl.ks_o = split_count(Hq * D / 64, static_cast<int>(std::min<long long>(want, 64)));
-    pl.ks_d = split_count(F / 64, static_cast<int>(std::min<long long>(want, 64)));
+    const long long want_o = std::max<long long>(1, num_sms / std::max<long long>(1, row_tiles * tok_tiles));
+    const long long want_d = std::max<long long>(1, num_sms / std::max<long long>(1, row_tiles * pl.tiles_f));
+    pl.ks_o = split_count(Hq * D / 64, static_cast<int>(std::min<long long>(want_o, 64)));
+    pl.ks_d = split_count(F / 64, static_cast<int>(std::min<long long>(want_d, 64)));
     auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
     size_t o = 0;
     pl.off_part_o = o; o += up(static_cast<size_t>(pl.ks_o) * T * Hd * 4);
@@ -1468,8 +1476,8 @@ int dm05_post_attention(const void *attn, const void *h, const void *scale, cons
     if (encode_2d(&tw_o, wo, static_cast<uint64_t>(A), static_cast<uint64_t>(Hd), 64) != DM05_OK ||
         encode_2d(&tw_gu, wgu, static_cast<uint64_t>(Hd), static_cast<uint64_t>(2) * F, 64) != DM05_OK ||
         encode_2d(&tw_d, wd, static_cast<uint64_t>(F), static_cast<uint64_t>(Hd), 64) != DM05_OK ||
-        encode_act(&tx_a, attn, B, S, A, D, pl.NT) != DM05_OK || encode_act(&tx_u, u, B, S, Hd, Hd, pl.NT) != DM05_OK ||
-        encode_act(&tx_m, m, B, S, F, F, pl.NT) != DM05_OK)
+        encode_act(&tx_a, attn, B, S, A, D, pl.NT) != DM05_OK || encode_act(&tx_u, u, 1, T, Hd, Hd, pl.NTf) != DM05_OK ||
+        encode_act(&tx_m, m, 1, T, F, F, pl.NTf) != DM05_OK)
         return DM05_ERR_CUDA;
 
     dm05::post::GemmParams gp{};
@@ -1502,13 +1510,16 @@ int dm05_post_attention(const void *attn, const void *h, const void *scale, cons
     rp.eps = eps;
     rc = launch_rows(dm05::post::adarms_rows, T, rp, stream);
     if (rc != DM05_OK) return rc;
-    // 3. GEGLU gate-up
+    // 3. GEGLU gate-up, over flat token tiles (one "sample" of T tokens)
     gp.part = nullptr;
     gp.m = m;
     gp.F = F;
     gp.xk_inner = Hd;
     gp.chunks_per_split = Hd / 64;
-    rc = launch_gemm(true, pl.NT, dim3(F / 64, tok_tiles, 1), tw_gu, tx_u, gp, num_sms, stream);
+    gp.S = T;
+    gp.tiles_per_sample = pl.tiles_f;
+    const unsigned flat_tiles = static_cast<unsigned>(pl.tiles_f);
+    rc = launch_gemm(true, pl.NTf, dim3(F / 64, flat_tiles, 1), tw_gu, tx_u, gp, num_sms, stream);
     if (rc != DM05_OK) return rc;
     // 4. MLP down: partial sums over ks_d K ranges
     gp.part = part_d;
@@ -1516,7 +1527,7 @@ int dm05_post_attention(const void *attn, const void *h, const void *scale, cons
     gp.N_rows = Hd;
     gp.xk_inner = F;
     gp.chunks_per_split = F / 64 / pl.ks_d;
-    rc = launch_gemm(false, pl.NT, dim3(Hd / 128, tok_tiles, pl.ks_d), tw_d, tx_m, gp, num_sms, stream);
+    rc = launch_gemm(false, pl.NTf, dim3(Hd / 128, flat_tiles, pl.ks_d), tw_d, tx_m, gp, num_sms, stream);
     if (rc != DM05_OK) return rc;
     // 5. gated residual
     rp.part = part_d;

@@ -58,7 +58,8 @@ struct GemmParams {
     __nv_bfloat16 *m;          // kGeglu: [T][F] bf16
     uint32_t *err;
     int T;                     // tokens (B * S)
-    int S;                     // tokens per sample: a token tile never crosses samples
+    int S;                     // tokens per "sample" of the activation map, which a token tile
+                               // never crosses (the attention output: S; u and m: all T tokens)
     int tiles_per_sample;      // ceil(S / NT)
     int xk_inner;              // K columns per row of the activation map's inner dimension
     int N_rows;                // rows of the weight (kPartial: output features)

@@ -1263,6 +1263,7 @@ namespace {
 // (no padding rows per sample, and 128-token tiles once B*S > 64).
 struct PostPlan {
     int NT = 64, tiles = 1, NTf = 64, tiles_f = 1, ks_o = 1, ks_d = 1;
+    bool geglu64 = false;  // GEGLU on M = 64 tiles: twice the CTAs when the M = 128 grid is under half the SMs
     size_t off_part_o = 0, off_h1 = 0, off_u = 0, off_m = 0, off_part_d = 0, total = 0;
 };
 
@@ -1290,6 +1291,7 @@ PostPlan post_plan(int B, int S, int Hq, int D, int Hd, int F, int num_sms)
     const long long want_d = std::max<long long>(1, num_sms / std::max<long long>(1, row_tiles * pl.tiles_f));
     pl.ks_o = split_count(Hq * D / 64, static_cast<int>(std::min<long long>(want_o, 64)));
     pl.ks_d = split_count(F / 64, static_cast<int>(std::min<long long>(want_d, 64)));
+    pl.geglu64 = 2LL * (F / 64) * pl.tiles_f <= num_sms;
     auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
     size_t o = 0;
     pl.off_part_o = o; o += up(static_cast<size_t>(pl.ks_o) * T * Hd * 4);
@@ -1347,7 +1349,8 @@ struct GemmVariant {
 template <int NT, int EPI, int ST>
 GemmVariant gemm_variant()
 {
-    return {&dm05::post::gemm_kernel<NT, EPI, ST>, dm05::post::GemmSmem<NT, ST>::kAllocBytes};
+    return {&dm05::post::gemm_kernel<NT, EPI, ST>,
+            dm05::post::GemmSmem<NT, ST, EPI == dm05::post::kGeglu64 ? 64 : 128>::kAllocBytes};
 }
 template <int NT, int EPI>
 GemmVariant gemm_variant_depth(bool deep)
@@ -1355,20 +1358,23 @@ GemmVariant gemm_variant_depth(bool deep)
     return deep ? gemm_variant<NT, EPI, dm05::post::deep_stages<NT>()>()
                 : gemm_variant<NT, EPI, dm05::post::shallow_stages<NT>()>();
 }
-GemmVariant gemm_variant_for(bool geglu, int NT, bool deep)
+GemmVariant gemm_variant_for(int epi, int NT, bool deep)
 {
-    if (geglu)
+    if (epi == dm05::post::kGeglu64)
+        return NT == 64 ? gemm_variant_depth<64, dm05::post::kGeglu64>(deep)
+                        : gemm_variant_depth<128, dm05::post::kGeglu64>(deep);
+    if (epi == dm05::post::kGeglu)
         return NT == 64 ? gemm_variant_depth<64, dm05::post::kGeglu>(deep)
                         : gemm_variant_depth<128, dm05::post::kGeglu>(deep);
     return NT == 64 ? gemm_variant_depth<64, dm05::post::kPartial>(deep)
                     : gemm_variant_depth<128, dm05::post::kPartial>(deep);
 }
 
-int launch_gemm(bool geglu, int NT, dim3 grid, const CUtensorMap &tw, const CUtensorMap &tx,
+int launch_gemm(int epi, int NT, dim3 grid, const CUtensorMap &tw, const CUtensorMap &tx,
                 const dm05::post::GemmParams &gp, int num_sms, cudaStream_t stream)
 {
     const long long ctas = static_cast<long long>(grid.x) * grid.y * grid.z;
-    const GemmVariant gv = gemm_variant_for(geglu, NT, ctas <= num_sms);
+    const GemmVariant gv = gemm_variant_for(epi, NT, ctas <= num_sms);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = dim3(dm05::post::kThreads, 1, 1);
@@ -1410,8 +1416,8 @@ int post_device_state(cudaStream_t stream, DeviceState **out)
         if (cs != cudaStreamCaptureStatusNone) return DM05_ERR_WORKSPACE;
         rc = device_state(true, &ds, stream);
         if (rc != DM05_OK) return rc;
-        for (int v = 0; v < 8; ++v) {
-            const GemmVariant gv = gemm_variant_for((v & 1) != 0, (v & 2) ? 128 : 64, (v & 4) != 0);
+        for (int v = 0; v < 12; ++v) {
+            const GemmVariant gv = gemm_variant_for(v % 3, (v / 3) & 1 ? 128 : 64, (v / 6) != 0);
             if (cudaFuncSetAttribute(gv.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, gv.smem) != cudaSuccess)
                 return DM05_ERR_CUDA;
         }
@@ -1474,7 +1480,7 @@ int dm05_post_attention(const void *attn, const void *h, const void *scale, cons
     CUtensorMap tw_o, tw_gu, tw_d, tx_a, tx_u, tx_m;
     const int A = Hq * D;
     if (encode_2d(&tw_o, wo, static_cast<uint64_t>(A), static_cast<uint64_t>(Hd), 64) != DM05_OK ||
-        encode_2d(&tw_gu, wgu, static_cast<uint64_t>(Hd), static_cast<uint64_t>(2) * F, 64) != DM05_OK ||
+        encode_2d(&tw_gu, wgu, static_cast<uint64_t>(Hd), static_cast<uint64_t>(2) * F, pl.geglu64 ? 32 : 64) != DM05_OK ||
         encode_2d(&tw_d, wd, static_cast<uint64_t>(F), static_cast<uint64_t>(Hd), 64) != DM05_OK ||
         encode_act(&tx_a, attn, B, S, A, D, pl.NT) != DM05_OK || encode_act(&tx_u, u, 1, T, Hd, Hd, pl.NTf) != DM05_OK ||
         encode_act(&tx_m, m, 1, T, F, F, pl.NTf) != DM05_OK)
@@ -1491,7 +1497,7 @@ int dm05_post_attention(const void *attn, const void *h, const void *scale, cons
     gp.N_rows = Hd;
     gp.xk_inner = D;
     gp.chunks_per_split = A / 64 / pl.ks_o;
-    rc = launch_gemm(false, pl.NT, dim3(Hd / 128, tok_tiles, pl.ks_o), tw_o, tx_a, gp, num_sms, stream);
+    rc = launch_gemm(dm05::post::kPartial, pl.NT, dim3(Hd / 128, tok_tiles, pl.ks_o), tw_o, tx_a, gp, num_sms, stream);
     if (rc != DM05_OK) return rc;
     // 2. residual, Adarms
     dm05::post::RowParams rp{};
@@ -1519,7 +1525,10 @@ int dm05_post_attention(const void *attn, const void *h, const void *scale, cons
     gp.S = T;
     gp.tiles_per_sample = pl.tiles_f;
     const unsigned flat_tiles = static_cast<unsigned>(pl.tiles_f);
-    rc = launch_gemm(true, pl.NTf, dim3(F / 64, flat_tiles, 1), tw_gu, tx_u, gp, num_sms, stream);
+    if (pl.geglu64)
+        rc = launch_gemm(dm05::post::kGeglu64, pl.NTf, dim3(F / 32, flat_tiles, 1), tw_gu, tx_u, gp, num_sms, stream);
+    else
+        rc = launch_gemm(dm05::post::kGeglu, pl.NTf, dim3(F / 64, flat_tiles, 1), tw_gu, tx_u, gp, num_sms, stream);
     if (rc != DM05_OK) return rc;
     // 4. MLP down: partial sums over ks_d K ranges
     gp.part = part_d;
@@ -1527,7 +1536,7 @@ int dm05_post_attention(const void *attn, const void *h, const void *scale, cons
     gp.N_rows = Hd;
     gp.xk_inner = F;
     gp.chunks_per_split = F / 64 / pl.ks_d;
-    rc = launch_gemm(false, pl.NTf, dim3(Hd / 128, flat_tiles, pl.ks_d), tw_d, tx_m, gp, num_sms, stream);
+    rc = launch_gemm(dm05::post::kPartial, pl.NTf, dim3(Hd / 128, flat_tiles, pl.ks_d), tw_d, tx_m, gp, num_sms, stream);
     if (rc != DM05_OK) return rc;
     // 5. gated residual
     rp.part = part_d;

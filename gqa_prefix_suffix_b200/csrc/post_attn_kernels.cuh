@@ -49,8 +49,9 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr uint32_t kEwTimeout = 0x2u;
 
 enum Epilogue : int {
-    kPartial = 0,  // fp32 partial tile -> part[split][token][row]
-    kGeglu = 1,    // rows: 64 gate + their 64 up rows -> m[token][f] = gelu_tanh(g) * up (bf16)
+    kPartial = 0,   // fp32 partial tile -> part[split][token][row]
+    kGeglu = 1,     // rows: 64 gate + their 64 up rows -> m[token][f] = gelu_tanh(g) * up (bf16)
+    kGeglu64 = 2,   // the same with M = 64: 32 gate + their 32 up rows (twice the CTAs for small grids)
 };
 
 struct GemmParams {
@@ -67,9 +68,9 @@ struct GemmParams {
     int chunks_per_split;      // K chunks each split covers
 };
 
-template <int NT, int STAGES>
+template <int NT, int STAGES, int MR = 128>
 struct GemmSmem {
-    static constexpr int kABytes = 128 * kChunk * 2;
+    static constexpr int kABytes = MR * kChunk * 2;  // MR weight rows of a K chunk
     static constexpr int kBBytes = NT * kChunk * 2;
     static constexpr int kStageBytes = kABytes + kBBytes;
     static constexpr int kStages = STAGES;
@@ -91,7 +92,8 @@ __device__ __forceinline__ float gelu_tanh(float z)
 // grid: x = row tile (128 weight rows), y = token tile (sample y / tiles,
 // its tokens [NT * (y % tiles), +NT)), z = K split.  kPartial: the tile is
 // weight rows [128 x, +128).  kGeglu: the tile is gate rows [64 x, +64)
-// followed by up rows [F + 64 x, +64).  The activation map is 4-D
+// followed by up rows [F + 64 x, +64); kGeglu64: gate rows [32 x, +32) and
+// up rows [F + 32 x, +32), an M = 64 MMA.  The activation map is 4-D
 // [B][K / xk_inner][S][xk_inner]: K column k of token (b, i) sits at
 // (k % xk_inner, i, k / xk_inner, b), which covers both a [B*S][K] matrix
 // (xk_inner = K) and the attention output [B][Hq][S][D] read as the tokens'
@@ -101,7 +103,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
                 const GemmParams p)
 {
-    using L = GemmSmem<NT, STAGES>;
+    constexpr int MR = EPI == kGeglu64 ? 64 : 128;  // MMA rows
+    constexpr int kHalf = MR / 2;                   // rows per weight box (two boxes per chunk)
+    using L = GemmSmem<NT, STAGES, MR>;
     static_assert(NT % 16 == 0 && NT >= 16 && NT <= 256, "N of an M=128 MMA");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -119,8 +123,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int split = blockIdx.z;
     const int c_begin = split * p.chunks_per_split;
     const int n_chunks = p.chunks_per_split;
-    const int row_a = EPI == kGeglu ? 64 * blockIdx.x : 128 * blockIdx.x;
-    const int row_b = EPI == kGeglu ? p.F + 64 * blockIdx.x : row_a + 64;
+    const int row_a = EPI == kPartial ? 128 * blockIdx.x : kHalf * blockIdx.x;
+    const int row_b = EPI == kPartial ? row_a + 64 : p.F + kHalf * blockIdx.x;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -156,14 +160,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int kc = (c_begin + c) * kChunk;
             ptx::mbar_arrive_expect_tx(&full[s], L::kStageBytes);
             ptx::tma_load_2d(a, &tm_w, &full[s], kc, row_a);
-            ptx::tma_load_2d(a + 64 * 128, &tm_w, &full[s], kc, row_b);
+            ptx::tma_load_2d(a + kHalf * 128, &tm_w, &full[s], kc, row_b);
             ptx::tma_load_4d(a + L::kABytes, &tm_x, &full[s], kc % p.xk_inner, i0, kc / p.xk_inner, bs);
         }
         for (int c = (n_chunks > kStages ? n_chunks - kStages : 0); c < n_chunks && !failed; ++c)
             if (!ptx::mbar_wait(&full[c % kStages], (c / kStages) & 1, kWaitLimitNs)) failed = true;
     } else if (warp == 1 && lane == 0) {
         // ------------------------------------------------ MMA issuer
-        constexpr uint32_t idesc = ptx::idesc_bf16_f32(128, NT, false);
+        constexpr uint32_t idesc = ptx::idesc_bf16_f32(MR, NT, false);
         const uint64_t adesc0 = ptx::sw128_desc(ptx::smem_addr(smem), 16, 1024);
         const uint64_t bdesc0 = ptx::sw128_desc(ptx::smem_addr(smem + L::kABytes), 16, 1024);
         bool ok = true;
@@ -205,6 +209,35 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int jj = j * 16 + e;
                 if (jj < n_tok) dst[static_cast<size_t>(jj) * p.N_rows] = __uint_as_float(o[e]);
             }
+        }
+    } else if (EPI == kGeglu64) {
+        // M = 64: tile row i sits in TMEM lane 32 (i / 16) + i % 16, so lanes
+        // 0-15 of warp w hold rows 16 w + lane (rows 0-31: gate rows, 32-63:
+        // the matching up rows).  Each thread then takes two adjacent
+        // features f, f + 1 (f = 32 x + 2 (lane % 16)) for the tokens
+        // t = threadIdx / 16 (mod 8): bf16x2 stores, 64 contiguous bytes per
+        // 16 threads and token.
+        constexpr int kUS = NT + 1;
+        float *rows_s = reinterpret_cast<float *>(smem);  // [64][NT + 1]
+        static_assert(64 * kUS * 4 <= L::kRingBytes, "the gate/up tile reuses the ring");
+#pragma unroll
+        for (int j = 0; j < NT / 16; ++j) {
+            uint32_t o[16];
+            ptx::tmem_ld16(tmem + lane_base + j * 16, o);
+            ptx::tmem_ld_wait();
+            if (lane < 16) {
+#pragma unroll
+                for (int e = 0; e < 16; ++e) rows_s[(16 * warp + lane) * kUS + j * 16 + e] = __uint_as_float(o[e]);
+            }
+        }
+        __syncthreads();
+        const int fl = 2 * (lane & 15);
+        const int f = 32 * blockIdx.x + fl;
+        for (int t = threadIdx.x >> 4; t < n_tok; t += kThreads / 16) {
+            const float g0 = rows_s[fl * kUS + t], g1 = rows_s[(fl + 1) * kUS + t];
+            const float u0 = rows_s[(32 + fl) * kUS + t], u1 = rows_s[(33 + fl) * kUS + t];
+            *reinterpret_cast<__nv_bfloat162 *>(p.m + static_cast<size_t>(tok0 + t) * p.F + f) =
+                __floats2bfloat162_rn(gelu_tanh(g0) * u0, gelu_tanh(g1) * u1);
         }
     } else {
         // lanes 0-63: gate rows, lanes 64-127: the matching up rows.  Every

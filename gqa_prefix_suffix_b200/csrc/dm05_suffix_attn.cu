@@ -1286,11 +1286,17 @@ PostPlan post_plan(int B, int S, int Hq, int D, int Hd, int F, int num_sms)
     pl.NTf = T <= 64 ? 64 : 128;
     pl.tiles_f = static_cast<int>((T + pl.NTf - 1) / pl.NTf);
     const long long row_tiles = Hd / 128;
-    // spread the two long-K projections over about one wave of CTAs
-    const long long want_o = std::max<long long>(1, num_sms / std::max<long long>(1, row_tiles * tok_tiles));
-    const long long want_d = std::max<long long>(1, num_sms / std::max<long long>(1, row_tiles * pl.tiles_f));
-    pl.ks_o = split_count(Hq * D / 64, static_cast<int>(std::min<long long>(want_o, 64)));
-    pl.ks_d = split_count(F / 64, static_cast<int>(std::min<long long>(want_d, 64)));
+    // spread the two long-K projections over about one wave of CTAs: of
+    // one-per-SM CTAs (deep rings) while that needs a split, else of
+    // two-per-SM CTAs (shallow rings) when those would add one
+    auto splits_for = [&](int chunks, long long tiles) {
+        tiles = std::max<long long>(1, tiles);
+        long long want = num_sms / tiles;
+        if (want < 2) want = (2LL * num_sms) / tiles;
+        return split_count(chunks, static_cast<int>(std::max<long long>(1, std::min<long long>(want, 64))));
+    };
+    pl.ks_o = splits_for(Hq * D / 64, row_tiles * tok_tiles);
+    pl.ks_d = splits_for(F / 64, row_tiles * pl.tiles_f);
     pl.geglu64 = 2LL * (F / 64) * pl.tiles_f <= num_sms;
     auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
     size_t o = 0;

@@ -78,7 +78,8 @@ struct Smem {
     static constexpr int kNumBars = 2 * kStages + 1;     // full[s], empty[s], mma done
     static constexpr int kSsOff = kBarOff + kNumBars * 8 + 8;   // own sums [NT], partner's sums [NT]
     static constexpr int kPosOff = kSsOff + 2 * NT * 4;         // the tile's token positions [NT]
-    static constexpr int kTmemSlotOff = kPosOff + NT * 4;
+    static constexpr int kRowOff = (kPosOff + NT * 4 + 7) / 8 * 8;  // each token's output row offset [NT]
+    static constexpr int kTmemSlotOff = kRowOff + NT * 8;
     static constexpr int kEnd = kTmemSlotOff + 16;
     static constexpr int kAllocBytes = kEnd + 1024;
 };
@@ -98,6 +99,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     float *ss_own = reinterpret_cast<float *>(smem + L::kSsOff);
     float *ss_peer = ss_own + NT;  // written by the other half of the head
     int *pos_s = reinterpret_cast<int *>(smem + L::kPosOff);
+    unsigned long long *row_s = reinterpret_cast<unsigned long long *>(smem + L::kRowOff);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kTmemSlotOff);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -263,37 +265,57 @@ __global__ void __launch_bounds__(kThreads, 1)
         inv_freq0 = exp2(-2.0 * static_cast<double>(fa) / static_cast<double>(D) * static_cast<double>(p.log2_theta));
         inv_freq1 = exp2(-2.0 * static_cast<double>(fa + 1) / static_cast<double>(D) * static_cast<double>(p.log2_theta));
     }
-    // the angle reduced to [-pi, pi] in double, then its sine and cosine by
-    // the hardware approximation (absolute error about 2^-21 on [-pi, pi],
-    // far below the bf16 rounding of the result)
-    auto rot = [](double ang, float &sn, float &cs) {
-        const double two_pi = 6.283185307179586, inv_two_pi = 0.15915494309189535;
-        ang = fma(-two_pi, rint(ang * inv_two_pi), ang);
-        __sincosf(static_cast<float>(ang), &sn, &cs);
+    // Angle pos * inv_freq reduced to [-pi, pi] in fp32 without losing the
+    // bits a large position carries: inv_freq is split into two floats, the
+    // product's rounding error is recovered with an fma, and 2 pi is split
+    // into three floats (Cody-Waite) with C1 = 6.28125 exact in few bits, so
+    // that k * C1 and ph - k * C1 are exact for |k| < 2^16.  Worst error over
+    // positions 0..4096 and all D / 2 frequencies (fp32 emulation against
+    // fp64): 2.4e-7 rad.  Sine and cosine by the hardware approximation
+    // (absolute error about 2^-21 on [-pi, pi]), far below the bf16 rounding.
+    const float ih0 = static_cast<float>(inv_freq0), il0 = static_cast<float>(inv_freq0 - static_cast<double>(ih0));
+    const float ih1 = static_cast<float>(inv_freq1), il1 = static_cast<float>(inv_freq1 - static_cast<double>(ih1));
+    auto rot = [](float pos, float ih, float il, float &sn, float &cs) {
+        const float ph = pos * ih;
+        const float pe = fmaf(pos, ih, -ph) + pos * il;  // the product's rounding error, plus the low part
+        const float k = rintf(ph * 0.159154943f);
+        float r = fmaf(-k, 6.28125f, ph);                // exact
+        r = fmaf(-k, 1.935307169e-03f, r);
+        r = fmaf(-k, 1.025313168e-11f, r) + pe;
+        __sincosf(r, &sn, &cs);
     };
     const int n_tok = min(NT, p.T - t0);
+    // per token, once: 1 / rms (in place of the own sums; the other half's
+    // writes ended at the cluster barrier), the position as a float, and the
+    // output row offset
+    float *pos_f = reinterpret_cast<float *>(pos_s);
+    if (threadIdx.x < n_tok) {
+        const int t = threadIdx.x, tok = t0 + t;
+        if (!is_v) ss_own[t] = rsqrtf((ss_own[t] + ss_peer[t]) / static_cast<float>(D) + p.eps);
+        pos_f[t] = static_cast<float>(pos_s[t]);  // exact: positions are below 2^24
+        const int bi = tok / p.S, i = tok - bi * p.S;
+        row_s[t] = ((static_cast<unsigned long long>(bi) * heads + h) * p.S + i) * D;
+    }
+    __syncthreads();
 #pragma unroll 4
     for (int t = warp; t < n_tok; t += kThreads / 32) {
-        const int tok = t0 + t;
         const float ya0 = Y[j0 * L::kYStride + t], ya1 = Y[(j0 + 1) * L::kYStride + t];
         const float yb0 = Y[(64 + j0) * L::kYStride + t], yb1 = Y[(65 + j0) * L::kYStride + t];
         float oa0 = ya0, oa1 = ya1, ob0 = yb0, ob1 = yb1;
         if (!is_v) {
-            const float ms = (ss_own[t] + ss_peer[t]) / static_cast<float>(D);
-            const float inv_rms = rsqrtf(ms + p.eps);
+            const float inv_rms = ss_own[t];
             const float a0 = ya0 * inv_rms * wa0, a1 = ya1 * inv_rms * wa1;
             const float b0 = yb0 * inv_rms * wb0, b1 = yb1 * inv_rms * wb1;
-            const double ps = static_cast<double>(pos_s[t]);
+            const float ps = pos_f[t];
             float sn0, cs0, sn1, cs1;
-            rot(ps * inv_freq0, sn0, cs0);
-            rot(ps * inv_freq1, sn1, cs1);
+            rot(ps, ih0, il0, sn0, cs0);
+            rot(ps, ih1, il1, sn1, cs1);
             oa0 = a0 * cs0 - b0 * sn0;
             ob0 = a0 * sn0 + b0 * cs0;
             oa1 = a1 * cs1 - b1 * sn1;
             ob1 = a1 * sn1 + b1 * cs1;
         }
-        const int bi = tok / p.S, i = tok - bi * p.S;
-        __nv_bfloat16 *row = dst_base + ((static_cast<size_t>(bi) * heads + h) * p.S + i) * D;
+        __nv_bfloat16 *row = dst_base + row_s[t];
         *reinterpret_cast<__nv_bfloat162 *>(row + fa) = __floats2bfloat162_rn(oa0, oa1);
         *reinterpret_cast<__nv_bfloat162 *>(row + fb) = __floats2bfloat162_rn(ob0, ob1);
     }

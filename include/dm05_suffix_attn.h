@@ -278,7 +278,9 @@ int dm05_prefix_prefill_plan(int B, int Hq, int Hkv, int P, int D, int *splits_p
  *   x          bf16  [B*S, H]                  hidden states of the action tokens
  *   w          bf16  [(Hq + 2*Hkv) * D, H]     QKV weight (row-major)
  *   q_norm_w, k_norm_w  bf16 [D]               QK-Norm weights
- *   positions  int32 [B*S]                     RoPE position of each token
+ *   positions  int32 [B*S]                     RoPE position of each token (the angle is
+ *                                              accurate to ~1e-6 rad for positions in
+ *                                              [0, 65536); larger ones lose precision)
  *   q, k, v    bf16  outputs as above
  *   eps > 0, theta > 1                          norm epsilon and RoPE base
  *

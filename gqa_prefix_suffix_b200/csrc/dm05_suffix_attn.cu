@@ -68,22 +68,25 @@ PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 auto *kKernel = &dm05::suffix_attn_kernel<kTileRows, kStages>;
 
 // Prologue variants: token tile NT (64 or 128) x ring depth (deep: one CTA per
-// SM for grids of about one wave; shallow: two per SM for larger grids).
+// SM for grids of about one wave; shallow: two per SM for larger grids), and
+// for small grids 64 feature rows per CTA (four CTAs per head).
 using PrologueFn = void (*)(CUtensorMap, CUtensorMap, dm05::prologue::Params);
 struct PrologueVariant {
     PrologueFn fn;
     int smem;
 };
-template <int NT, int ST>
+template <int NT, int ST, int MR>
 PrologueVariant prologue_variant()
 {
-    return {&dm05::prologue::qkv_prologue_kernel<NT, ST>, dm05::prologue::Smem<NT, ST>::kAllocBytes};
+    return {&dm05::prologue::qkv_prologue_kernel<NT, ST, MR>, dm05::prologue::Smem<NT, ST, MR>::kAllocBytes};
 }
-const PrologueVariant kPrologueVariants[4] = {
-    prologue_variant<64, dm05::prologue::deep_stages<64>()>(),
-    prologue_variant<64, dm05::prologue::shallow_stages<64>()>(),
-    prologue_variant<128, dm05::prologue::deep_stages<128>()>(),
-    prologue_variant<128, dm05::prologue::shallow_stages<128>()>(),
+const PrologueVariant kPrologueVariants[6] = {
+    prologue_variant<64, dm05::prologue::deep_stages<64>(), 128>(),
+    prologue_variant<64, dm05::prologue::shallow_stages<64>(), 128>(),
+    prologue_variant<128, dm05::prologue::deep_stages<128>(), 128>(),
+    prologue_variant<128, dm05::prologue::shallow_stages<128>(), 128>(),
+    prologue_variant<64, dm05::prologue::deep_stages<64, 64>(), 64>(),
+    prologue_variant<128, dm05::prologue::deep_stages<128, 64>(), 64>(),
 };
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -843,9 +846,15 @@ int dm05_suffix_qkv_prologue(const void *x, const void *w, const void *q_norm_w,
     }
     const int NT = small ? 64 : 128;
     const long long ctas = static_cast<long long>(2 * (Hq + 2 * Hkv)) * ((T + NT - 1) / NT);
-    const PrologueVariant &pv = kPrologueVariants[(small ? 0 : 2) + (ctas > 2LL * num_sms ? 1 : 0)];
+    // 64 feature rows per CTA (four per head) when 128-row CTAs would fill
+    // under half the SMs
+    const bool mr64 = 2 * ctas <= num_sms;
+    const int kq = mr64 ? 4 : 2;
+    const PrologueVariant &pv =
+        mr64 ? kPrologueVariants[small ? 4 : 5] : kPrologueVariants[(small ? 0 : 2) + (ctas > 2LL * num_sms ? 1 : 0)];
     CUtensorMap tm_w, tm_x;
-    if (encode_2d(&tm_w, w, static_cast<uint64_t>(H), static_cast<uint64_t>(Hq + 2 * Hkv) * D, 64) != DM05_OK ||
+    if (encode_2d(&tm_w, w, static_cast<uint64_t>(H), static_cast<uint64_t>(Hq + 2 * Hkv) * D, mr64 ? 32 : 64) !=
+            DM05_OK ||
         encode_2d(&tm_x, x, static_cast<uint64_t>(H), static_cast<uint64_t>(T), static_cast<uint32_t>(NT)) != DM05_OK)
         return DM05_ERR_CUDA;
     dm05::prologue::Params pp;
@@ -866,7 +875,7 @@ int dm05_suffix_qkv_prologue(const void *x, const void *w, const void *q_norm_w,
     pp.log2_theta = std::log2(theta);
 
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(2 * (Hq + 2 * Hkv)), static_cast<unsigned>((T + NT - 1) / NT), 1);
+    cfg.gridDim = dim3(static_cast<unsigned>(kq * (Hq + 2 * Hkv)), static_cast<unsigned>((T + NT - 1) / NT), 1);
     cfg.blockDim = dim3(dm05::prologue::kThreads, 1, 1);
     cfg.dynamicSmemBytes = static_cast<size_t>(pv.smem);
     cfg.stream = stream;
@@ -874,7 +883,7 @@ int dm05_suffix_qkv_prologue(const void *x, const void *w, const void *q_norm_w,
     at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     at[0].val.programmaticStreamSerializationAllowed = 1;
     at[1].id = cudaLaunchAttributeClusterDimension;
-    at[1].val.clusterDim.x = 2;  // the two halves of a head
+    at[1].val.clusterDim.x = static_cast<unsigned>(kq);  // the CTAs of a head
     at[1].val.clusterDim.y = 1;
     at[1].val.clusterDim.z = 1;
     cfg.attrs = at;

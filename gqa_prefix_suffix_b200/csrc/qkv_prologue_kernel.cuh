@@ -14,19 +14,21 @@
 // value heads are the plain projection.  Outputs go to q [B,Hq,S,D],
 // k [B,Hkv,S,D], v [B,Hkv,S,D], the layout the suffix attention reads.
 //
-// Design (one CTA = one head half x one tile of NT tokens):
+// Design (one CTA = MR feature rows of a head x one tile of NT tokens):
 //   * Swapped GEMM on tcgen05: D^T[features, tokens] = W_rows x X^T with
-//     M = 128 feature rows (A, K-major from the weight) and N = NT tokens
-//     (B, K-major from the hidden states), K = H in 64-column chunks staged by
-//     TMA (128-byte swizzle) in a ring.  The accumulator lives in TMEM.
-//   * A CTA's 128 feature rows are the two rotation partners of 64 pairs:
-//     features 64c + j (lanes j) and 64c + 128 + j (lanes 64 + j) of its head,
-//     so RoPE needs no data from another CTA.  The two halves of a head form a
-//     cluster of 2 and exchange their per-token sums of squares through
-//     distributed shared memory for the RMS norm.
-//   * Epilogue: TMEM -> shared memory [128][NT] fp32, per-token sums of
-//     squares, the exchange, then each thread produces rotated pairs and
-//     stores bf16 rows (consecutive threads write consecutive features).
+//     M = MR feature rows (A, K-major from the weight; MR = 128, or 64 when
+//     the grid is small, for twice the CTAs) and N = NT tokens (B, K-major
+//     from the hidden states), K = H in 64-column chunks staged by TMA
+//     (128-byte swizzle) in a ring.  The accumulator lives in TMEM.
+//   * A CTA's MR feature rows are the two rotation partners of MR / 2 pairs:
+//     features (MR/2) q + j (rows j) and (MR/2) q + 128 + j (rows MR/2 + j)
+//     of its head, so RoPE needs no data from another CTA.  The 256 / MR CTAs
+//     of a head form a cluster and exchange their per-token sums of squares
+//     through distributed shared memory for the RMS norm.
+//   * Epilogue: TMEM -> shared memory [MR][NT] fp32, per-token sums of
+//     squares, the exchange, per-token 1 / rms and output row, then each
+//     thread produces rotated pairs and stores bf16 (consecutive threads
+//     write consecutive features).
 #pragma once
 
 #include <cstdint>
@@ -44,10 +46,10 @@ constexpr int kThreads = 128;
 // stream's latency covered; shallow (about 96 KB, two CTAs per SM) when
 // the grid spans several waves, so that one CTA's copies overlap the
 // other's epilogue.
-template <int NT>
-constexpr int deep_stages() { return (192 * 1024) / (128 * 128 + NT * 128) > 8 ? 8 : (192 * 1024) / (128 * 128 + NT * 128); }
-template <int NT>
-constexpr int shallow_stages() { return (96 * 1024) / (128 * 128 + NT * 128); }
+template <int NT, int MR = 128>
+constexpr int deep_stages() { return (192 * 1024) / (MR * 128 + NT * 128) > 8 ? 8 : (192 * 1024) / (MR * 128 + NT * 128); }
+template <int NT, int MR = 128>
+constexpr int shallow_stages() { return (96 * 1024) / (MR * 128 + NT * 128); }
 constexpr int kChunk = 64;                 // K columns per stage (128 bytes of bf16)
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr uint32_t kEwTimeout = 0x2u;
@@ -63,50 +65,57 @@ struct Params {
     float log2_theta;          // log2(theta)
 };
 
-template <int NT, int STAGES>
+// MR feature rows per CTA (128, or 64 for small grids: twice the CTAs): the
+// head's D features in 256 / MR CTAs of a cluster.
+template <int NT, int STAGES, int MR = 128>
 struct Smem {
-    static constexpr int kABytes = 128 * kChunk * 2;     // 16 KB: 128 feature rows
+    static constexpr int kQ = 256 / MR;                  // CTAs (quarters or halves) per head
+    static constexpr int kABytes = MR * kChunk * 2;      // MR feature rows of a K chunk
     static constexpr int kBBytes = NT * kChunk * 2;      // NT token rows
     static constexpr int kStageBytes = kABytes + kBBytes;
     static constexpr int kStages = STAGES;
     static constexpr int kRingBytes = kStages * kStageBytes;
     static constexpr int kYStride = NT + 1;              // fp32 per feature row (odd: conflict-free row writes)
-    static constexpr int kYBytes = 128 * kYStride * 4;
+    static constexpr int kYBytes = MR * kYStride * 4;
     // the epilogue tile and the per-group sums of squares reuse the ring
     static_assert(kRingBytes >= kYBytes + kThreads * 4 * 4, "the epilogue tile reuses the ring");
     static constexpr int kBarOff = kRingBytes;
     static constexpr int kNumBars = 2 * kStages + 1;     // full[s], empty[s], mma done
-    static constexpr int kSsOff = kBarOff + kNumBars * 8 + 8;   // own sums [NT], partner's sums [NT]
-    static constexpr int kPosOff = kSsOff + 2 * NT * 4;         // the tile's token positions [NT]
+    static constexpr int kSsOff = kBarOff + kNumBars * 8 + 8;   // every CTA's sums of squares [kQ][NT]
+    static constexpr int kInvOff = kSsOff + kQ * NT * 4;        // 1 / rms per token [NT]
+    static constexpr int kPosOff = kInvOff + NT * 4;            // the tile's token positions [NT]
     static constexpr int kRowOff = (kPosOff + NT * 4 + 7) / 8 * 8;  // each token's output row offset [NT]
     static constexpr int kTmemSlotOff = kRowOff + NT * 8;
     static constexpr int kEnd = kTmemSlotOff + 16;
     static constexpr int kAllocBytes = kEnd + 1024;
 };
 
-template <int NT, int STAGES>
+template <int NT, int STAGES, int MR>
 __global__ void __launch_bounds__(kThreads, 1)
     qkv_prologue_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
                         const Params p)
 {
-    using L = Smem<NT, STAGES>;
+    static_assert(MR == 128 || MR == 64, "128 or 64 feature rows per CTA");
+    using L = Smem<NT, STAGES, MR>;
+    constexpr int kQ = L::kQ;
+    constexpr int kHalf = MR / 2;  // rows per weight box: features [kHalf q, +kHalf) and [128 + kHalf q, +kHalf)
     static_assert(NT % 16 == 0 && NT >= 16 && NT <= 256, "N of an M=128 MMA");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kBarOff);
     constexpr int kStages = L::kStages;
     uint64_t *full = bars, *empty = bars + kStages, *mma_done = bars + 2 * kStages;
-    float *ss_own = reinterpret_cast<float *>(smem + L::kSsOff);
-    float *ss_peer = ss_own + NT;  // written by the other half of the head
+    float *ss_all = reinterpret_cast<float *>(smem + L::kSsOff);  // [kQ][NT]: CTA r's sums at row r
+    float *inv_s = reinterpret_cast<float *>(smem + L::kInvOff);
     int *pos_s = reinterpret_cast<int *>(smem + L::kPosOff);
     unsigned long long *row_s = reinterpret_cast<unsigned long long *>(smem + L::kRowOff);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kTmemSlotOff);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // blockIdx.x = (head * 2 + half); blockIdx.y = token tile.  The two
-    // halves of a head are one cluster of 2.
-    const int half = blockIdx.x & 1;
-    const int hd = blockIdx.x >> 1;
+    // blockIdx.x = (head * kQ + qi); blockIdx.y = token tile.  The kQ CTAs
+    // of a head are one cluster.
+    const int qi = blockIdx.x % kQ;
+    const int hd = blockIdx.x / kQ;
     const int t0 = blockIdx.y * NT;
     const int D = p.D;
     const int n_chunks = p.H / kChunk;
@@ -137,8 +146,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = threadIdx.x - 64; i >= 0 && i < NT; i += kThreads - 64) pos_s[i] = t0 + i < p.T ? p.pos[t0 + i] : 0;
 
     bool failed = false;
-    // feature rows of this CTA: the head's rows [64*half, +64) then [64*half + 128, +64)
-    const int row_a = hd * D + 64 * half;
+    // feature rows of this CTA: the head's rows [kHalf*qi, +kHalf) then [kHalf*qi + 128, +kHalf)
+    const int row_a = hd * D + kHalf * qi;
     if (warp == 0 && lane == 0) {
         // ------------------------------------------------ TMA producer
         for (int c = 0; c < n_chunks; ++c) {
@@ -150,7 +159,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint8_t *a = smem + s * L::kStageBytes;
             ptx::mbar_arrive_expect_tx(&full[s], L::kStageBytes);
             ptx::tma_load_2d(a, &tm_w, &full[s], c * kChunk, row_a);
-            ptx::tma_load_2d(a + 64 * 128, &tm_w, &full[s], c * kChunk, row_a + 128);
+            ptx::tma_load_2d(a + kHalf * 128, &tm_w, &full[s], c * kChunk, row_a + 128);
             ptx::tma_load_2d(a + L::kABytes, &tm_x, &full[s], c * kChunk, t0);
         }
         // drain: every issued copy has landed before the CTA may exit
@@ -158,7 +167,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!ptx::mbar_wait(&full[c % kStages], (c / kStages) & 1, kWaitLimitNs)) failed = true;
     } else if (warp == 1 && lane == 0) {
         // ------------------------------------------------ MMA issuer
-        constexpr uint32_t idesc = ptx::idesc_bf16_f32(128, NT, false);
+        constexpr uint32_t idesc = ptx::idesc_bf16_f32(MR, NT, false);
         const uint64_t adesc0 = ptx::sw128_desc(ptx::smem_addr(smem), 16, 1024);
         const uint64_t bdesc0 = ptx::sw128_desc(ptx::smem_addr(smem + L::kABytes), 16, 1024);
         bool ok = true;
@@ -186,26 +195,31 @@ __global__ void __launch_bounds__(kThreads, 1)
     // all MMAs (and so every stage's copies) complete
     if (!ptx::mbar_wait(mma_done, 0, kWaitLimitNs)) failed = true;
     ptx::tc_fence_after_sync();
-    // TMEM lane = this thread's feature row, columns = tokens
-    float *Y = reinterpret_cast<float *>(smem);  // [128][kYStride]
-    const int r = threadIdx.x;
+    // columns = tokens; M = 128: TMEM lane = tile row; M = 64: tile row i sits
+    // in lane 32 (i / 16) + i % 16 (lanes 0-15 of each warp's quarter)
+    float *Y = reinterpret_cast<float *>(smem);  // [MR][kYStride]
+    const int r = MR == 128 ? threadIdx.x : 16 * warp + lane;
+    const bool holds_row = MR == 128 || lane < 16;
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
 #pragma unroll
     for (int j = 0; j < NT / 16; ++j) {
         uint32_t o[16];
         ptx::tmem_ld16(tmem + lane_base + j * 16, o);
         ptx::tmem_ld_wait();
+        if (holds_row) {
 #pragma unroll
-        for (int e = 0; e < 16; ++e) Y[r * L::kYStride + j * 16 + e] = __uint_as_float(o[e]);
+            for (int e = 0; e < 16; ++e) Y[r * L::kYStride + j * 16 + e] = __uint_as_float(o[e]);
+        }
     }
     __syncthreads();
     if (!is_v) {
-        // per-token sum of squares over this CTA's 128 features: thread
-        // (token t, feature group g) sums 128 / kGroups features with four
+        // per-token sum of squares over this CTA's MR features: thread
+        // (token t, feature group g) sums MR / kGroups features with four
         // independent chains; the groups' sums meet in shared memory, and the
-        // token's total goes to the other half of the head too (cluster of 2)
+        // token's sum goes to every CTA of the head (row qi of ss_all)
         constexpr int kGroups = kThreads / NT > 0 ? kThreads / NT : 1;
-        constexpr int kPer = 128 / kGroups;
+        constexpr int kPer = MR / kGroups;
+        static_assert(kPer % 4 == 0, "four chains");
         float *part = reinterpret_cast<float *>(smem + L::kYBytes);  // [kGroups][NT], after the tile
         for (int idx = threadIdx.x; idx < NT * kGroups; idx += kThreads) {
             const int t = idx % NT, g = idx / NT;
@@ -226,17 +240,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int t = threadIdx.x; t < NT; t += kThreads) {
             float acc = 0.0f;
             for (int g = 0; g < kGroups; ++g) acc += part[g * NT + t];
-            ss_own[t] = acc;
-            ptx::st_dsmem_f32(ptx::mapa(ptx::smem_addr(ss_peer + t), static_cast<uint32_t>(half ^ 1)), acc);
+            ss_all[qi * NT + t] = acc;
+            const uint32_t a = ptx::smem_addr(ss_all + qi * NT + t);
+#pragma unroll
+            for (int rr = 1; rr < kQ; ++rr)
+                ptx::st_dsmem_f32(ptx::mapa(a, static_cast<uint32_t>((qi + rr) % kQ)), acc);
         }
     }
-    ptx::cluster_sync();  // both halves' sums are in place (and no one still writes)
+    ptx::cluster_sync();  // every CTA's sums are in place (and no one still writes)
 
     // each thread: the two adjacent rotation pairs (fa, fa + D/2) and
-    // (fa + 1, fa + 1 + D/2), fa = 64 * half + 2 * lane, for the tokens
-    // t = warp (mod 4): bf16x2 stores, 32 lanes covering 128 contiguous bytes
-    const int j0 = 2 * lane;
-    const int fa = 64 * half + j0;  // feature index within the head (first of the two pairs)
+    // (fa + 1, fa + 1 + D/2), fa = kHalf * qi + j0, for the tokens
+    // t = tg (mod kGroupsT): bf16x2 stores, kTpt threads covering 4 kTpt
+    // contiguous bytes per token and half
+    constexpr int kTpt = kHalf / 2;              // threads per token
+    constexpr int kGroupsT = kThreads / kTpt;    // token groups
+    const int j0 = 2 * (threadIdx.x % kTpt);
+    const int tg = threadIdx.x / kTpt;
+    const int fa = kHalf * qi + j0;  // feature index within the head (first of the two pairs)
     const int fb = fa + D / 2;
     __nv_bfloat16 *dst_base;
     int heads, h;
@@ -285,25 +306,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         __sincosf(r, &sn, &cs);
     };
     const int n_tok = min(NT, p.T - t0);
-    // per token, once: 1 / rms (in place of the own sums; the other half's
-    // writes ended at the cluster barrier), the position as a float, and the
-    // output row offset
+    // per token, once: 1 / rms (every CTA's sums arrived before the cluster
+    // barrier), the position as a float, and the output row offset
     float *pos_f = reinterpret_cast<float *>(pos_s);
     if (threadIdx.x < n_tok) {
         const int t = threadIdx.x, tok = t0 + t;
-        if (!is_v) ss_own[t] = rsqrtf((ss_own[t] + ss_peer[t]) / static_cast<float>(D) + p.eps);
+        if (!is_v) {
+            float tot = 0.0f;
+            for (int rr = 0; rr < kQ; ++rr) tot += ss_all[rr * NT + t];  // the same order in every CTA
+            inv_s[t] = rsqrtf(tot / static_cast<float>(D) + p.eps);
+        }
         pos_f[t] = static_cast<float>(pos_s[t]);  // exact: positions are below 2^24
         const int bi = tok / p.S, i = tok - bi * p.S;
         row_s[t] = ((static_cast<unsigned long long>(bi) * heads + h) * p.S + i) * D;
     }
     __syncthreads();
 #pragma unroll 4
-    for (int t = warp; t < n_tok; t += kThreads / 32) {
+    for (int t = tg; t < n_tok; t += kGroupsT) {
         const float ya0 = Y[j0 * L::kYStride + t], ya1 = Y[(j0 + 1) * L::kYStride + t];
-        const float yb0 = Y[(64 + j0) * L::kYStride + t], yb1 = Y[(65 + j0) * L::kYStride + t];
+        const float yb0 = Y[(kHalf + j0) * L::kYStride + t], yb1 = Y[(kHalf + 1 + j0) * L::kYStride + t];
         float oa0 = ya0, oa1 = ya1, ob0 = yb0, ob1 = yb1;
         if (!is_v) {
-            const float inv_rms = ss_own[t];
+            const float inv_rms = inv_s[t];
             const float a0 = ya0 * inv_rms * wa0, a1 = ya1 * inv_rms * wa1;
             const float b0 = yb0 * inv_rms * wb0, b1 = yb1 * inv_rms * wb1;
             const float ps = pos_f[t];

@@ -240,7 +240,9 @@ def cover_launch():
     already queued when the event fires, so the timed region holds device work
     only, not the host's launch of the first replay."""
     import torch
-    torch.cuda._sleep(100_000)
+    sleep = getattr(torch.cuda, "_sleep", None)
+    if sleep is not None:
+        sleep(100_000)
 
 
 def warm_graphs(graphs, stream, min_passes=3, min_ms=200.0):

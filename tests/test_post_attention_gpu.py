@@ -2,14 +2,20 @@
 Adarms, GEGLU, MLP down + gated residual) against the fp64 oracle, element by
 element.
 
-Tolerance: the kernels accumulate in fp32, but the two GEMM inputs built on
-the way (u, the Adarms output, and m, the GEGLU output) are rounded to bf16
-before their projections (the tensor cores' input type), and out is rounded
-once to bf16.  The rounding of u and m perturbs each projection by about
-2^-9 of its terms' size, spread over their K terms; at the workloads' scale
-(every projection O(1)) this stays below the output rounding.  Bound: every
-element |out - ref| <= 2^-7 |ref| + 1e-2, and the mean error at most twice the
-mean error of the correctly rounded result plus 1e-3."""
+Tolerance, from the kernels' arithmetic: they accumulate in fp32, but the two
+GEMM inputs built on the way -- u (the Adarms output) and m (the GEGLU
+output) -- are rounded to bf16, the tensor cores' input type, and out is
+rounded once to bf16.  Each rounding is an independent error, uniform within
+half a bf16 ulp (variance ulp^2 / 12).  Linearised through the block:
+  Var(dg_f), Var(dup_f) = sum_k W_fk^2 Var(du_k)           (gate and up rows)
+  Var(dm_f) <= 2 (gelu'(g_f) up_f)^2 Var(dg_f) + 2 gelu(g_f)^2 Var(dup_f)
+               + ulp(m_f)^2 / 12                            (2x: their covariance)
+  sigma_ti^2 = gate_i^2 sum_f Wd_if^2 Var(dm_f)
+with g, up, m the exact (fp64) intermediates.  Every element must satisfy
+|out - ref| <= ulp(ref) + 6 sigma_ti + 1e-4 (one output ulp for the final
+rounding, 1e-4 for the fp32 sums), and the mean error must stay within twice
+the mean error of the correctly rounded result plus 1e-3.  Measured on 1.2M
+elements, the largest error minus half an output ulp is 3.6 sigma."""
 import numpy as np
 import pytest
 import torch
@@ -30,6 +36,42 @@ def cuda_ready():
     bd.lib()
 
 
+def bf16_ulp(x):
+    """The bf16 ulp at |x| (8 significant bits)."""
+    e = np.floor(np.log2(np.maximum(np.abs(x), 2.0 ** -126)))
+    return 2.0 ** (e - 7)
+
+
+def _gelu(z):
+    return 0.5 * z * (1.0 + np.tanh(0.7978845608028654 * (z + 0.044715 * z ** 3)))
+
+
+def _gelu_prime(z):
+    k0, k1 = 0.7978845608028654, 0.044715
+    t = np.tanh(k0 * (z + k1 * z ** 3))
+    return 0.5 * (1.0 + t) + 0.5 * z * (1.0 - t * t) * k0 * (1.0 + 3.0 * k1 * z * z)
+
+
+def rounding_sigma(inp, eps=1e-6):
+    """Per-element standard deviation of the error that the bf16 roundings of
+    u and m put into out (the model of the module docstring), from fp64
+    intermediates of the inputs alone."""
+    B, S, Hq, D, Hd, F = inp.B, inp.S, inp.Hq, inp.D, inp.Hd, inp.F
+    T = B * S
+    f = lambda x: x.float().double().numpy()
+    a = f(inp.attn).reshape(B, Hq, S, D).transpose(0, 2, 1, 3).reshape(T, Hq * D)
+    bi = np.repeat(np.arange(B), S)
+    h1 = f(inp.h) + a @ f(inp.wo).T
+    u = h1 / np.sqrt((h1 ** 2).mean(1, keepdims=True) + eps) * (1.0 + f(inp.scale)[bi]) + f(inp.shift)[bi]
+    wgu, wd = f(inp.wgu), f(inp.wd)
+    gu = u @ wgu.T
+    g, up = gu[:, :F], gu[:, F:]
+    var_gu = (bf16_ulp(u) ** 2 / 12.0) @ (wgu ** 2).T
+    var_m = (2.0 * (_gelu_prime(g) * up) ** 2 * var_gu[:, :F] + 2.0 * _gelu(g) ** 2 * var_gu[:, F:]
+             + bf16_ulp(_gelu(g) * up) ** 2 / 12.0)
+    return np.abs(f(inp.gate)[bi]) * np.sqrt(var_m @ (wd ** 2).T)
+
+
 def run_and_check(inp, what):
     d = inp.to("cuda")
     out = bd.post_attention(d.attn, d.h, d.scale, d.shift, d.gate, d.wo, d.wgu, d.wd)
@@ -41,9 +83,11 @@ def run_and_check(inp, what):
     g = out.float().cpu().double().numpy()
     err = np.abs(g - ref)
     floor = np.abs(torch.from_numpy(ref).to(torch.bfloat16).double().numpy() - ref).mean()
-    bound = 2.0 ** -7 * np.abs(ref) + 1e-2
+    sig = rounding_sigma(inp)
+    bound = bf16_ulp(ref) + 6.0 * sig + 1e-4
+    z = np.maximum(err - bf16_ulp(ref) / 2, 0.0) / sig
     print(f"[{what}] max err {err.max():.4g}, mean {err.mean():.4g} (rounding floor {floor:.4g}), "
-          f"max |ref| {np.abs(ref).max():.3g}")
+          f"max |ref| {np.abs(ref).max():.3g}, largest (err - ulp/2) / sigma {z.max():.3g}")
     assert (err <= bound).all(), f"{what}: {int((err > bound).sum())} elements over the bound, max {err.max():.4g}"
     assert err.mean() <= 2.0 * floor + 1e-3, f"{what}: mean err {err.mean():.4g}"
 
@@ -54,6 +98,10 @@ CASES = [
     (2, 7, 2, 128, 256, 320),
     (1, 50, 8, 256, 1024, 4096),
     (3, 70, 4, 64, 256, 512),       # S > 64: two token tiles per sample
+    # grids of several waves: 1200 tokens (the last 128-token tile holding
+    # 48), and 4800 tokens of a narrow MLP (last tile 64 tokens)
+    (24, 50, 8, 256, 1024, 4096),
+    (80, 60, 2, 64, 256, 1024),
 ]
 
 

@@ -1273,6 +1273,7 @@ namespace {
 struct PostPlan {
     int NT = 64, tiles = 1, NTf = 64, tiles_f = 1, ks_o = 1, ks_d = 1;
     bool geglu64 = false;  // GEGLU on M = 64 tiles: twice the CTAs when the M = 128 grid is under half the SMs
+    bool geglu_wide = false;  // and, within one wave, four-chunk stages (512 contiguous bytes per row)
     size_t off_part_o = 0, off_h1 = 0, off_u = 0, off_m = 0, off_part_d = 0, total = 0;
 };
 
@@ -1307,6 +1308,7 @@ PostPlan post_plan(int B, int S, int Hq, int D, int Hd, int F, int num_sms)
     pl.ks_o = splits_for(Hq * D / 64, row_tiles * tok_tiles);
     pl.ks_d = splits_for(F / 64, row_tiles * pl.tiles_f);
     pl.geglu64 = 2LL * (F / 64) * pl.tiles_f <= num_sms;
+    pl.geglu_wide = pl.geglu64 && (F / 32) * pl.tiles_f <= num_sms && Hd % 256 == 0;
     auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
     size_t o = 0;
     pl.off_part_o = o; o += up(static_cast<size_t>(pl.ks_o) * T * Hd * 4);
@@ -1319,6 +1321,36 @@ PostPlan post_plan(int B, int S, int Hq, int D, int Hd, int F, int num_sms)
 }
 
 std::vector<StreamWorkspace> g_post_ws;  // per (device, stream[, thread]) buffers of the post-attention block
+
+// The M = 64 GEGLU's four-chunk stages.  Weight [2F][K] viewed as 5-D
+// (64 columns, row r < F, half h (gate rows / up rows F + r), chunk c of a
+// 256-column group, group g): a box of 64 x 32 x 2 x 4 x 1 lands as four
+// chunk-major blocks of [32 gate rows, then their 32 up rows][128 B].
+int encode_gu_wide(CUtensorMap *map, const void *base, uint64_t K, uint64_t F)
+{
+    cuuint64_t dims[5] = {64, F, 2, 4, K / 256};
+    cuuint64_t strides[4] = {K * 2, F * K * 2, 128, 512};
+    cuuint32_t box[5] = {64, 32, 2, 4, 1};
+    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? DM05_OK : DM05_ERR_CUDA;
+}
+
+// Activation [T][K] viewed as 4-D (64 columns, token, chunk of a 256-column
+// group, group): a box of 64 x NT x 4 x 1 lands as four chunk-major [NT][128 B] blocks.
+int encode_act_wide(CUtensorMap *map, const void *base, uint64_t T, uint64_t K, int NT)
+{
+    cuuint64_t dims[4] = {64, T, 4, K / 256};
+    cuuint64_t strides[3] = {K * 2, 128, 512};
+    cuuint32_t box[4] = {64, static_cast<cuuint32_t>(NT), 4, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? DM05_OK : DM05_ERR_CUDA;
+}
 
 // activation viewed as 4-D [B][K / inner][S][inner]; boxes of 64 x NT x 1 x 1
 int encode_act(CUtensorMap *map, const void *base, int B, int S, int K, int inner, int NT)
@@ -1361,11 +1393,18 @@ struct GemmVariant {
     GemmFn fn;
     int smem;
 };
-template <int NT, int EPI, int ST>
+template <int NT, int EPI, int ST, int W = 1>
 GemmVariant gemm_variant()
 {
-    return {&dm05::post::gemm_kernel<NT, EPI, ST>,
-            dm05::post::GemmSmem<NT, ST, EPI == dm05::post::kGeglu64 ? 64 : 128>::kAllocBytes};
+    return {&dm05::post::gemm_kernel<NT, EPI, ST, W>,
+            dm05::post::GemmSmem<NT, ST, EPI == dm05::post::kGeglu64 ? 64 : 128, W>::kAllocBytes};
+}
+// the M = 64 GEGLU with four-chunk stages (one wave, deep ring)
+template <int NT>
+GemmVariant geglu64_wide_variant()
+{
+    constexpr int kSt = (192 * 1024) / (4 * (64 * 128 + NT * 128));
+    return gemm_variant<NT, dm05::post::kGeglu64, kSt, 4>();
 }
 template <int NT, int EPI>
 GemmVariant gemm_variant_depth(bool deep)
@@ -1386,10 +1425,13 @@ GemmVariant gemm_variant_for(int epi, int NT, bool deep)
 }
 
 int launch_gemm(int epi, int NT, dim3 grid, const CUtensorMap &tw, const CUtensorMap &tx,
-                const dm05::post::GemmParams &gp, int num_sms, cudaStream_t stream)
+                const dm05::post::GemmParams &gp, int num_sms, cudaStream_t stream, bool wide = false)
 {
     const long long ctas = static_cast<long long>(grid.x) * grid.y * grid.z;
-    const GemmVariant gv = gemm_variant_for(epi, NT, ctas <= num_sms);
+    // wide: the M = 64 GEGLU in four-chunk stages
+    const GemmVariant gv = !wide      ? gemm_variant_for(epi, NT, ctas <= num_sms)
+                           : NT == 64 ? geglu64_wide_variant<64>()
+                                      : geglu64_wide_variant<128>();
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = dim3(dm05::post::kThreads, 1, 1);
@@ -1431,8 +1473,10 @@ int post_device_state(cudaStream_t stream, DeviceState **out)
         if (cs != cudaStreamCaptureStatusNone) return DM05_ERR_WORKSPACE;
         rc = device_state(true, &ds, stream);
         if (rc != DM05_OK) return rc;
-        for (int v = 0; v < 12; ++v) {
-            const GemmVariant gv = gemm_variant_for(v % 3, (v / 3) & 1 ? 128 : 64, (v / 6) != 0);
+        for (int v = 0; v < 14; ++v) {
+            const GemmVariant gv = v < 12    ? gemm_variant_for(v % 3, (v / 3) & 1 ? 128 : 64, (v / 6) != 0)
+                                 : v == 12 ? geglu64_wide_variant<64>()
+                                           : geglu64_wide_variant<128>();
             if (cudaFuncSetAttribute(gv.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, gv.smem) != cudaSuccess)
                 return DM05_ERR_CUDA;
         }
@@ -1495,9 +1539,13 @@ int dm05_post_attention(const void *attn, const void *h, const void *scale, cons
     CUtensorMap tw_o, tw_gu, tw_d, tx_a, tx_u, tx_m;
     const int A = Hq * D;
     if (encode_2d(&tw_o, wo, static_cast<uint64_t>(A), static_cast<uint64_t>(Hd), 64) != DM05_OK ||
-        encode_2d(&tw_gu, wgu, static_cast<uint64_t>(Hd), static_cast<uint64_t>(2) * F, pl.geglu64 ? 32 : 64) != DM05_OK ||
+        (pl.geglu_wide ? encode_gu_wide(&tw_gu, wgu, static_cast<uint64_t>(Hd), static_cast<uint64_t>(F))
+                       : encode_2d(&tw_gu, wgu, static_cast<uint64_t>(Hd), static_cast<uint64_t>(2) * F,
+                                   pl.geglu64 ? 32 : 64)) != DM05_OK ||
         encode_2d(&tw_d, wd, static_cast<uint64_t>(F), static_cast<uint64_t>(Hd), 64) != DM05_OK ||
-        encode_act(&tx_a, attn, B, S, A, D, pl.NT) != DM05_OK || encode_act(&tx_u, u, 1, T, Hd, Hd, pl.NTf) != DM05_OK ||
+        encode_act(&tx_a, attn, B, S, A, D, pl.NT) != DM05_OK ||
+        (pl.geglu_wide ? encode_act_wide(&tx_u, u, static_cast<uint64_t>(T), static_cast<uint64_t>(Hd), pl.NTf)
+                       : encode_act(&tx_u, u, 1, T, Hd, Hd, pl.NTf)) != DM05_OK ||
         encode_act(&tx_m, m, 1, T, F, F, pl.NTf) != DM05_OK)
         return DM05_ERR_CUDA;
 
@@ -1541,7 +1589,8 @@ int dm05_post_attention(const void *attn, const void *h, const void *scale, cons
     gp.tiles_per_sample = pl.tiles_f;
     const unsigned flat_tiles = static_cast<unsigned>(pl.tiles_f);
     if (pl.geglu64)
-        rc = launch_gemm(dm05::post::kGeglu64, pl.NTf, dim3(F / 32, flat_tiles, 1), tw_gu, tx_u, gp, num_sms, stream);
+        rc = launch_gemm(dm05::post::kGeglu64, pl.NTf, dim3(F / 32, flat_tiles, 1), tw_gu, tx_u, gp, num_sms, stream,
+                         pl.geglu_wide);
     else
         rc = launch_gemm(dm05::post::kGeglu, pl.NTf, dim3(F / 64, flat_tiles, 1), tw_gu, tx_u, gp, num_sms, stream);
     if (rc != DM05_OK) return rc;

@@ -68,10 +68,13 @@ struct GemmParams {
     int chunks_per_split;      // K chunks each split covers
 };
 
-template <int NT, int STAGES, int MR = 128>
+// W = K chunks per ring stage: 1, or 4 (boxes of four chunks: each weight
+// and activation row is read as 512 contiguous bytes, landing as four
+// chunk-major [rows][128 B] blocks)
+template <int NT, int STAGES, int MR = 128, int W = 1>
 struct GemmSmem {
-    static constexpr int kABytes = MR * kChunk * 2;  // MR weight rows of a K chunk
-    static constexpr int kBBytes = NT * kChunk * 2;
+    static constexpr int kABytes = W * MR * kChunk * 2;  // MR weight rows of W K chunks
+    static constexpr int kBBytes = W * NT * kChunk * 2;
     static constexpr int kStageBytes = kABytes + kBBytes;
     static constexpr int kStages = STAGES;
     static constexpr int kRingBytes = kStages * kStageBytes;
@@ -98,14 +101,19 @@ __device__ __forceinline__ float gelu_tanh(float z)
 // (k % xk_inner, i, k / xk_inner, b), which covers both a [B*S][K] matrix
 // (xk_inner = K) and the attention output [B][Hq][S][D] read as the tokens'
 // heads concatenated (xk_inner = D).
-template <int NT, int EPI, int STAGES>
+// W = 4 (the M = 64 GEGLU within one wave): per stage one 5-D weight box
+// [4 chunks][gate, up][32 rows][64] and one 4-D activation box [4 chunks][NT
+// tokens][64] of the flat [T][K] map (tm_w and tm_x then use those views):
+// each weight and activation row is read as 512 contiguous bytes.
+template <int NT, int EPI, int STAGES, int W = 1>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
                 const GemmParams p)
 {
     constexpr int MR = EPI == kGeglu64 ? 64 : 128;  // MMA rows
     constexpr int kHalf = MR / 2;                   // rows per weight box (two boxes per chunk)
-    using L = GemmSmem<NT, STAGES, MR>;
+    static_assert(W == 1 || (W == 4 && EPI == kGeglu64), "four-chunk stages: the M = 64 GEGLU");
+    using L = GemmSmem<NT, STAGES, MR, W>;
     static_assert(NT % 16 == 0 && NT >= 16 && NT <= 256, "N of an M=128 MMA");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -122,7 +130,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int n_tok = min(NT, p.S - i0);                           // valid tokens of the tile
     const int split = blockIdx.z;
     const int c_begin = split * p.chunks_per_split;
-    const int n_chunks = p.chunks_per_split;
+    const int n_chunks = p.chunks_per_split / W;  // ring stages to stream (the host checks the division)
     const int row_a = EPI == kPartial ? 128 * blockIdx.x : kHalf * blockIdx.x;
     const int row_b = EPI == kPartial ? row_a + 64 : p.F + kHalf * blockIdx.x;
 
@@ -157,11 +165,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             }
             uint8_t *a = smem + s * L::kStageBytes;
-            const int kc = (c_begin + c) * kChunk;
             ptx::mbar_arrive_expect_tx(&full[s], L::kStageBytes);
-            ptx::tma_load_2d(a, &tm_w, &full[s], kc, row_a);
-            ptx::tma_load_2d(a + kHalf * 128, &tm_w, &full[s], kc, row_b);
-            ptx::tma_load_4d(a + L::kABytes, &tm_x, &full[s], kc % p.xk_inner, i0, kc / p.xk_inner, bs);
+            if constexpr (W == 4) {
+                // group g = K columns [256 g, +256): gate rows [32 x, +32) and
+                // their up rows (the 5-D view's half dimension), NT tokens
+                const int g = (c_begin / 4) + c;
+                ptx::tma_load_5d(a, &tm_w, &full[s], 0, kHalf * static_cast<int>(blockIdx.x), 0, 0, g);
+                ptx::tma_load_4d(a + L::kABytes, &tm_x, &full[s], 0, tok0, 0, g);
+            } else {
+                const int kc = (c_begin + c) * kChunk;
+                ptx::tma_load_2d(a, &tm_w, &full[s], kc, row_a);
+                ptx::tma_load_2d(a + kHalf * 128, &tm_w, &full[s], kc, row_b);
+                ptx::tma_load_4d(a + L::kABytes, &tm_x, &full[s], kc % p.xk_inner, i0, kc / p.xk_inner, bs);
+            }
         }
         for (int c = (n_chunks > kStages ? n_chunks - kStages : 0); c < n_chunks && !failed; ++c)
             if (!ptx::mbar_wait(&full[c % kStages], (c / kStages) & 1, kWaitLimitNs)) failed = true;
@@ -180,10 +196,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::tc_fence_after_sync();
             const uint64_t so = static_cast<uint64_t>((s * L::kStageBytes) >> 4);
 #pragma unroll
-            for (int kk = 0; kk < kChunk / 16; ++kk)
-                ptx::mma_bf16_ss(tmem, adesc0 + so + static_cast<uint64_t>((kk * 32) >> 4),
-                                 bdesc0 + so + static_cast<uint64_t>((kk * 32) >> 4), idesc,
-                                 (c > 0 || kk > 0) ? 1u : 0u);
+            for (int w = 0; w < W; ++w) {
+                // chunk w of the stage: [MR rows][128 B] and [NT rows][128 B] blocks
+                const uint64_t ao = so + static_cast<uint64_t>((w * MR * 128) >> 4);
+                const uint64_t bo = so + static_cast<uint64_t>((w * NT * 128) >> 4);
+#pragma unroll
+                for (int kk = 0; kk < kChunk / 16; ++kk)
+                    ptx::mma_bf16_ss(tmem, adesc0 + ao + static_cast<uint64_t>((kk * 32) >> 4),
+                                     bdesc0 + bo + static_cast<uint64_t>((kk * 32) >> 4), idesc,
+                                     (c > 0 || w > 0 || kk > 0) ? 1u : 0u);
+            }
             ptx::mma_commit(&empty[s]);
         }
         ptx::mma_commit(mma_done);

@@ -98,6 +98,11 @@ CASES = [
     (2, 7, 2, 128, 256, 320),
     (1, 50, 8, 256, 1024, 4096),
     (3, 70, 4, 64, 256, 512),       # S > 64: two token tiles per sample
+    # one-wave grids: 100 tokens in one 128-token tile (GEGLU on M = 64 in
+    # four-chunk stages, the ring wrapping over four 256-column groups), and
+    # F = 8192 (GEGLU on M = 128, MLP down split 16 ways of 8 chunks)
+    (1, 100, 8, 256, 1024, 2048),
+    (1, 64, 8, 256, 1024, 8192),
     # grids of several waves: 1200 tokens (the last 128-token tile holding
     # 48), and 4800 tokens of a narrow MLP (last tile 64 tokens)
     (24, 50, 8, 256, 1024, 4096),

@@ -75,18 +75,23 @@ struct PrologueVariant {
     PrologueFn fn;
     int smem;
 };
-template <int NT, int ST, int MR>
+template <int NT, int ST, int MR, int W = 1>
 PrologueVariant prologue_variant()
 {
-    return {&dm05::prologue::qkv_prologue_kernel<NT, ST, MR>, dm05::prologue::Smem<NT, ST, MR>::kAllocBytes};
+    return {&dm05::prologue::qkv_prologue_kernel<NT, ST, MR, W>, dm05::prologue::Smem<NT, ST, MR, W>::kAllocBytes};
 }
-const PrologueVariant kPrologueVariants[6] = {
+// the 64-row CTAs in four-chunk stages (one wave, about 192 KB of ring)
+template <int NT>
+constexpr int wide_stages() { return (192 * 1024) / (4 * (64 * 128 + NT * 128)); }
+const PrologueVariant kPrologueVariants[8] = {
     prologue_variant<64, dm05::prologue::deep_stages<64>(), 128>(),
     prologue_variant<64, dm05::prologue::shallow_stages<64>(), 128>(),
     prologue_variant<128, dm05::prologue::deep_stages<128>(), 128>(),
     prologue_variant<128, dm05::prologue::shallow_stages<128>(), 128>(),
     prologue_variant<64, dm05::prologue::deep_stages<64, 64>(), 64>(),
     prologue_variant<128, dm05::prologue::deep_stages<128, 64>(), 64>(),
+    prologue_variant<64, wide_stages<64>(), 64, 4>(),
+    prologue_variant<128, wide_stages<128>(), 64, 4>(),
 };
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -521,6 +526,41 @@ int encode_2d(CUtensorMap *map, const void *base, uint64_t cols, uint64_t rows, 
     return r == CUDA_SUCCESS ? DM05_OK : DM05_ERR_CUDA;
 }
 
+// Four-chunk ring stages read 256 columns of a row at once (512 contiguous
+// bytes) and land them as four chunk-major [box rows][128 B] blocks with
+// 128-byte swizzle, the layout the tensor-core descriptors read.
+//
+// Row-major bf16 [rows][K] viewed as 4-D (64 columns, row, 64-column chunk
+// of a 256-column group, group): boxes of 64 x box_rows x 4 x 1.
+int encode_wide4(CUtensorMap *map, const void *base, uint64_t rows, uint64_t K, uint32_t box_rows)
+{
+    cuuint64_t dims[4] = {64, rows, 4, K / 256};
+    cuuint64_t strides[3] = {K * 2, 128, 512};
+    cuuint32_t box[4] = {64, box_rows, 4, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? DM05_OK : DM05_ERR_CUDA;
+}
+
+// Row-major bf16 [rows][K] viewed as 5-D (64 columns, row r, pair half h --
+// row r or row r + pair --, chunk, group): a box of 64 x box_rows x 2 x 4 x 1
+// lands as four chunk-major blocks of [box_rows rows r, then their rows
+// r + pair][128 B] (the GEGLU's gate and up rows, the prologue's rotation
+// partners).  The row extent is rows - pair, so no box reaches past the matrix.
+int encode_pair5(CUtensorMap *map, const void *base, uint64_t rows, uint64_t K, uint64_t pair, uint32_t box_rows)
+{
+    cuuint64_t dims[5] = {64, rows - pair, 2, 4, K / 256};
+    cuuint64_t strides[4] = {K * 2, pair * K * 2, 128, 512};
+    cuuint32_t box[5] = {64, box_rows, 2, 4, 1};
+    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? DM05_OK : DM05_ERR_CUDA;
+}
+
 // Encodes the tensor maps and launches the kernel with plan `pl` on
 // `stream`; `err` is the device error word, `part` the partial-result area
 // (unused when pl.splits == 1).  Sizes and pointers are already checked.
@@ -849,14 +889,26 @@ int dm05_suffix_qkv_prologue(const void *x, const void *w, const void *q_norm_w,
     // 64 feature rows per CTA (four per head) when 128-row CTAs would fill
     // under half the SMs
     const bool mr64 = 2 * ctas <= num_sms;
+    // those in four-chunk stages when H is a whole number of 256-column groups
+    const bool wide = mr64 && H % 256 == 0;
     const int kq = mr64 ? 4 : 2;
     const PrologueVariant &pv =
-        mr64 ? kPrologueVariants[small ? 4 : 5] : kPrologueVariants[(small ? 0 : 2) + (ctas > 2LL * num_sms ? 1 : 0)];
+        wide   ? kPrologueVariants[small ? 6 : 7]
+        : mr64 ? kPrologueVariants[small ? 4 : 5]
+               : kPrologueVariants[(small ? 0 : 2) + (ctas > 2LL * num_sms ? 1 : 0)];
     CUtensorMap tm_w, tm_x;
-    if (encode_2d(&tm_w, w, static_cast<uint64_t>(H), static_cast<uint64_t>(Hq + 2 * Hkv) * D, mr64 ? 32 : 64) !=
-            DM05_OK ||
-        encode_2d(&tm_x, x, static_cast<uint64_t>(H), static_cast<uint64_t>(T), static_cast<uint32_t>(NT)) != DM05_OK)
+    const uint64_t w_rows = static_cast<uint64_t>(Hq + 2 * Hkv) * D;
+    if (wide) {
+        // the partner of feature row r is row r + 128 (D = 256)
+        if (encode_pair5(&tm_w, w, w_rows, static_cast<uint64_t>(H), 128, 32) != DM05_OK ||
+            encode_wide4(&tm_x, x, static_cast<uint64_t>(T), static_cast<uint64_t>(H), static_cast<uint32_t>(NT)) !=
+                DM05_OK)
+            return DM05_ERR_CUDA;
+    } else if (encode_2d(&tm_w, w, static_cast<uint64_t>(H), w_rows, mr64 ? 32 : 64) != DM05_OK ||
+               encode_2d(&tm_x, x, static_cast<uint64_t>(H), static_cast<uint64_t>(T), static_cast<uint32_t>(NT)) !=
+                   DM05_OK) {
         return DM05_ERR_CUDA;
+    }
     dm05::prologue::Params pp;
     pp.qw = static_cast<const __nv_bfloat16 *>(q_norm_w);
     pp.kw = static_cast<const __nv_bfloat16 *>(k_norm_w);
@@ -1322,36 +1374,6 @@ PostPlan post_plan(int B, int S, int Hq, int D, int Hd, int F, int num_sms)
 
 std::vector<StreamWorkspace> g_post_ws;  // per (device, stream[, thread]) buffers of the post-attention block
 
-// The M = 64 GEGLU's four-chunk stages.  Weight [2F][K] viewed as 5-D
-// (64 columns, row r < F, half h (gate rows / up rows F + r), chunk c of a
-// 256-column group, group g): a box of 64 x 32 x 2 x 4 x 1 lands as four
-// chunk-major blocks of [32 gate rows, then their 32 up rows][128 B].
-int encode_gu_wide(CUtensorMap *map, const void *base, uint64_t K, uint64_t F)
-{
-    cuuint64_t dims[5] = {64, F, 2, 4, K / 256};
-    cuuint64_t strides[4] = {K * 2, F * K * 2, 128, 512};
-    cuuint32_t box[5] = {64, 32, 2, 4, 1};
-    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(base), dims, strides, box, estr,
-                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? DM05_OK : DM05_ERR_CUDA;
-}
-
-// Activation [T][K] viewed as 4-D (64 columns, token, chunk of a 256-column
-// group, group): a box of 64 x NT x 4 x 1 lands as four chunk-major [NT][128 B] blocks.
-int encode_act_wide(CUtensorMap *map, const void *base, uint64_t T, uint64_t K, int NT)
-{
-    cuuint64_t dims[4] = {64, T, 4, K / 256};
-    cuuint64_t strides[3] = {K * 2, 128, 512};
-    cuuint32_t box[4] = {64, static_cast<cuuint32_t>(NT), 4, 1};
-    cuuint32_t estr[4] = {1, 1, 1, 1};
-    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, estr,
-                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? DM05_OK : DM05_ERR_CUDA;
-}
-
 // activation viewed as 4-D [B][K / inner][S][inner]; boxes of 64 x NT x 1 x 1
 int encode_act(CUtensorMap *map, const void *base, int B, int S, int K, int inner, int NT)
 {
@@ -1539,12 +1561,14 @@ int dm05_post_attention(const void *attn, const void *h, const void *scale, cons
     CUtensorMap tw_o, tw_gu, tw_d, tx_a, tx_u, tx_m;
     const int A = Hq * D;
     if (encode_2d(&tw_o, wo, static_cast<uint64_t>(A), static_cast<uint64_t>(Hd), 64) != DM05_OK ||
-        (pl.geglu_wide ? encode_gu_wide(&tw_gu, wgu, static_cast<uint64_t>(Hd), static_cast<uint64_t>(F))
+        (pl.geglu_wide ? encode_pair5(&tw_gu, wgu, static_cast<uint64_t>(2) * F, static_cast<uint64_t>(Hd),
+                                      static_cast<uint64_t>(F), 32)
                        : encode_2d(&tw_gu, wgu, static_cast<uint64_t>(Hd), static_cast<uint64_t>(2) * F,
                                    pl.geglu64 ? 32 : 64)) != DM05_OK ||
         encode_2d(&tw_d, wd, static_cast<uint64_t>(F), static_cast<uint64_t>(Hd), 64) != DM05_OK ||
         encode_act(&tx_a, attn, B, S, A, D, pl.NT) != DM05_OK ||
-        (pl.geglu_wide ? encode_act_wide(&tx_u, u, static_cast<uint64_t>(T), static_cast<uint64_t>(Hd), pl.NTf)
+        (pl.geglu_wide ? encode_wide4(&tx_u, u, static_cast<uint64_t>(T), static_cast<uint64_t>(Hd),
+                                      static_cast<uint32_t>(pl.NTf))
                        : encode_act(&tx_u, u, 1, T, Hd, Hd, pl.NTf)) != DM05_OK ||
         encode_act(&tx_m, m, 1, T, F, F, pl.NTf) != DM05_OK)
         return DM05_ERR_CUDA;

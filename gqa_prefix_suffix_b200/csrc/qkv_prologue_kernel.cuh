@@ -67,11 +67,13 @@ struct Params {
 
 // MR feature rows per CTA (128, or 64 for small grids: twice the CTAs): the
 // head's D features in 256 / MR CTAs of a cluster.
-template <int NT, int STAGES, int MR = 128>
+// W = K chunks per ring stage: 1, or 4 (one box of four chunks for each
+// operand: every weight and token row read as 512 contiguous bytes)
+template <int NT, int STAGES, int MR = 128, int W = 1>
 struct Smem {
     static constexpr int kQ = 256 / MR;                  // CTAs (quarters or halves) per head
-    static constexpr int kABytes = MR * kChunk * 2;      // MR feature rows of a K chunk
-    static constexpr int kBBytes = NT * kChunk * 2;      // NT token rows
+    static constexpr int kABytes = W * MR * kChunk * 2;  // MR feature rows of W K chunks
+    static constexpr int kBBytes = W * NT * kChunk * 2;  // NT token rows
     static constexpr int kStageBytes = kABytes + kBBytes;
     static constexpr int kStages = STAGES;
     static constexpr int kRingBytes = kStages * kStageBytes;
@@ -90,13 +92,18 @@ struct Smem {
     static constexpr int kAllocBytes = kEnd + 1024;
 };
 
-template <int NT, int STAGES, int MR>
+// W = 4: tm_w is the 5-D view (64 columns, row, partner half -- row + 128 --,
+// chunk of a 256-column group, group) with boxes of 64 x MR/2 x 2 x 4 x 1,
+// and tm_x the 4-D view (64 columns, token, chunk, group) with boxes of
+// 64 x NT x 4 x 1: each lands as four chunk-major [rows][128 B] blocks.
+template <int NT, int STAGES, int MR, int W = 1>
 __global__ void __launch_bounds__(kThreads, 1)
     qkv_prologue_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
                         const Params p)
 {
     static_assert(MR == 128 || MR == 64, "128 or 64 feature rows per CTA");
-    using L = Smem<NT, STAGES, MR>;
+    static_assert(W == 1 || W == 4, "one or four K chunks per stage");
+    using L = Smem<NT, STAGES, MR, W>;
     constexpr int kQ = L::kQ;
     constexpr int kHalf = MR / 2;  // rows per weight box: features [kHalf q, +kHalf) and [128 + kHalf q, +kHalf)
     static_assert(NT % 16 == 0 && NT >= 16 && NT <= 256, "N of an M=128 MMA");
@@ -118,7 +125,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int hd = blockIdx.x / kQ;
     const int t0 = blockIdx.y * NT;
     const int D = p.D;
-    const int n_chunks = p.H / kChunk;
+    const int n_chunks = p.H / kChunk / W;  // ring stages to stream (W = 4: the host checks H % 256)
     const bool is_v = hd >= p.Hq + p.Hkv;
 
     if (threadIdx.x == 0) {
@@ -158,9 +165,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             uint8_t *a = smem + s * L::kStageBytes;
             ptx::mbar_arrive_expect_tx(&full[s], L::kStageBytes);
-            ptx::tma_load_2d(a, &tm_w, &full[s], c * kChunk, row_a);
-            ptx::tma_load_2d(a + kHalf * 128, &tm_w, &full[s], c * kChunk, row_a + 128);
-            ptx::tma_load_2d(a + L::kABytes, &tm_x, &full[s], c * kChunk, t0);
+            if constexpr (W == 4) {
+                ptx::tma_load_5d(a, &tm_w, &full[s], 0, row_a, 0, 0, c);
+                ptx::tma_load_4d(a + L::kABytes, &tm_x, &full[s], 0, t0, 0, c);
+            } else {
+                ptx::tma_load_2d(a, &tm_w, &full[s], c * kChunk, row_a);
+                ptx::tma_load_2d(a + kHalf * 128, &tm_w, &full[s], c * kChunk, row_a + 128);
+                ptx::tma_load_2d(a + L::kABytes, &tm_x, &full[s], c * kChunk, t0);
+            }
         }
         // drain: every issued copy has landed before the CTA may exit
         for (int c = (n_chunks > kStages ? n_chunks - kStages : 0); c < n_chunks && !failed; ++c)
@@ -180,10 +192,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::tc_fence_after_sync();
             const uint64_t so = static_cast<uint64_t>((s * L::kStageBytes) >> 4);
 #pragma unroll
-            for (int kk = 0; kk < kChunk / 16; ++kk)
-                ptx::mma_bf16_ss(tmem, adesc0 + so + static_cast<uint64_t>((kk * 32) >> 4),
-                                 bdesc0 + so + static_cast<uint64_t>((kk * 32) >> 4), idesc,
-                                 (c > 0 || kk > 0) ? 1u : 0u);
+            for (int w = 0; w < W; ++w) {
+                // chunk w of the stage: [MR rows][128 B] and [NT rows][128 B] blocks
+                const uint64_t ao = so + static_cast<uint64_t>((w * MR * 128) >> 4);
+                const uint64_t bo = so + static_cast<uint64_t>((w * NT * 128) >> 4);
+#pragma unroll
+                for (int kk = 0; kk < kChunk / 16; ++kk)
+                    ptx::mma_bf16_ss(tmem, adesc0 + ao + static_cast<uint64_t>((kk * 32) >> 4),
+                                     bdesc0 + bo + static_cast<uint64_t>((kk * 32) >> 4), idesc,
+                                     (c > 0 || w > 0 || kk > 0) ? 1u : 0u);
+            }
             ptx::mma_commit(&empty[s]);
         }
         ptx::mma_commit(mma_done);

@@ -19,7 +19,9 @@
 //     M = MR feature rows (A, K-major from the weight; MR = 128, or 64 when
 //     the grid is small, for twice the CTAs) and N = NT tokens (B, K-major
 //     from the hidden states), K = H in 64-column chunks staged by TMA
-//     (128-byte swizzle) in a ring.  The accumulator lives in TMEM.
+//     (128-byte swizzle) in a ring.  The accumulator lives in TMEM.  The
+//     64-row CTAs (one wave) stage four chunks at a time, so that every
+//     weight and token row is read as 512 contiguous bytes.
 //   * A CTA's MR feature rows are the two rotation partners of MR / 2 pairs:
 //     features (MR/2) q + j (rows j) and (MR/2) q + 128 + j (rows MR/2 + j)
 //     of its head, so RoPE needs no data from another CTA.  The 256 / MR CTAs
@@ -102,7 +104,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const Params p)
 {
     static_assert(MR == 128 || MR == 64, "128 or 64 feature rows per CTA");
-    static_assert(W == 1 || W == 4, "one or four K chunks per stage");
+    static_assert(W == 1 || (W == 4 && MR == 64), "four K chunks per stage: the 64-row CTAs");
     using L = Smem<NT, STAGES, MR, W>;
     constexpr int kQ = L::kQ;
     constexpr int kHalf = MR / 2;  // rows per weight box: features [kHalf q, +kHalf) and [128 + kHalf q, +kHalf)

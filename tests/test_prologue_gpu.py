@@ -59,6 +59,8 @@ CASES = [
     (1, 50, 64, 8, 4, 900),            # one K chunk
     (1, 50, 2048, 4, 4, 900),          # one query head per key head
     (1, 16, 1024, 8, 1, 7),            # one key head
+    (1, 20, 768, 8, 4, 300),           # three 256-column groups (four-chunk stages, ring not wrapped)
+    (2, 30, 1280, 8, 4, [11, 3000]),   # five groups: the three-stage ring wraps
 ]
 
 

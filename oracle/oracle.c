@@ -511,7 +511,7 @@ int oracle_post_attention(const uint16_t *attn, const uint16_t *h, const uint16_
     return failed ? -7 : 0;
 }
 
-/* Number of OpenMP threads this build can use (1 without OpenMP). */
+/* Number of OpenMP threads the oracle can use (1 when compiled without OpenMP). */
 int oracle_max_threads(void)
 {
 #ifdef _OPENMP
